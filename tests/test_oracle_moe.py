@@ -1,0 +1,124 @@
+"""Pins for the oracle's expert grouping, SwiGLU expert MLP and layer combine (CPU only)."""
+import types
+
+import numpy as np
+import torch
+
+import oracle
+from oracle.moe import QuantTensor, _bf16_round
+from workloads import TINY, activations, router_weight, expert_weight
+
+
+def _cfg(shape):
+    return types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
+                                 topk=shape.topk, routed_scale=shape.routed_scale)
+
+
+def test_permutation_against_loop_and_invariants():
+    rng = np.random.default_rng(0)
+    T, k, E = 37, 8, 32
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    counts, offsets, perm, inv = oracle.permutation(idx, E)
+    # plain loop: walk experts, then tokens in order
+    want = [t * k + j for e in range(E) for t in range(T) for j in range(k) if idx[t, j] == e]
+    assert perm.tolist() == want
+    assert counts.sum() == T * k and offsets[-1] == T * k
+    np.testing.assert_array_equal(np.diff(offsets), counts)
+    np.testing.assert_array_equal(perm[inv.reshape(-1)], np.arange(T * k))
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(idx.reshape(-1)[seg] == e) and np.all(np.diff(seg // k) > 0)
+
+
+def test_permutation_empty_experts():
+    idx = np.array([[3, 1], [3, 1]])
+    counts, offsets, perm, inv = oracle.permutation(idx, 6)
+    assert counts.tolist() == [0, 2, 0, 2, 0, 0]
+    assert offsets.tolist() == [0, 0, 2, 2, 4, 4, 4]
+    assert perm.tolist() == [1, 3, 0, 2]
+
+
+def _qt(w):
+    return oracle.quantize_tensor(w.float().numpy())
+
+
+def test_expert_mlp_one_hot_input_closed_form():
+    """x = v * e_k picks column k of the gate/up weights: h_i = silu(v Wg[i,k]) * v Wu[i,k]."""
+    H, I = 64, 32
+    gate = _qt(expert_weight(TINY, 0, "gate")[:I, :H] * 40)
+    up = _qt(expert_weight(TINY, 0, "up")[:I, :H] * 40)
+    down = _qt(expert_weight(TINY, 0, "down")[:H, :I] * 40)
+    v, k = 1.5, 11
+    x = np.zeros((1, H))
+    x[0, k] = v
+    res = oracle.expert_mlp(x, gate, up, down, np.float32(0.01))
+    wg = gate.dequant()[:, k]
+    wu = up.dequant()[:, k]
+    h = (v * wg) / (1 + np.exp(-v * wg)) * (v * wu)
+    np.testing.assert_allclose(res["h"][0], h, rtol=1e-14, atol=1e-300)
+    # y = dequant(requant(h)) @ Wd^T, written as a per-output loop
+    hh = oracle.dequantize(res["hq_codes"], res["hq_scales"], np.float32(0.01))[0]
+    wd = down.dequant()
+    y = np.array([sum(hh[i] * wd[n, i] for i in range(I)) for n in range(H)])
+    np.testing.assert_allclose(res["y"][0], y, rtol=1e-12, atol=1e-15)
+
+
+def test_swiglu_special_values():
+    H, I = 32, 16
+    zero = QuantTensor(np.zeros((I, H // 2), np.uint8), np.zeros((I, H // 16), np.uint8), np.float32(1))
+    up = _qt(expert_weight(TINY, 1, "up")[:I, :H])
+    down = _qt(expert_weight(TINY, 1, "down")[:H, :I])
+    res = oracle.expert_mlp(np.ones((2, H)), zero, up, down, np.float32(0.01))
+    assert np.all(res["h"] == 0) and np.all(res["y"] == 0)
+
+
+def _tiny_layer(T=24):
+    shape = TINY
+    x = activations(T, shape).float().numpy()
+    wr = router_weight(shape).numpy()
+    ex = {e: tuple(_qt(expert_weight(shape, e, w)) for w in ("gate", "up", "down")) for e in range(shape.E)}
+    g_h = np.full(shape.E, np.float32(0.002), dtype=np.float32)
+    return shape, x, wr, ex, g_h
+
+
+def test_layer_combine_matches_dense_formulation():
+    """Gathered per-expert evaluation == every expert on every token, then a dense [T, E]
+    weight matrix; pins the pair/slot/expert indexing of the combine."""
+    shape, x, wr, ex, g_h = _tiny_layer()
+    cfg = _cfg(shape)
+    res = oracle.moe_forward(x, wr, cfg, lambda e: ex[e], g_h)
+    r = res["route"]
+    xhat = oracle.dequantize(res["xq_codes"], res["xq_scales"], res["g_x"])
+    dense_w = np.zeros((x.shape[0], shape.E))
+    np.put_along_axis(dense_w, r.idx, r.w, axis=1)
+    y_all = np.stack([oracle.expert_mlp(xhat, *ex[e], g_h[e])["y"] for e in range(shape.E)], axis=1)
+    out = np.einsum("te,teh->th", dense_w, y_all)
+    np.testing.assert_allclose(res["out"], out, rtol=1e-12, atol=1e-12)
+
+
+def test_layer_sampled_tokens_equal_full_run():
+    shape, x, wr, ex, g_h = _tiny_layer()
+    cfg = _cfg(shape)
+    full = oracle.moe_forward(x, wr, cfg, lambda e: ex[e], g_h)
+    part = oracle.moe_forward(x, wr, cfg, lambda e: ex[e], g_h, tokens=[3, 17, 5])
+    np.testing.assert_allclose(part["out"], full["out"][[3, 17, 5]], rtol=1e-12, atol=1e-15)
+
+
+def test_single_expert_layer_is_scaled_expert():
+    shape, x, wr, ex, g_h = _tiny_layer(8)
+    cfg = types.SimpleNamespace(E=shape.E, n_groups=1, topk_groups=1, topk=1, routed_scale=2.5)
+    res = oracle.moe_forward(x, wr, cfg, lambda e: ex[e], g_h)
+    xhat = oracle.dequantize(res["xq_codes"], res["xq_scales"], res["g_x"])
+    for t in range(8):
+        e = res["route"].idx[t, 0]
+        y = oracle.expert_mlp(xhat[t:t + 1], *ex[e], g_h[e])["y"][0]
+        np.testing.assert_allclose(res["out"][t], 2.5 * y, rtol=1e-12, atol=1e-15)
+
+
+def test_bf16_rounding_matches_torch():
+    v = np.random.default_rng(0).standard_normal(100000) * 3
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    # torch rounds FP64 -> BF16 via FP32; away from double-rounding cases they agree
+    v32 = v.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(_bf16_round(v32), torch.from_numpy(v32).to(torch.bfloat16).double().numpy())
+    assert np.mean(_bf16_round(v) == ref) > 0.999
