@@ -1,0 +1,215 @@
+/*
+ * nvfp4moe — NVFP4 (W4A4) group-limited mixture-of-experts layer for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libnvfp4moe.so.  The layer it computes:
+ *
+ *   * Router ("Reflection releases Beam ...", section "Mixture-of-Experts details"):
+ *     sigmoid scores s = 1/(1+exp(-x.W_r^T)) over E experts; experts split into
+ *     n_groups contiguous groups; keep the topk_groups groups with the largest sum of
+ *     their two best scores; select the topk best experts inside the kept groups;
+ *     weights w = routed_scale * s / sum(selected s).  Computed in FP32 (section
+ *     "Residual stream and numerical decisions").
+ *   * Experts: SwiGLU MLPs, y = W_down (silu(W_gate x) * (W_up x)), whose weights and
+ *     input activations are NVFP4 ("NVFP4 quantization", section "Quantization
+ *     scheme"): 4-bit E2M1 values, one FP8 E4M3 scale per 16 consecutive values along a
+ *     row, one FP32 global scale per tensor; a value decodes to E2M1 * E4M3 * global.
+ *   * Output: out[t] = sum over the token's selected experts of w * y, as BF16.
+ *
+ * Quantisation rule (the pages give the format, not the rule; this is the library's
+ * reading, with every FP32 step one IEEE round-to-nearest-even operation):
+ *     g   = A / 2688 (A = max|x| of the tensor; A == 0 -> g = 1)
+ *     r_t = 1 / (6 g)
+ *     S_b = E4M3_rn_satfinite(amax_b * r_t)      (block of 16 values, unsigned)
+ *     d_b = E4M3(S_b) * g,  r_b = (d_b == 0) ? 0 : 1 / d_b
+ *     c_i = E2M1_rn_satfinite(x_i * r_b)         (sign kept, also for zero)
+ *     byte j of a row holds c_{2j} in its low nibble and c_{2j+1} in its high nibble.
+ *   The layer input is quantised with a dynamic global scale (its own amax, all tokens of
+ *   the call); the SwiGLU intermediate h (FP32) with a static per-expert global scale g_h
+ *   supplied with the weights.
+ *
+ * Conventions for every call:
+ *   * Tensor pointers are DEVICE pointers owned by the caller unless stated otherwise;
+ *     row-major, densely packed.  BF16 is the IEEE bfloat16 bit pattern (uint16).
+ *   * `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous
+ *     on it and allocate nothing; they return after enqueueing work.
+ *   * Argument and shape errors are reported synchronously by the return code and
+ *     nothing is enqueued.  Errors found on the device (non-finite input, a bounded
+ *     wait that ran out) are OR-ed into a status word at the start of the caller's
+ *     workspace; nvfp4moe_status_read() returns it once the stream has finished.
+ *   * Workspaces are caller-allocated device memory, 256-byte aligned, of at least the
+ *     size the matching *_workspace_bytes() function returns.  A workspace must not be
+ *     used by two calls that can run at the same time.
+ *   * Scale layouts: NVFP4MOE_SCALES_LINEAR is [rows][cols/16] bytes.
+ *     NVFP4MOE_SCALES_SWIZZLED is the 128x4 tile layout of block-scaled tensor-core
+ *     operands: rows padded to a multiple of 128 and scale columns to a multiple of 4
+ *     (padding written as zero), 512-byte tiles of 128 rows x 4 scale columns ordered
+ *     row-tile-major then column tile, scale (r, c) at byte
+ *     (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4 inside its tile.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4MOE_API __attribute__((visibility("default")))
+#else
+#define NVFP4MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+typedef enum {
+  NVFP4MOE_OK = 0,
+  NVFP4MOE_ERR_ARG = -1,        /* NULL pointer, misaligned pointer, bad enum value */
+  NVFP4MOE_ERR_SHAPE = -2,      /* shape outside the supported limits */
+  NVFP4MOE_ERR_CUDA = -3,       /* a CUDA runtime/driver call failed */
+  NVFP4MOE_ERR_WORKSPACE = -4,  /* workspace smaller than required */
+  NVFP4MOE_ERR_NONFINITE = -5,  /* device status: the input held NaN or Inf */
+  NVFP4MOE_ERR_TIMEOUT = -6,    /* device status: a bounded wait inside a kernel ran out */
+  NVFP4MOE_ERR_DEVICE = -7      /* current device is not compute capability 10.0 */
+} nvfp4moe_status;
+
+enum { NVFP4MOE_SCALES_LINEAR = 0, NVFP4MOE_SCALES_SWIZZLED = 1 };
+
+/* Layer configuration.  Defaults (nvfp4moe_cfg_default) are the Beam layer:
+ * E=256, n_groups=8, topk_groups=4, topk=8, H=5120, I=2560, routed_scale=2.5
+ * ("Reflection releases Beam ...", sections "Model architecture and attention" and
+ * "Mixture-of-Experts details").
+ * Limits: H % 256 == 0, I % 128 == 0, 1 <= E <= 256, E % n_groups == 0,
+ * E / n_groups <= 32, 1 <= topk_groups <= n_groups <= 32, 1 <= topk <= 8,
+ * topk <= topk_groups * (E / n_groups). */
+typedef struct {
+  int32_t E;
+  int32_t n_groups;
+  int32_t topk_groups;
+  int32_t topk;
+  int32_t H;
+  int32_t I;
+  float routed_scale;
+} nvfp4moe_cfg;
+
+/* Fills *cfg with the Beam defaults.  Returns NVFP4MOE_ERR_ARG if cfg is NULL. */
+NVFP4MOE_API int nvfp4moe_cfg_default(nvfp4moe_cfg* cfg);
+
+/* Checks *cfg against the limits above: NVFP4MOE_OK or NVFP4MOE_ERR_SHAPE / _ARG. */
+NVFP4MOE_API int nvfp4moe_cfg_check(const nvfp4moe_cfg* cfg);
+
+/* ---------------------------------------------------------------- quantize ----
+ * quantize_nvfp4(x) -> codes + block scales + global scale
+ * ("NVFP4 quantization", section "Quantization scheme"; rule in the file header).
+ *
+ *   x_bf16   [rows][cols] BF16, cols % 64 == 0, rows >= 0.
+ *   g_in     NULL: the global scale is computed from max|x| (dynamic).  Otherwise a
+ *            device pointer to one FP32 global scale used as given (static).
+ *   codes    out, [rows][cols/2] bytes (even element in the low nibble).
+ *   scales   out, E4M3 block scales in `scale_layout` (linear: rows*cols/16 bytes;
+ *            swizzled: nvfp4moe_swizzled_scale_bytes(rows, cols/16) bytes).
+ *   g_out    out, device pointer to one FP32: the global scale used (may be NULL).
+ *   ws       workspace of nvfp4moe_quantize_workspace_bytes(rows, cols) bytes.
+ * A non-finite max|x| (dynamic scale) sets NVFP4MOE_ERR_NONFINITE in the status word;
+ * codes and scales are then unspecified. */
+NVFP4MOE_API size_t nvfp4moe_quantize_workspace_bytes(int64_t rows, int64_t cols);
+NVFP4MOE_API size_t nvfp4moe_swizzled_scale_bytes(int64_t rows, int64_t cols16);
+NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const float* g_in,
+                      uint8_t* codes, uint8_t* scales, int32_t scale_layout, float* g_out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------- route ----
+ * route(hidden, W_router) -> top-k experts and weights
+ * ("Reflection releases Beam ...", section "Mixture-of-Experts details").
+ *
+ *   hidden_bf16 [T][H] BF16;  w_router [E][H] FP32;  logit_bias [E] FP32 or NULL
+ *   (added to the logits before the sigmoid; the Beam router has none).
+ *   idx  out [T][topk] int32: selected experts by score descending, equal scores by
+ *        lower expert index (the same rule picks the groups).
+ *   w    out [T][topk] FP32: routed_scale * s / sum(selected s).
+ * Logits are FP32 sums of FP32 products; each is accumulated in runs of at most 32
+ * products, and the runs (at most H/32 + 32 of them, plus the bias) are added in a fixed
+ * order, so |logit - exact| <= (32 + H/32 + 33) * 2^-24 * sum_h |x_h W_eh| (+ |bias|). */
+NVFP4MOE_API size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
+NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
+                   const float* w_router, const float* logit_bias, int32_t* idx, float* w,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------------- experts ----
+ * Library-owned, repacked copy of the E experts' NVFP4 weights (the operand layout of
+ * the grouped GEMMs).  nvfp4moe_experts_create allocates it (device memory of the
+ * current device, about E * 3 * H * I * 0.5625 bytes) and is the only allocating call;
+ * nvfp4moe_experts_destroy frees it. */
+typedef struct nvfp4moe_experts nvfp4moe_experts;
+
+/* One expert's tensors, as nvfp4moe_quantize produces them with linear scales.
+ * Device pointers: gate/up codes [I][H/2], scales [I][H/16]; down codes [H][I/2],
+ * scales [H][I/16].  Global scales are host values.  g_h is the static global scale
+ * of the SwiGLU intermediate (input of the down projection). */
+typedef struct {
+  const uint8_t* gate_codes;
+  const uint8_t* gate_scales;
+  const uint8_t* up_codes;
+  const uint8_t* up_scales;
+  const uint8_t* down_codes;
+  const uint8_t* down_scales;
+  float g_gate;
+  float g_up;
+  float g_down;
+  float g_h;
+} nvfp4moe_expert_tensors;
+
+NVFP4MOE_API int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out);
+/* Copies expert e (0 <= e < E) into the handle, on `stream`.  The caller's buffers may be
+ * reused once the stream has passed this call. */
+NVFP4MOE_API int nvfp4moe_experts_set(nvfp4moe_experts* experts, int32_t e, const nvfp4moe_expert_tensors* t,
+                         void* stream);
+NVFP4MOE_API void nvfp4moe_experts_destroy(nvfp4moe_experts* experts);
+/* The handle's configuration (copied out). */
+NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_cfg* cfg);
+
+/* ----------------------------------------------------------------- forward ----
+ * moe_forward(hidden, experts) -> out: the whole layer (route, quantise x, group the
+ * token/expert pairs by expert, gate/up GEMM + SwiGLU + requantisation of h, down GEMM
+ * + weighted combine, BF16 output).
+ *
+ *   hidden_bf16 [T][H] BF16, 1 <= T <= T_max of the workspace;  w_router [E][H] FP32;
+ *   logit_bias [E] FP32 or NULL;  out_bf16 [T][H] BF16 (out).
+ *   dbg  NULL on the hot path.  Otherwise every non-NULL member receives a copy of that
+ *        intermediate (sizes below), for checking the layer step by step.
+ *   ws   workspace of nvfp4moe_forward_workspace_bytes(cfg, T_max) bytes. */
+typedef struct {
+  int32_t* idx;        /* [T][topk] selected experts */
+  float* w;            /* [T][topk] routing weights */
+  float* g_x;          /* [1] global scale of the quantised layer input */
+  uint8_t* xq_codes;   /* [T][H/2] quantised layer input */
+  uint8_t* xq_scales;  /* [T][H/16] its block scales, linear */
+  int32_t* counts;     /* [E] pairs per expert */
+  int32_t* offsets;    /* [E+1] exclusive scan of counts */
+  int32_t* perm;       /* [T*topk] pair ids (t*topk + j) grouped by expert, tokens ascending */
+  uint8_t* hq_codes;   /* [T*topk][I/2] quantised SwiGLU intermediate, rows in perm order */
+  uint8_t* hq_scales;  /* [T*topk][I/16] its block scales, linear */
+} nvfp4moe_debug;
+
+NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
+NVFP4MOE_API int nvfp4moe_forward(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
+                     const float* w_router, const float* logit_bias, void* out_bf16,
+                     const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ status ----
+ * Waits for `stream`, then returns the device-side status of the last call that used
+ * workspace `ws` (NVFP4MOE_OK, _ERR_NONFINITE or _ERR_TIMEOUT; _ERR_CUDA if the wait or
+ * the read failed). */
+NVFP4MOE_API int nvfp4moe_status_read(const void* ws, void* stream);
+NVFP4MOE_API const char* nvfp4moe_status_string(int status);
+
+/* Number of kernels the last nvfp4moe_forward / _route / _quantize call on this host
+ * thread enqueued (for launch accounting in benchmarks). */
+NVFP4MOE_API int32_t nvfp4moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4MOE_H */

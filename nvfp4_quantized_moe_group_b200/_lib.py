@@ -1,0 +1,276 @@
+"""ctypes binding of libnvfp4moe.so: argument marshalling only.
+
+Every call forwards torch tensors' device pointers and the current CUDA stream to the
+C ABI declared in include/nvfp4moe.h; all arithmetic runs in the library's sm_100a
+kernels.  torch is used for device memory (outputs and workspaces) and streams.
+Loading fails loudly when the library is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libnvfp4moe.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "nvfp4moe.h")
+
+OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_WORKSPACE, ERR_NONFINITE, ERR_TIMEOUT, ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6, -7
+SCALES_LINEAR, SCALES_SWIZZLED = 0, 1
+
+
+class NvFp4MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int32), ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("routed_scale", ctypes.c_float)]
+
+    def __repr__(self):
+        return (f"Cfg(E={self.E}, n_groups={self.n_groups}, topk_groups={self.topk_groups}, "
+                f"topk={self.topk}, H={self.H}, I={self.I}, routed_scale={self.routed_scale})")
+
+
+class ExpertTensors(ctypes.Structure):
+    _fields_ = [("gate_codes", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p),
+                ("up_codes", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+                ("down_codes", ctypes.c_void_p), ("down_scales", ctypes.c_void_p),
+                ("g_gate", ctypes.c_float), ("g_up", ctypes.c_float), ("g_down", ctypes.c_float),
+                ("g_h", ctypes.c_float)]
+
+
+class Debug(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("idx", "w", "g_x", "xq_codes", "xq_scales", "counts", "offsets",
+                                               "perm", "hq_codes", "hq_scales")]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "nvfp4moe_cfg_default": (ctypes.c_int, [ctypes.POINTER(Cfg)]),
+    "nvfp4moe_cfg_check": (ctypes.c_int, [ctypes.POINTER(Cfg)]),
+    "nvfp4moe_quantize_workspace_bytes": (_SZ, [_I64, _I64]),
+    "nvfp4moe_swizzled_scale_bytes": (_SZ, [_I64, _I64]),
+    "nvfp4moe_quantize": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, ctypes.c_int32, _P, _P, _SZ, _P]),
+    "nvfp4moe_route_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
+    "nvfp4moe_route": (ctypes.c_int, [ctypes.POINTER(Cfg), _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nvfp4moe_experts_create": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.POINTER(_P)]),
+    "nvfp4moe_experts_set": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(ExpertTensors), _P]),
+    "nvfp4moe_experts_destroy": (None, [_P]),
+    "nvfp4moe_experts_cfg": (ctypes.c_int, [_P, ctypes.POINTER(Cfg)]),
+    "nvfp4moe_forward_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
+    "nvfp4moe_forward": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_status_read": (ctypes.c_int, [_P, _P]),
+    "nvfp4moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nvfp4moe_last_launch_count": (ctypes.c_int32, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m nvfp4_quantized_moe_group_b200.build` (needs nvcc 12.9)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the entry points include/nvfp4moe.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"NVFP4MOE_API\s+[\w\s\*]+?\b(nvfp4moe_\w+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise NvFp4MoeError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's allocator returns blocks aligned to at least 512 bytes
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def cfg_default() -> Cfg:
+    c = Cfg()
+    _check(lib().nvfp4moe_cfg_default(ctypes.byref(c)), "nvfp4moe_cfg_default")
+    return c
+
+
+def make_cfg(E, n_groups, topk_groups, topk, H, I, routed_scale=2.5) -> Cfg:
+    c = Cfg(E, n_groups, topk_groups, topk, H, I, routed_scale)
+    _check(lib().nvfp4moe_cfg_check(ctypes.byref(c)), "nvfp4moe_cfg_check")
+    return c
+
+
+def last_launch_count() -> int:
+    return int(lib().nvfp4moe_last_launch_count())
+
+
+def status_read(ws: torch.Tensor, stream=None) -> int:
+    return int(lib().nvfp4moe_status_read(_ptr(ws), _stream(stream)))
+
+
+def swizzled_scale_bytes(rows: int, cols16: int) -> int:
+    return int(lib().nvfp4moe_swizzled_scale_bytes(rows, cols16))
+
+
+def quantize_workspace_bytes(rows: int, cols: int) -> int:
+    return int(lib().nvfp4moe_quantize_workspace_bytes(rows, cols))
+
+
+def quantize(x: torch.Tensor, g: torch.Tensor | None = None, swizzled: bool = False, ws=None, out=None,
+             stream=None):
+    """quantize_nvfp4(x) -> (codes [rows, cols/2] u8, scales u8, g [1] f32).
+
+    ``g``: None for a dynamic global scale, else a 1-element CUDA float32 tensor.
+    Scales are [rows, cols/16] (linear) or the flat swizzled array.
+    """
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 CUDA tensor")
+    rows, cols = x.shape
+    dev = x.device
+    if out is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+        if swizzled:
+            scales = torch.empty(swizzled_scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
+        else:
+            scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+        g_out = torch.empty(1, dtype=torch.float32, device=dev)
+    else:
+        codes, scales, g_out = out
+    if ws is None:
+        ws = _workspace(quantize_workspace_bytes(rows, cols), dev)
+    st = lib().nvfp4moe_quantize(_ptr(x), rows, cols, _ptr(g), _ptr(codes), _ptr(scales),
+                                 SCALES_SWIZZLED if swizzled else SCALES_LINEAR, _ptr(g_out), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    _check(st, "nvfp4moe_quantize")
+    return codes, scales, g_out
+
+
+def route_workspace_bytes(cfg: Cfg, T: int) -> int:
+    return int(lib().nvfp4moe_route_workspace_bytes(ctypes.byref(cfg), T))
+
+
+def route(cfg: Cfg, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None, ws=None,
+          stream=None):
+    """route(hidden, W_router) -> (idx [T, topk] int32, w [T, topk] float32)."""
+    T = x.shape[0]
+    dev = x.device
+    idx = torch.empty((T, cfg.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.topk), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(route_workspace_bytes(cfg, T), dev)
+    st = lib().nvfp4moe_route(ctypes.byref(cfg), _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(idx), _ptr(w),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "nvfp4moe_route")
+    return idx, w
+
+
+class Experts:
+    """Library-owned NVFP4 expert weights (nvfp4moe_experts_create / _set / _destroy)."""
+
+    def __init__(self, cfg: Cfg):
+        self.cfg = cfg
+        h = ctypes.c_void_p()
+        _check(lib().nvfp4moe_experts_create(ctypes.byref(cfg), ctypes.byref(h)), "nvfp4moe_experts_create")
+        self.handle = h
+
+    def set(self, e: int, gate, up, down, g_h: float, stream=None):
+        """gate/up/down: (codes, linear scales, global scale as float) from quantize()."""
+        t = ExpertTensors(gate[0].data_ptr(), gate[1].data_ptr(), up[0].data_ptr(), up[1].data_ptr(),
+                          down[0].data_ptr(), down[1].data_ptr(), float(gate[2]), float(up[2]),
+                          float(down[2]), float(g_h))
+        _check(lib().nvfp4moe_experts_set(self.handle, int(e), ctypes.byref(t), _stream(stream)),
+               "nvfp4moe_experts_set")
+
+    def set_from_bf16(self, e: int, gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor, g_h: float,
+                      stream=None):
+        """Quantise BF16 gate [I, H], up [I, H], down [H, I] with nvfp4moe_quantize (dynamic
+        per-tensor global scales, linear block scales) and copy them into expert e."""
+        q = [quantize(w, stream=stream) for w in (gate, up, down)]
+        gs = torch.cat([t[2] for t in q]).cpu().tolist()
+        self.set(e, (q[0][0], q[0][1], gs[0]), (q[1][0], q[1][1], gs[1]), (q[2][0], q[2][1], gs[2]), g_h,
+                 stream=stream)
+        return gs
+
+    def close(self):
+        if self.handle:
+            lib().nvfp4moe_experts_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def forward_workspace_bytes(cfg: Cfg, T_max: int) -> int:
+    return int(lib().nvfp4moe_forward_workspace_bytes(ctypes.byref(cfg), T_max))
+
+
+def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
+            out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None):
+    """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug)."""
+    cfg = experts.cfg
+    T, H = x.shape
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(cfg, T), dev)
+    dbg = None
+    tensors = None
+    if debug:
+        k, E, I = cfg.topk, cfg.E, cfg.I
+        tensors = {
+            "idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "w": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "g_x": torch.empty(1, dtype=torch.float32, device=dev),
+            "xq_codes": torch.empty((T, H // 2), dtype=torch.uint8, device=dev),
+            "xq_scales": torch.empty((T, H // 16), dtype=torch.uint8, device=dev),
+            "counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "hq_codes": torch.empty((T * k, I // 2), dtype=torch.uint8, device=dev),
+            "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
+        }
+        dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
+    st = lib().nvfp4moe_forward(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(out),
+                                ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(st, "nvfp4moe_forward")
+    if debug:
+        return out, tensors
+    return out

@@ -1,0 +1,557 @@
+// C ABI of libnvfp4moe: argument checking, workspace layout and the launch sequences of the
+// quantize / route / forward calls.  Declarations and contracts are in nvfp4moe.h.
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace nvfp4moe;
+
+struct nvfp4moe_experts {
+  nvfp4moe_cfg cfg;
+  int device;
+  uint8_t* w13_codes;   // [E][2I][H/2], gate and up rows interleaved per 128-row tile
+  uint8_t* w13_sf;      // swizzled, [E][2I/128 tiles][H/64 column tiles][512]
+  uint8_t* wd_codes;    // [E][H][I/2]
+  uint8_t* wd_sf;       // swizzled, [E][H/128][I/64][512]
+  float* g_gate;        // [E] device
+  float* g_up;
+  float* g_h;
+  float* alpha_down;    // [E] g_h * g_down
+  CUtensorMap tma_w13;
+  CUtensorMap tma_wd;
+};
+
+namespace {
+
+thread_local int32_t g_launches = 0;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA; }
+
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  return (major == 10 && minor == 0) ? NVFP4MOE_OK : NVFP4MOE_ERR_DEVICE;
+}
+
+// Carves a workspace into 256-byte aligned pieces.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
+
+struct QuantWs {
+  WsHeader* hdr;
+  uint32_t* partials;
+  size_t bytes;
+};
+
+QuantWs carve_quant(void* ws) {
+  Carver c(ws);
+  QuantWs q;
+  q.hdr = c.take<WsHeader>(1);
+  q.partials = c.take<uint32_t>(kMaxAmaxPartials);
+  q.bytes = c.off;
+  return q;
+}
+
+struct RouteWs {
+  WsHeader* hdr;
+  float* parts;
+  size_t bytes;
+};
+
+RouteWs carve_route(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
+  Carver c(ws);
+  RouteWs r;
+  r.hdr = c.take<WsHeader>(1);
+  r.parts = c.take<float>(router_parts_elems(T, cfg.E, cfg.H));
+  r.bytes = c.off;
+  return r;
+}
+
+int64_t rows_capacity(const nvfp4moe_cfg& cfg, int64_t T) {
+  const int64_t pairs = T * cfg.topk;
+  const int64_t pad = 127 * (pairs < cfg.E ? pairs : cfg.E);
+  return round128(pairs + pad);
+}
+
+struct ForwardWs {
+  WsHeader* hdr;
+  uint32_t* partials;
+  float* g_x;
+  float* parts;
+  int32_t* idx;
+  float* wts;
+  uint8_t* xq_codes;
+  uint8_t* xq_sf;
+  float* acc;
+  int32_t* chunk_counts;
+  int32_t* chunk_base;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile_prefix;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* row_pair;
+  uint8_t* a_codes;
+  uint8_t* a_sf;
+  uint8_t* hq_codes;
+  uint8_t* hq_sf;
+  int64_t rows_cap;
+  size_t bytes;
+};
+
+ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
+  Carver c(ws);
+  ForwardWs f;
+  const int64_t pairs = T * cfg.topk;
+  const int64_t n_chunks = (T + kPermChunkTokens - 1) / kPermChunkTokens;
+  f.rows_cap = rows_capacity(cfg, T);
+  f.hdr = c.take<WsHeader>(1);
+  f.partials = c.take<uint32_t>(kMaxAmaxPartials);
+  f.g_x = c.take<float>(1);
+  f.parts = c.take<float>(router_parts_elems(T, cfg.E, cfg.H));
+  f.idx = c.take<int32_t>(pairs);
+  f.wts = c.take<float>(pairs);
+  f.xq_codes = c.take<uint8_t>(T * cfg.H / 2);
+  f.xq_sf = c.take<uint8_t>(round128(T) * cfg.H / 16);
+  f.acc = c.take<float>(T * cfg.H);
+  f.chunk_counts = c.take<int32_t>(n_chunks * cfg.E);
+  f.chunk_base = c.take<int32_t>(n_chunks * cfg.E);
+  f.counts = c.take<int32_t>(cfg.E);
+  f.offsets = c.take<int32_t>(cfg.E + 1);
+  f.mtile_prefix = c.take<int32_t>(cfg.E + 1);
+  f.perm = c.take<int32_t>(pairs);
+  f.inv = c.take<int32_t>(pairs);
+  f.row_pair = c.take<int32_t>(f.rows_cap);
+  f.a_codes = c.take<uint8_t>(f.rows_cap * cfg.H / 2);
+  f.a_sf = c.take<uint8_t>(f.rows_cap * cfg.H / 16);
+  f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg.I / 2);
+  f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg.I / 16);
+  f.bytes = c.off;
+  return f;
+}
+
+__global__ void set_expert_scalars_kernel(float* g_gate, float* g_up, float* g_h, float* alpha, int e,
+                                          float gg, float gu, float gh, float gd) {
+  g_gate[e] = gg;
+  g_up[e] = gu;
+  g_h[e] = gh;
+  alpha[e] = __fmul_rn(gh, gd);
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4moe_cfg_default(nvfp4moe_cfg* cfg) {
+  if (cfg == nullptr) return NVFP4MOE_ERR_ARG;
+  cfg->E = 256;
+  cfg->n_groups = 8;
+  cfg->topk_groups = 4;
+  cfg->topk = 8;
+  cfg->H = 5120;
+  cfg->I = 2560;
+  cfg->routed_scale = 2.5f;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_cfg_check(const nvfp4moe_cfg* c) {
+  if (c == nullptr) return NVFP4MOE_ERR_ARG;
+  if (c->H <= 0 || c->I <= 0 || c->H % 256 != 0 || c->I % 128 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (c->E < 1 || c->E > 256 || c->n_groups < 1 || c->n_groups > 32 || c->E % c->n_groups != 0)
+    return NVFP4MOE_ERR_SHAPE;
+  if (c->E / c->n_groups > 32) return NVFP4MOE_ERR_SHAPE;
+  if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return NVFP4MOE_ERR_SHAPE;
+  if (c->topk < 1 || c->topk > 8 || c->topk > c->topk_groups * (c->E / c->n_groups))
+    return NVFP4MOE_ERR_SHAPE;
+  if (!(c->routed_scale == c->routed_scale)) return NVFP4MOE_ERR_ARG;
+  return NVFP4MOE_OK;
+}
+
+size_t nvfp4moe_swizzled_scale_bytes(int64_t rows, int64_t cols16) {
+  if (rows < 0 || cols16 < 0) return 0;
+  return (size_t)round128(rows) * (size_t)((cols16 + 3) / 4 * 4);
+}
+
+size_t nvfp4moe_quantize_workspace_bytes(int64_t rows, int64_t cols) {
+  (void)rows;
+  (void)cols;
+  return carve_quant(nullptr).bytes;
+}
+
+int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const float* g_in, uint8_t* codes,
+                      uint8_t* scales, int32_t scale_layout, float* g_out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  g_launches = 0;
+  if (rows < 0 || cols <= 0 || cols % 64 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (scale_layout != NVFP4MOE_SCALES_LINEAR && scale_layout != NVFP4MOE_SCALES_SWIZZLED)
+    return NVFP4MOE_ERR_ARG;
+  if (ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
+  if ((rows > 0 || scale_layout == NVFP4MOE_SCALES_SWIZZLED) && (scales == nullptr || !aligned(scales, 4)))
+    return NVFP4MOE_ERR_ARG;
+  if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || !aligned(x_bf16, 16) || !aligned(codes, 16)))
+    return NVFP4MOE_ERR_ARG;
+  const QuantWs q = carve_quant(ws);
+  if (ws_bytes < q.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  int blocks = 0;
+  if (g_in == nullptr) {
+    blocks = amax_partial_blocks(rows * cols);
+    if (launch_amax_partial(x_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess)
+      return NVFP4MOE_ERR_CUDA;
+    ++g_launches;
+  }
+  QuantizeArgs a{};
+  a.x = static_cast<const uint16_t*>(x_bf16);
+  a.rows = rows;
+  a.rows_padded = scale_layout == NVFP4MOE_SCALES_SWIZZLED ? round128(rows) : rows;
+  a.cols = cols;
+  a.g_in = g_in;
+  a.partials = q.partials;
+  a.n_partials = blocks;
+  a.codes = codes;
+  a.scales = scales;
+  a.swizzled = scale_layout == NVFP4MOE_SCALES_SWIZZLED;
+  a.n_col_tiles = cols / 64;
+  a.g_out = g_out;
+  a.zero_out = nullptr;
+  a.status = &q.hdr->status;
+  if (launch_quantize(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  return NVFP4MOE_OK;
+}
+
+size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T) {
+  if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || T < 0) return 0;
+  return carve_route(nullptr, *cfg, T > 0 ? T : 1).bytes;
+}
+
+int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, const float* w_router,
+                   const float* logit_bias, int32_t* idx, float* w, void* ws, size_t ws_bytes,
+                   void* stream) {
+  g_launches = 0;
+  int st = nvfp4moe_cfg_check(cfg);
+  if (st != NVFP4MOE_OK) return st;
+  if (T < 0 || T > (1 << 24)) return NVFP4MOE_ERR_SHAPE;
+  if (ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
+  if (T > 0 && (hidden_bf16 == nullptr || w_router == nullptr || idx == nullptr || w == nullptr ||
+                !aligned(hidden_bf16, 16) || !aligned(w_router, 16)))
+    return NVFP4MOE_ERR_ARG;
+  const RouteWs r = carve_route(ws, *cfg, T > 0 ? T : 1);
+  if (ws_bytes < r.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&r.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (T == 0) return NVFP4MOE_OK;
+  RouterArgs a{};
+  a.x = static_cast<const uint16_t*>(hidden_bf16);
+  a.w = w_router;
+  a.bias = logit_bias;
+  a.parts = r.parts;
+  a.idx = idx;
+  a.wts = w;
+  a.T = T;
+  a.H = cfg->H;
+  a.E = cfg->E;
+  a.n_groups = cfg->n_groups;
+  a.topk_groups = cfg->topk_groups;
+  a.topk = cfg->topk;
+  a.routed_scale = cfg->routed_scale;
+  if (launch_router(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 2;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out) {
+  if (out == nullptr) return NVFP4MOE_ERR_ARG;
+  *out = nullptr;
+  int st = nvfp4moe_cfg_check(cfg);
+  if (st != NVFP4MOE_OK) return st;
+  st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  nvfp4moe_experts* x = new nvfp4moe_experts();
+  std::memset(x, 0, sizeof(*x));
+  x->cfg = *cfg;
+  cudaGetDevice(&x->device);
+  const int64_t E = cfg->E, H = cfg->H, I = cfg->I;
+  const size_t w13 = (size_t)E * 2 * I * H / 2, w13sf = (size_t)E * 2 * I * H / 16;
+  const size_t wd = (size_t)E * H * I / 2, wdsf = (size_t)E * H * I / 16;
+  bool ok = cudaMalloc(&x->w13_codes, w13) == cudaSuccess && cudaMalloc(&x->w13_sf, w13sf) == cudaSuccess &&
+            cudaMalloc(&x->wd_codes, wd) == cudaSuccess && cudaMalloc(&x->wd_sf, wdsf) == cudaSuccess &&
+            cudaMalloc(&x->g_gate, E * sizeof(float)) == cudaSuccess &&
+            cudaMalloc(&x->g_up, E * sizeof(float)) == cudaSuccess &&
+            cudaMalloc(&x->g_h, E * sizeof(float)) == cudaSuccess &&
+            cudaMalloc(&x->alpha_down, E * sizeof(float)) == cudaSuccess;
+  ok = ok && make_tma_2d(&x->tma_w13, x->w13_codes, H / 2, (uint64_t)E * 2 * I, kBlockN) == 0;
+  ok = ok && make_tma_2d(&x->tma_wd, x->wd_codes, I / 2, (uint64_t)E * H, kBlockN) == 0;
+  if (!ok) {
+    nvfp4moe_experts_destroy(x);
+    return NVFP4MOE_ERR_CUDA;
+  }
+  *out = x;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e, const nvfp4moe_expert_tensors* t, void* stream) {
+  g_launches = 0;
+  if (x == nullptr || t == nullptr) return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = x->cfg;
+  if (e < 0 || e >= c.E) return NVFP4MOE_ERR_ARG;
+  if (!t->gate_codes || !t->gate_scales || !t->up_codes || !t->up_scales || !t->down_codes || !t->down_scales)
+    return NVFP4MOE_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t H = c.H, I = c.I;
+  const size_t tile_gu = (size_t)128 * H / 2;  // bytes of 128 rows of gate/up codes
+  uint8_t* w13 = x->w13_codes + (size_t)e * 2 * I * H / 2;
+  // gate tile j -> packed tile 2j, up tile j -> packed tile 2j+1
+  if (cudaMemcpy2DAsync(w13, 2 * tile_gu, t->gate_codes, tile_gu, tile_gu, I / 128, cudaMemcpyDeviceToDevice,
+                        s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  if (cudaMemcpy2DAsync(w13 + tile_gu, 2 * tile_gu, t->up_codes, tile_gu, tile_gu, I / 128,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(x->wd_codes + (size_t)e * H * I / 2, t->down_codes, (size_t)H * I / 2,
+                      cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  uint8_t* w13sf = x->w13_sf + (size_t)e * 2 * I * H / 16;
+  if (launch_repack_sf(t->gate_scales, (int)I, (int)(H / 16), w13sf, H / 64, (2 << 8) | 0, s) != cudaSuccess ||
+      launch_repack_sf(t->up_scales, (int)I, (int)(H / 16), w13sf, H / 64, (2 << 8) | 1, s) != cudaSuccess ||
+      launch_repack_sf(t->down_scales, (int)H, (int)(I / 16), x->wd_sf + (size_t)e * H * I / 16, I / 64,
+                       (1 << 8) | 0, s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  set_expert_scalars_kernel<<<1, 1, 0, s>>>(x->g_gate, x->g_up, x->g_h, x->alpha_down, e, t->g_gate, t->g_up,
+                                            t->g_h, t->g_down);
+  if (cudaGetLastError() != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 4;
+  return NVFP4MOE_OK;
+}
+
+void nvfp4moe_experts_destroy(nvfp4moe_experts* x) {
+  if (x == nullptr) return;
+  cudaFree(x->w13_codes);
+  cudaFree(x->w13_sf);
+  cudaFree(x->wd_codes);
+  cudaFree(x->wd_sf);
+  cudaFree(x->g_gate);
+  cudaFree(x->g_up);
+  cudaFree(x->g_h);
+  cudaFree(x->alpha_down);
+  delete x;
+}
+
+int nvfp4moe_experts_cfg(const nvfp4moe_experts* x, nvfp4moe_cfg* cfg) {
+  if (x == nullptr || cfg == nullptr) return NVFP4MOE_ERR_ARG;
+  *cfg = x->cfg;
+  return NVFP4MOE_OK;
+}
+
+size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) {
+  if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || T_max < 1) return 0;
+  return carve_forward(nullptr, *cfg, T_max).bytes;
+}
+
+int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
+                     const float* logit_bias, void* out_bf16, const nvfp4moe_debug* dbg, void* ws,
+                     size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (x == nullptr) return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = x->cfg;
+  if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
+  if (hidden_bf16 == nullptr || w_router == nullptr || out_bf16 == nullptr || ws == nullptr)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(out_bf16, 16) || !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  const ForwardWs f = carve_forward(ws, c, T);
+  if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t pairs = T * c.topk;
+
+  CUtensorMap tma_a, tma_h;
+  if (make_tma_2d(&tma_a, f.a_codes, c.H / 2, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_h, f.hq_codes, c.I / 2, f.rows_cap, kBlockM) != 0)
+    return NVFP4MOE_ERR_CUDA;
+
+  if (cudaMemsetAsync(&f.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  const int blocks = amax_partial_blocks(T * c.H);
+  if (launch_amax_partial(hidden_bf16, T * c.H, f.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  RouterArgs r{};
+  r.x = static_cast<const uint16_t*>(hidden_bf16);
+  r.w = w_router;
+  r.bias = logit_bias;
+  r.parts = f.parts;
+  r.idx = f.idx;
+  r.wts = f.wts;
+  r.T = T;
+  r.H = c.H;
+  r.E = c.E;
+  r.n_groups = c.n_groups;
+  r.topk_groups = c.topk_groups;
+  r.topk = c.topk;
+  r.routed_scale = c.routed_scale;
+  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 2;
+
+  QuantizeArgs q{};
+  q.x = static_cast<const uint16_t*>(hidden_bf16);
+  q.rows = T;
+  q.rows_padded = round128(T);
+  q.cols = c.H;
+  q.g_in = nullptr;
+  q.partials = f.partials;
+  q.n_partials = blocks;
+  q.codes = f.xq_codes;
+  q.scales = f.xq_sf;
+  q.swizzled = 1;
+  q.n_col_tiles = c.H / 64;
+  q.g_out = f.g_x;
+  q.zero_out = f.acc;
+  q.status = &f.hdr->status;
+  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  PermArgs pa{};
+  pa.idx = f.idx;
+  pa.T = T;
+  pa.topk = c.topk;
+  pa.E = c.E;
+  pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
+  pa.chunk_counts = f.chunk_counts;
+  pa.chunk_base = f.chunk_base;
+  pa.counts = f.counts;
+  pa.offsets = f.offsets;
+  pa.mtile_prefix = f.mtile_prefix;
+  pa.perm = f.perm;
+  pa.inv = f.inv;
+  pa.row_pair = f.row_pair;
+  if (launch_permute(pa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 3;
+
+  GatherArgs ga{};
+  ga.xq_codes = f.xq_codes;
+  ga.xq_sf = f.xq_sf;
+  ga.idx = f.idx;
+  ga.inv = f.inv;
+  ga.offsets = f.offsets;
+  ga.mtile_prefix = f.mtile_prefix;
+  ga.a_codes = f.a_codes;
+  ga.a_sf = f.a_sf;
+  ga.n_pairs = pairs;
+  ga.topk = c.topk;
+  ga.H = c.H;
+  if (launch_gather(ga, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  const int grid = num_sms();
+  GemmArgs g{};
+  g.sfa = f.a_sf;
+  g.sfb = x->w13_sf;
+  g.mtile_prefix = f.mtile_prefix;
+  g.counts = f.counts;
+  g.E = c.E;
+  g.K = c.H;
+  g.n_total = 2 * c.I;
+  g.status = &f.hdr->status;
+  g.hq_codes = f.hq_codes;
+  g.hq_sf = f.hq_sf;
+  g.g_x = f.g_x;
+  g.g_gate = x->g_gate;
+  g.g_up = x->g_up;
+  g.g_h = x->g_h;
+  g.I = c.I;
+  g.acc = f.acc;
+  g.row_pair = f.row_pair;
+  g.wts = f.wts;
+  g.alpha_down = x->alpha_down;
+  g.topk = c.topk;
+  g.H = c.H;
+  if (launch_gemm_gateup(tma_a, x->tma_w13, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  g.sfa = f.hq_sf;
+  g.sfb = x->wd_sf;
+  g.K = c.I;
+  g.n_total = c.H;
+  if (launch_gemm_down(tma_h, x->tma_wd, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H};
+  if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  if (dbg != nullptr) {
+    bool ok = true;
+    if (dbg->idx) ok &= cudaMemcpyAsync(dbg->idx, f.idx, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->w) ok &= cudaMemcpyAsync(dbg->w, f.wts, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->g_x) ok &= cudaMemcpyAsync(dbg->g_x, f.g_x, 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->xq_codes)
+      ok &= cudaMemcpyAsync(dbg->xq_codes, f.xq_codes, T * c.H / 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->xq_scales)
+      ok &= launch_unswizzle_rows(f.xq_sf, c.H / 64, nullptr, T, c.H / 16, dbg->xq_scales, s) == cudaSuccess;
+    if (dbg->counts) ok &= cudaMemcpyAsync(dbg->counts, f.counts, c.E * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->offsets)
+      ok &= cudaMemcpyAsync(dbg->offsets, f.offsets, (c.E + 1) * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->perm) ok &= cudaMemcpyAsync(dbg->perm, f.perm, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->hq_codes && dbg->hq_scales)
+      ok &= launch_export_hq(f.hq_codes, f.hq_sf, f.perm, f.idx, f.offsets, f.mtile_prefix, pairs, c.I,
+                             dbg->hq_codes, dbg->hq_scales, s) == cudaSuccess;
+    if (!ok) return NVFP4MOE_ERR_CUDA;
+  }
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_status_read(const void* ws, void* stream) {
+  if (ws == nullptr) return NVFP4MOE_ERR_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (v & kStatusTimeout) return NVFP4MOE_ERR_TIMEOUT;
+  if (v & kStatusNonFinite) return NVFP4MOE_ERR_NONFINITE;
+  return NVFP4MOE_OK;
+}
+
+const char* nvfp4moe_status_string(int status) {
+  switch (status) {
+    case NVFP4MOE_OK: return "ok";
+    case NVFP4MOE_ERR_ARG: return "invalid argument";
+    case NVFP4MOE_ERR_SHAPE: return "unsupported shape";
+    case NVFP4MOE_ERR_CUDA: return "CUDA call failed";
+    case NVFP4MOE_ERR_WORKSPACE: return "workspace too small";
+    case NVFP4MOE_ERR_NONFINITE: return "non-finite input";
+    case NVFP4MOE_ERR_TIMEOUT: return "bounded device wait ran out";
+    case NVFP4MOE_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
+    default: return "unknown status";
+  }
+}
+
+int32_t nvfp4moe_last_launch_count(void) { return g_launches; }
+
+}  // extern "C"

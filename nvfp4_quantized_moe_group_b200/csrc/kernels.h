@@ -1,0 +1,143 @@
+// Internal kernel interfaces of libnvfp4moe (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4moe {
+
+constexpr int kMaxAmaxPartials = 1024;   // blocks of the amax pass
+constexpr int kBlockM = 128;             // token rows per GEMM tile / expert segment padding
+constexpr int kBlockN = 256;             // output columns per GEMM tile
+constexpr int kBlockK = 256;             // K values per pipeline stage (128 bytes of E2M1)
+constexpr int kPermChunkTokens = 128;    // tokens per chunk of the grouping kernels
+
+struct QuantizeArgs {
+  const uint16_t* x;       // [rows][cols] bf16
+  int64_t rows;
+  int64_t rows_padded;     // rows rounded up to 128 in the swizzled layout, else rows
+  int64_t cols;
+  const float* g_in;       // static scale or nullptr
+  const uint32_t* partials;
+  int n_partials;
+  uint8_t* codes;
+  uint8_t* scales;
+  int swizzled;
+  int64_t n_col_tiles;     // ceil(cols/16/4)
+  float* g_out;
+  float* zero_out;         // optional [rows][cols] fp32 zeroed alongside (layer accumulator)
+  uint32_t* status;
+};
+
+struct RouterArgs {
+  const uint16_t* x;       // [T][H] bf16
+  const float* w;          // [E][H]
+  const float* bias;       // [E] or nullptr
+  float* parts;            // [ksplit][T][E]
+  int32_t* idx;            // [T][topk]
+  float* wts;              // [T][topk]
+  int64_t T;
+  int H, E, n_groups, topk_groups, topk;
+  float routed_scale;
+  int ksplit, k_slice;
+};
+
+struct PermArgs {
+  const int32_t* idx;      // [T][topk]
+  int64_t T;
+  int topk, E;
+  int n_chunks;
+  int32_t* chunk_counts;   // [n_chunks][E]
+  int32_t* chunk_base;     // [n_chunks][E]
+  int32_t* counts;         // [E]
+  int32_t* offsets;        // [E+1]
+  int32_t* mtile_prefix;   // [E+1] cumulative 128-row tiles
+  int32_t* perm;           // [T*topk]
+  int32_t* inv;            // [T*topk]
+  int32_t* row_pair;       // [rows_cap] pair id of each padded row, -1 for padding
+};
+
+struct GatherArgs {
+  const uint8_t* xq_codes;   // [T][H/2]
+  const uint8_t* xq_sf;      // swizzled, rows = tokens
+  const int32_t* idx;
+  const int32_t* inv;
+  const int32_t* offsets;
+  const int32_t* mtile_prefix;
+  uint8_t* a_codes;          // [rows_cap][H/2]
+  uint8_t* a_sf;             // swizzled, rows = padded rows
+  int64_t n_pairs;
+  int topk;
+  int H;
+};
+
+struct GemmArgs {
+  const uint8_t* sfa;          // swizzled scales of A (padded rows)
+  const uint8_t* sfb;          // swizzled scales of B, experts back to back
+  const int32_t* mtile_prefix; // [E+1]
+  const int32_t* counts;       // [E]
+  int E;
+  int K;                       // reduction length
+  int n_total;                 // B rows per expert (2I for gate/up, H for down)
+  uint32_t* status;
+  // gate/up epilogue
+  uint8_t* hq_codes;           // [rows_cap][I/2]
+  uint8_t* hq_sf;              // swizzled [rows_cap][I/16]
+  const float* g_x;            // device scalar
+  const float* g_gate;         // [E]
+  const float* g_up;           // [E]
+  const float* g_h;            // [E]
+  int I;
+  // down epilogue
+  float* acc;                  // [T][H]
+  const int32_t* row_pair;     // [rows_cap]
+  const float* wts;            // [T*topk]
+  const float* alpha_down;     // [E] = g_h * g_down
+  int topk;
+  int H;
+};
+
+struct FinalizeArgs {
+  const float* acc;
+  uint16_t* out;
+  int64_t n;  // elements, multiple of 8
+};
+
+// quantize.cu
+int amax_partial_blocks(int64_t n_elems);
+cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partials, int blocks,
+                                cudaStream_t stream);
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+
+// route.cu
+int router_ksplit(int64_t T, int E, int H);
+size_t router_parts_elems(int64_t T_max, int E, int H);
+cudaError_t launch_router(RouterArgs a, cudaStream_t stream);
+
+// permute.cu
+cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream);
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream);
+cudaError_t launch_unswizzle_rows(const uint8_t* sf, int64_t n_col_tiles, const int32_t* src_rows,
+                                  int64_t n_rows, int cols16, uint8_t* out, cudaStream_t stream);
+cudaError_t launch_export_hq(const uint8_t* hq_codes, const uint8_t* hq_sf, const int32_t* perm,
+                             const int32_t* idx, const int32_t* offsets, const int32_t* mtile_prefix,
+                             int64_t n_pairs, int I, uint8_t* out_codes, uint8_t* out_sf,
+                             cudaStream_t stream);
+cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_t* swz,
+                             int64_t n_col_tiles, int tile_mul_add /* (mul << 8) | add */,
+                             cudaStream_t stream);
+
+// gemm.cu
+cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_b, const GemmArgs& a,
+                               int grid, cudaStream_t stream);
+cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_b, const GemmArgs& a,
+                             int grid, cudaStream_t stream);
+// Encodes a 2D byte tensor map [rows][row_bytes] with a 128-byte x box_rows box, 128B swizzle.
+int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows);
+
+int num_sms();
+
+}  // namespace nvfp4moe

@@ -1,0 +1,227 @@
+// Grouping of (token, slot) pairs by expert and the byte-moving kernels around the grouped
+// GEMMs: stable counting sort into 128-row-padded expert segments, gather of quantised
+// rows into those segments, FP32 -> BF16 output, scale-layout conversions.
+// Only the top-8 of 256 experts run per token ("Reflection releases Beam ...", section
+// "Mixture-of-Experts details"), so the pairs are grouped by expert before the expert GEMMs.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4moe {
+
+// Per chunk of kPermChunkTokens tokens: how many of its pairs go to each expert.
+__global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
+  __shared__ int hist[256];
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t p0 = (int64_t)blockIdx.x * kPermChunkTokens * a.topk;
+  const int64_t p1 = min(p0 + (int64_t)kPermChunkTokens * a.topk, a.T * a.topk);
+  for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&hist[a.idx[p]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+    a.chunk_counts[(int64_t)blockIdx.x * a.E + e] = hist[e];
+}
+
+// One block, one thread per expert: per-chunk bases, counts, offsets (exclusive scan),
+// 128-row tile prefix, and -1 in every padding row of every segment.
+__global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
+  __shared__ int s_cnt[256];
+  __shared__ int s_tiles[256];
+  const int e = threadIdx.x;
+  int running = 0;
+  if (e < a.E) {
+    for (int c = 0; c < a.n_chunks; ++c) {
+      const int v = a.chunk_counts[(int64_t)c * a.E + e];
+      a.chunk_base[(int64_t)c * a.E + e] = running;
+      running += v;
+    }
+  }
+  s_cnt[e] = e < a.E ? running : 0;
+  s_tiles[e] = e < a.E ? (running + kBlockM - 1) / kBlockM : 0;
+  __syncthreads();
+  if (e == 0) {
+    int off = 0, tiles = 0;
+    for (int i = 0; i < a.E; ++i) {
+      const int c = s_cnt[i], t = s_tiles[i];
+      a.offsets[i] = off;
+      a.mtile_prefix[i] = tiles;
+      s_cnt[i] = off;
+      s_tiles[i] = tiles;
+      off += c;
+      tiles += t;
+    }
+    a.offsets[a.E] = off;
+    a.mtile_prefix[a.E] = tiles;
+  }
+  __syncthreads();
+  if (e < a.E) {
+    const int off = s_cnt[e];
+    a.counts[e] = running;
+    for (int c = 0; c < a.n_chunks; ++c) a.chunk_base[(int64_t)c * a.E + e] += off;
+    const int64_t r0 = (int64_t)s_tiles[e] * kBlockM;
+    const int64_t r1 = r0 + (int64_t)((running + kBlockM - 1) / kBlockM) * kBlockM;
+    for (int64_t r = r0 + running; r < r1; ++r) a.row_pair[r] = -1;
+  }
+}
+
+// One warp per chunk walks its pairs in order, so pairs of one expert keep ascending pair
+// (and token) order: a stable counting sort.
+__global__ void __launch_bounds__(32) perm_scatter_kernel(PermArgs a) {
+  __shared__ int run[256];
+  const int lane = threadIdx.x;
+  const int c = blockIdx.x;
+  for (int e = lane; e < a.E; e += 32) run[e] = a.chunk_base[(int64_t)c * a.E + e];
+  __syncwarp();
+  const int64_t p0 = (int64_t)c * kPermChunkTokens * a.topk;
+  const int64_t p1 = min(p0 + (int64_t)kPermChunkTokens * a.topk, a.T * a.topk);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t base = p0; base < p1; base += 32) {
+    const int64_t p = base + lane;
+    const bool valid = p < p1;
+    const int e = valid ? a.idx[p] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt);
+    if (valid) {
+      const int pos = run[e] + rank;
+      a.perm[pos] = (int32_t)p;
+      a.inv[p] = pos;
+      const int64_t row = (int64_t)a.mtile_prefix[e] * kBlockM + (pos - a.offsets[e]);
+      a.row_pair[row] = (int32_t)p;
+    }
+    __syncwarp();
+    if (valid && rank == 0) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream) {
+  perm_count_kernel<<<a.n_chunks, 256, 0, stream>>>(a);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  perm_scan_kernel<<<1, 256, 0, stream>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  perm_scatter_kernel<<<a.n_chunks, 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// One warp per pair: copy the token's quantised row (codes and its swizzled scale groups)
+// into the pair's row of the expert segment.
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  const int64_t pair = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (pair >= a.n_pairs) return;
+  const int e = a.idx[pair];
+  const int64_t token = pair / a.topk;
+  const int64_t row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[pair] - a.offsets[e]);
+  const int64_t row_bytes = a.H >> 1;
+  const uint4* src = reinterpret_cast<const uint4*>(a.xq_codes + token * row_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(a.a_codes + row * row_bytes);
+  for (int64_t i = lane; i < row_bytes / 16; i += 32) dst[i] = __ldg(src + i);
+  const int64_t n_ct = a.H >> 6;  // 4-scale column groups per row
+  for (int64_t ct = lane; ct < n_ct; ct += 32) {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(a.xq_sf + swz_offset(token, ct * 4, n_ct));
+    *reinterpret_cast<uint32_t*>(a.a_sf + swz_offset(row, ct * 4, n_ct)) = v;
+  }
+}
+
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream) {
+  if (a.n_pairs == 0) return cudaSuccess;
+  gather_kernel<<<(unsigned)((a.n_pairs + 7) / 8), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// out = bf16(acc), 8 values per thread.
+__global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
+  const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8;
+  if (i >= a.n) return;
+  const float4 p = *reinterpret_cast<const float4*>(a.acc + i);
+  const float4 q = *reinterpret_cast<const float4*>(a.acc + i + 4);
+  const float v[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j]));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j + 1]));
+    w[j] = lo | (hi << 16);
+  }
+  *reinterpret_cast<uint4*>(a.out + i) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream) {
+  if (a.n == 0) return cudaSuccess;
+  const int64_t threads = a.n / 8;
+  finalize_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// Linear [n_rows][cols16] scales from swizzled storage: row i of the output is row
+// src_rows[i] (or i when src_rows is null) of the swizzled tensor.
+__global__ void __launch_bounds__(256) unswizzle_rows_kernel(const uint8_t* sf, int64_t n_col_tiles,
+                                                             const int32_t* src_rows, int64_t n_rows,
+                                                             int cols16, uint8_t* out) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n_rows * cols16) return;
+  const int64_t r = i / cols16;
+  const int c = (int)(i - r * cols16);
+  const int64_t sr = src_rows ? src_rows[r] : r;
+  out[i] = sf[swz_offset(sr, c, n_col_tiles)];
+}
+
+cudaError_t launch_unswizzle_rows(const uint8_t* sf, int64_t n_col_tiles, const int32_t* src_rows,
+                                  int64_t n_rows, int cols16, uint8_t* out, cudaStream_t stream) {
+  const int64_t n = n_rows * cols16;
+  if (n == 0) return cudaSuccess;
+  unswizzle_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(sf, n_col_tiles, src_rows,
+                                                                         n_rows, cols16, out);
+  return cudaGetLastError();
+}
+
+// Debug export of the requantised SwiGLU intermediate: row pos of the output (perm order)
+// is the padded segment row of pair perm[pos].
+__global__ void __launch_bounds__(256) export_hq_kernel(const uint8_t* hq_codes, const uint8_t* hq_sf,
+                                                        const int32_t* perm, const int32_t* idx,
+                                                        const int32_t* offsets,
+                                                        const int32_t* mtile_prefix, int64_t n_pairs,
+                                                        int I, uint8_t* out_codes, uint8_t* out_sf) {
+  const int64_t pos = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (pos >= n_pairs) return;
+  const int e = idx[perm[pos]];
+  const int64_t row = (int64_t)mtile_prefix[e] * kBlockM + (pos - offsets[e]);
+  for (int j = lane; j < I / 2; j += 32) out_codes[pos * (I / 2) + j] = hq_codes[row * (I / 2) + j];
+  for (int c = lane; c < I / 16; c += 32) out_sf[pos * (I / 16) + c] = hq_sf[swz_offset(row, c, I / 64)];
+}
+
+cudaError_t launch_export_hq(const uint8_t* hq_codes, const uint8_t* hq_sf, const int32_t* perm,
+                             const int32_t* idx, const int32_t* offsets, const int32_t* mtile_prefix,
+                             int64_t n_pairs, int I, uint8_t* out_codes, uint8_t* out_sf,
+                             cudaStream_t stream) {
+  if (n_pairs == 0) return cudaSuccess;
+  export_hq_kernel<<<(unsigned)((n_pairs + 7) / 8), 256, 0, stream>>>(
+      hq_codes, hq_sf, perm, idx, offsets, mtile_prefix, n_pairs, I, out_codes, out_sf);
+  return cudaGetLastError();
+}
+
+// Linear [rows][cols16] weight scales -> swizzled operand storage.  Source row tile j is
+// placed at destination row tile j * tile_mul + tile_add (gate/up interleave: 2, 0 / 2, 1).
+__global__ void __launch_bounds__(256) repack_sf_kernel(const uint8_t* linear, int rows, int cols16,
+                                                        uint8_t* swz, int64_t n_col_tiles, int tile_mul,
+                                                        int tile_add) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= (int64_t)rows * cols16) return;
+  const int r = (int)(i / cols16);
+  const int c = (int)(i - (int64_t)r * cols16);
+  const int64_t dr = (int64_t)((r >> 7) * tile_mul + tile_add) * kBlockM + (r & 127);
+  swz[swz_offset(dr, c, n_col_tiles)] = linear[i];
+}
+
+cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_t* swz,
+                             int64_t n_col_tiles, int tile_mul_add, cudaStream_t stream) {
+  const int64_t n = (int64_t)rows * cols16;
+  const int tile_mul = tile_mul_add >> 8, tile_add = tile_mul_add & 0xFF;
+  repack_sf_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(linear, rows, cols16, swz,
+                                                                    n_col_tiles, tile_mul, tile_add);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

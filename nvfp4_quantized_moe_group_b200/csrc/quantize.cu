@@ -1,0 +1,147 @@
+// NVFP4 activation quantisation (quantize_nvfp4): global amax, per-16 block E4M3 scale,
+// E2M1 codes with round-to-nearest-even, two codes per byte, linear or swizzled scales.
+// Format: "NVFP4 quantization", section "Quantization scheme" (E2M1 values, one E4M3 scale
+// per 16 values, one FP32 global scale per tensor); the scale rule is the library's reading
+// stated in nvfp4moe.h.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4moe {
+
+// Per-block maximum of |x| as the BF16 magnitude bit pattern (bits & 0x7FFF).  Integer
+// maxima are exact and order-free; a pattern >= 0x7F80 means Inf or NaN was seen.
+__global__ void __launch_bounds__(256) amax_partial_kernel(const uint4* __restrict__ x, int64_t n_vec,
+                                                           uint32_t* __restrict__ partials) {
+  uint32_t m = 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(x + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m = max(m, w[j] & 0x7FFFu);
+      m = max(m, (w[j] >> 16) & 0x7FFFu);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) partials[blockIdx.x] = m;
+  }
+}
+
+// One thread quantises 64 consecutive values of a row (4 blocks of 16).  Rows in
+// [rows, rows_padded) only write zero scales (swizzled layout padding).
+__global__ void __launch_bounds__(256) quantize_kernel(QuantizeArgs a) {
+  __shared__ float s_g;
+  __shared__ int s_bad;
+  if (threadIdx.x < 32) {
+    float g;
+    int bad = 0;
+    if (a.g_in != nullptr) {
+      g = *a.g_in;
+    } else {
+      uint32_t m = 0;
+      for (int i = threadIdx.x; i < a.n_partials; i += 32) m = max(m, a.partials[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      bad = m >= 0x7F80u;
+      g = global_scale_from_amax(__uint_as_float(m << 16));
+    }
+    if (threadIdx.x == 0) {
+      s_g = g;
+      s_bad = bad;
+      if (blockIdx.x == 0) {
+        if (bad) raise_status(a.status, kStatusNonFinite);
+        if (a.g_out != nullptr) *a.g_out = g;
+      }
+    }
+  }
+  __syncthreads();
+  if (s_bad) return;
+  const float g = s_g;
+  const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
+
+  const int64_t chunks_per_row = a.cols >> 6;
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t r = idx / chunks_per_row;
+  const int64_t q = idx - r * chunks_per_row;
+  if (r >= a.rows_padded) return;
+
+  if (a.zero_out != nullptr && r < a.rows) {
+    float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + q * 64);
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = zero;
+  }
+
+  uint32_t sc = 0;
+  if (r < a.rows) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + q * 64);
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __ldg(src + i);
+    uint32_t out[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t w[8] = {v[2 * b].x, v[2 * b].y, v[2 * b].z, v[2 * b].w,
+                             v[2 * b + 1].x, v[2 * b + 1].y, v[2 * b + 1].z, v[2 * b + 1].w};
+      float f[16];
+      uint32_t mb = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        mb = max(mb, w[j] & 0x7FFFu);
+        mb = max(mb, (w[j] >> 16) & 0x7FFFu);
+      }
+      float r_b;
+      const uint32_t s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
+      sc |= s << (8 * b);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
+      out[2 * b] = cvt_e2m1x8(f);
+      out[2 * b + 1] = cvt_e2m1x8(f + 8);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + q * 32);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+  uint32_t* sdst;
+  if (a.swizzled) {
+    sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, q * 4, a.n_col_tiles));
+  } else {
+    sdst = reinterpret_cast<uint32_t*>(a.scales + r * (a.cols >> 4) + q * 4);
+  }
+  *sdst = sc;
+}
+
+int amax_partial_blocks(int64_t n_elems) {
+  const int64_t n_vec = n_elems / 8;
+  int64_t blocks = (n_vec + 255) / 256;
+  if (blocks > kMaxAmaxPartials) blocks = kMaxAmaxPartials;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partials, int blocks,
+                                cudaStream_t stream) {
+  amax_partial_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), n_elems / 8,
+                                                  partials);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
+  const int64_t threads = a.rows_padded * (a.cols >> 6);
+  const int64_t blocks = threads > 0 ? (threads + 255) / 256 : 1;  // one block still writes g_out
+  quantize_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

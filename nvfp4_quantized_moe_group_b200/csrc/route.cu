@@ -1,0 +1,212 @@
+// Group-limited sigmoid router ("Reflection releases Beam ...", section "Mixture-of-Experts
+// details"): FP32 logits x.W_r^T, sigmoid scores, group score = sum of the two best scores of
+// each group, keep the best topk_groups groups, pick the topk best experts inside them,
+// weights = routed_scale * s / sum(selected s).  FP32 throughout (section "Residual stream and
+// numerical decisions").
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4moe {
+
+namespace {
+constexpr int kTM = 64;   // tokens per CTA tile
+constexpr int kTN = 64;   // experts per CTA tile
+constexpr int kTK = 32;   // K chunk; each chunk is summed into a fresh partial
+}  // namespace
+
+// Split-K FP32 logits: parts[ks][t][e] = sum over this CTA's K slice of x[t][k] * W[e][k].
+// Each 32-product chunk is accumulated into a fresh register (one FMA chain of at most 32),
+// then added to the running slice sum, which keeps the rounding-error bound at
+// (32 + slice/32) units of 2^-24 instead of growing with H.
+__global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
+  __shared__ __align__(16) float xs[kTK][kTM + 4];
+  __shared__ __align__(16) float ws[kTK][kTN + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15;  // expert quad
+  const int ty = tid >> 4;  // token quad
+  const int64_t t0 = (int64_t)blockIdx.x * kTM;
+  const int e0 = blockIdx.y * kTN;
+  const int64_t k_begin = (int64_t)blockIdx.z * a.k_slice;
+  const int64_t k_end = k_begin + a.k_slice;
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  // global -> shared mapping: x tile 64 rows x 32 bf16 (4 threads per row, 8 bf16 each);
+  // W tile 64 rows x 32 fp32 (4 threads per row, 8 floats each).
+  const int lr = tid >> 2;
+  const int lc = (tid & 3) * 8;
+  for (int64_t k0 = k_begin; k0 < k_end; k0 += kTK) {
+    {
+      const int64_t t = t0 + lr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t < a.T) v = __ldg(reinterpret_cast<const uint4*>(a.x + t * a.H + k0 + lc));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xs[lc + 2 * j][lr] = __uint_as_float(w[j] << 16);
+        xs[lc + 2 * j + 1][lr] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+      const int e = e0 + lr;
+      float4 p = make_float4(0.f, 0.f, 0.f, 0.f), q = p;
+      if (e < a.E) {
+        const float4* src = reinterpret_cast<const float4*>(a.w + (int64_t)e * a.H + k0 + lc);
+        p = __ldg(src);
+        q = __ldg(src + 1);
+      }
+      ws[lc + 0][lr] = p.x; ws[lc + 1][lr] = p.y; ws[lc + 2][lr] = p.z; ws[lc + 3][lr] = p.w;
+      ws[lc + 4][lr] = q.x; ws[lc + 5][lr] = q.y; ws[lc + 6][lr] = q.z; ws[lc + 7][lr] = q.w;
+    }
+    __syncthreads();
+    float part[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < kTK; ++k) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
+      const float4 wv = *reinterpret_cast<const float4*>(&ws[k][tx * 4]);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = __fmaf_rn(xa[i], wa[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = __fadd_rn(acc[i][j], part[i][j]);
+    __syncthreads();
+  }
+  float* out = a.parts + (int64_t)blockIdx.z * a.T * a.E;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + ty * 4 + i;
+    if (t >= a.T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < a.E) out[t * a.E + e] = acc[i][j];
+    }
+  }
+}
+
+// One warp per token: sum the split-K parts in order, add the bias, sigmoid, group-limited
+// top-k, weights.  Equal scores go to the lower index (groups and experts).
+__global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
+  __shared__ float s_sc[8][256];
+  __shared__ float s_gsc[8][32];
+  __shared__ int s_keep[8][32];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+  if (t >= a.T) return;
+  float* sc = s_sc[warp];
+  const int E = a.E, G = a.n_groups, gs = a.E / a.n_groups;
+
+  // scores; lane holds experts lane, lane+32, ...
+  for (int e = lane; e < E; e += 32) {
+    float l = a.parts[t * E + e];
+    for (int ks = 1; ks < a.ksplit; ++ks) l = __fadd_rn(l, a.parts[((int64_t)ks * a.T + t) * E + e]);
+    if (a.bias != nullptr) l = __fadd_rn(l, a.bias[e]);
+    sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
+  }
+  __syncwarp();
+  // group scores: sum of the two best scores of each group
+  if (lane < G) {
+    float b1 = -1.f, b2 = -1.f;
+    for (int j = 0; j < gs; ++j) {
+      const float v = sc[lane * gs + j];
+      if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+    }
+    s_gsc[warp][lane] = gs >= 2 ? __fadd_rn(b1, b2) : b1;
+  }
+  __syncwarp();
+  if (lane < G) {
+    const float mine = s_gsc[warp][lane];
+    int rank = 0;
+    for (int g = 0; g < G; ++g) {
+      const float o = s_gsc[warp][g];
+      rank += (o > mine) || (o == mine && g < lane);
+    }
+    s_keep[warp][lane] = rank < a.topk_groups;
+  }
+  __syncwarp();
+  // candidates: this lane's experts in kept groups; k rounds of warp argmax
+  float cand[8];
+  int n_mine = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    cand[i] = (e < E && s_keep[warp][e / gs]) ? sc[e] : -1.0f;
+    n_mine += e < E;
+  }
+  (void)n_mine;
+  float sel_s[8];
+  int sel_e[8];
+  float sum = 0.f;
+  for (int j = 0; j < a.topk; ++j) {
+    float best = -1.0f;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (cand[i] > best) { best = cand[i]; be = e; }   // e ascends with i: ties keep lower e
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ob > best || (ob == best && oe < be)) { best = ob; be = oe; }
+    }
+    sel_s[j] = best;
+    sel_e[j] = be;
+    sum = __fadd_rn(sum, best);
+    if ((be & 31) == lane) cand[be >> 5] = -1.0f;
+  }
+  if (lane < a.topk) {
+    float s = 0.f;
+    int e = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j == lane) { s = sel_s[j]; e = sel_e[j]; }
+    a.idx[t * a.topk + lane] = e;
+    a.wts[t * a.topk + lane] = __fdiv_rn(__fmul_rn(a.routed_scale, s), sum);
+  }
+}
+
+int router_ksplit(int64_t T, int E, int H) {
+  const int64_t tiles = ((T + kTM - 1) / kTM) * ((E + kTN - 1) / kTN);
+  int ks = 1;
+  while (ks < 32 && tiles * ks * 2 <= 2 * 148 && (H / kTK) % (ks * 2) == 0) ks *= 2;
+  return ks;
+}
+
+size_t router_parts_elems(int64_t T_max, int E, int H) {
+  size_t best = 0;
+  // ksplit depends on T only through the number of 64-token tiles
+  for (int64_t c = 1; c <= (T_max + kTM - 1) / kTM; ++c) {
+    const int64_t T = c * kTM < T_max ? c * kTM : T_max;
+    const size_t n = (size_t)router_ksplit(T, E, H) * (size_t)T * (size_t)E;
+    if (n > best) best = n;
+  }
+  return best;
+}
+
+cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
+  a.ksplit = router_ksplit(a.T, a.E, a.H);
+  a.k_slice = a.H / a.ksplit;
+  dim3 grid((unsigned)((a.T + kTM - 1) / kTM), (unsigned)((a.E + kTN - 1) / kTN), (unsigned)a.ksplit);
+  router_logits_kernel<<<grid, 256, 0, stream>>>(a);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  router_topk_kernel<<<(unsigned)((a.T + 7) / 8), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

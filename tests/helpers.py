@@ -1,0 +1,169 @@
+"""Shared test plumbing: oracle-side layer construction, the router near-tie protocol and
+output tolerances.  Oracle calls only: nothing here reads a value computed by the CUDA
+library except the GPU results under test, which are only compared."""
+from __future__ import annotations
+
+import math
+import multiprocessing as mp
+import os
+import types
+
+import numpy as np
+import torch
+
+import oracle
+from workloads import TINY, BEAM, activations, router_weight, expert_weight, zipf_bias
+from tests.conftest import read_golden
+
+U = 2.0 ** -24
+
+
+def cfg_ns(shape):
+    return types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
+                                 topk=shape.topk, routed_scale=shape.routed_scale)
+
+
+def intermediate_scales(shape) -> np.ndarray:
+    """Static g_h[e] of the layer, as written by tests/golden/make_intermediate_scales.py."""
+    name = {TINY: "tiny", BEAM: "beam"}[shape]
+    rows = read_golden(f"intermediate_scales_{name}.txt")
+    g = np.array([int(h, 16) for _, h, _ in rows], dtype=np.uint32).view(np.float32)
+    assert len(g) == shape.E
+    return g
+
+
+# ------------------------------------------------------------------ router ----
+
+def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
+    """Bound on |FP32 logit - exact| the library documents for nvfp4moe_route:
+    (32 + H/32 + 33) * 2^-24 * sum_h |x_h W_eh| (+ 2^-24 |bias|)."""
+    b = (32 + H // 32 + 33) * U * (np.abs(x) @ np.abs(wr).T)
+    if bias is not None:
+        b = b + U * np.abs(np.asarray(bias, dtype=np.float64))[None, :]
+    return b
+
+
+def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6):
+    """Near-tie protocol.  A token is clean when every routing decision has a margin larger
+    than the FP32 error bound; clean tokens must match the oracle bit for bit (experts and
+    their order).  Other tokens must pick an admissible selection: experts from groups and
+    scores within the error bound of the exact choice.  Weights are compared (relative
+    tolerance) against the oracle's weights of the GPU's own selection.
+    Returns (clean token mask, number of flagged tokens)."""
+    T, K = gpu_idx.shape
+    gs = shape.E // shape.n_groups
+    bl = router_logit_bound(x, wr, bias, shape.H)
+    s = r.scores
+    eps_s = bl * s * (1 - s) + 8 * U                       # sigmoid: Lipschitz s(1-s) + its own rounding
+    eps = eps_s.max(axis=1)                                # per token
+    dgrp = 2 * eps + 2 * U                                 # error of one group score
+    clean = (r.expert_margin > 2 * eps) & (r.group_margin > 2 * dgrp) & (r.order_margin > 2 * eps)
+    n_flag = int((~clean).sum())
+    # clean tokens: exact
+    mism = clean & (gpu_idx != r.idx).any(axis=1)
+    assert not mism.any(), f"{int(mism.sum())} clean tokens routed differently, e.g. {np.flatnonzero(mism)[:5]}"
+    # every token: a valid, admissible selection
+    for t in range(T):
+        sel = gpu_idx[t]
+        assert len(set(sel.tolist())) == K and sel.min() >= 0 and sel.max() < shape.E
+        if clean[t]:
+            continue
+        kth = np.sort(s[t, r.idx[t]])[0]
+        g4 = np.sort(r.group_scores[t])[::-1][shape.topk_groups - 1]
+        assert np.all(s[t, sel] >= kth - 2 * eps[t]), f"token {t}: expert score below admissible range"
+        assert np.all(r.group_scores[t, sel // gs] >= g4 - 2 * dgrp[t]), f"token {t}: group not admissible"
+    # weights of the GPU's selection
+    ssel = np.take_along_axis(s, gpu_idx.astype(np.int64), axis=1)
+    w_ref = shape.routed_scale * ssel / ssel.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(gpu_w, w_ref, rtol=w_rtol, atol=0)
+    return clean, n_flag
+
+
+# ------------------------------------------------------------------ experts ----
+
+def oracle_expert(shape, e: int, seed: int = 0):
+    """Expert e quantised by the oracle from the seeded BF16 weights."""
+    return tuple(oracle.quantize_tensor(expert_weight(shape, e, w, seed=seed).float().numpy())
+                 for w in ("gate", "up", "down"))
+
+
+def _expert_job(args):
+    shape, e, xhat, g_h = args
+    gate, up, down = oracle_expert(shape, e)
+    res = oracle.expert_mlp(xhat, gate, up, down, np.float32(g_h))
+    return e, res["y"], res["h"], res["hq_codes"], res["hq_scales"], (gate.g, up.g, down.g)
+
+
+def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, tokens=None, workers=None):
+    """Oracle layer output for the given tokens: routing of all tokens, expert MLPs of the
+    sampled tokens (experts evaluated in a spawn process pool when there are many)."""
+    cfg = cfg_ns(shape)
+    r = oracle.route(x, wr, cfg, bias)
+    xc, xs, gx = oracle.quantize(np.asarray(x, dtype=np.float32))
+    T = x.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    need = {}
+    for i, t in enumerate(tokens):
+        for j in range(cfg.topk):
+            need.setdefault(int(r.idx[t, j]), []).append((i, int(t), j))
+    jobs = []
+    for e, rows in sorted(need.items()):
+        ts = np.array([t for _, t, _ in rows])
+        jobs.append((shape, e, oracle.dequantize(xc[ts], xs[ts], gx), float(g_h[e])))
+    if workers is None:
+        workers = min(len(jobs), max(1, len(os.sched_getaffinity(0)) // 2)) if len(jobs) > 8 else 1
+    if workers > 1:
+        with mp.get_context("spawn").Pool(workers) as pool:
+            results = pool.map(_expert_job, jobs)
+    else:
+        results = [_expert_job(j) for j in jobs]
+    out = np.zeros((len(tokens), x.shape[1]))
+    inter = {}
+    for e, y, h, hc, hs, _ in results:
+        for n, (i, t, j) in enumerate(need[e]):
+            out[i] += r.w[t, j] * y[n]
+            inter[(t, j)] = (h[n], hc[n], hs[n])
+    return {"route": r, "xq_codes": xc, "xq_scales": xs, "g_x": gx, "tokens": tokens, "out": out,
+            "inter": inter}
+
+
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half a BF16 unit in the last place at |v| (the output format's own rounding)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 8)
+
+
+def check_output(gpu_out: np.ndarray, ref: np.ndarray, max_abs=2e-2, rel_fro=5e-3):
+    """Layer output tolerance: max-abs 2e-2 (plus the BF16 output rounding of each value)
+    and relative Frobenius 5e-3 against the oracle's FP64 output."""
+    err = np.abs(gpu_out - ref)
+    lim = max_abs + bf16_half_ulp(ref)
+    bad = err > lim
+    assert not bad.any(), f"{int(bad.sum())} outputs beyond tolerance; worst {err.max():.4g}"
+    fro = np.linalg.norm(gpu_out - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert fro <= rel_fro, f"relative Frobenius error {fro:.3g}"
+    return float(err.max()), float(fro)
+
+
+E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def requant_near_tie(h: np.ndarray, g_h: float, rel=1e-4) -> tuple[np.ndarray, np.ndarray]:
+    """Where the requantisation of h (FP64) sits within a relative ``rel`` of a rounding
+    boundary: per block (E4M3 scale) and per element (E2M1 code).  A kernel whose FP32 h
+    differs from the exact value by less than that may round the other way there."""
+    h = np.asarray(h, dtype=np.float64)
+    n = h.shape[-1]
+    hb = h.reshape(-1, n // 16, 16)
+    r_t = 1.0 / (6.0 * g_h)
+    q = np.abs(hb).max(axis=2) * r_t
+    grid = oracle.e4m3_table()[:127]
+    mids = (grid[:-1] + grid[1:]) / 2
+    dq = np.min(np.abs(q[..., None] - mids[None, None, :]), axis=-1)
+    block_tie = dq <= rel * np.maximum(q, 2.0 ** -9)
+    S = oracle.e4m3_encode(q.astype(np.float32))
+    d = oracle.e4m3_decode(S) * g_h
+    v = np.abs(hb) / np.where(d == 0, np.inf, d)[..., None]
+    dv = np.min(np.abs(v[..., None] - E2M1_MIDS), axis=-1)
+    elem_tie = dv <= rel * np.maximum(v, 0.25)
+    return block_tie.reshape(h.shape[:-1] + (n // 16,)), elem_tie.reshape(h.shape)
