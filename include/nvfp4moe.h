@@ -128,9 +128,10 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
  *   idx  out [T][topk] int32: selected experts by score descending, equal scores by
  *        lower expert index (the same rule picks the groups).
  *   w    out [T][topk] FP32: routed_scale * s / sum(selected s).
- * Logits are FP32 sums of FP32 products; each is accumulated in runs of at most 32
- * products, and the runs (at most H/32 + 32 of them, plus the bias) are added in a fixed
- * order, so |logit - exact| <= (32 + H/32 + 33) * 2^-24 * sum_h |x_h W_eh| (+ |bias|). */
+ * Logits: FP32 products accumulated in FP32 runs of at most 32 products; the runs, the
+ * split-K parts and the bias are added in FP64 and the logit is rounded to FP32 once, so
+ * |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
+ * Scores are 1 / (1 + expf(-logit)) in FP32. */
 NVFP4MOE_API size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
 NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
                    const float* w_router, const float* logit_bias, int32_t* idx, float* w,

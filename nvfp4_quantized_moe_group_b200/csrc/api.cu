@@ -76,7 +76,7 @@ QuantWs carve_quant(void* ws) {
 
 struct RouteWs {
   WsHeader* hdr;
-  float* parts;
+  double* parts;
   size_t bytes;
 };
 
@@ -84,7 +84,7 @@ RouteWs carve_route(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   Carver c(ws);
   RouteWs r;
   r.hdr = c.take<WsHeader>(1);
-  r.parts = c.take<float>(router_parts_elems(T, cfg.E, cfg.H));
+  r.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
   r.bytes = c.off;
   return r;
 }
@@ -99,7 +99,7 @@ struct ForwardWs {
   WsHeader* hdr;
   uint32_t* partials;
   float* g_x;
-  float* parts;
+  double* parts;
   int32_t* idx;
   float* wts;
   uint8_t* xq_codes;
@@ -130,7 +130,7 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.hdr = c.take<WsHeader>(1);
   f.partials = c.take<uint32_t>(kMaxAmaxPartials);
   f.g_x = c.take<float>(1);
-  f.parts = c.take<float>(router_parts_elems(T, cfg.E, cfg.H));
+  f.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
   f.idx = c.take<int32_t>(pairs);
   f.wts = c.take<float>(pairs);
   f.xq_codes = c.take<uint8_t>(T * cfg.H / 2);
@@ -209,8 +209,7 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   if (scale_layout != NVFP4MOE_SCALES_LINEAR && scale_layout != NVFP4MOE_SCALES_SWIZZLED)
     return NVFP4MOE_ERR_ARG;
   if (ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
-  if ((rows > 0 || scale_layout == NVFP4MOE_SCALES_SWIZZLED) && (scales == nullptr || !aligned(scales, 4)))
-    return NVFP4MOE_ERR_ARG;
+  if (rows > 0 && (scales == nullptr || !aligned(scales, 4))) return NVFP4MOE_ERR_ARG;
   if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || !aligned(x_bf16, 16) || !aligned(codes, 16)))
     return NVFP4MOE_ERR_ARG;
   const QuantWs q = carve_quant(ws);

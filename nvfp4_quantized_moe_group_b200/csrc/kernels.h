@@ -35,7 +35,7 @@ struct RouterArgs {
   const uint16_t* x;       // [T][H] bf16
   const float* w;          // [E][H]
   const float* bias;       // [E] or nullptr
-  float* parts;            // [ksplit][T][E]
+  double* parts;           // [ksplit][T][E]
   int32_t* idx;            // [T][topk]
   float* wts;              // [T][topk]
   int64_t T;

@@ -14,10 +14,11 @@ constexpr int kTN = 64;   // experts per CTA tile
 constexpr int kTK = 32;   // K chunk; each chunk is summed into a fresh partial
 }  // namespace
 
-// Split-K FP32 logits: parts[ks][t][e] = sum over this CTA's K slice of x[t][k] * W[e][k].
-// Each 32-product chunk is accumulated into a fresh register (one FMA chain of at most 32),
-// then added to the running slice sum, which keeps the rounding-error bound at
-// (32 + slice/32) units of 2^-24 instead of growing with H.
+// Split-K logits: parts[ks][t][e] = sum over this CTA's K slice of x[t][k] * W[e][k].
+// Each 32-product chunk is an FP32 FMA chain into a fresh register; the chunk sums are
+// added in FP64 (and so are the split-K parts and the bias), and the logit is rounded to
+// FP32 once.  The error is then at most 32 * 2^-24 * sum|x W| + 2^-24 |logit| (plus FP64
+// terms), independent of H.
 __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
   __shared__ __align__(16) float xs[kTK][kTM + 4];
   __shared__ __align__(16) float ws[kTK][kTN + 4];
@@ -29,11 +30,11 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
   const int64_t k_begin = (int64_t)blockIdx.z * a.k_slice;
   const int64_t k_end = k_begin + a.k_slice;
 
-  float acc[4][4];
+  double acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
 
   // global -> shared mapping: x tile 64 rows x 32 bf16 (4 threads per row, 8 bf16 each);
   // W tile 64 rows x 32 fp32 (4 threads per row, 8 floats each).
@@ -80,10 +81,10 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = __fadd_rn(acc[i][j], part[i][j]);
+      for (int j = 0; j < 4; ++j) acc[i][j] = __dadd_rn(acc[i][j], (double)part[i][j]);
     __syncthreads();
   }
-  float* out = a.parts + (int64_t)blockIdx.z * a.T * a.E;
+  double* out = a.parts + (int64_t)blockIdx.z * a.T * a.E;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t t = t0 + ty * 4 + i;
@@ -111,9 +112,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
 
   // scores; lane holds experts lane, lane+32, ...
   for (int e = lane; e < E; e += 32) {
-    float l = a.parts[t * E + e];
-    for (int ks = 1; ks < a.ksplit; ++ks) l = __fadd_rn(l, a.parts[((int64_t)ks * a.T + t) * E + e]);
-    if (a.bias != nullptr) l = __fadd_rn(l, a.bias[e]);
+    double ld = a.parts[t * E + e];
+    for (int ks = 1; ks < a.ksplit; ++ks) ld = __dadd_rn(ld, a.parts[((int64_t)ks * a.T + t) * E + e]);
+    if (a.bias != nullptr) ld = __dadd_rn(ld, (double)a.bias[e]);
+    const float l = __double2float_rn(ld);
     sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
   }
   __syncwarp();

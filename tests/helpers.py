@@ -36,11 +36,12 @@ def intermediate_scales(shape) -> np.ndarray:
 
 def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
     """Bound on |FP32 logit - exact| the library documents for nvfp4moe_route:
-    (32 + H/32 + 33) * 2^-24 * sum_h |x_h W_eh| (+ 2^-24 |bias|)."""
-    b = (32 + H // 32 + 33) * U * (np.abs(x) @ np.abs(wr).T)
+    32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (FP64 terms covered by a 2^-40 margin)."""
+    sabs = np.abs(x) @ np.abs(wr).T
+    logit = x @ wr.T
     if bias is not None:
-        b = b + U * np.abs(np.asarray(bias, dtype=np.float64))[None, :]
-    return b
+        logit = logit + np.asarray(bias, dtype=np.float64)[None, :]
+    return 32 * U * sabs + U * np.abs(logit) + 2.0 ** -40 * (sabs + 1)
 
 
 def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6):
@@ -151,7 +152,9 @@ E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
 def requant_near_tie(h: np.ndarray, g_h: float, rel=1e-4) -> tuple[np.ndarray, np.ndarray]:
     """Where the requantisation of h (FP64) sits within a relative ``rel`` of a rounding
     boundary: per block (E4M3 scale) and per element (E2M1 code).  A kernel whose FP32 h
-    differs from the exact value by less than that may round the other way there."""
+    differs from the exact value by less than that may round the other way there.  An
+    element whose scaled value is within ``rel`` of zero has an ambiguous sign: +0 and -0
+    (codes 0x0 and 0x8) both decode to zero."""
     h = np.asarray(h, dtype=np.float64)
     n = h.shape[-1]
     hb = h.reshape(-1, n // 16, 16)
@@ -165,5 +168,5 @@ def requant_near_tie(h: np.ndarray, g_h: float, rel=1e-4) -> tuple[np.ndarray, n
     d = oracle.e4m3_decode(S) * g_h
     v = np.abs(hb) / np.where(d == 0, np.inf, d)[..., None]
     dv = np.min(np.abs(v[..., None] - E2M1_MIDS), axis=-1)
-    elem_tie = dv <= rel * np.maximum(v, 0.25)
+    elem_tie = (dv <= rel * np.maximum(v, 0.25)) | (v <= rel)
     return block_tie.reshape(h.shape[:-1] + (n // 16,)), elem_tie.reshape(h.shape)
