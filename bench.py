@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 W4A4 group-limited MoE layer on B200.
+
+One step = one nvfp4moe_forward over one batch of tokens: route, quantise, group by
+expert, gate/up grouped GEMM + SwiGLU + requantisation, down grouped GEMM + weighted
+combine, BF16 output.  Default workload: the Beam-shape decode layer (16 tokens, hidden
+5120, 256 experts of intermediate 2560 in 8 groups of 32, top-4 groups, top-8 experts,
+x2.5), synthetic seeded inputs, random-init NVFP4 weights.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload decode|prefill|skewed|sweepT]
+    python bench.py --impl reference ...      # the CPU oracle on bounded samples
+
+Multi-GPU (launched with torch.distributed.run): every rank holds a full replica of the
+layer and routes its own batch (data parallel, no collective on the data path; weak
+scaling); the reported time is the maximum over ranks.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, BEAM, LayerShape, activations, router_weight, expert_weight, zipf_bias  # noqa: E402
+
+METRIC = "NVFP4 MoE-layer tokens/s; % of FP4 tensor peak (prefill) / HBM BW (decode)"
+FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense FP4 : BF16 tensor ratio
+E2M1_BYTES = 0.5                    # per value
+E4M3_PER16 = 1.0 / 16.0             # block-scale bytes per value
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def intermediate_scales(E: int) -> np.ndarray:
+    """Static SwiGLU-intermediate global scales written by the oracle calibration script."""
+    path = os.path.join(ROOT, "tests", "golden", "intermediate_scales_beam.txt")
+    vals = []
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if line:
+                vals.append(int(line[1], 16))
+    return np.array(vals, dtype=np.uint32).view(np.float32)[:E]
+
+
+# ------------------------------------------------------------------- clocks ----
+
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in _REASONS.items() if self.reasons & b], "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------- layer ----
+
+def layer_shape(E: int | None) -> LayerShape:
+    if E is None or E == BEAM.E:
+        return BEAM
+    # same hidden / intermediate sizes, fewer experts (8 groups): a smaller layer for profiling
+    return LayerShape(H=BEAM.H, I=BEAM.I, E=E, n_groups=8, topk_groups=4, topk=8, routed_scale=2.5,
+                      wr_std=BEAM.wr_std, w_std=BEAM.w_std)
+
+
+def build_layer(moe, shape: LayerShape):
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    ex = moe.Experts(cfg)
+    g_h = intermediate_scales(shape.E)
+    for e in range(shape.E):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    torch.cuda.synchronize()
+    return cfg, ex
+
+
+def algorithmic(shape: LayerShape, T: int, counts: np.ndarray):
+    """Algorithmic bytes / FLOPs of one step, from the routing the step actually produced."""
+    H, I, k = shape.H, shape.I, shape.topk
+    hit = int((counts > 0).sum())
+    pairs = T * k
+    per_val = E2M1_BYTES + E4M3_PER16                      # 0.5625 bytes per NVFP4 value
+    w13 = 2 * I * H * per_val + 8                          # gate + up codes, scales, globals
+    wd = H * I * per_val + 8
+    gateup_bytes = hit * w13 + pairs * H * per_val + pairs * I * per_val
+    layer_bytes = hit * (w13 + wd) + T * H * 2 + T * H * 2 + shape.E * H * 4
+    flops = 2.0 * pairs * (2 * I * H + H * I)
+    gateup_flops = 2.0 * pairs * 2 * I * H
+    return {"experts_hit": hit, "gateup_bytes": gateup_bytes, "layer_bytes": layer_bytes, "flops": flops,
+            "gateup_flops": gateup_flops}
+
+
+def _oracle_cfg(shape: LayerShape):
+    import types
+    return types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
+                                 topk=shape.topk, routed_scale=shape.routed_scale)
+
+
+def _blas_threads() -> int:
+    from threadpoolctl import threadpool_info
+    return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+
+
+def _oracle_experts(shape: LayerShape, experts):
+    """NVFP4 weights of the given experts, quantised by the oracle (the oracle's counterpart of
+    nvfp4moe_experts_create: prepared once, outside any timed region)."""
+    import oracle
+    return {e: tuple(oracle.quantize_tensor(expert_weight(shape, e, n).float().numpy())
+                     for n in ("gate", "up", "down")) for e in experts}
+
+
+def cpu_baseline_oracle(shape: LayerShape, wl, x_cpu, wr_cpu, bias_cpu, n_tokens=2):
+    """The oracle on a bounded sample of the step: routing and input quantisation of every
+    token, then the layer output of ``n_tokens`` tokens (their 8 experts' FP64 SwiGLU MLPs on
+    dequantised weights).  Expert weights are quantised beforehand, untimed, as the library's
+    experts are."""
+    import oracle
+    g_h = intermediate_scales(shape.E)
+    cfg = _oracle_cfg(shape)
+    x = x_cpu.float().numpy()
+    t0 = time.perf_counter()
+    r = oracle.route(x.astype(np.float64), wr_cpu.numpy(), cfg, None if bias_cpu is None else bias_cpu.numpy())
+    xc, xs, gx = oracle.quantize(x)
+    elapsed = time.perf_counter() - t0
+    toks = list(range(min(n_tokens, wl.T)))
+    qex = _oracle_experts(shape, sorted({int(e) for t in toks for e in r.idx[t]}))
+    t0 = time.perf_counter()
+    for t in toks:
+        xhat = oracle.dequantize(xc[t:t + 1], xs[t:t + 1], gx)
+        for j in range(shape.topk):
+            e = int(r.idx[t, j])
+            oracle.expert_mlp(xhat, *qex[e], np.float32(g_h[e]))
+    elapsed += time.perf_counter() - t0
+    return {"value": len(toks) / elapsed, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"routing + input quantisation of all {wl.T} tokens and the layer output of {len(toks)} "
+                      f"token(s) ({shape.topk} experts each, FP64 MLP on dequantised NVFP4 weights; weight "
+                      f"quantisation done beforehand, untimed); {elapsed:.1f} s of CPU work"}
+
+
+# --------------------------------------------------------------------- main ----
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_ours(args, world, rank, local):
+    import nvfp4_quantized_moe_group_b200 as moe
+    wl = WORKLOADS[args.workload]
+    shape = layer_shape(args.experts) if args.experts else wl.shape
+    T = wl.T
+    cfg, ex = build_layer(moe, shape)
+    x_cpu = activations(T, shape, seed=wl.seed + rank, rms_rows=wl.rms_rows)
+    wr_cpu = router_weight(shape)
+    bias_cpu = zipf_bias(shape.E) if wl.zipf else None
+    x = x_cpu.cuda()
+    wr = wr_cpu.cuda()
+    bias = None if bias_cpu is None else bias_cpu.cuda()
+    out = torch.empty((T, shape.H), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(moe.forward_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    # routing of this batch (for the algorithmic byte count) and a status check
+    _, dbg = moe.forward(ex, x, wr, bias, out=out, ws=ws, debug=True)
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"forward status {moe.status_string(st)}")
+    alg = algorithmic(shape, T, dbg["counts"].cpu().numpy())
+    launches_per_step = moe.last_launch_count()
+    del dbg
+
+    timers = [moe.StageTimer() for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        moe.forward(ex, x, wr, bias, out=out, ws=ws)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: K back-to-back steps, inputs resident in HBM
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        torch.cuda.nvtx.range_push("timed")
+        start.record(stream)
+        for k in range(args.steps):
+            moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=timers[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+    barrier(world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
+    stage = {n: statistics.mean(t.stage_ms()[n] for t in timers) for n in moe.STAGES}
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"forward status {moe.status_string(st)}")
+
+    # ---- end to end: pinned host input -> device, forward, device -> pinned host output
+    x_host = x_cpu.pin_memory()
+    out_host = torch.empty((T, shape.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(args.warmup):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.forward(ex, x_dev, wr, bias, out=out, ws=ws)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.forward(ex, x_dev, wr, bias, out=out, ws=ws)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    p = peaks()
+    ms_step = elapsed_ms / args.steps
+    tokens_per_s = world * T * args.steps / (elapsed_ms / 1e3)
+    # dominant kernel: the gate/up grouped GEMM (2/3 of the weight bytes and FLOPs)
+    gu_s = stage["gateup"] / 1e3
+    t_bytes = alg["gateup_bytes"] / (p["hbm_gbs"] * 1e9)
+    fp4_peak = p["bf16_tflops_sustained"] * FP4_OVER_BF16
+    t_flops = alg["gateup_flops"] / (fp4_peak * 1e12)
+    if t_bytes >= t_flops:
+        roof = {"bound": "hbm", "achieved": alg["gateup_bytes"] / gu_s / 1e9, "peak": p["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": alg["gateup_flops"] / gu_s / 1e12, "peak": fp4_peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
+    roof["peak_source"] = (f"{p['source']} hbm_gbs" if roof["bound"] == "hbm"
+                           else f"{p['source']} bf16_tflops_sustained x {FP4_OVER_BF16:g} (nominal FP4:BF16)")
+    layer_s = ms_step / 1e3
+    layer_roof = {"bytes_per_step": alg["layer_bytes"], "flops_per_step": alg["flops"],
+                  "hbm_frac": alg["layer_bytes"] / layer_s / (p["hbm_gbs"] * 1e9),
+                  "fp4_frac": alg["flops"] / layer_s / (fp4_peak * 1e12)}
+    res = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
+        "data": "synthetic (seeded counter-hash inputs; random-init NVFP4 weights)",
+        "config": {"workload": wl.describe() if not args.experts else wl.describe() + f" (E={shape.E} variant)",
+                   "T_per_rank": T, "experts_hit": alg["experts_hit"], "parallelism": f"dp{world} (replicas)",
+                   "l2": "no flush: every step streams the routed experts' weights "
+                         f"({alg['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"},
+        "roofline": roof, "layer_roofline": layer_roof,
+        "stage_ms": stage,
+        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_oracle(shape, wl, x_cpu, wr_cpu, bias_cpu)
+    ex.close()
+    return res
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm.  Each step is a bounded sample of the workload's step:
+    routing and input quantisation of all its tokens plus one (token, slot) pair's expert
+    (FP64 SwiGLU MLP on dequantised NVFP4 weights); the steps cycle through the 8 pairs of
+    token 0, whose experts are quantised once beforehand (untimed).  A pair is 1/topk token."""
+    import oracle
+    wl = WORKLOADS[args.workload]
+    shape = layer_shape(args.experts) if args.experts else wl.shape
+    T = wl.T
+    g_h = intermediate_scales(shape.E)
+    x = activations(T, shape, seed=wl.seed, rms_rows=wl.rms_rows).float().numpy()
+    wr = router_weight(shape).numpy()
+    bias = zipf_bias(shape.E).numpy() if wl.zipf else None
+    cfg = _oracle_cfg(shape)
+    r0 = oracle.route(x.astype(np.float64), wr, cfg, bias)
+    qex = _oracle_experts(shape, [int(e) for e in r0.idx[0]])
+
+    def step(i):
+        j = i % shape.topk
+        t0 = time.perf_counter()
+        r = oracle.route(x.astype(np.float64), wr, cfg, bias)
+        xc, xs, gx = oracle.quantize(x)
+        e = int(r.idx[0, j])
+        oracle.expert_mlp(oracle.dequantize(xc[:1], xs[:1], gx), *qex[e], np.float32(g_h[e]))
+        return time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        step(i)
+    total = sum(step(args.warmup + i) for i in range(args.steps))
+    value = (args.steps / shape.topk) / total
+    sample = (f"each step: routing + input quantisation of all {T} tokens of the {wl.name} workload and one "
+              f"(token, slot) pair's expert MLP (a pair is 1/{shape.topk} token); experts quantised beforehand")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.describe(), "T_per_rank": T},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+
+    world, rank, local = init_dist()
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

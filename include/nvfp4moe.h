@@ -180,6 +180,19 @@ NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_
  *   dbg  NULL on the hot path.  Otherwise every non-NULL member receives a copy of that
  *        intermediate (sizes below), for checking the layer step by step.
  *   ws   workspace of nvfp4moe_forward_workspace_bytes(cfg, T_max) bytes. */
+/* Stages of nvfp4moe_forward, in launch order (for nvfp4moe_debug.events). */
+enum {
+  NVFP4MOE_STAGE_AMAX = 0,      /* global amax of the input */
+  NVFP4MOE_STAGE_ROUTE = 1,     /* router logits + group-limited top-k */
+  NVFP4MOE_STAGE_QUANTIZE = 2,  /* NVFP4 quantisation of the input (+ accumulator zeroing) */
+  NVFP4MOE_STAGE_PERMUTE = 3,   /* grouping of pairs by expert */
+  NVFP4MOE_STAGE_GATHER = 4,    /* quantised rows into expert segments */
+  NVFP4MOE_STAGE_GATEUP = 5,    /* gate/up grouped GEMM + SwiGLU + requantisation */
+  NVFP4MOE_STAGE_DOWN = 6,      /* down grouped GEMM + weighted combine */
+  NVFP4MOE_STAGE_FINALIZE = 7,  /* FP32 accumulator -> BF16 output */
+  NVFP4MOE_NUM_STAGES = 8
+};
+
 typedef struct {
   int32_t* idx;        /* [T][topk] selected experts */
   float* w;            /* [T][topk] routing weights */
@@ -191,6 +204,9 @@ typedef struct {
   int32_t* perm;       /* [T*topk] pair ids (t*topk + j) grouped by expert, tokens ascending */
   uint8_t* hq_codes;   /* [T*topk][I/2] quantised SwiGLU intermediate, rows in perm order */
   uint8_t* hq_scales;  /* [T*topk][I/16] its block scales, linear */
+  void* const* events; /* NULL, or 2 * NVFP4MOE_NUM_STAGES cudaEvent_t created by the caller:
+                          events[2s] / events[2s+1] are recorded on the stream right before /
+                          after stage s (timing of the stages inside a forward) */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);

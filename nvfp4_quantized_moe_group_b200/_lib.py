@@ -45,9 +45,29 @@ class ExpertTensors(ctypes.Structure):
                 ("g_h", ctypes.c_float)]
 
 
+DEBUG_FIELDS = ("idx", "w", "g_x", "xq_codes", "xq_scales", "counts", "offsets", "perm", "hq_codes",
+                "hq_scales")
+STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "finalize")
+
+
 class Debug(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("idx", "w", "g_x", "xq_codes", "xq_scales", "counts", "offsets",
-                                               "perm", "hq_codes", "hq_scales")]
+    _fields_ = [(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class StageTimer:
+    """CUDA events recorded around every stage of a forward call (nvfp4moe_debug.events)."""
+
+    def __init__(self):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))]
+        for e in self.events:       # materialise the underlying cudaEvent_t
+            e.record()
+        torch.cuda.synchronize()
+        self.array = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+
+    def stage_ms(self) -> dict:
+        """Elapsed milliseconds of each stage of the last recorded forward (synchronises)."""
+        self.events[-1].synchronize()
+        return {name: self.events[2 * i].elapsed_time(self.events[2 * i + 1]) for i, name in enumerate(STAGES)}
 
 
 _lib = None
@@ -241,8 +261,10 @@ def forward_workspace_bytes(cfg: Cfg, T_max: int) -> int:
 
 
 def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
-            out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None):
-    """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug)."""
+            out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None,
+            timer: StageTimer | None = None):
+    """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug).
+    ``timer``: a StageTimer whose events are recorded around each stage."""
     cfg = experts.cfg
     T, H = x.shape
     dev = x.device
@@ -267,6 +289,10 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
             "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
         }
         dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
+    if timer is not None:
+        if dbg is None:
+            dbg = Debug()
+        dbg.events = ctypes.cast(timer.array, ctypes.POINTER(ctypes.c_void_p))
     st = lib().nvfp4moe_forward(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(out),
                                 ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
                                 _stream(stream))

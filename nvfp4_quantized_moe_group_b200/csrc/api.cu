@@ -160,6 +160,14 @@ __global__ void set_expert_scalars_kernel(float* g_gate, float* g_up, float* g_h
   alpha[e] = __fmul_rn(gh, gd);
 }
 
+struct StageEvents {
+  void* const* ev;
+  cudaStream_t s;
+  void mark(int stage, int which) const {
+    if (ev != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(ev[2 * stage + which]), s);
+  }
+};
+
 }  // namespace
 
 extern "C" {
@@ -398,9 +406,12 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
       make_tma_2d(&tma_h, f.hq_codes, c.I / 2, f.rows_cap, kBlockM) != 0)
     return NVFP4MOE_ERR_CUDA;
 
+  const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
   if (cudaMemsetAsync(&f.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   const int blocks = amax_partial_blocks(T * c.H);
+  ev.mark(NVFP4MOE_STAGE_AMAX, 0);
   if (launch_amax_partial(hidden_bf16, T * c.H, f.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_AMAX, 1);
   ++g_launches;
 
   RouterArgs r{};
@@ -417,7 +428,9 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   r.topk_groups = c.topk_groups;
   r.topk = c.topk;
   r.routed_scale = c.routed_scale;
+  ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
   if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
   g_launches += 2;
 
   QuantizeArgs q{};
@@ -435,7 +448,9 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   q.g_out = f.g_x;
   q.zero_out = f.acc;
   q.status = &f.hdr->status;
+  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
   if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
   ++g_launches;
 
   PermArgs pa{};
@@ -452,7 +467,9 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   pa.perm = f.perm;
   pa.inv = f.inv;
   pa.row_pair = f.row_pair;
+  ev.mark(NVFP4MOE_STAGE_PERMUTE, 0);
   if (launch_permute(pa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
   g_launches += 3;
 
   GatherArgs ga{};
@@ -467,7 +484,9 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   ga.n_pairs = pairs;
   ga.topk = c.topk;
   ga.H = c.H;
+  ev.mark(NVFP4MOE_STAGE_GATHER, 0);
   if (launch_gather(ga, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_GATHER, 1);
   ++g_launches;
 
   const int grid = num_sms();
@@ -493,17 +512,23 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   g.alpha_down = x->alpha_down;
   g.topk = c.topk;
   g.H = c.H;
+  ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
   if (launch_gemm_gateup(tma_a, x->tma_w13, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
   ++g_launches;
   g.sfa = f.hq_sf;
   g.sfb = x->wd_sf;
   g.K = c.I;
   g.n_total = c.H;
+  ev.mark(NVFP4MOE_STAGE_DOWN, 0);
   if (launch_gemm_down(tma_h, x->tma_wd, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 
   FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H};
+  ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
   if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_FINALIZE, 1);
   ++g_launches;
 
   if (dbg != nullptr) {
