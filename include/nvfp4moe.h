@@ -137,6 +137,28 @@ NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16
                    const float* w_router, const float* logit_bias, int32_t* idx, float* w,
                    void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------ route, no allocation ----
+ * The pages have no counterpart of this call; it exists for callers that cannot allocate
+ * device memory: a host runtime that passes the library only its input and output buffers
+ * and allows no device allocation after start-up, or a host framework that owns every
+ * device allocation and gives the libraries it embeds no allocator.  Such a caller has no
+ * workspace to pass to nvfp4moe_route.
+ *
+ * Same arguments and results as nvfp4moe_route (same kernels, identical idx and w), minus
+ * the workspace.  The router's scratch is a fixed array of 9,699,584 bytes of device memory
+ * declared by the library; every GPU that loads the library holds it until the process
+ * exits.  Limit: the split-K partial sums must fit, which holds whenever T * E <= 1,212,416
+ * (T <= 4736 for 256 experts); larger calls return NVFP4MOE_ERR_WORKSPACE and enqueue
+ * nothing.  The call allocates nothing.
+ *   * The first call on a device looks up that device's address of the array (once per
+ *     device, with the device current); make that first call before any stream capture.
+ *   * All calls share the one array, which keeps the contents of the last call.  Calls whose
+ *     work can overlap on the GPU (different streams, or different host threads, on the
+ *     same device) race on it; serialise them. */
+NVFP4MOE_API int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
+                                        const float* w_router, const float* logit_bias, int32_t* idx,
+                                        float* w, void* stream);
+
 /* ----------------------------------------------------------------- experts ----
  * Library-owned, repacked copy of the E experts' NVFP4 weights (the operand layout of
  * the grouped GEMMs).  nvfp4moe_experts_create allocates it (device memory of the

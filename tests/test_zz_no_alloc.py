@@ -1,0 +1,76 @@
+"""nvfp4moe_route_noalloc: the router for callers that cannot allocate device memory.
+
+Such callers (a host runtime that hands the library only input and output buffers and
+forbids device allocation after start-up, or a host framework that owns all device memory)
+cannot provide the workspace nvfp4moe_route needs, so this entry point keeps the router's
+scratch in a fixed device array of the library.  These tests call it through the C ABI and
+check it against nvfp4moe_route on consecutive calls (the array keeps the previous call's
+contents), and check that a call beyond the array's capacity is refused.  The file is
+collected last so that a failure here does not hide the other GPU tests.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_quantized_moe_group_b200 as moe
+from workloads import TINY, BEAM, activations, router_weight, zipf_bias
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    moe.lib()
+
+
+def _route_noalloc(cfg, x, wr, bias, idx, w):
+    f = moe.lib().nvfp4moe_route_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(moe.Cfg), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    return f(ctypes.byref(cfg), ptr(x), x.shape[0], ptr(wr), ptr(bias), ptr(idx), ptr(w),
+             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def _cfg(shape):
+    return moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                        shape.routed_scale)
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_matches_route_on_consecutive_calls(order):
+    cases = [(BEAM, 4096, False, None), (BEAM, 16, True, None), (TINY, 64, False, None),
+             (BEAM, 1000, False, zipf_bias(256))]
+    if order:
+        cases = cases[::-1]
+    for shape, T, rms, bias in cases:
+        cfg = _cfg(shape)
+        x = activations(T, shape, rms_rows=rms).cuda()
+        wr = router_weight(shape).cuda()
+        b = None if bias is None else bias.cuda()
+        idx = torch.full((T, shape.topk), -1, dtype=torch.int32, device="cuda")
+        w = torch.full((T, shape.topk), -1.0, dtype=torch.float32, device="cuda")
+        assert _route_noalloc(cfg, x, wr, b, idx, w) == moe.OK
+        ref_idx, ref_w = moe.route(cfg, x, wr, b)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx.cpu().numpy())
+        np.testing.assert_allclose(w.cpu().numpy(), ref_w.cpu().numpy(), rtol=2e-6, atol=0)
+
+
+def test_refuses_calls_beyond_capacity():
+    cfg = _cfg(BEAM)
+    wr = router_weight(BEAM).cuda()
+    x = activations(4737, BEAM).cuda()
+    idx = torch.empty((4737, 8), dtype=torch.int32, device="cuda")
+    w = torch.empty((4737, 8), dtype=torch.float32, device="cuda")
+    assert _route_noalloc(cfg, x, wr, None, idx, w) == moe.ERR_WORKSPACE
+    x = x[:4736].contiguous()
+    assert _route_noalloc(cfg, x, wr, None, idx[:4736], w[:4736]) == moe.OK
+    ref_idx, _ = moe.route(cfg, x, wr)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx[:4736].cpu().numpy(), ref_idx.cpu().numpy())
