@@ -202,13 +202,17 @@ NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_
  *   dbg  NULL on the hot path.  Otherwise every non-NULL member receives a copy of that
  *        intermediate (sizes below), for checking the layer step by step.
  *   ws   workspace of nvfp4moe_forward_workspace_bytes(cfg, T_max) bytes. */
-/* Stages of nvfp4moe_forward, in launch order (for nvfp4moe_debug.events). */
+/* Stages of nvfp4moe_forward (for nvfp4moe_debug.events).  Launch order: ROUTE, PERMUTE,
+ * QUANTIZE, GATEUP, DOWN, FINALIZE.  The input's global amax is computed inside ROUTE and
+ * the rows are written into the expert segments inside QUANTIZE, so the AMAX and GATHER
+ * events are recorded back to back (zero time). */
 enum {
-  NVFP4MOE_STAGE_AMAX = 0,      /* global amax of the input */
-  NVFP4MOE_STAGE_ROUTE = 1,     /* router logits + group-limited top-k */
-  NVFP4MOE_STAGE_QUANTIZE = 2,  /* NVFP4 quantisation of the input (+ accumulator zeroing) */
+  NVFP4MOE_STAGE_AMAX = 0,      /* global amax of the input (inside ROUTE) */
+  NVFP4MOE_STAGE_ROUTE = 1,     /* router logits (+ amax partials) + group-limited top-k */
+  NVFP4MOE_STAGE_QUANTIZE = 2,  /* NVFP4 quantisation of the input into the expert segments
+                                   (+ accumulator zeroing) */
   NVFP4MOE_STAGE_PERMUTE = 3,   /* grouping of pairs by expert */
-  NVFP4MOE_STAGE_GATHER = 4,    /* quantised rows into expert segments */
+  NVFP4MOE_STAGE_GATHER = 4,    /* (inside QUANTIZE) */
   NVFP4MOE_STAGE_GATEUP = 5,    /* gate/up grouped GEMM + SwiGLU + requantisation */
   NVFP4MOE_STAGE_DOWN = 6,      /* down grouped GEMM + weighted combine */
   NVFP4MOE_STAGE_FINALIZE = 7,  /* FP32 accumulator -> BF16 output */
@@ -228,7 +232,8 @@ typedef struct {
   uint8_t* hq_scales;  /* [T*topk][I/16] its block scales, linear */
   void* const* events; /* NULL, or 2 * NVFP4MOE_NUM_STAGES cudaEvent_t created by the caller:
                           events[2s] / events[2s+1] are recorded on the stream right before /
-                          after stage s (timing of the stages inside a forward) */
+                          after stage s (timing of the stages inside a forward); NULL entries
+                          are skipped */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);

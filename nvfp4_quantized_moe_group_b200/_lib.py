@@ -55,19 +55,32 @@ class Debug(ctypes.Structure):
 
 
 class StageTimer:
-    """CUDA events recorded around every stage of a forward call (nvfp4moe_debug.events)."""
+    """CUDA events recorded around stages of a forward call (nvfp4moe_debug.events).
+    ``stages``: the stage names to time (default all)."""
 
-    def __init__(self):
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(STAGES))]
-        for e in self.events:       # materialise the underlying cudaEvent_t
-            e.record()
+    def __init__(self, stages=STAGES):
+        self.stages = [s for s in STAGES if s in stages]
+        self.events = {}
+        for name in self.stages:
+            pair = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for e in pair:          # materialise the underlying cudaEvent_t
+                e.record()
+            self.events[name] = pair
         torch.cuda.synchronize()
-        self.array = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+        handles = []
+        for name in STAGES:
+            pair = self.events.get(name)
+            handles += [pair[0].cuda_event, pair[1].cuda_event] if pair else [None, None]
+        self.array = (ctypes.c_void_p * len(handles))(*handles)
 
     def stage_ms(self) -> dict:
-        """Elapsed milliseconds of each stage of the last recorded forward (synchronises)."""
-        self.events[-1].synchronize()
-        return {name: self.events[2 * i].elapsed_time(self.events[2 * i + 1]) for i, name in enumerate(STAGES)}
+        """Elapsed milliseconds of each timed stage of the last recorded forward (synchronises)."""
+        out = {}
+        for name in self.stages:
+            a, b = self.events[name]
+            b.synchronize()
+            out[name] = a.elapsed_time(b)
+        return out
 
 
 _lib = None

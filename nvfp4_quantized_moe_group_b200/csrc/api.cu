@@ -11,16 +11,14 @@ using namespace nvfp4moe;
 struct nvfp4moe_experts {
   nvfp4moe_cfg cfg;
   int device;
-  uint8_t* w13_codes;   // [E][2I][H/2], gate and up rows interleaved per 128-row tile
-  uint8_t* w13_sf;      // swizzled, [E][2I/128 tiles][H/64 column tiles][512]
-  uint8_t* wd_codes;    // [E][H][I/2]
+  uint8_t* w13_codes;   // tiled (see launch_tile_weights), gate/up rows interleaved per 64-row group
+  uint8_t* w13_sf;      // swizzled, [E][2I/128 row tiles][H/64 column tiles][512]
+  uint8_t* wd_codes;    // tiled, [E][H/128][ceil(I/256)][128][128]
   uint8_t* wd_sf;       // swizzled, [E][H/128][I/64][512]
   float* g_gate;        // [E] device
   float* g_up;
   float* g_h;
   float* alpha_down;    // [E] g_h * g_down
-  CUtensorMap tma_w13;
-  CUtensorMap tma_wd;
 };
 
 namespace {
@@ -128,7 +126,8 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   const int64_t n_chunks = (T + kPermChunkTokens - 1) / kPermChunkTokens;
   f.rows_cap = rows_capacity(cfg, T);
   f.hdr = c.take<WsHeader>(1);
-  f.partials = c.take<uint32_t>(kMaxAmaxPartials);
+  const int n_part = router_amax_partials(T, cfg.E, cfg.H);
+  f.partials = c.take<uint32_t>(n_part > kMaxAmaxPartials ? n_part : kMaxAmaxPartials);
   f.g_x = c.take<float>(1);
   f.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
   f.idx = c.take<int32_t>(pairs);
@@ -164,7 +163,8 @@ struct StageEvents {
   void* const* ev;
   cudaStream_t s;
   void mark(int stage, int which) const {
-    if (ev != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(ev[2 * stage + which]), s);
+    if (ev != nullptr && ev[2 * stage + which] != nullptr)
+      cudaEventRecord(static_cast<cudaEvent_t>(ev[2 * stage + which]), s);
   }
 };
 
@@ -307,16 +307,16 @@ int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out) {
   x->cfg = *cfg;
   cudaGetDevice(&x->device);
   const int64_t E = cfg->E, H = cfg->H, I = cfg->I;
-  const size_t w13 = (size_t)E * 2 * I * H / 2, w13sf = (size_t)E * 2 * I * H / 16;
-  const size_t wd = (size_t)E * H * I / 2, wdsf = (size_t)E * H * I / 16;
+  // tiled codes: K padded to a multiple of 256 values (128 bytes)
+  const size_t w13 = (size_t)E * 2 * I * ((H + 255) / 256 * 128), w13sf = (size_t)E * 2 * I * H / 16;
+  const size_t wd = (size_t)E * H * ((I + 255) / 256 * 128), wdsf = (size_t)E * H * I / 16;
   bool ok = cudaMalloc(&x->w13_codes, w13) == cudaSuccess && cudaMalloc(&x->w13_sf, w13sf) == cudaSuccess &&
             cudaMalloc(&x->wd_codes, wd) == cudaSuccess && cudaMalloc(&x->wd_sf, wdsf) == cudaSuccess &&
             cudaMalloc(&x->g_gate, E * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&x->g_up, E * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&x->g_h, E * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&x->alpha_down, E * sizeof(float)) == cudaSuccess;
-  ok = ok && make_tma_2d(&x->tma_w13, x->w13_codes, H / 2, (uint64_t)E * 2 * I, kBlockN) == 0;
-  ok = ok && make_tma_2d(&x->tma_wd, x->wd_codes, I / 2, (uint64_t)E * H, kBlockN) == 0;
+  ok = ok && cudaMemset(x->w13_codes, 0, w13) == cudaSuccess && cudaMemset(x->wd_codes, 0, wd) == cudaSuccess;
   if (!ok) {
     nvfp4moe_experts_destroy(x);
     return NVFP4MOE_ERR_CUDA;
@@ -334,28 +334,27 @@ int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e, const nvfp4moe_expert_t
     return NVFP4MOE_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t H = c.H, I = c.I;
-  const size_t tile_gu = (size_t)128 * H / 2;  // bytes of 128 rows of gate/up codes
-  uint8_t* w13 = x->w13_codes + (size_t)e * 2 * I * H / 2;
-  // gate tile j -> packed tile 2j, up tile j -> packed tile 2j+1
-  if (cudaMemcpy2DAsync(w13, 2 * tile_gu, t->gate_codes, tile_gu, tile_gu, I / 128, cudaMemcpyDeviceToDevice,
-                        s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
-  if (cudaMemcpy2DAsync(w13 + tile_gu, 2 * tile_gu, t->up_codes, tile_gu, tile_gu, I / 128,
-                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
-  if (cudaMemcpyAsync(x->wd_codes + (size_t)e * H * I / 2, t->down_codes, (size_t)H * I / 2,
-                      cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+  // gate/up rows are interleaved in groups of half a GEMM column tile: packed group 2j holds
+  // gate rows [64j, 64j+64), group 2j+1 the up rows of the same features
+  constexpr int kG = kBlockN / 2;
+  const size_t w13_expert = (size_t)2 * I * ((H + 255) / 256 * 128);
+  const size_t wd_expert = (size_t)H * ((I + 255) / 256 * 128);
+  uint8_t* w13 = x->w13_codes + (size_t)e * w13_expert;
+  if (launch_tile_weights(t->gate_codes, (int)I, (int)(H / 2), w13, kG, 2, 0, s) != cudaSuccess ||
+      launch_tile_weights(t->up_codes, (int)I, (int)(H / 2), w13, kG, 2, 1, s) != cudaSuccess ||
+      launch_tile_weights(t->down_codes, (int)H, (int)(I / 2), x->wd_codes + (size_t)e * wd_expert, (int)H, 1, 0,
+                          s) != cudaSuccess)
     return NVFP4MOE_ERR_CUDA;
   uint8_t* w13sf = x->w13_sf + (size_t)e * 2 * I * H / 16;
-  if (launch_repack_sf(t->gate_scales, (int)I, (int)(H / 16), w13sf, H / 64, (2 << 8) | 0, s) != cudaSuccess ||
-      launch_repack_sf(t->up_scales, (int)I, (int)(H / 16), w13sf, H / 64, (2 << 8) | 1, s) != cudaSuccess ||
-      launch_repack_sf(t->down_scales, (int)H, (int)(I / 16), x->wd_sf + (size_t)e * H * I / 16, I / 64,
-                       (1 << 8) | 0, s) != cudaSuccess)
+  if (launch_repack_sf(t->gate_scales, (int)I, (int)(H / 16), w13sf, H / 64, kG, 2, 0, s) != cudaSuccess ||
+      launch_repack_sf(t->up_scales, (int)I, (int)(H / 16), w13sf, H / 64, kG, 2, 1, s) != cudaSuccess ||
+      launch_repack_sf(t->down_scales, (int)H, (int)(I / 16), x->wd_sf + (size_t)e * H * I / 16, I / 64, (int)H,
+                       1, 0, s) != cudaSuccess)
     return NVFP4MOE_ERR_CUDA;
   set_expert_scalars_kernel<<<1, 1, 0, s>>>(x->g_gate, x->g_up, x->g_h, x->alpha_down, e, t->g_gate, t->g_up,
                                             t->g_h, t->g_down);
   if (cudaGetLastError() != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  g_launches += 4;
+  g_launches += 7;
   return NVFP4MOE_OK;
 }
 
@@ -401,19 +400,17 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t pairs = T * c.topk;
 
-  CUtensorMap tma_a, tma_h;
+  CUtensorMap tma_a, tma_a32, tma_h, tma_h32;
   if (make_tma_2d(&tma_a, f.a_codes, c.H / 2, f.rows_cap, kBlockM) != 0 ||
-      make_tma_2d(&tma_h, f.hq_codes, c.I / 2, f.rows_cap, kBlockM) != 0)
+      make_tma_2d(&tma_a32, f.a_codes, c.H / 2, f.rows_cap, 32) != 0 ||
+      make_tma_2d(&tma_h, f.hq_codes, c.I / 2, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_h32, f.hq_codes, c.I / 2, f.rows_cap, 32) != 0)
     return NVFP4MOE_ERR_CUDA;
 
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
   if (cudaMemsetAsync(&f.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  const int blocks = amax_partial_blocks(T * c.H);
-  ev.mark(NVFP4MOE_STAGE_AMAX, 0);
-  if (launch_amax_partial(hidden_bf16, T * c.H, f.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_AMAX, 1);
-  ++g_launches;
 
+  // route: logits (with the per-block maxima of |x| for the global scale) + top-k
   RouterArgs r{};
   r.x = static_cast<const uint16_t*>(hidden_bf16);
   r.w = w_router;
@@ -428,31 +425,15 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   r.topk_groups = c.topk_groups;
   r.topk = c.topk;
   r.routed_scale = c.routed_scale;
+  r.amax_partials = f.partials;
+  ev.mark(NVFP4MOE_STAGE_AMAX, 0);
+  ev.mark(NVFP4MOE_STAGE_AMAX, 1);
   ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
   if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
   g_launches += 2;
 
-  QuantizeArgs q{};
-  q.x = static_cast<const uint16_t*>(hidden_bf16);
-  q.rows = T;
-  q.rows_padded = round128(T);
-  q.cols = c.H;
-  q.g_in = nullptr;
-  q.partials = f.partials;
-  q.n_partials = blocks;
-  q.codes = f.xq_codes;
-  q.scales = f.xq_sf;
-  q.swizzled = 1;
-  q.n_col_tiles = c.H / 64;
-  q.g_out = f.g_x;
-  q.zero_out = f.acc;
-  q.status = &f.hdr->status;
-  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
-  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
-  ++g_launches;
-
+  // group the (token, slot) pairs by expert
   PermArgs pa{};
   pa.idx = f.idx;
   pa.T = T;
@@ -468,29 +449,44 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   pa.inv = f.inv;
   pa.row_pair = f.row_pair;
   ev.mark(NVFP4MOE_STAGE_PERMUTE, 0);
-  if (launch_permute(pa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
-  g_launches += 3;
 
-  GatherArgs ga{};
-  ga.xq_codes = f.xq_codes;
-  ga.xq_sf = f.xq_sf;
-  ga.idx = f.idx;
-  ga.inv = f.inv;
-  ga.offsets = f.offsets;
-  ga.mtile_prefix = f.mtile_prefix;
-  ga.a_codes = f.a_codes;
-  ga.a_sf = f.a_sf;
-  ga.n_pairs = pairs;
-  ga.topk = c.topk;
-  ga.H = c.H;
+  // quantise x and write each token's row into its expert-segment rows (zeroes the
+  // accumulator alongside); the token-major copy is only kept for the debug export
+  const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
+  QuantizeArgs q{};
+  q.x = static_cast<const uint16_t*>(hidden_bf16);
+  q.rows = T;
+  q.rows_padded = keep_xq ? round128(T) : T;
+  q.cols = c.H;
+  q.g_in = nullptr;
+  q.partials = f.partials;
+  q.n_partials = router_amax_partials(T, c.E, c.H);
+  q.codes = keep_xq ? f.xq_codes : nullptr;
+  q.scales = keep_xq ? f.xq_sf : nullptr;
+  q.swizzled = 1;
+  q.n_col_tiles = c.H / 64;
+  q.g_out = f.g_x;
+  q.zero_out = f.acc;
+  q.status = &f.hdr->status;
+  q.idx = f.idx;
+  q.inv = f.inv;
+  q.offsets = f.offsets;
+  q.mtile_prefix = f.mtile_prefix;
+  q.topk = c.topk;
+  q.seg_codes = f.a_codes;
+  q.seg_sf = f.a_sf;
+  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
+  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
   ev.mark(NVFP4MOE_STAGE_GATHER, 0);
-  if (launch_gather(ga, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_GATHER, 1);
   ++g_launches;
 
   const int grid = num_sms();
   GemmArgs g{};
+  g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
   g.sfb = x->w13_sf;
   g.mtile_prefix = f.mtile_prefix;
@@ -513,15 +509,16 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   g.topk = c.topk;
   g.H = c.H;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
-  if (launch_gemm_gateup(tma_a, x->tma_w13, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
   ++g_launches;
+  g.b_tiles = x->wd_codes;
   g.sfa = f.hq_sf;
   g.sfb = x->wd_sf;
   g.K = c.I;
   g.n_total = c.H;
   ev.mark(NVFP4MOE_STAGE_DOWN, 0);
-  if (launch_gemm_down(tma_h, x->tma_wd, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_down(tma_h, tma_h32, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 

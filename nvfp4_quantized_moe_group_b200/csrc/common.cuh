@@ -80,6 +80,13 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float r_t, float g, 
   return s;
 }
 
+// Approximate reciprocal (rcp.approx, about 1 ulp), for x >= 1.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Global scale from a tensor amax: A / 2688, or 1 when A == 0.
 __device__ __forceinline__ float global_scale_from_amax(float a) {
   return (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);

@@ -10,7 +10,7 @@ namespace nvfp4moe {
 
 constexpr int kMaxAmaxPartials = 1024;   // blocks of the amax pass
 constexpr int kBlockM = 128;             // token rows per GEMM tile / expert segment padding
-constexpr int kBlockN = 256;             // output columns per GEMM tile
+constexpr int kBlockN = 128;             // output columns per GEMM tile
 constexpr int kBlockK = 256;             // K values per pipeline stage (128 bytes of E2M1)
 constexpr int kPermChunkTokens = 128;    // tokens per chunk of the grouping kernels
 
@@ -29,6 +29,15 @@ struct QuantizeArgs {
   float* g_out;
   float* zero_out;         // optional [rows][cols] fp32 zeroed alongside (layer accumulator)
   uint32_t* status;
+  // optional scatter into expert segments: row t also goes to the padded segment row of
+  // each of its pairs (t*topk + j), codes [seg rows][cols/2], swizzled scales
+  const int32_t* idx;
+  const int32_t* inv;
+  const int32_t* offsets;
+  const int32_t* mtile_prefix;
+  int topk;
+  uint8_t* seg_codes;
+  uint8_t* seg_sf;
 };
 
 struct RouterArgs {
@@ -42,6 +51,7 @@ struct RouterArgs {
   int H, E, n_groups, topk_groups, topk;
   float routed_scale;
   int ksplit, k_slice;
+  uint32_t* amax_partials;  // optional: per-CTA max |x| (BF16 magnitude bits) for the global scale
 };
 
 struct PermArgs {
@@ -59,21 +69,8 @@ struct PermArgs {
   int32_t* row_pair;       // [rows_cap] pair id of each padded row, -1 for padding
 };
 
-struct GatherArgs {
-  const uint8_t* xq_codes;   // [T][H/2]
-  const uint8_t* xq_sf;      // swizzled, rows = tokens
-  const int32_t* idx;
-  const int32_t* inv;
-  const int32_t* offsets;
-  const int32_t* mtile_prefix;
-  uint8_t* a_codes;          // [rows_cap][H/2]
-  uint8_t* a_sf;             // swizzled, rows = padded rows
-  int64_t n_pairs;
-  int topk;
-  int H;
-};
-
 struct GemmArgs {
+  const uint8_t* b_tiles;      // weights, tiled: [E][n_total/128][ceil(K/256)][128 rows][128 B], swizzled
   const uint8_t* sfa;          // swizzled scales of A (padded rows)
   const uint8_t* sfb;          // swizzled scales of B, experts back to back
   const int32_t* mtile_prefix; // [E+1]
@@ -114,11 +111,14 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 // route.cu
 int router_ksplit(int64_t T, int E, int H);
 size_t router_parts_elems(int64_t T_max, int E, int H);
+// Number of amax partials the logits kernel writes for T tokens (grid x * split-K).
+int router_amax_partials(int64_t T, int E, int H);
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream);
 
 // permute.cu
-cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream);
-cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
+// Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.
+constexpr int kPermSmallPairs = 4096;
+cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream, int* launches);
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream);
 cudaError_t launch_unswizzle_rows(const uint8_t* sf, int64_t n_col_tiles, const int32_t* src_rows,
                                   int64_t n_rows, int cols16, uint8_t* out, cudaStream_t stream);
@@ -126,15 +126,22 @@ cudaError_t launch_export_hq(const uint8_t* hq_codes, const uint8_t* hq_sf, cons
                              const int32_t* idx, const int32_t* offsets, const int32_t* mtile_prefix,
                              int64_t n_pairs, int I, uint8_t* out_codes, uint8_t* out_sf,
                              cudaStream_t stream);
+// Source row r goes to destination row (r / group) * group * mul + add * group + r % group.
 cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_t* swz,
-                             int64_t n_col_tiles, int tile_mul_add /* (mul << 8) | add */,
-                             cudaStream_t stream);
+                             int64_t n_col_tiles, int group, int mul, int add, cudaStream_t stream);
 
 // gemm.cu
-cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_b, const GemmArgs& a,
+// tma_a / tma_a32: the A rows with a 128-row / 32-row box (both 128 bytes wide).
+cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                                int grid, cudaStream_t stream);
-cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_b, const GemmArgs& a,
+cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                              int grid, cudaStream_t stream);
+// Weight codes [rows][row_bytes] -> tiled operand layout: source row r is packed row
+// (r / group) * group * mul + add * group + r % group; packed rows form 128-row tiles, each
+// split into 128-byte K blocks stored as contiguous 16 KB images of the 128-byte-swizzled
+// shared-memory tile.  The destination must be zero where row_bytes is not a multiple of 128.
+cudaError_t launch_tile_weights(const uint8_t* src, int rows, int row_bytes, uint8_t* dst, int group, int mul,
+                                int add, cudaStream_t stream);
 // Encodes a 2D byte tensor map [rows][row_bytes] with a 128-byte x box_rows box, 128B swizzle.
 int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows);
 

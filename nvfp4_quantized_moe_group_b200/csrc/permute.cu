@@ -1,6 +1,6 @@
 // Grouping of (token, slot) pairs by expert and the byte-moving kernels around the grouped
-// GEMMs: stable counting sort into 128-row-padded expert segments, gather of quantised
-// rows into those segments, FP32 -> BF16 output, scale-layout conversions.
+// GEMMs: stable counting sort into 128-row-padded expert segments, FP32 -> BF16 output,
+// scale-layout conversions.
 // Only the top-8 of 256 experts run per token ("Reflection releases Beam ...", section
 // "Mixture-of-Experts details"), so the pairs are grouped by expert before the expert GEMMs.
 #include "common.cuh"
@@ -35,30 +35,32 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
       running += v;
     }
   }
+  const int tiles = e < a.E ? (running + kBlockM - 1) / kBlockM : 0;
   s_cnt[e] = e < a.E ? running : 0;
-  s_tiles[e] = e < a.E ? (running + kBlockM - 1) / kBlockM : 0;
+  s_tiles[e] = tiles;
   __syncthreads();
-  if (e == 0) {
-    int off = 0, tiles = 0;
-    for (int i = 0; i < a.E; ++i) {
-      const int c = s_cnt[i], t = s_tiles[i];
-      a.offsets[i] = off;
-      a.mtile_prefix[i] = tiles;
-      s_cnt[i] = off;
-      s_tiles[i] = tiles;
-      off += c;
-      tiles += t;
-    }
-    a.offsets[a.E] = off;
-    a.mtile_prefix[a.E] = tiles;
+  // inclusive scans (Hillis-Steele) of counts and tiles over the 256 threads
+  for (int d = 1; d < 256; d <<= 1) {
+    const int vc = e >= d ? s_cnt[e - d] : 0;
+    const int vt = e >= d ? s_tiles[e - d] : 0;
+    __syncthreads();
+    s_cnt[e] += vc;
+    s_tiles[e] += vt;
+    __syncthreads();
   }
-  __syncthreads();
   if (e < a.E) {
-    const int off = s_cnt[e];
+    const int off = s_cnt[e] - running;       // exclusive
+    const int tile0 = s_tiles[e] - tiles;
+    a.offsets[e] = off;
+    a.mtile_prefix[e] = tile0;
     a.counts[e] = running;
+    if (e == a.E - 1) {
+      a.offsets[a.E] = off + running;
+      a.mtile_prefix[a.E] = tile0 + tiles;
+    }
     for (int c = 0; c < a.n_chunks; ++c) a.chunk_base[(int64_t)c * a.E + e] += off;
-    const int64_t r0 = (int64_t)s_tiles[e] * kBlockM;
-    const int64_t r1 = r0 + (int64_t)((running + kBlockM - 1) / kBlockM) * kBlockM;
+    const int64_t r0 = (int64_t)tile0 * kBlockM;
+    const int64_t r1 = r0 + (int64_t)tiles * kBlockM;
     for (int64_t r = r0 + running; r < r1; ++r) a.row_pair[r] = -1;
   }
 }
@@ -93,7 +95,73 @@ __global__ void __launch_bounds__(32) perm_scatter_kernel(PermArgs a) {
   }
 }
 
-cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream) {
+// Small inputs: histogram, scan and the stable scatter in one block (the scatter walks the
+// pairs in order with one warp, like perm_scatter_kernel does per chunk).
+__global__ void __launch_bounds__(256) perm_small_kernel(PermArgs a) {
+  __shared__ int s_cnt[256];
+  __shared__ int s_tiles[256];
+  __shared__ int run[256];
+  const int e = threadIdx.x;
+  s_cnt[e] = 0;
+  __syncthreads();
+  const int64_t n = a.T * a.topk;
+  for (int64_t p = e; p < n; p += blockDim.x) atomicAdd(&s_cnt[a.idx[p]], 1);
+  __syncthreads();
+  const int count = e < a.E ? s_cnt[e] : 0;
+  const int tiles = (count + kBlockM - 1) / kBlockM;
+  s_tiles[e] = tiles;
+  __syncthreads();
+  for (int d = 1; d < 256; d <<= 1) {
+    const int vc = e >= d ? s_cnt[e - d] : 0;
+    const int vt = e >= d ? s_tiles[e - d] : 0;
+    __syncthreads();
+    s_cnt[e] += vc;
+    s_tiles[e] += vt;
+    __syncthreads();
+  }
+  if (e < a.E) {
+    const int off = s_cnt[e] - count;
+    const int tile0 = s_tiles[e] - tiles;
+    a.offsets[e] = off;
+    a.mtile_prefix[e] = tile0;
+    a.counts[e] = count;
+    run[e] = off;
+    if (e == a.E - 1) {
+      a.offsets[a.E] = off + count;
+      a.mtile_prefix[a.E] = tile0 + tiles;
+    }
+    const int64_t r0 = (int64_t)tile0 * kBlockM;
+    for (int64_t r = r0 + count; r < r0 + (int64_t)tiles * kBlockM; ++r) a.row_pair[r] = -1;
+  }
+  __syncthreads();
+  if (e >= 32) return;
+  const int lane = e;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t base = 0; base < n; base += 32) {
+    const int64_t p = base + lane;
+    const bool valid = p < n;
+    const int ex = valid ? a.idx[p] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ex);
+    const int rank = __popc(peers & lt);
+    if (valid) {
+      const int pos = run[ex] + rank;
+      a.perm[pos] = (int32_t)p;
+      a.inv[p] = pos;
+      a.row_pair[(int64_t)a.mtile_prefix[ex] * kBlockM + (pos - a.offsets[ex])] = (int32_t)p;
+    }
+    __syncwarp();
+    if (valid && rank == 0) run[ex] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream, int* launches) {
+  if (a.T * a.topk <= kPermSmallPairs) {
+    perm_small_kernel<<<1, 256, 0, stream>>>(a);
+    *launches += 1;
+    return cudaGetLastError();
+  }
+  *launches += 3;
   perm_count_kernel<<<a.n_chunks, 256, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -101,32 +169,6 @@ cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream) {
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   perm_scatter_kernel<<<a.n_chunks, 32, 0, stream>>>(a);
-  return cudaGetLastError();
-}
-
-// One warp per pair: copy the token's quantised row (codes and its swizzled scale groups)
-// into the pair's row of the expert segment.
-__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
-  const int64_t pair = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (pair >= a.n_pairs) return;
-  const int e = a.idx[pair];
-  const int64_t token = pair / a.topk;
-  const int64_t row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[pair] - a.offsets[e]);
-  const int64_t row_bytes = a.H >> 1;
-  const uint4* src = reinterpret_cast<const uint4*>(a.xq_codes + token * row_bytes);
-  uint4* dst = reinterpret_cast<uint4*>(a.a_codes + row * row_bytes);
-  for (int64_t i = lane; i < row_bytes / 16; i += 32) dst[i] = __ldg(src + i);
-  const int64_t n_ct = a.H >> 6;  // 4-scale column groups per row
-  for (int64_t ct = lane; ct < n_ct; ct += 32) {
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(a.xq_sf + swz_offset(token, ct * 4, n_ct));
-    *reinterpret_cast<uint32_t*>(a.a_sf + swz_offset(row, ct * 4, n_ct)) = v;
-  }
-}
-
-cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream) {
-  if (a.n_pairs == 0) return cudaSuccess;
-  gather_kernel<<<(unsigned)((a.n_pairs + 7) / 8), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -202,25 +244,49 @@ cudaError_t launch_export_hq(const uint8_t* hq_codes, const uint8_t* hq_sf, cons
   return cudaGetLastError();
 }
 
-// Linear [rows][cols16] weight scales -> swizzled operand storage.  Source row tile j is
-// placed at destination row tile j * tile_mul + tile_add (gate/up interleave: 2, 0 / 2, 1).
+// Linear [rows][cols16] weight scales -> swizzled operand storage.  Source row r goes to
+// destination row (r / group) * group * mul + add * group + r % group (gate/up interleave:
+// group 64, mul 2, add 0 for gate and 1 for up).
 __global__ void __launch_bounds__(256) repack_sf_kernel(const uint8_t* linear, int rows, int cols16,
-                                                        uint8_t* swz, int64_t n_col_tiles, int tile_mul,
-                                                        int tile_add) {
+                                                        uint8_t* swz, int64_t n_col_tiles, int group, int mul,
+                                                        int add) {
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= (int64_t)rows * cols16) return;
   const int r = (int)(i / cols16);
   const int c = (int)(i - (int64_t)r * cols16);
-  const int64_t dr = (int64_t)((r >> 7) * tile_mul + tile_add) * kBlockM + (r & 127);
+  const int64_t dr = (int64_t)(r / group) * group * mul + (int64_t)add * group + r % group;
   swz[swz_offset(dr, c, n_col_tiles)] = linear[i];
 }
 
 cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_t* swz,
-                             int64_t n_col_tiles, int tile_mul_add, cudaStream_t stream) {
+                             int64_t n_col_tiles, int group, int mul, int add, cudaStream_t stream) {
   const int64_t n = (int64_t)rows * cols16;
-  const int tile_mul = tile_mul_add >> 8, tile_add = tile_mul_add & 0xFF;
-  repack_sf_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(linear, rows, cols16, swz,
-                                                                    n_col_tiles, tile_mul, tile_add);
+  repack_sf_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(linear, rows, cols16, swz, n_col_tiles,
+                                                                    group, mul, add);
+  return cudaGetLastError();
+}
+
+// One thread per 16-byte chunk of a weight row.
+__global__ void __launch_bounds__(256) tile_weights_kernel(const uint8_t* src, int rows, int row_bytes,
+                                                           uint8_t* dst, int group, int mul, int add) {
+  const int chunks = row_bytes / 16;
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= (int64_t)rows * chunks) return;
+  const int r = (int)(i / chunks);
+  const int j = (int)(i - (int64_t)r * chunks);
+  const int64_t pr = (int64_t)(r / group) * group * mul + (int64_t)add * group + r % group;
+  const int64_t tile = pr >> 7;
+  const int rr = (int)(pr & 127);
+  const int kb_count = (row_bytes + 127) / 128;
+  const int kb = j >> 3, c = j & 7;
+  const int64_t off = ((tile * kb_count + kb) * 128 + rr) * 128 + ((c ^ (rr & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + (int64_t)r * row_bytes + j * 16);
+}
+
+cudaError_t launch_tile_weights(const uint8_t* src, int rows, int row_bytes, uint8_t* dst, int group, int mul,
+                                int add, cudaStream_t stream) {
+  const int64_t n = (int64_t)rows * (row_bytes / 16);
+  tile_weights_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(src, rows, row_bytes, dst, group, mul, add);
   return cudaGetLastError();
 }
 

@@ -109,10 +109,24 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantizeArgs a) {
       out[2 * b] = cvt_e2m1x8(f);
       out[2 * b + 1] = cvt_e2m1x8(f + 8);
     }
-    uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + q * 32);
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    if (a.codes != nullptr) {
+      uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + q * 32);
+      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    if (a.seg_codes != nullptr) {
+      for (int j = 0; j < a.topk; ++j) {
+        const int64_t p = r * a.topk + j;
+        const int e = a.idx[p];
+        const int64_t row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
+        uint4* dst = reinterpret_cast<uint4*>(a.seg_codes + row * (a.cols >> 1) + q * 32);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, q * 4, a.n_col_tiles)) = sc;
+      }
+    }
   }
+  if (a.scales == nullptr) return;
   uint32_t* sdst;
   if (a.swizzled) {
     sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, q * 4, a.n_col_tiles));

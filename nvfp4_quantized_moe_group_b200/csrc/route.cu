@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
   // W tile 64 rows x 32 fp32 (4 threads per row, 8 floats each).
   const int lr = tid >> 2;
   const int lc = (tid & 3) * 8;
+  uint32_t mag = 0;  // max BF16 magnitude bits of the x elements this thread loads
   for (int64_t k0 = k_begin; k0 < k_end; k0 += kTK) {
     {
       const int64_t t = t0 + lr;
@@ -50,6 +51,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
       for (int j = 0; j < 4; ++j) {
         xs[lc + 2 * j][lr] = __uint_as_float(w[j] << 16);
         xs[lc + 2 * j + 1][lr] = __uint_as_float(w[j] & 0xFFFF0000u);
+        mag = max(mag, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
       }
       const int e = e0 + lr;
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f), q = p;
@@ -84,6 +86,21 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
       for (int j = 0; j < 4; ++j) acc[i][j] = __dadd_rn(acc[i][j], (double)part[i][j]);
     __syncthreads();
   }
+  // the CTAs of the first expert tile together load every x element exactly once: they
+  // also produce the per-block maxima of |x| for the global activation scale
+  if (a.amax_partials != nullptr && blockIdx.y == 0) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+    __shared__ uint32_t red[8];
+    if ((tid & 31) == 0) red[tid >> 5] = mag;
+    __syncthreads();
+    if (tid < 32) {
+      mag = tid < 8 ? red[tid] : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+      if (tid == 0) a.amax_partials[blockIdx.z * gridDim.x + blockIdx.x] = mag;
+    }
+  }
   double* out = a.parts + (int64_t)blockIdx.z * a.T * a.E;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -97,27 +114,37 @@ __global__ void __launch_bounds__(256) router_logits_kernel(RouterArgs a) {
   }
 }
 
-// One warp per token: sum the split-K parts in order, add the bias, sigmoid, group-limited
-// top-k, weights.  Equal scores go to the lower index (groups and experts).
+// One token per block.  Phase 1: thread e sums expert e's split-K parts in FP64 (the
+// loads of consecutive experts are coalesced and independent across parts), adds the bias,
+// rounds the logit to FP32 once and takes the sigmoid.  Phase 2: warp 0 does the
+// group-limited top-k.  Equal scores go to the lower index (groups and experts).
 __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
-  __shared__ float s_sc[8][256];
-  __shared__ float s_gsc[8][32];
-  __shared__ int s_keep[8][32];
-  const int warp = threadIdx.x >> 5;
+  __shared__ float s_sc[256];
+  __shared__ float s_gsc[32];
+  __shared__ int s_keep[32];
   const int lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
-  float* sc = s_sc[warp];
   const int E = a.E, G = a.n_groups, gs = a.E / a.n_groups;
-
-  // scores; lane holds experts lane, lane+32, ...
-  for (int e = lane; e < E; e += 32) {
-    double ld = a.parts[t * E + e];
-    for (int ks = 1; ks < a.ksplit; ++ks) ld = __dadd_rn(ld, a.parts[((int64_t)ks * a.T + t) * E + e]);
-    if (a.bias != nullptr) ld = __dadd_rn(ld, (double)a.bias[e]);
-    const float l = __double2float_rn(ld);
-    sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
+  const int64_t t = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const double* src = a.parts + t * E + e;
+    const int64_t step = a.T * E;
+    double acc = 0.0;
+    int ks = 0;
+    for (; ks + 8 <= a.ksplit; ks += 8) {
+      double v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = src[(int64_t)(ks + j) * step];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = __dadd_rn(acc, v[j]);
+    }
+    for (; ks < a.ksplit; ++ks) acc = __dadd_rn(acc, src[(int64_t)ks * step]);
+    if (a.bias != nullptr) acc = __dadd_rn(acc, (double)a.bias[e]);
+    const float l = __double2float_rn(acc);
+    s_sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
   }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  float* sc = s_sc;
   __syncwarp();
   // group scores: sum of the two best scores of each group
   if (lane < G) {
@@ -126,33 +153,32 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
       const float v = sc[lane * gs + j];
       if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
     }
-    s_gsc[warp][lane] = gs >= 2 ? __fadd_rn(b1, b2) : b1;
+    s_gsc[lane] = gs >= 2 ? __fadd_rn(b1, b2) : b1;
   }
   __syncwarp();
   if (lane < G) {
-    const float mine = s_gsc[warp][lane];
+    const float mine = s_gsc[lane];
     int rank = 0;
     for (int g = 0; g < G; ++g) {
-      const float o = s_gsc[warp][g];
+      const float o = s_gsc[g];
       rank += (o > mine) || (o == mine && g < lane);
     }
-    s_keep[warp][lane] = rank < a.topk_groups;
+    s_keep[lane] = rank < a.topk_groups;
   }
   __syncwarp();
   // candidates: this lane's experts in kept groups; k rounds of warp argmax
   float cand[8];
-  int n_mine = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
-    cand[i] = (e < E && s_keep[warp][e / gs]) ? sc[e] : -1.0f;
-    n_mine += e < E;
+    cand[i] = (e < E && s_keep[e / gs]) ? sc[e] : -1.0f;
   }
-  (void)n_mine;
-  float sel_s[8];
-  int sel_e[8];
+  float my_s = 0.0f;   // lane j keeps selection j
+  int my_e = 0;
   float sum = 0.f;
-  for (int j = 0; j < a.topk; ++j) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= a.topk) break;
     float best = -1.0f;
     int be = 0x7FFFFFFF;
 #pragma unroll
@@ -166,19 +192,15 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ob > best || (ob == best && oe < be)) { best = ob; be = oe; }
     }
-    sel_s[j] = best;
-    sel_e[j] = be;
+    if (lane == j) { my_s = best; my_e = be; }
     sum = __fadd_rn(sum, best);
-    if ((be & 31) == lane) cand[be >> 5] = -1.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (be == lane + 32 * i) cand[i] = -1.0f;
   }
   if (lane < a.topk) {
-    float s = 0.f;
-    int e = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j == lane) { s = sel_s[j]; e = sel_e[j]; }
-    a.idx[t * a.topk + lane] = e;
-    a.wts[t * a.topk + lane] = __fdiv_rn(__fmul_rn(a.routed_scale, s), sum);
+    a.idx[t * a.topk + lane] = my_e;
+    a.wts[t * a.topk + lane] = __fdiv_rn(__fmul_rn(a.routed_scale, my_s), sum);
   }
 }
 
@@ -200,6 +222,10 @@ size_t router_parts_elems(int64_t T_max, int E, int H) {
   return best;
 }
 
+int router_amax_partials(int64_t T, int E, int H) {
+  return (int)((T + kTM - 1) / kTM) * router_ksplit(T, E, H);
+}
+
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
   a.ksplit = router_ksplit(a.T, a.E, a.H);
   a.k_slice = a.H / a.ksplit;
@@ -207,7 +233,7 @@ cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
   router_logits_kernel<<<grid, 256, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  router_topk_kernel<<<(unsigned)((a.T + 7) / 8), 256, 0, stream>>>(a);
+  router_topk_kernel<<<(unsigned)a.T, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
