@@ -39,6 +39,35 @@ E2M1_BYTES = 0.5                    # per value
 E4M3_PER16 = 1.0 / 16.0             # block-scale bytes per value
 
 
+def kernel_source_hash() -> str:
+    """SHA-256 over the sources of the grouped GEMM kernels (ties a stored ncu traffic figure
+    to the kernel version it was measured on)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "nvfp4_quantized_moe_group_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload: str, experts_hit: int):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary, scaled to
+    this run's experts hit (traffic is proportional to the weight tiles streamed); None when
+    the summary was taken on other kernel sources or another workload."""
+    path = os.path.join(ROOT, "profiles", "gemm_gateup_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if len(line) >= 2:
+                vals[line[0]] = line[1]
+    if vals.get("source_sha256") != kernel_source_hash() or vals.get("workload") != workload:
+        return None
+    return float(vals["dram_bytes_per_launch"]) / float(vals["experts_hit"]) * experts_hit
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -49,9 +78,13 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def intermediate_scales(E: int) -> np.ndarray:
-    """Static SwiGLU-intermediate global scales written by the oracle calibration script."""
-    path = os.path.join(ROOT, "tests", "golden", "intermediate_scales_beam.txt")
+def intermediate_scales(shape: LayerShape) -> np.ndarray:
+    """Static SwiGLU-intermediate global scales written by the oracle calibration script
+    (the tiny layer's own file; Beam-shape layers use the Beam file's first E entries)."""
+    from workloads import TINY
+    name = "tiny" if shape == TINY else "beam"
+    E = shape.E
+    path = os.path.join(ROOT, "tests", "golden", f"intermediate_scales_{name}.txt")
     vals = []
     with open(path) as f:
         for line in f:
@@ -130,7 +163,7 @@ def build_layer(moe, shape: LayerShape):
     cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
                        shape.routed_scale)
     ex = moe.Experts(cfg)
-    g_h = intermediate_scales(shape.E)
+    g_h = intermediate_scales(shape)
     for e in range(shape.E):
         ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")),
                          float(g_h[e]))
@@ -179,7 +212,7 @@ def cpu_baseline_oracle(shape: LayerShape, wl, x_cpu, wr_cpu, bias_cpu, n_tokens
     dequantised weights).  Expert weights are quantised beforehand, untimed, as the library's
     experts are."""
     import oracle
-    g_h = intermediate_scales(shape.E)
+    g_h = intermediate_scales(shape)
     cfg = _oracle_cfg(shape)
     x = x_cpu.float().numpy()
     t0 = time.perf_counter()
@@ -217,6 +250,11 @@ def init_dist():
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
+
+
+def tokens_per_second(world: int, tokens_per_rank: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: tokens of every rank over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (elapsed_ms / 1e3)
 
 
 def max_over_ranks(v: float, world: int) -> float:
@@ -314,7 +352,7 @@ def run_ours(args, world, rank, local):
 
     p = peaks()
     ms_step = elapsed_ms / args.steps
-    tokens_per_s = world * T * args.steps / (elapsed_ms / 1e3)
+    tokens_per_s = tokens_per_second(world, T, args.steps, elapsed_ms)
     # dominant kernel: the gate/up grouped GEMM (2/3 of the weight bytes and FLOPs)
     gu_s = gateup_ms / 1e3
     t_bytes = alg["gateup_bytes"] / (p["hbm_gbs"] * 1e9)
@@ -326,7 +364,8 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "tensor", "achieved": alg["gateup_flops"] / gu_s / 1e12, "peak": fp4_peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = stored_traffic(args.workload if not args.experts else f"{args.workload}-e{shape.E}",
+                                     alg["experts_hit"])
     roof["kernel"] = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
     roof["peak_source"] = (f"{p['source']} hbm_gbs" if roof["bound"] == "hbm"
                            else f"{p['source']} bf16_tflops_sustained x {FP4_OVER_BF16:g} (nominal FP4:BF16)")
@@ -345,7 +384,7 @@ def run_ours(args, world, rank, local):
                          f"({alg['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"},
         "roofline": roof, "layer_roofline": layer_roof,
         "stage_ms": stage,
-        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": tokens_per_second(world, T, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
@@ -365,7 +404,7 @@ def run_reference(args, world, rank):
     wl = WORKLOADS[args.workload]
     shape = layer_shape(args.experts) if args.experts else wl.shape
     T = wl.T
-    g_h = intermediate_scales(shape.E)
+    g_h = intermediate_scales(shape)
     x = activations(T, shape, seed=wl.seed, rms_rows=wl.rms_rows).float().numpy()
     wr = router_weight(shape).numpy()
     bias = zipf_bias(shape.E).numpy() if wl.zipf else None

@@ -57,6 +57,7 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort_flag;
   int prefix[257];
+  int counts[256];
 };
 
 struct Work {
@@ -67,8 +68,7 @@ struct Work {
   int rows_valid; // rows of this tile that hold a pair
 };
 
-__device__ __forceinline__ Work decode_work(const int* prefix, int w, int E, int ntn,
-                                            const int32_t* __restrict__ counts) {
+__device__ __forceinline__ Work decode_work(const int* prefix, int w, int E, int ntn, const int* counts) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -113,7 +113,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i <= p.E; i += kThreads) s.prefix[i] = p.mtile_prefix[i];
+  for (int i = threadIdx.x; i <= p.E; i += kThreads) {
+    s.prefix[i] = p.mtile_prefix[i];
+    if (i < p.E) s.counts[i] = p.counts[i];
+  }
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&s.full[st], 1);
@@ -154,7 +157,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       const uint64_t pol_a = policy_evict_last();
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Work wk = decode_work(s.prefix, w, p.E, ntn, p.counts);
+        const Work wk = decode_work(s.prefix, w, p.E, ntn, s.counts);
         const int arow = wk.mtile * kBlockM;
         const bool a_small = wk.rows_valid <= 32;
         const uint32_t a_bytes = a_small ? 32u * 128u : (uint32_t)kABytes;
@@ -242,7 +245,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     const int row_l = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      const Work wk = decode_work(s.prefix, w, p.E, ntn, p.counts);
+      const Work wk = decode_work(s.prefix, w, p.E, ntn, s.counts);
       const int buf = it & 1;
       const uint32_t acc_par = ((uint32_t)it >> 1) & 1u;
       const int64_t row = (int64_t)wk.mtile * kBlockM + row_l;
