@@ -395,6 +395,45 @@ def run_ours(args, world, rank, local):
     return res
 
 
+def run_quantize(args, world, rank, local):
+    """Standalone quantize_nvfp4 on 32768 x 5120 BF16 activations with a dynamic global scale
+    and swizzled scales: the amax pass reads x once, the quantise pass reads it again and
+    writes codes + scales, so the algorithmic bytes are 2 * 2 * rows * cols + rows * cols * 9/16."""
+    import nvfp4_quantized_moe_group_b200 as moe
+    rows, cols = 32768, BEAM.H
+    x = activations(rows, BEAM, seed=rank, device="cuda")
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(moe.swizzled_scale_bytes(rows, cols // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(moe.quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g))
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        start.record()
+        for _ in range(args.steps):
+            moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g))
+        stop.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    launches = moe.last_launch_count()
+    if moe.status_read(ws) != moe.OK:
+        raise RuntimeError("quantize status")
+    nbytes = 2 * rows * cols * 2 + rows * cols // 2 + rows * cols // 16
+    p = peaks()
+    gbs = world * nbytes / (ms / 1e3) / 1e9
+    return {"metric": "quantize_nvfp4 HBM GB/s (32768x5120 BF16, dynamic global scale, swizzled scales)",
+            "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e2m1",
+            "data": "synthetic", "config": {"workload": "quantize 32768x5120", "bytes_per_step": nbytes,
+                                            "l2": "input 335 MB > 126 MB L2 (no flush)"},
+            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": p["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / world / p["hbm_gbs"], "traffic": None},
+            "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm.  Each step is a bounded sample of the workload's step:
     routing and input quantisation of all its tokens plus one (token, slot) pair's expert
@@ -442,7 +481,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize"])
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -459,7 +498,8 @@ def main():
 
     world, rank, local = init_dist()
     try:
-        res = run_ours(args, world, rank, local)
+        res = run_quantize(args, world, rank, local) if args.workload == "quantize" else \
+            run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
