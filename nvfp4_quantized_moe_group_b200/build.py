@@ -58,6 +58,8 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
         return LIB
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
+    if os.path.exists(LIB):
+        os.remove(LIB)  # a failed build must not leave an out-of-date library behind
     objs = []
     extra = ["-Xptxas", "-v"] if ptxas_info else []
     procs = []

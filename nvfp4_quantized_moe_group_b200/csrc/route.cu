@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(256) router_logits_big_kernel(RouterArgs a) {
   if (a.amax_partials != nullptr && blockIdx.y == 0) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
-    __shared__ uint32_t red[8];
+    uint32_t* red = reinterpret_cast<uint32_t*>(&xs[0][0][0]);  // tiles are no longer read
     if ((tid & 31) == 0) red[tid >> 5] = mag;
     __syncthreads();
     if (tid < 32) {
