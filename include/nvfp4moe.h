@@ -131,7 +131,7 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
  * Logits: FP32 products accumulated in FP32 runs of at most 32 products; the runs, the
  * split-K parts and the bias are added in FP64 and the logit is rounded to FP32 once, so
  * |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
- * Scores are 1 / (1 + expf(-logit)) in FP32. */
+ * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same kernels. */
 NVFP4MOE_API size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
 NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
                    const float* w_router, const float* logit_bias, int32_t* idx, float* w,
@@ -234,6 +234,7 @@ typedef struct {
                           events[2s] / events[2s+1] are recorded on the stream right before /
                           after stage s (timing of the stages inside a forward); NULL entries
                           are skipped */
+  float* logits;       /* [T][E] FP32 router logits (bias included) the selection used */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);

@@ -51,7 +51,8 @@ STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "f
 
 
 class Debug(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
+    _fields_ = ([(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
+                + [("logits", ctypes.c_void_p)])
 
 
 class StageTimer:
@@ -300,6 +301,7 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
             "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
             "hq_codes": torch.empty((T * k, I // 2), dtype=torch.uint8, device=dev),
             "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
+            "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
         }
         dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
     if timer is not None:

@@ -425,7 +425,9 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   r.topk_groups = c.topk_groups;
   r.topk = c.topk;
   r.routed_scale = c.routed_scale;
+  r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
   r.amax_partials = f.partials;
+  const int n_partials = router_amax_partials(T, c.E, c.H);
   ev.mark(NVFP4MOE_STAGE_AMAX, 0);
   ev.mark(NVFP4MOE_STAGE_AMAX, 1);
   ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
@@ -462,7 +464,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   q.cols = c.H;
   q.g_in = nullptr;
   q.partials = f.partials;
-  q.n_partials = router_amax_partials(T, c.E, c.H);
+  q.n_partials = n_partials;
   q.codes = keep_xq ? f.xq_codes : nullptr;
   q.scales = keep_xq ? f.xq_sf : nullptr;
   q.swizzled = 1;

@@ -52,6 +52,7 @@ struct RouterArgs {
   float routed_scale;
   int ksplit, k_slice;
   uint32_t* amax_partials;  // optional: per-CTA max |x| (BF16 magnitude bits) for the global scale
+  float* logits_out;        // optional [T][E]: the FP32 logits (bias included) the top-k used
 };
 
 struct PermArgs {
@@ -114,6 +115,10 @@ size_t router_parts_elems(int64_t T_max, int E, int H);
 // Number of amax partials the logits kernel writes for T tokens (grid x * split-K).
 int router_amax_partials(int64_t T, int E, int H);
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream);
+// The top-k stage alone (sums a.ksplit split-K parts of a.parts).
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);
+
+
 
 // permute.cu
 // Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.

@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
     for (; ks < a.ksplit; ++ks) acc = __dadd_rn(acc, src[(int64_t)ks * step]);
     if (a.bias != nullptr) acc = __dadd_rn(acc, (double)a.bias[e]);
     const float l = __double2float_rn(acc);
+    if (a.logits_out != nullptr) a.logits_out[t * E + e] = l;
     s_sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
   }
   __syncthreads();
@@ -362,6 +363,10 @@ cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
     router_logits_kernel<<<grid, 256, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  return launch_router_topk(a, stream);
+}
+
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
   router_topk_kernel<<<(unsigned)a.T, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -129,3 +129,24 @@ def test_beam_prefill_layer_sampled():
 
 def test_beam_skewed_layer_sampled():
     run_layer(BEAM, 16384, tokens=[3, 16383], bias=zipf_bias(256))
+
+
+@pytest.mark.parametrize("T", [200, 600, 4096])
+def test_router_logits_within_documented_bound(T):
+    """Every FP32 logit the selection used (small-T and large-T logits kernels) lies within
+    the documented 32 * 2^-24 * sum|x W| + 2^-24 |logit| of the exact value."""
+    from tests.helpers import router_logit_bound
+    ex = gpu_experts(BEAM)
+    x = activations(T, BEAM, seed=3)
+    wr = router_weight(BEAM)
+    _, dbg = moe.forward(ex, x.cuda(), wr.cuda(), debug=True)
+    torch.cuda.synchronize()
+    xn = x.float().numpy().astype(np.float64)
+    wn = wr.numpy().astype(np.float64)
+    exact = xn @ wn.T
+    got = dbg["logits"].cpu().numpy().astype(np.float64)
+    bound = router_logit_bound(xn, wn, None, BEAM.H)
+    err = np.abs(got - exact)
+    assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
+    # the bound is not vacuous: errors are a small fraction of it
+    assert np.max(err / bound) < 0.5
