@@ -131,7 +131,9 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
  * Logits: FP32 products accumulated in FP32 runs of at most 32 products; the runs, the
  * split-K parts and the bias are added in FP64 and the logit is rounded to FP32 once, so
  * |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
- * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same kernels. */
+ * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same arithmetic
+ * and bound (for T <= 64 in its fused front-end kernel).  A NaN logit raises
+ * NVFP4MOE_ERR_NONFINITE in the status word and ranks below every finite score. */
 NVFP4MOE_API size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
 NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
                    const float* w_router, const float* logit_bias, int32_t* idx, float* w,
@@ -205,7 +207,9 @@ NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_
 /* Stages of nvfp4moe_forward (for nvfp4moe_debug.events).  Launch order: ROUTE, PERMUTE,
  * QUANTIZE, GATEUP, DOWN, FINALIZE.  The input's global amax is computed inside ROUTE and
  * the rows are written into the expert segments inside QUANTIZE, so the AMAX and GATHER
- * events are recorded back to back (zero time). */
+ * events are recorded back to back (zero time).  For T <= 64 (when the device can hold the
+ * cooperative grid) ROUTE is one fused launch that also groups the pairs and quantises x,
+ * and the PERMUTE and QUANTIZE events are recorded back to back after it. */
 enum {
   NVFP4MOE_STAGE_AMAX = 0,      /* global amax of the input (inside ROUTE) */
   NVFP4MOE_STAGE_ROUTE = 1,     /* router logits (+ amax partials) + group-limited top-k */

@@ -129,7 +129,12 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   const int n_part = router_amax_partials(T, cfg.E, cfg.H);
   f.partials = c.take<uint32_t>(n_part > kMaxAmaxPartials ? n_part : kMaxAmaxPartials);
   f.g_x = c.take<float>(1);
-  f.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
+  size_t n_parts = router_parts_elems(T, cfg.E, cfg.H);
+  if (T <= kFrontMaxT) {
+    const size_t nf = (size_t)front_ksplit(cfg.E, cfg.H) * (size_t)T * (size_t)cfg.E;
+    if (nf > n_parts) n_parts = nf;
+  }
+  f.parts = c.take<double>(n_parts);
   f.idx = c.take<int32_t>(pairs);
   f.wts = c.take<float>(pairs);
   f.xq_codes = c.take<uint8_t>(T * cfg.H / 2);
@@ -290,6 +295,7 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   a.topk_groups = cfg->topk_groups;
   a.topk = cfg->topk;
   a.routed_scale = cfg->routed_scale;
+  a.status = &r.hdr->status;
   if (launch_router(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   g_launches += 2;
   return NVFP4MOE_OK;
@@ -408,83 +414,131 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
     return NVFP4MOE_ERR_CUDA;
 
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
-  if (cudaMemsetAsync(&f.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-
-  // route: logits (with the per-block maxima of |x| for the global scale) + top-k
-  RouterArgs r{};
-  r.x = static_cast<const uint16_t*>(hidden_bf16);
-  r.w = w_router;
-  r.bias = logit_bias;
-  r.parts = f.parts;
-  r.idx = f.idx;
-  r.wts = f.wts;
-  r.T = T;
-  r.H = c.H;
-  r.E = c.E;
-  r.n_groups = c.n_groups;
-  r.topk_groups = c.topk_groups;
-  r.topk = c.topk;
-  r.routed_scale = c.routed_scale;
-  r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
-  r.amax_partials = f.partials;
-  const int n_partials = router_amax_partials(T, c.E, c.H);
-  ev.mark(NVFP4MOE_STAGE_AMAX, 0);
-  ev.mark(NVFP4MOE_STAGE_AMAX, 1);
-  ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
-  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
-  g_launches += 2;
-
-  // group the (token, slot) pairs by expert
-  PermArgs pa{};
-  pa.idx = f.idx;
-  pa.T = T;
-  pa.topk = c.topk;
-  pa.E = c.E;
-  pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
-  pa.chunk_counts = f.chunk_counts;
-  pa.chunk_base = f.chunk_base;
-  pa.counts = f.counts;
-  pa.offsets = f.offsets;
-  pa.mtile_prefix = f.mtile_prefix;
-  pa.perm = f.perm;
-  pa.inv = f.inv;
-  pa.row_pair = f.row_pair;
-  ev.mark(NVFP4MOE_STAGE_PERMUTE, 0);
-  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
-
-  // quantise x and write each token's row into its expert-segment rows (zeroes the
-  // accumulator alongside); the token-major copy is only kept for the debug export
+  // status word and grid-barrier counter
+  if (cudaMemsetAsync(&f.hdr->status, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
-  QuantizeArgs q{};
-  q.x = static_cast<const uint16_t*>(hidden_bf16);
-  q.rows = T;
-  q.rows_padded = keep_xq ? round128(T) : T;
-  q.cols = c.H;
-  q.g_in = nullptr;
-  q.partials = f.partials;
-  q.n_partials = n_partials;
-  q.codes = keep_xq ? f.xq_codes : nullptr;
-  q.scales = keep_xq ? f.xq_sf : nullptr;
-  q.swizzled = 1;
-  q.n_col_tiles = c.H / 64;
-  q.g_out = f.g_x;
-  q.zero_out = f.acc;
-  q.status = &f.hdr->status;
-  q.idx = f.idx;
-  q.inv = f.inv;
-  q.offsets = f.offsets;
-  q.mtile_prefix = f.mtile_prefix;
-  q.topk = c.topk;
-  q.seg_codes = f.a_codes;
-  q.seg_sf = f.a_sf;
-  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
-  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
-  ev.mark(NVFP4MOE_STAGE_GATHER, 0);
-  ev.mark(NVFP4MOE_STAGE_GATHER, 1);
-  ++g_launches;
+
+  if (front_supported(T, c.E, c.H)) {
+    // small T: route, amax, grouping and quantise-scatter in one cooperative launch
+    FrontArgs fa{};
+    fa.x = static_cast<const uint16_t*>(hidden_bf16);
+    fa.w = w_router;
+    fa.bias = logit_bias;
+    fa.T = T;
+    fa.H = c.H;
+    fa.E = c.E;
+    fa.n_groups = c.n_groups;
+    fa.topk_groups = c.topk_groups;
+    fa.topk = c.topk;
+    fa.routed_scale = c.routed_scale;
+    fa.parts = f.parts;
+    fa.amax_partials = f.partials;
+    fa.idx = f.idx;
+    fa.wts = f.wts;
+    fa.logits_out = dbg != nullptr ? dbg->logits : nullptr;
+    fa.counts = f.counts;
+    fa.offsets = f.offsets;
+    fa.mtile_prefix = f.mtile_prefix;
+    fa.perm = f.perm;
+    fa.inv = f.inv;
+    fa.row_pair = f.row_pair;
+    fa.seg_codes = f.a_codes;
+    fa.seg_sf = f.a_sf;
+    fa.n_col_tiles = c.H / 64;
+    fa.xq_codes = keep_xq ? f.xq_codes : nullptr;
+    fa.xq_sf = keep_xq ? f.xq_sf : nullptr;
+    fa.g_out = f.g_x;
+    fa.acc = f.acc;
+    fa.status = &f.hdr->status;
+    fa.barrier = &f.hdr->barrier;
+    ev.mark(NVFP4MOE_STAGE_AMAX, 0);
+    ev.mark(NVFP4MOE_STAGE_AMAX, 1);
+    ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
+    if (launch_front(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
+    for (int stage : {NVFP4MOE_STAGE_PERMUTE, NVFP4MOE_STAGE_QUANTIZE, NVFP4MOE_STAGE_GATHER}) {
+      ev.mark(stage, 0);
+      ev.mark(stage, 1);
+    }
+    ++g_launches;
+  } else {
+
+    // route: logits (with the per-block maxima of |x| for the global scale) + top-k
+    RouterArgs r{};
+    r.x = static_cast<const uint16_t*>(hidden_bf16);
+    r.w = w_router;
+    r.bias = logit_bias;
+    r.parts = f.parts;
+    r.idx = f.idx;
+    r.wts = f.wts;
+    r.T = T;
+    r.H = c.H;
+    r.E = c.E;
+    r.n_groups = c.n_groups;
+    r.topk_groups = c.topk_groups;
+    r.topk = c.topk;
+    r.routed_scale = c.routed_scale;
+    r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
+    r.amax_partials = f.partials;
+    r.status = &f.hdr->status;
+    const int n_partials = router_amax_partials(T, c.E, c.H);
+    ev.mark(NVFP4MOE_STAGE_AMAX, 0);
+    ev.mark(NVFP4MOE_STAGE_AMAX, 1);
+    ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
+    if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
+    g_launches += 2;
+
+    // group the (token, slot) pairs by expert
+    PermArgs pa{};
+    pa.idx = f.idx;
+    pa.T = T;
+    pa.topk = c.topk;
+    pa.E = c.E;
+    pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
+    pa.chunk_counts = f.chunk_counts;
+    pa.chunk_base = f.chunk_base;
+    pa.counts = f.counts;
+    pa.offsets = f.offsets;
+    pa.mtile_prefix = f.mtile_prefix;
+    pa.perm = f.perm;
+    pa.inv = f.inv;
+    pa.row_pair = f.row_pair;
+    ev.mark(NVFP4MOE_STAGE_PERMUTE, 0);
+    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
+
+    // quantise x and write each token's row into its expert-segment rows (zeroes the
+    // accumulator alongside); the token-major copy is only kept for the debug export
+    QuantizeArgs q{};
+    q.x = static_cast<const uint16_t*>(hidden_bf16);
+    q.rows = T;
+    q.rows_padded = keep_xq ? round128(T) : T;
+    q.cols = c.H;
+    q.g_in = nullptr;
+    q.partials = f.partials;
+    q.n_partials = n_partials;
+    q.codes = keep_xq ? f.xq_codes : nullptr;
+    q.scales = keep_xq ? f.xq_sf : nullptr;
+    q.swizzled = 1;
+    q.n_col_tiles = c.H / 64;
+    q.g_out = f.g_x;
+    q.zero_out = f.acc;
+    q.status = &f.hdr->status;
+    q.idx = f.idx;
+    q.inv = f.inv;
+    q.offsets = f.offsets;
+    q.mtile_prefix = f.mtile_prefix;
+    q.topk = c.topk;
+    q.seg_codes = f.a_codes;
+    q.seg_sf = f.a_sf;
+    ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
+    if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
+    ev.mark(NVFP4MOE_STAGE_GATHER, 0);
+    ev.mark(NVFP4MOE_STAGE_GATHER, 1);
+    ++g_launches;
+  }
 
   const int grid = num_sms();
   GemmArgs g{};

@@ -21,7 +21,8 @@ enum : uint32_t {
 // Every workspace starts with this header.
 struct WsHeader {
   uint32_t status;
-  uint32_t pad[63];
+  uint32_t barrier;   // grid-barrier counter of the fused front kernel
+  uint32_t pad[62];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

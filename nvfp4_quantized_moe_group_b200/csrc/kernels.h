@@ -53,6 +53,7 @@ struct RouterArgs {
   int ksplit, k_slice;
   uint32_t* amax_partials;  // optional: per-CTA max |x| (BF16 magnitude bits) for the global scale
   float* logits_out;        // optional [T][E]: the FP32 logits (bias included) the top-k used
+  uint32_t* status;         // kStatusNonFinite is raised here for a NaN logit (may be nullptr)
 };
 
 struct PermArgs {
@@ -97,6 +98,38 @@ struct GemmArgs {
   int H;
 };
 
+// Fused front end for T <= kFrontMaxT (front.cu).
+constexpr int kFrontMaxT = 64;
+struct FrontArgs {
+  const uint16_t* x;        // [T][H] bf16
+  const float* w;           // router weight [E][H]
+  const float* bias;        // [E] or nullptr
+  int64_t T;
+  int H, E, n_groups, topk_groups, topk;
+  float routed_scale;
+  int ksplit, k_slice;      // set by launch_front
+  double* parts;            // [ksplit][T][E]
+  uint32_t* amax_partials;  // [ksplit]
+  int32_t* idx;             // [T][topk]
+  float* wts;               // [T][topk]
+  float* logits_out;        // optional [T][E]
+  int32_t* counts;          // [E]
+  int32_t* offsets;         // [E+1]
+  int32_t* mtile_prefix;    // [E+1]
+  int32_t* perm;            // [T*topk]
+  int32_t* inv;             // [T*topk]
+  int32_t* row_pair;        // [rows_cap]
+  uint8_t* seg_codes;       // [rows_cap][H/2]
+  uint8_t* seg_sf;          // swizzled [rows_cap][H/16]
+  int64_t n_col_tiles;      // H / 64
+  uint8_t* xq_codes;        // optional token-major copy [T][H/2]
+  uint8_t* xq_sf;           // swizzled, with xq_codes
+  float* g_out;             // global scale of x
+  float* acc;               // [T][H] FP32, zeroed
+  uint32_t* status;
+  uint32_t* barrier;        // zero at launch
+};
+
 struct FinalizeArgs {
   const float* acc;
   uint16_t* out;
@@ -119,6 +152,14 @@ cudaError_t launch_router(RouterArgs a, cudaStream_t stream);
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);
 
 
+
+// front.cu
+// True when the fused front end runs for T tokens on the current device (T <= kFrontMaxT and
+// its cooperative grid fits).
+bool front_supported(int64_t T, int E, int H);
+// Split-K partials the front kernel writes: ksplit * T * E doubles.
+int front_ksplit(int E, int H);
+cudaError_t launch_front(FrontArgs a, cudaStream_t stream);
 
 // permute.cu
 // Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.

@@ -5,6 +5,7 @@
 // numerical decisions").
 #include "common.cuh"
 #include "kernels.h"
+#include "route_topk.cuh"
 
 namespace nvfp4moe {
 
@@ -233,14 +234,11 @@ __global__ void __launch_bounds__(256) router_logits_big_kernel(RouterArgs a) {
 
 // One token per block.  Phase 1: thread e sums expert e's split-K parts in FP64 (the
 // loads of consecutive experts are coalesced and independent across parts), adds the bias,
-// rounds the logit to FP32 once and takes the sigmoid.  Phase 2: warp 0 does the
+// rounds the logit to FP32 once and takes the sigmoid.  Phase 2: the block does the
 // group-limited top-k.  Equal scores go to the lower index (groups and experts).
-__global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
+__global__ void __launch_bounds__(kTopkThreads) router_topk_kernel(RouterArgs a) {
   __shared__ float s_sc[256];
-  __shared__ float s_gsc[32];
-  __shared__ int s_keep[32];
-  const int lane = threadIdx.x & 31;
-  const int E = a.E, G = a.n_groups, gs = a.E / a.n_groups;
+  const int E = a.E;
   const int64_t t = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const double* src = a.parts + t * E + e;
@@ -258,68 +256,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterArgs a) {
     if (a.bias != nullptr) acc = __dadd_rn(acc, (double)a.bias[e]);
     const float l = __double2float_rn(acc);
     if (a.logits_out != nullptr) a.logits_out[t * E + e] = l;
-    s_sc[e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
+    s_sc[e] = router_sigmoid(l);
   }
   __syncthreads();
-  if (threadIdx.x >= 32) return;
-  float* sc = s_sc;
-  __syncwarp();
-  // group scores: sum of the two best scores of each group
-  if (lane < G) {
-    float b1 = -1.f, b2 = -1.f;
-    for (int j = 0; j < gs; ++j) {
-      const float v = sc[lane * gs + j];
-      if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
-    }
-    s_gsc[lane] = gs >= 2 ? __fadd_rn(b1, b2) : b1;
-  }
-  __syncwarp();
-  if (lane < G) {
-    const float mine = s_gsc[lane];
-    int rank = 0;
-    for (int g = 0; g < G; ++g) {
-      const float o = s_gsc[g];
-      rank += (o > mine) || (o == mine && g < lane);
-    }
-    s_keep[lane] = rank < a.topk_groups;
-  }
-  __syncwarp();
-  // candidates: this lane's experts in kept groups; k rounds of warp argmax
-  float cand[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    cand[i] = (e < E && s_keep[e / gs]) ? sc[e] : -1.0f;
-  }
-  float my_s = 0.0f;   // lane j keeps selection j
-  int my_e = 0;
-  float sum = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j >= a.topk) break;
-    float best = -1.0f;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (cand[i] > best) { best = cand[i]; be = e; }   // e ascends with i: ties keep lower e
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ob > best || (ob == best && oe < be)) { best = ob; be = oe; }
-    }
-    if (lane == j) { my_s = best; my_e = be; }
-    sum = __fadd_rn(sum, best);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (be == lane + 32 * i) cand[i] = -1.0f;
-  }
-  if (lane < a.topk) {
-    a.idx[t * a.topk + lane] = my_e;
-    a.wts[t * a.topk + lane] = __fdiv_rn(__fmul_rn(a.routed_scale, my_s), sum);
-  }
+  route_topk_block(s_sc, E, a.n_groups, a.topk_groups, a.topk, a.routed_scale, a.idx + t * a.topk,
+                   a.wts + t * a.topk, a.status);
 }
 
 static int tile_tokens(int64_t T) { return T >= kBigMinT ? kBigTM : kTM; }
@@ -367,7 +308,7 @@ cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
 }
 
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
-  router_topk_kernel<<<(unsigned)a.T, 256, 0, stream>>>(a);
+  router_topk_kernel<<<(unsigned)a.T, kTopkThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,7 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
   a.topk_groups = cfg->topk_groups;
   a.topk = cfg->topk;
   a.routed_scale = cfg->routed_scale;
+  a.status = &hdr->status;
   return launch_router(a, s) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
 }
 

@@ -131,10 +131,11 @@ def test_beam_skewed_layer_sampled():
     run_layer(BEAM, 16384, tokens=[3, 16383], bias=zipf_bias(256))
 
 
-@pytest.mark.parametrize("T", [200, 600, 4096])
+@pytest.mark.parametrize("T", [16, 64, 200, 600, 4096])
 def test_router_logits_within_documented_bound(T):
-    """Every FP32 logit the selection used (small-T and large-T logits kernels) lies within
-    the documented 32 * 2^-24 * sum|x W| + 2^-24 |logit| of the exact value."""
+    """Every FP32 logit the selection used (fused front-end kernel for T <= 64, large-T logits
+    kernel above) lies within the documented 32 * 2^-24 * sum|x W| + 2^-24 |logit| of the
+    exact value."""
     from tests.helpers import router_logit_bound
     ex = gpu_experts(BEAM)
     x = activations(T, BEAM, seed=3)
@@ -150,3 +151,52 @@ def test_router_logits_within_documented_bound(T):
     assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
     # the bound is not vacuous: errors are a small fraction of it
     assert np.max(err / bound) < 0.5
+
+
+@pytest.mark.parametrize("T", [16, 130])
+def test_nonfinite_router_weight_reported(T):
+    """A NaN in the router weight makes one expert's logits NaN: the forward reports
+    NONFINITE, and the selection still holds topk distinct in-range experts per token (the NaN
+    expert ranks last), so the grouping and the GEMMs stay inside their buffers."""
+    ex = gpu_experts(BEAM)
+    x = activations(T, BEAM, seed=5)
+    wr = router_weight(BEAM).clone()
+    wr[3, 7] = float("nan")
+    ws = torch.empty(moe.forward_workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
+    _, dbg = moe.forward(ex, x.cuda(), wr.cuda(), ws=ws, debug=True)
+    assert moe.status_read(ws) == moe.ERR_NONFINITE
+    idx = dbg["idx"].cpu().numpy()
+    assert ((idx >= 0) & (idx < BEAM.E)).all()
+    assert all(len(set(row.tolist())) == BEAM.topk for row in idx)
+    assert not (idx == 3).any()
+    counts = dbg["counts"].cpu().numpy()
+    assert counts.sum() == T * BEAM.topk
+
+
+def test_front_end_odd_group_layout():
+    """The fused front end (T <= 64) with a partial expert tile (E = 48) and groups of 12:
+    routing under the near-tie protocol, grouping, and the quantised input bit-exact."""
+    from tests.test_gpu_route import ODD_SHAPES
+    shape = ODD_SHAPES["gs12"]
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    ex = moe.Experts(cfg)
+    for e in range(shape.E):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")), 1.0)
+    for T in (20, 64):
+        x = activations(T, shape, seed=11)
+        wr = router_weight(shape)
+        ws = torch.empty(moe.forward_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+        _, dbg = moe.forward(ex, x.cuda(), wr.cuda(), ws=ws, debug=True)
+        assert moe.status_read(ws) == moe.OK
+        xn = x.float().numpy()
+        r = oracle.route(xn.astype(np.float64), wr.numpy(), cfg_ns(shape), None)
+        idx = dbg["idx"].cpu().numpy()
+        check_routing(idx, dbg["w"].cpu().numpy(), r, xn.astype(np.float64), wr.numpy().astype(np.float64),
+                      None, shape)
+        check_grouping(dbg, idx, shape.E)
+        xc, xs, gx = oracle.quantize(xn.astype(np.float32))
+        assert np.float32(dbg["g_x"].item()) == gx
+        np.testing.assert_array_equal(dbg["xq_codes"].cpu().numpy(), xc)
+        np.testing.assert_array_equal(dbg["xq_scales"].cpu().numpy(), xs)
+    ex.close()

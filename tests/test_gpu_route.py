@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import nvfp4_quantized_moe_group_b200 as moe
-from workloads import TINY, BEAM, activations, router_weight, zipf_bias
+from workloads import TINY, BEAM, LayerShape, activations, router_weight, zipf_bias
 from tests.helpers import cfg_ns, check_routing
 
 pytestmark = pytest.mark.gpu
@@ -62,3 +62,24 @@ def test_beam_skewed_zipf_bias():
 def test_ragged_token_counts():
     for T in (3, 65, 130):
         _run(BEAM, T)
+
+
+# Group layouts beyond Beam's: a group size that is not a power of two (the in-group ranks
+# go through shared memory instead of shuffles), one expert per group (the group score is
+# its single score), every group kept, and more than 32 selection candidates.
+ODD_SHAPES = {
+    "gs12": LayerShape(H=256, I=128, E=48, n_groups=4, topk_groups=2, topk=6, routed_scale=2.5,
+                       wr_std=1.0 / 16.0, w_std=0.02),
+    "gs1": LayerShape(H=256, I=128, E=8, n_groups=8, topk_groups=4, topk=3, routed_scale=1.0,
+                      wr_std=1.0 / 16.0, w_std=0.02),
+    "all_groups": LayerShape(H=256, I=128, E=64, n_groups=2, topk_groups=2, topk=8, routed_scale=2.5,
+                             wr_std=1.0 / 16.0, w_std=0.02),
+    "64_candidates": LayerShape(H=512, I=128, E=256, n_groups=8, topk_groups=8, topk=8, routed_scale=2.5,
+                                wr_std=512 ** -0.5, w_std=0.02),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ODD_SHAPES))
+@pytest.mark.parametrize("T", [16, 100])
+def test_group_layouts(name, T):
+    _run(ODD_SHAPES[name], T)
