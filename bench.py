@@ -44,7 +44,7 @@ def kernel_source_hash() -> str:
     to the kernel version it was measured on)."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("gemm.cu", "common.cuh", "kernels.h"):
+    for name in ("gemm.cu", "gemm.h", "common.cuh"):
         with open(os.path.join(ROOT, "nvfp4_quantized_moe_group_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -100,50 +100,76 @@ _REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown"
             0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
 
-class ClockSampler:
-    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+_SAMPLER_CODE = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[1]))
+period = float(sys.argv[2])
+get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    try:
+        print("s", time.monotonic(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get_reasons(h)),
+              flush=True)
+    except Exception:
+        pass
+    time.sleep(period)
+"""
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs, from a
+    child process (a thread here would wait on the interpreter lock while the main thread
+    launches kernels)."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        import subprocess
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
-        self._stop = threading.Event()
+        self._proc = None
+        self._lines = []
         self._thread = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            import pynvml  # noqa: F401  (only to know that the child can use it)
+            self._proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_CODE, str(device_index), str(period_s)],
+                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            first = self._proc.stdout.readline().split()
+            if first and first[0] == "max":
+                self.max_mhz = int(first[1])
+            else:                      # NVML could not start in the child
+                self._proc.wait()
+                self._proc = None
         except Exception:
-            self._nv = None
-        self.period = period_s
+            self._proc = None
 
-    def _run(self):
-        nv = self._nv
-        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(get_reasons(self._h))
-            except Exception:
-                pass
-            time.sleep(self.period)
+    def _reader(self):
+        for line in self._proc.stdout:
+            self._lines.append(line)
 
     def __enter__(self):
-        if self._nv is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
+        self._t0 = time.monotonic()
+        if self._proc is not None:
+            self._lines.clear()
+            self._thread = threading.Thread(target=self._reader, daemon=True)
             self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._thread is not None:
+        t1 = time.monotonic()
+        if self._proc is not None:
+            self._proc.terminate()
+            self._proc.wait()
             self._thread.join()
+            for line in self._lines:   # samples taken inside the region only
+                f = line.split()
+                if len(f) == 4 and f[0] == "s" and self._t0 <= float(f[1]) <= t1:
+                    self.samples.append(int(f[2]))
+                    self.reasons |= int(f[3])
 
     def summary(self):
-        if self._nv is None:
+        if self._proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in _REASONS.items() if self.reasons & b], "samples": len(self.samples)}
@@ -478,7 +504,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize"])

@@ -128,8 +128,10 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
  *   idx  out [T][topk] int32: selected experts by score descending, equal scores by
  *        lower expert index (the same rule picks the groups).
  *   w    out [T][topk] FP32: routed_scale * s / sum(selected s).
- * Logits: FP32 products accumulated in FP32 runs of at most 32 products; the runs, the
- * split-K parts and the bias are added in FP64 and the logit is rounded to FP32 once, so
+ * Logits: FP32 products accumulated in FP32 so that every product passes through at most
+ * 32 FP32 roundings (FMA chains of at most 32 products, or of at most 20 products added by
+ * a 3-level FP32 tree); these partial sums, the split-K parts and the bias are added in
+ * FP64 and the logit is rounded to FP32 once, so
  * |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
  * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same arithmetic
  * and bound (for T <= 64 in its fused front-end kernel).  A NaN logit raises

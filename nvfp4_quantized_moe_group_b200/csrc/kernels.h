@@ -6,12 +6,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "gemm.h"
+
 namespace nvfp4moe {
 
 constexpr int kMaxAmaxPartials = 1024;   // blocks of the amax pass
-constexpr int kBlockM = 128;             // token rows per GEMM tile / expert segment padding
-constexpr int kBlockN = 128;             // output columns per GEMM tile
-constexpr int kBlockK = 256;             // K values per pipeline stage (128 bytes of E2M1)
 constexpr int kPermChunkTokens = 128;    // tokens per chunk of the grouping kernels
 
 struct QuantizeArgs {
@@ -71,32 +70,6 @@ struct PermArgs {
   int32_t* row_pair;       // [rows_cap] pair id of each padded row, -1 for padding
 };
 
-struct GemmArgs {
-  const uint8_t* b_tiles;      // weights, tiled: [E][n_total/128][ceil(K/256)][128 rows][128 B], swizzled
-  const uint8_t* sfa;          // swizzled scales of A (padded rows)
-  const uint8_t* sfb;          // swizzled scales of B, experts back to back
-  const int32_t* mtile_prefix; // [E+1]
-  const int32_t* counts;       // [E]
-  int E;
-  int K;                       // reduction length
-  int n_total;                 // B rows per expert (2I for gate/up, H for down)
-  uint32_t* status;
-  // gate/up epilogue
-  uint8_t* hq_codes;           // [rows_cap][I/2]
-  uint8_t* hq_sf;              // swizzled [rows_cap][I/16]
-  const float* g_x;            // device scalar
-  const float* g_gate;         // [E]
-  const float* g_up;           // [E]
-  const float* g_h;            // [E]
-  int I;
-  // down epilogue
-  float* acc;                  // [T][H]
-  const int32_t* row_pair;     // [rows_cap]
-  const float* wts;            // [T*topk]
-  const float* alpha_down;     // [E] = g_h * g_down
-  int topk;
-  int H;
-};
 
 // Fused front end for T <= kFrontMaxT (front.cu).
 constexpr int kFrontMaxT = 64;
@@ -175,21 +148,6 @@ cudaError_t launch_export_hq(const uint8_t* hq_codes, const uint8_t* hq_sf, cons
 // Source row r goes to destination row (r / group) * group * mul + add * group + r % group.
 cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_t* swz,
                              int64_t n_col_tiles, int group, int mul, int add, cudaStream_t stream);
-
-// gemm.cu
-// tma_a / tma_a32: the A rows with a 128-row / 32-row box (both 128 bytes wide).
-cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                               int grid, cudaStream_t stream);
-cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                             int grid, cudaStream_t stream);
-// Weight codes [rows][row_bytes] -> tiled operand layout: source row r is packed row
-// (r / group) * group * mul + add * group + r % group; packed rows form 128-row tiles, each
-// split into 128-byte K blocks stored as contiguous 16 KB images of the 128-byte-swizzled
-// shared-memory tile.  The destination must be zero where row_bytes is not a multiple of 128.
-cudaError_t launch_tile_weights(const uint8_t* src, int rows, int row_bytes, uint8_t* dst, int group, int mul,
-                                int add, cudaStream_t stream);
-// Encodes a 2D byte tensor map [rows][row_bytes] with a 128-byte x box_rows box, 128B swizzle.
-int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows);
 
 int num_sms();
 
