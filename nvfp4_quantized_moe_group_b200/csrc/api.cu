@@ -342,7 +342,7 @@ int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e, const nvfp4moe_expert_t
   const int64_t H = c.H, I = c.I;
   // gate/up rows are interleaved in groups of half a GEMM column tile: packed group 2j holds
   // gate rows [64j, 64j+64), group 2j+1 the up rows of the same features
-  constexpr int kG = kBlockN / 2;
+  constexpr int kG = kWeightTileRows / 2;
   const size_t w13_expert = (size_t)2 * I * ((H + 255) / 256 * 128);
   const size_t wd_expert = (size_t)H * ((I + 255) / 256 * 128);
   uint8_t* w13 = x->w13_codes + (size_t)e * w13_expert;
@@ -541,6 +541,8 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   }
 
   const int grid = num_sms();
+  // down GEMM: the deeper pipeline when segments average under 32 rows (decode-sized)
+  const bool deep_down = T * c.topk < 32 * c.E;
   GemmArgs g{};
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
@@ -574,7 +576,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   g.K = c.I;
   g.n_total = c.H;
   ev.mark(NVFP4MOE_STAGE_DOWN, 0);
-  if (launch_gemm_down(tma_h, tma_h32, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_down(tma_h, tma_h32, g, grid, deep_down, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 
