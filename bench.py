@@ -123,7 +123,7 @@ class ClockSampler:
     child process (a thread here would wait on the interpreter lock while the main thread
     launches kernels)."""
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.025):
         import subprocess
         self.samples = []
         self.reasons = 0
@@ -333,7 +333,7 @@ def run_ours(args, world, rank, local):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
         torch.cuda.nvtx.range_push("timed")
         start.record(stream)
         for k in range(args.steps):
@@ -437,7 +437,7 @@ def run_quantize(args, world, rank, local):
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
         start.record()
         for _ in range(args.steps):
             moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g))
@@ -505,6 +505,8 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--clock-period-ms", type=float, default=25.0,
+                    help="NVML clock sampling period during the timed region")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize"])
