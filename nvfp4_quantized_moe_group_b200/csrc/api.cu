@@ -31,7 +31,6 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA; }
 
 int check_device() {
   int dev = 0, major = 0, minor = 0;
@@ -541,8 +540,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   }
 
   const int grid = num_sms();
-  // down GEMM: the deeper pipeline when segments average under 32 rows (decode-sized)
-  const bool deep_down = T * c.topk < 32 * c.E;
+  const bool decode_cfg = T * c.topk < 32 * c.E;   // segments average fewer than 32 rows
   GemmArgs g{};
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
@@ -567,7 +565,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   g.topk = c.topk;
   g.H = c.H;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
-  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
   ++g_launches;
   g.b_tiles = x->wd_codes;
@@ -576,7 +574,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   g.K = c.I;
   g.n_total = c.H;
   ev.mark(NVFP4MOE_STAGE_DOWN, 0);
-  if (launch_gemm_down(tma_h, tma_h32, g, grid, deep_down, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 

@@ -17,8 +17,9 @@
 //   gate/up:  each 128-column half holds 64 gate and 64 up columns of the same features:
 //             h = silu(g_x g_gate acc_gate) * (g_x g_up acc_up) in FP32, requantised to
 //             NVFP4 with the expert's static scale g_h (the down GEMM's A operand);
-//   down:     acc_out[token] += w * g_h * g_down * acc, staged through shared memory so each
-//             warp issues FP32 vector reductions over contiguous row pieces.
+//   down:     acc_out[token] += w * g_h * g_down * acc by FP32 vector reductions, each adding
+//             whole row pieces (staged through shared memory, or straight from the 16x256b
+//             register layout when segments hold few rows).
 // Every wait is bounded; a wait that runs out sets the timeout bit of the status word and
 // the CTA winds down (waits for its own copies and tensor-core work, frees tensor memory).
 //
@@ -47,29 +48,30 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kN = 256;
 constexpr int kNT = kN / 128;                       // 128-row weight tiles per item
 
-// kDeep (down GEMM only): 4 pipeline stages and 8-column epilogue staging, for batches whose
-// segments hold few rows; else 3 stages and 32-column staging (whole 128-byte row pieces per
-// reduction, better when every row of a tile holds a pair).
-template <bool kGateUp, bool kDeep>
+// kDecode: segments average fewer than 32 rows.  The epilogues then read the whole
+// accumulator before any arithmetic (gate/up) and reduce straight from the 16x256b register
+// layout (down), and the down GEMM keeps 4 stages.  With full segments the gate/up epilogue
+// frees the accumulator after its first 32-feature chunk, and the down GEMM stages 32-column
+// pieces through shared memory (whole 128-byte row pieces per reduction, 3 stages): both
+// measured faster there.
+template <bool kGateUp, bool kDecode>
 struct Cfg {
-  static constexpr int kStages = (kGateUp || kDeep) ? 4 : 3;
-  static constexpr bool kStaging = !kGateUp;
-  static constexpr int kStageCols = kDeep ? 8 : 32;
+  static constexpr int kStages = (kGateUp || kDecode) ? 4 : 3;
+  static constexpr bool kStaging = !kGateUp && !kDecode;
   static constexpr uint32_t kSfCol0 = kN;                        // the accumulator first
   static constexpr uint32_t kSfColsA = 16;                       // 4 K steps x 4 columns
   static constexpr uint32_t kSfColsPerStage = kSfColsA + 16 * kNT;
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory columns");
 };
 
-template <bool kGateUp, bool kDeep>
+template <bool kGateUp, bool kDecode>
 struct __align__(1024) Smem {
-  using C = Cfg<kGateUp, kDeep>;
+  using C = Cfg<kGateUp, kDecode>;
   uint8_t a[C::kStages][kABytes];
   uint8_t b[C::kStages][kNT * kTileBytes];
   uint8_t sfa[C::kStages][4 * kAtomBytes];
   uint8_t sfb[C::kStages][kNT * 4 * kAtomBytes];
-  // down: per epilogue warp, 32 rows x kStageCols columns (+1 against bank conflicts)
-  float stage_out[C::kStaging ? kEpiWarps : 1][32][C::kStageCols + 1];
+  float stage_out[C::kStaging ? kEpiWarps : 1][32][33];  // down, full segments: per epilogue warp
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
   uint64_t acc_full;
@@ -78,6 +80,31 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// 16 lanes x 128 columns of FP32 from tensor memory (16x256b shape, 16 repetitions along the
+// columns): thread i receives, for k = 0..15, lane (i / 4) columns 8k + 2 (i % 4) + {0, 1} in
+// r[4k], r[4k + 1] and lane (i / 4 + 8) at the same columns in r[4k + 2], r[4k + 3].
+__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+}
 
 struct Work {
   int e;          // expert
@@ -154,13 +181,13 @@ __device__ __forceinline__ void quant_store32(const float* h, float gh, float r_
   }
 }
 
-template <bool kGateUp, bool kDeep>
+template <bool kGateUp, bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a32,
                 const GemmArgs p) {
-  using C = Cfg<kGateUp, kDeep>;
+  using C = Cfg<kGateUp, kDecode>;
   constexpr int kStages = C::kStages;
-  using S = Smem<kGateUp, kDeep>;
+  using S = Smem<kGateUp, kDecode>;
   extern __shared__ uint8_t smem_raw[];
   S& s = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
@@ -300,7 +327,6 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     const int q = warp & 3;              // tensor-memory lane quarter this warp may read
     const int half = (warp - 2) >> 2;    // which half of the tile's columns it handles
     const int row_l = q * 32 + lane;
-    constexpr int kChunks = kN / 64;     // 32-wide column chunks of a warp's half
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
       const Work wk = decode_work(p.mtile_prefix, w, p.E, ntn, p.counts);
@@ -350,51 +376,86 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         // [128 half, +64) are their gate, [128 half + 64, +64) their up projections
         const int t = wk.nt * kNT + half;
         const int tcol = half * 128;
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          uint32_t G[32], U[32];
-          tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
-          tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
+        if constexpr (kDecode) {
+          // all four 32-column chunks into registers first, then the accumulator is released
+          uint32_t G0[32], U0[32], G1[32], U1[32];
+          tmem_ld_32x32b_x32(t_row + tcol, G0);
+          tmem_ld_32x32b_x32(t_row + tcol + 64, U0);
+          tmem_ld_32x32b_x32(t_row + tcol + 32, G1);
+          tmem_ld_32x32b_x32(t_row + tcol + 96, U1);
           tmem_ld_wait();
-          if (pr == 1) release();
+          release();
           float h[32];
-          swiglu32(G, U, sg, su, h);
-          quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, p, n_ct);
-        }
-      } else {
-        uint32_t R[kChunks][32];
+          swiglu32(G0, U0, sg, su, h);
+          quant_store32(h, gh, r_t, valid, row, t * 64, p, n_ct);
+          swiglu32(G1, U1, sg, su, h);
+          quant_store32(h, gh, r_t, valid, row, t * 64 + 32, p, n_ct);
+        } else {
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + half * (kN / 2) + c * 32, R[c]);
+          for (int pr = 0; pr < 2; ++pr) {
+            uint32_t G[32], U[32];
+            tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
+            tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
+            tmem_ld_wait();
+            if (pr == 1) release();
+            float h[32];
+            swiglu32(G, U, sg, su, h);
+            quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, p, n_ct);
+          }
+        }
+      } else if constexpr (kDecode) {
+        // two 16-lane blocks of this warp's rows, 128 columns each, in the 16x256b layout:
+        // four consecutive threads hold one row's 8 consecutive columns, so every reduction
+        // instruction adds whole 32-byte sectors of 8 token rows
+        uint32_t V[2][64];
+        tmem_ld_16x256b_x16(t_row + half * (kN / 2), V[0]);
+        tmem_ld_16x256b_x16(t_row + (16u << 16) + half * (kN / 2), V[1]);
         tmem_ld_wait();
         release();
-        // staged through shared memory so that each reduction instruction covers whole row
-        // pieces: with W = kStageCols columns, one pass reduces 32 / (W / 4) rows x 4W bytes
-        constexpr int W = C::kStageCols;
-        constexpr int kLanesPerRow = W / 4;
-        constexpr int kRowsPerPass = 32 / kLanesPerRow;
-        const float scale = c0s;
-        float (*st)[W + 1] = s.stage_out[warp - 2];
-        const int sub = lane / kLanesPerRow;          // row of this lane inside a pass
-        const int col = (lane % kLanesPerRow) * 4;    // its 4 columns inside the piece
+        const int cq = 2 * (lane & 3);   // this thread's column pair inside each 8-column group
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
+        for (int lh = 0; lh < 2; ++lh) {
 #pragma unroll
-          for (int c8 = 0; c8 < 32; c8 += W) {
-            const int c0 = half * (kN / 2) + c * 32 + c8;
+          for (int rr = 0; rr < 2; ++rr) {
+            const int r = 16 * lh + 8 * rr + (lane >> 2);   // row inside the warp's 32
+            const int tok = __shfl_sync(0xffffffffu, token, r);
+            const float sc = __shfl_sync(0xffffffffu, c0s, r);
+            if (tok >= 0) {
+              float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + half * (kN / 2) + cq;
 #pragma unroll
-            for (int j = 0; j < W; ++j) st[lane][j] = __fmul_rn(__uint_as_float(R[c][c8 + j]), scale);
-            __syncwarp();
-#pragma unroll
-            for (int pass = 0; pass < 32 / kRowsPerPass; ++pass) {
-              const int r = pass * kRowsPerPass + sub;
-              const int tok = __shfl_sync(0xffffffffu, token, r);
-              if (tok >= 0) {
-                float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + c0 + col;
-                red_add_v4(dst, st[r][col], st[r][col + 1], st[r][col + 2], st[r][col + 3]);
-              }
+              for (int k = 0; k < 16; ++k)
+                red_add_v2(dst + 8 * k, __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr]), sc),
+                           __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr + 1]), sc));
             }
-            __syncwarp();
           }
+        }
+      } else {
+        uint32_t R[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + half * (kN / 2) + c * 32, R[c]);
+        tmem_ld_wait();
+        release();
+        // staged through shared memory: each reduction instruction adds 4 rows x 128 bytes
+        const float scale = c0s;
+        float (*st)[33] = s.stage_out[warp - 2];
+        const int sub = lane >> 3;        // which of the 4 rows this lane writes per pass
+        const int col = (lane & 7) * 4;   // its 4 columns inside the 32-column chunk
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int c0 = half * (kN / 2) + c * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) st[lane][j] = __fmul_rn(__uint_as_float(R[c][j]), scale);
+          __syncwarp();
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            const int r = pass * 4 + sub;
+            const int tok = __shfl_sync(0xffffffffu, token, r);
+            if (tok >= 0) {
+              float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + c0 + col;
+              red_add_v4(dst, st[r][col], st[r][col + 1], st[r][col + 2], st[r][col + 3]);
+            }
+          }
+          __syncwarp();
         }
       }
     }
@@ -408,14 +469,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   }
 }
 
-template <bool kGateUp, bool kDeep>
+template <bool kGateUp, bool kDecode>
 cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a, int grid,
                         cudaStream_t stream) {
-  const size_t smem = sizeof(Smem<kGateUp, kDeep>) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDeep>,
+  const size_t smem = sizeof(Smem<kGateUp, kDecode>) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  moe_gemm_kernel<kGateUp, kDeep><<<grid, kThreads, smem, stream>>>(tma_a, tma_a32, a);
+  moe_gemm_kernel<kGateUp, kDecode><<<grid, kThreads, smem, stream>>>(tma_a, tma_a32, a);
   return cudaGetLastError();
 }
 
@@ -438,19 +499,21 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-static_assert(sizeof(Smem<true, false>) + 1024 <= 232448, "gate/up GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, false>) + 1024 <= 232448, "down GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, true>) + 1024 <= 232448, "down GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                               int grid, cudaStream_t stream) {
-  return launch_gemm<true, false>(tma_a, tma_a32, a, grid, stream);
+                               int grid, bool decode, cudaStream_t stream) {
+  return decode ? launch_gemm<true, true>(tma_a, tma_a32, a, grid, stream)
+                : launch_gemm<true, false>(tma_a, tma_a32, a, grid, stream);
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                             int grid, bool deep, cudaStream_t stream) {
-  return deep ? launch_gemm<false, true>(tma_a, tma_a32, a, grid, stream)
-              : launch_gemm<false, false>(tma_a, tma_a32, a, grid, stream);
+                             int grid, bool decode, cudaStream_t stream) {
+  return decode ? launch_gemm<false, true>(tma_a, tma_a32, a, grid, stream)
+                : launch_gemm<false, false>(tma_a, tma_a32, a, grid, stream);
 }
 
 int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {

@@ -42,11 +42,11 @@ struct GemmArgs {
 // gemm.cu
 // tma_a / tma_a32: the A rows with a 128-row / 32-row box (both 128 bytes wide).  Work items
 // are 256 output columns wide: n_total (2I, H) must be a multiple of 256.
+// decode: the configuration for segments that average fewer than 32 rows.
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                               int grid, cudaStream_t stream);
-// deep: 4 pipeline stages and narrow epilogue staging (batches whose segments hold few rows).
+                               int grid, bool decode, cudaStream_t stream);
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                             int grid, bool deep, cudaStream_t stream);
+                             int grid, bool decode, cudaStream_t stream);
 // Weight codes [rows][row_bytes] -> tiled operand layout: source row r is packed row
 // (r / group) * group * mul + add * group + r % group; packed rows form 128-row tiles, each
 // split into 128-byte K blocks stored as contiguous 16 KB images of the 128-byte-swizzled
