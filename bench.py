@@ -376,6 +376,29 @@ def run_ours(args, world, rank, local):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
 
+    # ---- the same step replayed from a CUDA graph (one capture, K replays; launch cost removed)
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream()
+    cap_stream.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap_stream):
+        moe.forward(ex, x, wr, bias, out=out, ws=ws)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    graph_ms = max_over_ranks(g0.elapsed_time(g1), world)
+    del graph
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"forward status after graph replay {moe.status_string(st)}")
+
     p = peaks()
     ms_step = elapsed_ms / args.steps
     tokens_per_s = tokens_per_second(world, T, args.steps, elapsed_ms)
@@ -414,6 +437,9 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
+        "graph": {"value": tokens_per_second(world, T, args.steps, graph_ms), "unit": "tokens/s",
+                  "ms_per_step": graph_ms / args.steps,
+                  "note": "the same forward captured once in a CUDA graph and replayed K times"},
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline_oracle(shape, wl, x_cpu, wr_cpu, bias_cpu)

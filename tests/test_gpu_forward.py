@@ -200,3 +200,36 @@ def test_front_end_odd_group_layout():
         np.testing.assert_array_equal(dbg["xq_codes"].cpu().numpy(), xc)
         np.testing.assert_array_equal(dbg["xq_scales"].cpu().numpy(), xs)
     ex.close()
+
+
+def test_cuda_graph_replay_matches_eager():
+    """The whole forward (cooperative front end included) captured in a CUDA graph replays to
+    the eager call's routing, grouping and requantised intermediate bit for bit, and to its
+    output within one BF16 unit in the last place (the 8 expert outputs of a token are added
+    with FP32 atomics, in no fixed order), with a clean status word."""
+    ex = gpu_experts(TINY)
+    for T in (16, 130):
+        x = activations(T, TINY, seed=7).cuda()
+        wr = router_weight(TINY).cuda()
+        ws = torch.empty(moe.forward_workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
+        out = torch.empty((T, TINY.H), dtype=torch.bfloat16, device="cuda")
+        _, dbg_ref = moe.forward(ex, x, wr, out=out, ws=ws, debug=True)
+        torch.cuda.synchronize()
+        ref = out.clone()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=s):
+            moe.forward(ex, x, wr, out=out, ws=ws)
+        out.zero_()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        assert moe.status_read(ws) == moe.OK
+        diff = (out.float() - ref.float()).abs()
+        assert bool((diff <= 2.0 ** -7 * ref.float().abs() + 1e-30).all())
+        # the deterministic intermediates, from one more eager call after the replays
+        _, dbg = moe.forward(ex, x, wr, out=out, ws=ws, debug=True)
+        for key in ("idx", "w", "perm", "hq_codes", "hq_scales"):
+            assert torch.equal(dbg[key], dbg_ref[key]), key
+        del g
