@@ -18,7 +18,9 @@ Sources followed (page titles of the pages describing the method):
   8 groups of 32, keep 4 groups by the sum of each group's top two scores,
   top 8 experts inside them, outputs combined with normalised router weights
   scaled by 2.5; section "Residual stream and numerical decisions": the router
-  and the SwiGLU product are computed in FP32.
+  and the SwiGLU product are computed in FP32; the residual stream adds the sublayer
+  output of step k with weight 1/sqrt(k) and keeps the stream with sqrt((k-1)/k), and
+  norms are computed in FP32 (``residual.py``).
 * "Beam-1.0 auf 4x NVIDIA RTX PRO 6000 ..." (eurokommerz), section "Drei
   Checkpoints und was sie speichern": experts in blocks of 16 values, an
   expert is about 22 MB = 39.3M parameters x 0.5625 bytes.
@@ -39,3 +41,4 @@ from .formats import (  # noqa: F401
 )
 from .router import route, RouteResult  # noqa: F401
 from .moe import permutation, expert_mlp, moe_forward, QuantTensor, quantize_tensor  # noqa: F401
+from .residual import rmsnorm, rmsnorm_scale, residual_weights, residual_add  # noqa: F401
