@@ -39,6 +39,9 @@ E2M1_BYTES = 0.5                    # per value
 E4M3_PER16 = 1.0 / 16.0             # block-scale bytes per value
 
 
+RESIDUAL_STEP = 30   # residual step k of the timed fused-residual forward (a mid-depth MoE block)
+
+
 def kernel_source_hash() -> str:
     """SHA-256 over the sources of the grouped GEMM kernels (ties a stored ncu traffic figure
     to the kernel version it was measured on)."""
@@ -399,6 +402,26 @@ def run_ours(args, world, rank, local):
     if st != moe.OK:
         raise RuntimeError(f"forward status after graph replay {moe.status_string(st)}")
 
+    # ---- the layer fused with its residual-stream neighbours (RMSNorm in, weighted add out)
+    h_res = (x.float() * 3.0).to(torch.bfloat16)
+    gamma = torch.ones(shape.H, dtype=torch.float32, device="cuda")
+    h_out = torch.empty_like(h_res)
+    for _ in range(args.warmup):
+        moe.forward_residual(ex, h_res, gamma, 1e-6, RESIDUAL_STEP, wr, bias, out=h_out, ws=ws)
+    torch.cuda.synchronize()
+    barrier(world)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record()
+    for _ in range(args.steps):
+        moe.forward_residual(ex, h_res, gamma, 1e-6, RESIDUAL_STEP, wr, bias, out=h_out, ws=ws)
+    r1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    residual_ms = max_over_ranks(r0.elapsed_time(r1), world)
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"residual forward status {moe.status_string(st)}")
+
     p = peaks()
     ms_step = elapsed_ms / args.steps
     tokens_per_s = tokens_per_second(world, T, args.steps, elapsed_ms)
@@ -437,6 +460,10 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
+        "residual": {"value": tokens_per_second(world, T, args.steps, residual_ms), "unit": "tokens/s",
+                     "ms_per_step": residual_ms / args.steps, "step_k": RESIDUAL_STEP,
+                     "note": "nvfp4moe_forward_residual: RMSNorm of the residual stream, the layer, and "
+                             "the weighted residual add in finalize"},
         "graph": {"value": tokens_per_second(world, T, args.steps, graph_ms), "unit": "tokens/s",
                   "ms_per_step": graph_ms / args.steps,
                   "note": "the same forward captured once in a CUDA graph and replayed K times"},

@@ -241,6 +241,7 @@ typedef struct {
                           after stage s (timing of the stages inside a forward); NULL entries
                           are skipped */
   float* logits;       /* [T][E] FP32 router logits (bias included) the selection used */
+  uint16_t* x_norm;    /* [T][H] BF16 layer input computed by nvfp4moe_forward_residual */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
@@ -254,6 +255,27 @@ NVFP4MOE_API int nvfp4moe_forward(const nvfp4moe_experts* experts, const void* h
  * the read failed). */
 NVFP4MOE_API int nvfp4moe_status_read(const void* ws, void* stream);
 NVFP4MOE_API const char* nvfp4moe_status_string(int status);
+
+/* ------------------------------------------------------- forward, residual ----
+ * The layer with its neighbours on the residual stream fused in ("Reflection releases Beam
+ * ...", section "Residual stream and numerical decisions": at step k a sublayer output is
+ * added with weight 1/sqrt(k) and the stream kept with weight sqrt((k-1)/k); norms in FP32):
+ *
+ *   x  = bf16(fp32(fp32(h * r) * gamma)),  r = fp32(1 / sqrt(mean_j h[t][j]^2 + eps))
+ *        (mean, root and reciprocal in FP64; the RMSNorm of the residual stream)
+ *   h' = bf16(fp32(a * h) + fp32(b * moe(x))),  a = fp32(sqrt((k-1)/k)), b = fp32(1/sqrt(k))
+ *        (moe(x) is the FP32 accumulator nvfp4moe_forward rounds to BF16; here it goes into
+ *        the residual add without that rounding)
+ *
+ *   h_bf16 [T][H] BF16 residual stream;  gamma [H] FP32 norm weight (16-byte aligned);
+ *   eps >= 0;  step_k >= 1 (k = 1 keeps only the layer output);  h_out_bf16 [T][H] BF16
+ *   (out), may be h_bf16 itself (in-place update of the stream).  w_router, logit_bias,
+ *   dbg, ws as for nvfp4moe_forward (same workspace size); dbg->x_norm receives x.
+ * One more launch than nvfp4moe_forward (the norm); the residual add is part of finalize. */
+NVFP4MOE_API int nvfp4moe_forward_residual(const nvfp4moe_experts* experts, const void* h_bf16, int64_t T,
+                                           const float* gamma, float eps, int32_t step_k,
+                                           const float* w_router, const float* logit_bias, void* h_out_bf16,
+                                           const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels the last nvfp4moe_forward / _route / _quantize call on this host
  * thread enqueued (for launch accounting in benchmarks). */

@@ -52,7 +52,7 @@ STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "f
 
 class Debug(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
-                + [("logits", ctypes.c_void_p)])
+                + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p)])
 
 
 class StageTimer:
@@ -103,6 +103,8 @@ _SIGS = {
     "nvfp4moe_experts_cfg": (ctypes.c_int, [_P, ctypes.POINTER(Cfg)]),
     "nvfp4moe_forward_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_forward": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_forward_residual": (ctypes.c_int, [_P, _P, _I64, _P, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
+                                                 ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_status_read": (ctypes.c_int, [_P, _P]),
     "nvfp4moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4moe_last_launch_count": (ctypes.c_int32, []),
@@ -274,6 +276,51 @@ def forward_workspace_bytes(cfg: Cfg, T_max: int) -> int:
     return int(lib().nvfp4moe_forward_workspace_bytes(ctypes.byref(cfg), T_max))
 
 
+def _debug_tensors(cfg: Cfg, T: int, H: int, dev, x_norm: bool = False) -> dict:
+    k, E, I = cfg.topk, cfg.E, cfg.I
+    tensors = {
+        "idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+        "w": torch.empty((T, k), dtype=torch.float32, device=dev),
+        "g_x": torch.empty(1, dtype=torch.float32, device=dev),
+        "xq_codes": torch.empty((T, H // 2), dtype=torch.uint8, device=dev),
+        "xq_scales": torch.empty((T, H // 16), dtype=torch.uint8, device=dev),
+        "counts": torch.empty(E, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+        "hq_codes": torch.empty((T * k, I // 2), dtype=torch.uint8, device=dev),
+        "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
+        "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
+    }
+    if x_norm:
+        tensors["x_norm"] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    return tensors
+
+
+def forward_residual(experts: Experts, h: torch.Tensor, gamma: torch.Tensor, eps: float, step_k: int,
+                     w_router: torch.Tensor, bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, debug: bool = False, stream=None):
+    """The layer fused with its residual-stream neighbours (nvfp4moe_forward_residual):
+    h' = bf16(a h + b moe(rmsnorm(h) gamma)) for residual step ``step_k``.  ``out`` may be ``h``
+    (in-place update).  Returns h' (and the intermediates, x_norm included, if debug)."""
+    cfg = experts.cfg
+    T, H = h.shape
+    dev = h.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(cfg, T), dev)
+    tensors = _debug_tensors(cfg, T, H, dev, x_norm=True) if debug else None
+    dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()}) if debug else None
+    st = lib().nvfp4moe_forward_residual(experts.handle, _ptr(h), T, _ptr(gamma), float(eps), int(step_k),
+                                         _ptr(w_router), _ptr(bias), _ptr(out),
+                                         ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
+                                         _stream(stream))
+    _check(st, "nvfp4moe_forward_residual")
+    if debug:
+        return out, tensors
+    return out
+
+
 def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
             out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None,
             timer: StageTimer | None = None):
@@ -289,20 +336,7 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
     dbg = None
     tensors = None
     if debug:
-        k, E, I = cfg.topk, cfg.E, cfg.I
-        tensors = {
-            "idx": torch.empty((T, k), dtype=torch.int32, device=dev),
-            "w": torch.empty((T, k), dtype=torch.float32, device=dev),
-            "g_x": torch.empty(1, dtype=torch.float32, device=dev),
-            "xq_codes": torch.empty((T, H // 2), dtype=torch.uint8, device=dev),
-            "xq_scales": torch.empty((T, H // 16), dtype=torch.uint8, device=dev),
-            "counts": torch.empty(E, dtype=torch.int32, device=dev),
-            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
-            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
-            "hq_codes": torch.empty((T * k, I // 2), dtype=torch.uint8, device=dev),
-            "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
-            "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
-        }
+        tensors = _debug_tensors(cfg, T, H, dev)
         dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
     if timer is not None:
         if dbg is None:

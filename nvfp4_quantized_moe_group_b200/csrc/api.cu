@@ -1,5 +1,6 @@
 // C ABI of libnvfp4moe: argument checking, workspace layout and the launch sequences of the
 // quantize / route / forward calls.  Declarations and contracts are in nvfp4moe.h.
+#include <cmath>
 #include <cstring>
 #include <vector>
 
@@ -114,6 +115,7 @@ struct ForwardWs {
   uint8_t* a_sf;
   uint8_t* hq_codes;
   uint8_t* hq_sf;
+  uint16_t* x_norm;        // residual forward: the normalised layer input
   int64_t rows_cap;
   size_t bytes;
 };
@@ -151,6 +153,7 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.a_sf = c.take<uint8_t>(f.rows_cap * cfg.H / 16);
   f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg.I / 2);
   f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg.I / 16);
+  f.x_norm = c.take<uint16_t>(T * cfg.H);
   f.bytes = c.off;
   return f;
 }
@@ -162,6 +165,12 @@ __global__ void set_expert_scalars_kernel(float* g_gate, float* g_up, float* g_h
   g_h[e] = gh;
   alpha[e] = __fmul_rn(gh, gd);
 }
+
+// Weighted residual add fused into finalize: out = bf16(a * h + b * layer output).
+struct Residual {
+  const uint16_t* h;
+  float a, b;
+};
 
 struct StageEvents {
   void* const* ev;
@@ -387,9 +396,10 @@ size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) 
   return carve_forward(nullptr, *cfg, T_max).bytes;
 }
 
-int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
-                     const float* logit_bias, void* out_bf16, const nvfp4moe_debug* dbg, void* ws,
-                     size_t ws_bytes, void* stream) {
+// The layer; with res, finalize adds the output into the residual stream.
+static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
+                        const float* logit_bias, void* out_bf16, const Residual* res, const nvfp4moe_debug* dbg,
+                        void* ws, size_t ws_bytes, void* stream) {
   g_launches = 0;
   if (x == nullptr) return NVFP4MOE_ERR_ARG;
   const nvfp4moe_cfg& c = x->cfg;
@@ -578,7 +588,8 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 
-  FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H};
+  FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,
+                  res != nullptr ? res->a : 0.0f, res != nullptr ? res->b : 0.0f};
   ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
   if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_FINALIZE, 1);
@@ -603,6 +614,43 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
     if (!ok) return NVFP4MOE_ERR_CUDA;
   }
   return NVFP4MOE_OK;
+}
+
+int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
+                     const float* logit_bias, void* out_bf16, const nvfp4moe_debug* dbg, void* ws,
+                     size_t ws_bytes, void* stream) {
+  return forward_core(x, hidden_bf16, T, w_router, logit_bias, out_bf16, nullptr, dbg, ws, ws_bytes, stream);
+}
+
+int nvfp4moe_forward_residual(const nvfp4moe_experts* x, const void* h_bf16, int64_t T, const float* gamma,
+                              float eps, int32_t step_k, const float* w_router, const float* logit_bias,
+                              void* h_out_bf16, const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes,
+                              void* stream) {
+  g_launches = 0;
+  if (x == nullptr) return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = x->cfg;
+  if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
+  if (h_bf16 == nullptr || gamma == nullptr || w_router == nullptr || h_out_bf16 == nullptr || ws == nullptr)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(h_bf16, 16) || !aligned(gamma, 16) || !aligned(h_out_bf16, 16) || !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  if (step_k < 1 || !(eps >= 0.0f) || eps > 3.0e38f) return NVFP4MOE_ERR_ARG;
+  const ForwardWs f = carve_forward(ws, c, T);
+  if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word is reset by the forward that follows; the norm raises nothing
+  RmsNormArgs na{static_cast<const uint16_t*>(h_bf16), gamma, eps, T, c.H, f.x_norm};
+  if (launch_rmsnorm(na, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  const Residual r{static_cast<const uint16_t*>(h_bf16), (float)std::sqrt((double)(step_k - 1) / (double)step_k),
+                   (float)(1.0 / std::sqrt((double)step_k))};
+  st = forward_core(x, f.x_norm, T, w_router, logit_bias, h_out_bf16, &r, dbg, ws, ws_bytes, stream);
+  g_launches += 1;
+  if (st == NVFP4MOE_OK && dbg != nullptr && dbg->x_norm != nullptr &&
+      cudaMemcpyAsync(dbg->x_norm, f.x_norm, (size_t)T * c.H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  return st;
 }
 
 int nvfp4moe_status_read(const void* ws, void* stream) {

@@ -107,6 +107,19 @@ struct FinalizeArgs {
   const float* acc;
   uint16_t* out;
   int64_t n;  // elements, multiple of 8
+  // optional weighted residual add: out = bf16(fp32(a * res) + fp32(b * acc)); res may be out
+  const uint16_t* res;
+  float a, b;
+};
+
+// RMSNorm of the residual stream into the layer input (residual.cu).
+struct RmsNormArgs {
+  const uint16_t* h;       // [T][H] bf16 residual stream
+  const float* gamma;      // [H]
+  float eps;
+  int64_t T;
+  int H;                   // multiple of 8
+  uint16_t* x;             // [T][H] bf16 out
 };
 
 // quantize.cu
@@ -133,6 +146,9 @@ bool front_supported(int64_t T, int E, int H);
 // Split-K partials the front kernel writes: ksplit * T * E doubles.
 int front_ksplit(int E, int H);
 cudaError_t launch_front(FrontArgs a, cudaStream_t stream);
+
+// residual.cu
+cudaError_t launch_rmsnorm(const RmsNormArgs& a, cudaStream_t stream);
 
 // permute.cu
 // Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.

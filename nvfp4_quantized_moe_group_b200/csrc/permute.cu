@@ -172,13 +172,25 @@ cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream, int* launches
   return cudaGetLastError();
 }
 
-// out = bf16(acc), 8 values per thread.
+// out = bf16(acc), or with the residual stream bf16(fp32(a * res) + fp32(b * acc)) (the
+// weighted residual add of "Reflection releases Beam ...", section "Residual stream and
+// numerical decisions"); 8 values per thread.  res may alias out: each thread reads its 8
+// residual values before it writes them.
 __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
   const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8;
   if (i >= a.n) return;
   const float4 p = *reinterpret_cast<const float4*>(a.acc + i);
   const float4 q = *reinterpret_cast<const float4*>(a.acc + i + 4);
-  const float v[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+  float v[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+  if (a.res != nullptr) {
+    const uint4 r = *reinterpret_cast<const uint4*>(a.res + i);
+    const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __fadd_rn(__fmul_rn(a.a, __uint_as_float(rw[j] << 16)), __fmul_rn(a.b, v[2 * j]));
+      v[2 * j + 1] = __fadd_rn(__fmul_rn(a.a, __uint_as_float(rw[j] & 0xFFFF0000u)), __fmul_rn(a.b, v[2 * j + 1]));
+    }
+  }
   uint32_t w[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
