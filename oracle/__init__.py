@@ -21,6 +21,8 @@ Sources followed (page titles of the pages describing the method):
   and the SwiGLU product are computed in FP32; the residual stream adds the sublayer
   output of step k with weight 1/sqrt(k) and keeps the stream with sqrt((k-1)/k), and
   norms are computed in FP32 (``residual.py``).
+* "NVFP4 quantization", section "Quantization method": the post-training block-scale search
+  that minimises the Hessian-weighted error (``local_hessian.py``).
 * "Beam-1.0 auf 4x NVIDIA RTX PRO 6000 ..." (eurokommerz), section "Drei
   Checkpoints und was sie speichern": experts in blocks of 16 values, an
   expert is about 22 MB = 39.3M parameters x 0.5625 bytes.
@@ -42,3 +44,4 @@ from .formats import (  # noqa: F401
 from .router import route, RouteResult  # noqa: F401
 from .moe import permutation, expert_mlp, moe_forward, QuantTensor, quantize_tensor  # noqa: F401
 from .residual import rmsnorm, rmsnorm_scale, residual_weights, residual_add  # noqa: F401
+from .local_hessian import quantize_local_hessian, hessian_blocks, candidate_offsets  # noqa: F401
