@@ -513,6 +513,65 @@ def run_quantize(args, world, rank, local):
             "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
 
 
+FP32_LANES_PER_SM = 128   # FP32 FMA lanes per B200 SM (4 partitions x 32)
+
+
+def run_quantize_lh(args, world, rank, local):
+    """Local-Hessian weight quantisation of one Beam expert per step: gate [2560, 5120], up
+    [2560, 5120] and down [5120, 2560], m = 4 (9 candidate scales per block), local Hessian
+    blocks of 256 synthetic calibration tokens.  FP32-ALU bound: per block and candidate the
+    kernel does a 16x16 matrix-vector product and a dot product (272 FMAs) plus ~40 other
+    operations; the roofline counts 2 x 272 FLOP per block-candidate against the FP32 FMA peak
+    of the SMs at the maximum SM clock."""
+    import nvfp4_quantized_moe_group_b200 as moe
+    import oracle
+    H, I, m = BEAM.H, BEAM.I, 4
+    shapes = [(I, H), (I, H), (H, I)]
+    mats, hess = [], []
+    for j, (rows, cols) in enumerate(shapes):
+        mats.append(expert_weight(BEAM, j, ("gate", "up", "down")[j], device="cuda"))
+        x = activations(256, LayerShape(H=cols, I=I, E=1, n_groups=1, topk_groups=1, topk=1, routed_scale=1.0,
+                                        wr_std=1.0, w_std=0.02), seed=70 + j + rank)
+        hess.append(torch.from_numpy(oracle.hessian_blocks(x.float().numpy()).astype(np.float32)).cuda())
+    ws = torch.empty(moe.quantize_workspace_bytes(H, H), dtype=torch.uint8, device="cuda")
+
+    def step():
+        for w, hb in zip(mats, hess):
+            moe.quantize_weights_lh(w, hb, m, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
+        start.record()
+        for _ in range(args.steps):
+            step()
+        stop.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    if moe.status_read(ws) != moe.OK:
+        raise RuntimeError("local-Hessian quantize status")
+    blocks = sum(r * c // 16 for r, c in shapes)
+    flops = blocks * (2 * m + 1) * 2 * 272
+    clk = clocks.summary()
+    max_mhz = clk["sm_max_mhz"] or 1965
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    peak = sms * FP32_LANES_PER_SM * 2 * max_mhz * 1e6 / 1e12
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"metric": "local-Hessian NVFP4 weight quantisation, Beam experts/s (m = 4)",
+            "value": world * 1e3 / ms, "unit": "experts/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16->e2m1 (fp32 search)", "data": "synthetic",
+            "config": {"workload": "quantize_lh: gate/up 2560x5120 + down 5120x2560, m=4, 256 calibration tokens",
+                       "blocks_per_step": blocks},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": "SMs x 128 FP32 lanes x 2 FLOP x max SM clock"},
+            "gpu_launches": 2 * len(shapes) * args.steps, "clocks": clk}
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm.  Each step is a bounded sample of the workload's step:
     routing and input quantisation of all its tokens plus one (token, slot) pair's expert
@@ -562,7 +621,7 @@ def main():
                     help="NVML clock sampling period during the timed region")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize"])
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize", "quantize_lh"])
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -579,8 +638,12 @@ def main():
 
     world, rank, local = init_dist()
     try:
-        res = run_quantize(args, world, rank, local) if args.workload == "quantize" else \
-            run_ours(args, world, rank, local)
+        if args.workload == "quantize":
+            res = run_quantize(args, world, rank, local)
+        elif args.workload == "quantize_lh":
+            res = run_quantize_lh(args, world, rank, local)
+        else:
+            res = run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -119,6 +119,29 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
                       uint8_t* codes, uint8_t* scales, int32_t scale_layout, float* g_out,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- weights, local-Hessian scales ----
+ * Weight quantisation with the block-scale search of "NVFP4 quantization", section
+ * "Quantization method": for each 16-value block, candidate scales are tried and the one
+ * minimising the Hessian-weighted error dW^T H dW is kept.
+ *
+ *   w_bf16 [rows][cols] BF16 weight matrix (rows >= 1, cols % 16 == 0, 16-byte aligned);
+ *   hess_blocks [cols/16][16][16] FP32: for each 16-column block, the 16x16 diagonal block of
+ *       H = X^T X over calibration inputs X of this projection (shared by all rows);
+ *   m  0..16: candidates are the E4M3 scale codes S0-m .. S0+m (clamped to 1..0x7E) around the
+ *       round-to-nearest code S0 of nvfp4moe_quantize's rule; a zero block keeps scale 0;
+ *       m = 0 gives exactly nvfp4moe_quantize with linear scales;
+ *   codes out [rows][cols/2] (8-byte aligned), scales out [rows][cols/16] linear, g_out out
+ *       device scalar: the global scale fp32(amax / 2688) of the matrix.
+ * For each candidate the codes follow the quantisation rule with that block scale, and the
+ * error is computed in FP32; a candidate replaces the best only when its error is strictly
+ * smaller, in the visiting order S0, S0-1, S0+1, ..., S0-m, S0+m.  The outputs feed
+ * nvfp4moe_experts_set.  Workspace: nvfp4moe_quantize_workspace_bytes.  A non-finite weight
+ * raises NVFP4MOE_ERR_NONFINITE in the status word (nvfp4moe_status_read). */
+NVFP4MOE_API int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, int64_t cols,
+                                              const float* hess_blocks, int32_t m, uint8_t* codes,
+                                              uint8_t* scales, float* g_out, void* ws, size_t ws_bytes,
+                                              void* stream);
+
 /* ------------------------------------------------------------------- route ----
  * route(hidden, W_router) -> top-k experts and weights
  * ("Reflection releases Beam ...", section "Mixture-of-Experts details").

@@ -95,6 +95,7 @@ _SIGS = {
     "nvfp4moe_quantize_workspace_bytes": (_SZ, [_I64, _I64]),
     "nvfp4moe_swizzled_scale_bytes": (_SZ, [_I64, _I64]),
     "nvfp4moe_quantize": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, ctypes.c_int32, _P, _P, _SZ, _P]),
+    "nvfp4moe_quantize_weights_lh": (ctypes.c_int, [_P, _I64, _I64, _P, ctypes.c_int32, _P, _P, _P, _P, _SZ, _P]),
     "nvfp4moe_route_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_route": (ctypes.c_int, [ctypes.POINTER(Cfg), _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
     "nvfp4moe_experts_create": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.POINTER(_P)]),
@@ -211,6 +212,28 @@ def quantize(x: torch.Tensor, g: torch.Tensor | None = None, swizzled: bool = Fa
                                  SCALES_SWIZZLED if swizzled else SCALES_LINEAR, _ptr(g_out), _ptr(ws),
                                  ws.numel(), _stream(stream))
     _check(st, "nvfp4moe_quantize")
+    return codes, scales, g_out
+
+
+def quantize_weights_lh(w: torch.Tensor, hess_blocks: torch.Tensor, m: int = 4, ws=None, stream=None):
+    """Weight quantisation with the local-Hessian block-scale search
+    (nvfp4moe_quantize_weights_lh): w [rows, cols] bf16, hess_blocks [cols/16, 16, 16] float32
+    -> (codes [rows, cols/2] u8, linear scales [rows, cols/16] u8, g [1] f32)."""
+    if w.dtype != torch.bfloat16 or not w.is_cuda or w.dim() != 2 or not w.is_contiguous():
+        raise TypeError("w must be a contiguous 2-D bfloat16 CUDA tensor")
+    rows, cols = w.shape
+    if hess_blocks.dtype != torch.float32 or tuple(hess_blocks.shape) != (cols // 16, 16, 16) \
+            or not hess_blocks.is_contiguous():
+        raise TypeError("hess_blocks must be a contiguous float32 tensor [cols/16, 16, 16]")
+    dev = w.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    g_out = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(quantize_workspace_bytes(rows, cols), dev)
+    st = lib().nvfp4moe_quantize_weights_lh(_ptr(w), rows, cols, _ptr(hess_blocks), int(m), _ptr(codes),
+                                            _ptr(scales), _ptr(g_out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "nvfp4moe_quantize_weights_lh")
     return codes, scales, g_out
 
 

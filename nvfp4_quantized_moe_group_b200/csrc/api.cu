@@ -266,6 +266,34 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   return NVFP4MOE_OK;
 }
 
+int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, int64_t cols, const float* hess_blocks,
+                                 int32_t m, uint8_t* codes, uint8_t* scales, float* g_out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (rows < 1 || cols <= 0 || cols % 16 != 0 || cols / 16 > 65535) return NVFP4MOE_ERR_SHAPE;
+  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (m < 0 || m > 16) return NVFP4MOE_ERR_ARG;
+  if (w_bf16 == nullptr || hess_blocks == nullptr || codes == nullptr || scales == nullptr || g_out == nullptr ||
+      ws == nullptr)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(w_bf16, 16) || !aligned(hess_blocks, 4) || !aligned(codes, 8) || !aligned(g_out, 4) ||
+      !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  const QuantWs q = carve_quant(ws);
+  if (ws_bytes < q.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  const int blocks = amax_partial_blocks(rows * cols);
+  if (launch_amax_partial(w_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  LhArgs la{static_cast<const uint16_t*>(w_bf16), rows, cols, hess_blocks, m, q.partials, blocks, codes, scales,
+            g_out, &q.hdr->status};
+  if (launch_lh_quantize(la, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches = 2;
+  return NVFP4MOE_OK;
+}
+
 size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T) {
   if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || T < 0) return 0;
   return carve_route(nullptr, *cfg, T > 0 ? T : 1).bytes;

@@ -150,6 +150,22 @@ cudaError_t launch_front(FrontArgs a, cudaStream_t stream);
 // residual.cu
 cudaError_t launch_rmsnorm(const RmsNormArgs& a, cudaStream_t stream);
 
+// local_hessian.cu: block-scale search for weight quantisation.
+struct LhArgs {
+  const uint16_t* w;       // [rows][cols] bf16
+  int64_t rows;
+  int64_t cols;            // multiple of 16
+  const float* hess;       // [cols/16][16][16] local Hessian blocks
+  int m;                   // candidates S0 - m .. S0 + m
+  const uint32_t* partials;
+  int n_partials;
+  uint8_t* codes;          // [rows][cols/2]
+  uint8_t* scales;         // [rows][cols/16] linear
+  float* g_out;
+  uint32_t* status;
+};
+cudaError_t launch_lh_quantize(const LhArgs& a, cudaStream_t stream);
+
 // permute.cu
 // Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.
 constexpr int kPermSmallPairs = 4096;
