@@ -21,6 +21,8 @@ Sources followed (page titles of the pages describing the method):
   and the SwiGLU product are computed in FP32; the residual stream adds the sublayer
   output of step k with weight 1/sqrt(k) and keeps the stream with sqrt((k-1)/k), and
   norms are computed in FP32 (``residual.py``).
+* "FP8 quantization", sections "Quantization scheme" and "Quantization method": the FP8 W8A8
+  variant, per-output-channel weight scales and per-token activation scales (``fp8.py``).
 * "NVFP4 quantization", section "Quantization method": the post-training block-scale search
   that minimises the Hessian-weighted error (``local_hessian.py``).
 * "Beam-1.0 auf 4x NVIDIA RTX PRO 6000 ..." (eurokommerz), section "Drei
@@ -45,3 +47,4 @@ from .router import route, RouteResult  # noqa: F401
 from .moe import permutation, expert_mlp, moe_forward, QuantTensor, quantize_tensor  # noqa: F401
 from .residual import rmsnorm, rmsnorm_scale, residual_weights, residual_add  # noqa: F401
 from .local_hessian import quantize_local_hessian, hessian_blocks, candidate_offsets  # noqa: F401
+from . import fp8  # noqa: F401
