@@ -216,6 +216,51 @@ def algorithmic(shape: LayerShape, T: int, counts: np.ndarray):
             "gateup_flops": gateup_flops}
 
 
+def run_fp8(moe, shape: LayerShape, cfg, x, wr, bias, T: int, steps: int, warmup: int, world: int) -> dict:
+    """The FP8 W8A8 variant of the layer (nvfp4moe_forward_fp8) on the same batch: its own
+    experts quantised per output channel, K device-timed steps, and its HBM roofline (E4M3
+    weights of the routed experts, one byte per value, plus FP32 channel scales)."""
+    ex = moe.Fp8Experts(cfg)
+    for e in range(shape.E):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")))
+    ws = torch.empty(moe.forward_fp8_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, shape.H), dtype=torch.bfloat16, device="cuda")
+    _, dbg = moe.forward_fp8(ex, x, wr, bias, out=out, ws=ws, debug=True)
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"fp8 forward status {moe.status_string(st)}")
+    hit = int((dbg["counts"].cpu().numpy() > 0).sum())
+    launches = moe.last_launch_count()
+    del dbg
+    for _ in range(warmup):
+        moe.forward_fp8(ex, x, wr, bias, out=out, ws=ws)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(steps):
+        moe.forward_fp8(ex, x, wr, bias, out=out, ws=ws)
+    f1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(f0.elapsed_time(f1), world) / steps
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"fp8 forward status {moe.status_string(st)}")
+    ex.close()
+    H, I = shape.H, shape.I
+    w_bytes = hit * (3 * H * I + 4 * (2 * I + H))
+    layer_bytes = w_bytes + T * H * 2 * 2 + shape.E * H * 4
+    p = peaks()
+    return {"value": tokens_per_second(world, T, steps, ms * steps), "unit": "tokens/s", "ms_per_step": ms,
+            "experts_hit": hit, "gpu_launches_per_step": launches,
+            "layer_roofline": {"bound": "hbm", "bytes_per_step": layer_bytes,
+                               "achieved": layer_bytes / (ms / 1e3) / 1e9, "peak": p["hbm_gbs"], "unit": "GB/s",
+                               "frac": layer_bytes / (ms / 1e3) / (p["hbm_gbs"] * 1e9)},
+            "note": "nvfp4moe_forward_fp8: E4M3 weights with per-channel scales, per-token E4M3 activations, "
+                    "tcgen05 kind::f8f6f4 grouped GEMMs; same batch and routing as the NVFP4 line"}
+
+
 def _oracle_cfg(shape: LayerShape):
     import types
     return types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
@@ -422,6 +467,8 @@ def run_ours(args, world, rank, local):
     if st != moe.OK:
         raise RuntimeError(f"residual forward status {moe.status_string(st)}")
 
+    fp8 = None if args.no_fp8 else run_fp8(moe, shape, cfg, x, wr, bias, T, args.steps, args.warmup, world)
+
     p = peaks()
     ms_step = elapsed_ms / args.steps
     tokens_per_s = tokens_per_second(world, T, args.steps, elapsed_ms)
@@ -468,6 +515,8 @@ def run_ours(args, world, rank, local):
                   "ms_per_step": graph_ms / args.steps,
                   "note": "the same forward captured once in a CUDA graph and replayed K times"},
     }
+    if fp8 is not None:
+        res["fp8"] = fp8
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline_oracle(shape, wl, x_cpu, wr_cpu, bias_cpu)
     ex.close()
@@ -624,6 +673,7 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize", "quantize_lh"])
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 W8A8 variant's measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -265,6 +265,8 @@ typedef struct {
                           are skipped */
   float* logits;       /* [T][E] FP32 router logits (bias included) the selection used */
   uint16_t* x_norm;    /* [T][H] BF16 layer input computed by nvfp4moe_forward_residual */
+  uint8_t* xq8_codes;  /* [T][H] E4M3 layer input of nvfp4moe_forward_fp8 */
+  float* xq8_scales;   /* [T] its per-token scales */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
@@ -299,6 +301,56 @@ NVFP4MOE_API int nvfp4moe_forward_residual(const nvfp4moe_experts* experts, cons
                                            const float* gamma, float eps, int32_t step_k,
                                            const float* w_router, const float* logit_bias, void* h_out_bf16,
                                            const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------- FP8 W8A8 variant ----
+ * The same layer with FP8 experts ("FP8 quantization", section "Quantization scheme": E4M3
+ * weights with a fixed scale per output channel, E4M3 input activations with a scale per
+ * token computed at run time; the router stays in high precision; section "Quantization
+ * method": round to nearest).  Rule for one row v (a weight output channel, a token's input
+ * row, or a pair's SwiGLU product):
+ *   s = fp32(max|v| / 448)  (s = 1 when max|v| = 0),  code = E4M3_rn_satfinite(fp32(v / s))
+ * (IEEE division, sign kept).  The down projection's input is the SwiGLU product h in FP32,
+ * quantised per (token, slot) row.  The GEMMs multiply E4M3 codes with FP32 accumulation and
+ * apply the row scales in the epilogue; routing, grouping and the weighted combine are the
+ * NVFP4 layer's.
+ *
+ * nvfp4moe_quantize_fp8: x_bf16 [rows][cols] BF16 (16-byte aligned, cols % 16 == 0) ->
+ *   codes [rows][cols] (8-byte aligned) and scales [rows] FP32.  Workspace:
+ *   nvfp4moe_quantize_workspace_bytes.  A non-finite row raises NVFP4MOE_ERR_NONFINITE in the
+ *   status word and leaves that row's outputs unwritten. */
+NVFP4MOE_API int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_t* codes,
+                                       float* scales, void* ws, size_t ws_bytes, void* stream);
+
+/* Library-owned FP8 experts (about E * 3 * H * I bytes of device memory), laid out for the
+ * FP8 grouped GEMMs; same life cycle as nvfp4moe_experts. */
+typedef struct nvfp4moe_fp8_experts nvfp4moe_fp8_experts;
+
+/* One expert's FP8 tensors, as nvfp4moe_quantize_fp8 produces them.  Device pointers:
+ * gate/up codes [I][H] (16-byte aligned), scales [I] FP32; down codes [H][I] (16-byte
+ * aligned), scales [H] FP32. */
+typedef struct {
+  const uint8_t* gate_codes;
+  const float* gate_scales;
+  const uint8_t* up_codes;
+  const float* up_scales;
+  const uint8_t* down_codes;
+  const float* down_scales;
+} nvfp4moe_fp8_expert_tensors;
+
+NVFP4MOE_API int nvfp4moe_fp8_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_fp8_experts** out);
+/* Copies expert e into the handle on `stream` (experts never set hold zero weights). */
+NVFP4MOE_API int nvfp4moe_fp8_experts_set(nvfp4moe_fp8_experts* experts, int32_t e,
+                                          const nvfp4moe_fp8_expert_tensors* t, void* stream);
+NVFP4MOE_API void nvfp4moe_fp8_experts_destroy(nvfp4moe_fp8_experts* experts);
+
+/* The FP8 layer: arguments as nvfp4moe_forward, with its own workspace size.  dbg: idx, w,
+ * counts, offsets, perm, logits, xq8_codes and xq8_scales are filled; the NVFP4-specific
+ * members and events are ignored.  Launches: router (2), grouping (1 or 3), quantise-scatter,
+ * gate/up GEMM, requantisation of h, down GEMM, finalize. */
+NVFP4MOE_API size_t nvfp4moe_forward_fp8_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
+NVFP4MOE_API int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* experts, const void* hidden_bf16, int64_t T,
+                                      const float* w_router, const float* logit_bias, void* out_bf16,
+                                      const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels the last nvfp4moe_forward / _route / _quantize call on this host
  * thread enqueued (for launch accounting in benchmarks). */

@@ -52,7 +52,14 @@ STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "f
 
 class Debug(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
-                + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p)])
+                + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p), ("xq8_codes", ctypes.c_void_p),
+                   ("xq8_scales", ctypes.c_void_p)])
+
+
+class Fp8ExpertTensors(ctypes.Structure):
+    _fields_ = [("gate_codes", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p),
+                ("up_codes", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+                ("down_codes", ctypes.c_void_p), ("down_scales", ctypes.c_void_p)]
 
 
 class StageTimer:
@@ -106,6 +113,12 @@ _SIGS = {
     "nvfp4moe_forward": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_forward_residual": (ctypes.c_int, [_P, _P, _I64, _P, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
                                                  ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_quantize_fp8": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "nvfp4moe_fp8_experts_create": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.POINTER(_P)]),
+    "nvfp4moe_fp8_experts_set": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(Fp8ExpertTensors), _P]),
+    "nvfp4moe_fp8_experts_destroy": (None, [_P]),
+    "nvfp4moe_forward_fp8_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
+    "nvfp4moe_forward_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_status_read": (ctypes.c_int, [_P, _P]),
     "nvfp4moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4moe_last_launch_count": (ctypes.c_int32, []),
@@ -369,6 +382,99 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
                                 ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
                                 _stream(stream))
     _check(st, "nvfp4moe_forward")
+    if debug:
+        return out, tensors
+    return out
+
+
+# ------------------------------------------------------------------ FP8 W8A8 variant ----
+
+def quantize_fp8(x: torch.Tensor, ws=None, stream=None):
+    """Per-row FP8 quantisation (nvfp4moe_quantize_fp8): x [rows, cols] bf16 ->
+    (codes [rows, cols] u8 E4M3, scales [rows] f32)."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 CUDA tensor")
+    rows, cols = x.shape
+    dev = x.device
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(quantize_workspace_bytes(rows, cols), dev)
+    st = lib().nvfp4moe_quantize_fp8(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _ptr(ws), ws.numel(),
+                                     _stream(stream))
+    _check(st, "nvfp4moe_quantize_fp8")
+    return codes, scales
+
+
+class Fp8Experts:
+    """Library-owned FP8 expert weights (nvfp4moe_fp8_experts_create / _set / _destroy)."""
+
+    def __init__(self, cfg: Cfg):
+        self.cfg = cfg
+        h = ctypes.c_void_p()
+        _check(lib().nvfp4moe_fp8_experts_create(ctypes.byref(cfg), ctypes.byref(h)),
+               "nvfp4moe_fp8_experts_create")
+        self.handle = h
+
+    def set(self, e: int, gate, up, down, stream=None):
+        """gate/up/down: (codes, scales) from quantize_fp8()."""
+        t = Fp8ExpertTensors(gate[0].data_ptr(), gate[1].data_ptr(), up[0].data_ptr(), up[1].data_ptr(),
+                             down[0].data_ptr(), down[1].data_ptr())
+        _check(lib().nvfp4moe_fp8_experts_set(self.handle, int(e), ctypes.byref(t), _stream(stream)),
+               "nvfp4moe_fp8_experts_set")
+
+    def set_from_bf16(self, e: int, gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor, stream=None):
+        """Quantise BF16 gate [I, H], up [I, H], down [H, I] per output channel and copy them in."""
+        q = [quantize_fp8(w, stream=stream) for w in (gate, up, down)]
+        self.set(e, q[0], q[1], q[2], stream=stream)
+        return q
+
+    def close(self):
+        if self.handle:
+            lib().nvfp4moe_fp8_experts_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def forward_fp8_workspace_bytes(cfg: Cfg, T_max: int) -> int:
+    return int(lib().nvfp4moe_forward_fp8_workspace_bytes(ctypes.byref(cfg), T_max))
+
+
+def forward_fp8(experts: Fp8Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
+                out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False,
+                stream=None):
+    """The FP8 W8A8 layer (nvfp4moe_forward_fp8) -> out [T, H] bf16 (and intermediates if debug)."""
+    cfg = experts.cfg
+    T, H = x.shape
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = _workspace(forward_fp8_workspace_bytes(cfg, T), dev)
+    tensors = None
+    dbg = None
+    if debug:
+        k, E = cfg.topk, cfg.E
+        tensors = {
+            "idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "w": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "perm": torch.empty(T * k, dtype=torch.int32, device=dev),
+            "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
+            "xq8_codes": torch.empty((T, H), dtype=torch.uint8, device=dev),
+            "xq8_scales": torch.empty(T, dtype=torch.float32, device=dev),
+        }
+        dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
+    st = lib().nvfp4moe_forward_fp8(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(out),
+                                    ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
+                                    _stream(stream))
+    _check(st, "nvfp4moe_forward_fp8")
     if debug:
         return out, tensors
     return out

@@ -22,6 +22,16 @@ struct nvfp4moe_experts {
   float* alpha_down;    // [E] g_h * g_down
 };
 
+// FP8 W8A8 experts ("FP8 quantization", section "Quantization scheme").
+struct nvfp4moe_fp8_experts {
+  nvfp4moe_cfg cfg;
+  int device;
+  uint8_t* w13_codes;   // tiled like the NVFP4 codes with 128-value K blocks, gate/up interleaved per 64 rows
+  float* w13_scale;     // [E][2I] channel scales in the same interleaved order
+  uint8_t* wd_codes;    // tiled, [E][H/128][I/128][128][128]
+  float* wd_scale;      // [E][H]
+};
+
 namespace {
 
 thread_local int32_t g_launches = 0;
@@ -154,6 +164,60 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg.I / 2);
   f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg.I / 16);
   f.x_norm = c.take<uint16_t>(T * cfg.H);
+  f.bytes = c.off;
+  return f;
+}
+
+struct ForwardFp8Ws {
+  WsHeader* hdr;
+  uint32_t* partials;
+  double* parts;
+  int32_t* idx;
+  float* wts;
+  float* acc;
+  int32_t* chunk_counts;
+  int32_t* chunk_base;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile_prefix;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* row_pair;
+  uint8_t* a_codes;     // [rows_cap][H] E4M3
+  float* a_scale;       // [rows_cap]
+  float* h32;           // [rows_cap][I]
+  uint8_t* hq;          // [rows_cap][I] E4M3
+  float* h_scale;       // [rows_cap]
+  int64_t rows_cap;
+  size_t bytes;
+};
+
+ForwardFp8Ws carve_forward_fp8(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
+  Carver c(ws);
+  ForwardFp8Ws f;
+  const int64_t pairs = T * cfg.topk;
+  const int64_t n_chunks = (T + kPermChunkTokens - 1) / kPermChunkTokens;
+  f.rows_cap = rows_capacity(cfg, T);
+  f.hdr = c.take<WsHeader>(1);
+  const int n_part = router_amax_partials(T, cfg.E, cfg.H);
+  f.partials = c.take<uint32_t>(n_part > kMaxAmaxPartials ? n_part : kMaxAmaxPartials);
+  f.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
+  f.idx = c.take<int32_t>(pairs);
+  f.wts = c.take<float>(pairs);
+  f.acc = c.take<float>(T * cfg.H);
+  f.chunk_counts = c.take<int32_t>(n_chunks * cfg.E);
+  f.chunk_base = c.take<int32_t>(n_chunks * cfg.E);
+  f.counts = c.take<int32_t>(cfg.E);
+  f.offsets = c.take<int32_t>(cfg.E + 1);
+  f.mtile_prefix = c.take<int32_t>(cfg.E + 1);
+  f.perm = c.take<int32_t>(pairs);
+  f.inv = c.take<int32_t>(pairs);
+  f.row_pair = c.take<int32_t>(f.rows_cap);
+  f.a_codes = c.take<uint8_t>(f.rows_cap * cfg.H);
+  f.a_scale = c.take<float>(f.rows_cap);
+  f.h32 = c.take<float>(f.rows_cap * cfg.I);
+  f.hq = c.take<uint8_t>(f.rows_cap * cfg.I);
+  f.h_scale = c.take<float>(f.rows_cap);
   f.bytes = c.off;
   return f;
 }
@@ -679,6 +743,211 @@ int nvfp4moe_forward_residual(const nvfp4moe_experts* x, const void* h_bf16, int
       cudaMemcpyAsync(dbg->x_norm, f.x_norm, (size_t)T * c.H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return NVFP4MOE_ERR_CUDA;
   return st;
+}
+
+int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_t* codes, float* scales, void* ws,
+                          size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (rows < 1 || cols <= 0 || cols % 16 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (x_bf16 == nullptr || codes == nullptr || scales == nullptr || ws == nullptr) return NVFP4MOE_ERR_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(codes, 8) || !aligned(scales, 4) || !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  const QuantWs q = carve_quant(ws);
+  if (ws_bytes < q.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  Fp8RowsArgs fa{static_cast<const uint16_t*>(x_bf16), rows, cols, codes, scales, &q.hdr->status};
+  if (launch_fp8_quantize_rows(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches = 1;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_fp8_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_fp8_experts** out) {
+  if (out == nullptr) return NVFP4MOE_ERR_ARG;
+  *out = nullptr;
+  int st = nvfp4moe_cfg_check(cfg);
+  if (st != NVFP4MOE_OK) return st;
+  st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  nvfp4moe_fp8_experts* x = new nvfp4moe_fp8_experts();
+  std::memset(x, 0, sizeof(*x));
+  x->cfg = *cfg;
+  cudaGetDevice(&x->device);
+  const int64_t E = cfg->E, H = cfg->H, I = cfg->I;
+  const size_t w13 = (size_t)E * 2 * I * H, wd = (size_t)E * H * I;
+  const bool ok = cudaMalloc(&x->w13_codes, w13) == cudaSuccess && cudaMalloc(&x->wd_codes, wd) == cudaSuccess &&
+                  cudaMalloc(&x->w13_scale, (size_t)E * 2 * I * sizeof(float)) == cudaSuccess &&
+                  cudaMalloc(&x->wd_scale, (size_t)E * H * sizeof(float)) == cudaSuccess &&
+                  cudaMemset(x->w13_codes, 0, w13) == cudaSuccess && cudaMemset(x->wd_codes, 0, wd) == cudaSuccess &&
+                  cudaMemset(x->w13_scale, 0, (size_t)E * 2 * I * sizeof(float)) == cudaSuccess &&
+                  cudaMemset(x->wd_scale, 0, (size_t)E * H * sizeof(float)) == cudaSuccess;
+  if (!ok) {
+    nvfp4moe_fp8_experts_destroy(x);
+    return NVFP4MOE_ERR_CUDA;
+  }
+  *out = x;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_fp8_experts_set(nvfp4moe_fp8_experts* x, int32_t e, const nvfp4moe_fp8_expert_tensors* t,
+                             void* stream) {
+  g_launches = 0;
+  if (x == nullptr || t == nullptr) return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = x->cfg;
+  if (e < 0 || e >= c.E) return NVFP4MOE_ERR_ARG;
+  if (!t->gate_codes || !t->gate_scales || !t->up_codes || !t->up_scales || !t->down_codes || !t->down_scales)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(t->gate_codes, 16) || !aligned(t->up_codes, 16) || !aligned(t->down_codes, 16))
+    return NVFP4MOE_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t H = c.H, I = c.I;
+  constexpr int kG = kWeightTileRows / 2;
+  uint8_t* w13 = x->w13_codes + (size_t)e * 2 * I * H;
+  // gate/up rows interleaved in groups of 64 (packed group 2j: gate rows [64j, 64j+64), 2j+1: up rows)
+  if (launch_tile_weights(t->gate_codes, (int)I, (int)H, w13, kG, 2, 0, s) != cudaSuccess ||
+      launch_tile_weights(t->up_codes, (int)I, (int)H, w13, kG, 2, 1, s) != cudaSuccess ||
+      launch_tile_weights(t->down_codes, (int)H, (int)I, x->wd_codes + (size_t)e * H * I, (int)H, 1, 0, s) !=
+          cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  float* sc = x->w13_scale + (size_t)e * 2 * I;
+  const size_t gb = kG * sizeof(float);
+  if (cudaMemcpy2DAsync(sc, 2 * gb, t->gate_scales, gb, gb, I / kG, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpy2DAsync(sc + kG, 2 * gb, t->up_scales, gb, gb, I / kG, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(x->wd_scale + (size_t)e * H, t->down_scales, H * sizeof(float), cudaMemcpyDeviceToDevice,
+                      s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  g_launches = 3;
+  return NVFP4MOE_OK;
+}
+
+void nvfp4moe_fp8_experts_destroy(nvfp4moe_fp8_experts* x) {
+  if (x == nullptr) return;
+  cudaFree(x->w13_codes);
+  cudaFree(x->w13_scale);
+  cudaFree(x->wd_codes);
+  cudaFree(x->wd_scale);
+  delete x;
+}
+
+size_t nvfp4moe_forward_fp8_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) {
+  if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || T_max < 1) return 0;
+  return carve_forward_fp8(nullptr, *cfg, T_max).bytes;
+}
+
+int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
+                         const float* logit_bias, void* out_bf16, const nvfp4moe_debug* dbg, void* ws,
+                         size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (x == nullptr) return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = x->cfg;
+  if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
+  if (hidden_bf16 == nullptr || w_router == nullptr || out_bf16 == nullptr || ws == nullptr)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(out_bf16, 16) || !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  const ForwardFp8Ws f = carve_forward_fp8(ws, c, T);
+  if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t pairs = T * c.topk;
+  CUtensorMap tma_a, tma_a32, tma_h, tma_h32;
+  if (make_tma_2d(&tma_a, f.a_codes, c.H, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_a32, f.a_codes, c.H, f.rows_cap, 32) != 0 ||
+      make_tma_2d(&tma_h, f.hq, c.I, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_h32, f.hq, c.I, f.rows_cap, 32) != 0)
+    return NVFP4MOE_ERR_CUDA;
+  if (cudaMemsetAsync(&f.hdr->status, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+
+  RouterArgs r{};
+  r.x = static_cast<const uint16_t*>(hidden_bf16);
+  r.w = w_router;
+  r.bias = logit_bias;
+  r.parts = f.parts;
+  r.idx = f.idx;
+  r.wts = f.wts;
+  r.T = T;
+  r.H = c.H;
+  r.E = c.E;
+  r.n_groups = c.n_groups;
+  r.topk_groups = c.topk_groups;
+  r.topk = c.topk;
+  r.routed_scale = c.routed_scale;
+  r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
+  r.amax_partials = f.partials;
+  r.status = &f.hdr->status;
+  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 2;
+
+  PermArgs pa{};
+  pa.idx = f.idx;
+  pa.T = T;
+  pa.topk = c.topk;
+  pa.E = c.E;
+  pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
+  pa.chunk_counts = f.chunk_counts;
+  pa.chunk_base = f.chunk_base;
+  pa.counts = f.counts;
+  pa.offsets = f.offsets;
+  pa.mtile_prefix = f.mtile_prefix;
+  pa.perm = f.perm;
+  pa.inv = f.inv;
+  pa.row_pair = f.row_pair;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+
+  Fp8ScatterArgs qa{static_cast<const uint16_t*>(hidden_bf16), T, c.H, c.topk, f.idx, f.inv, f.offsets,
+                    f.mtile_prefix, f.a_codes, f.a_scale, f.acc,
+                    dbg != nullptr ? dbg->xq8_codes : nullptr, dbg != nullptr ? dbg->xq8_scales : nullptr,
+                    &f.hdr->status};
+  if (launch_fp8_quantize_scatter(qa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+
+  const int grid = num_sms();
+  const bool decode_cfg = T * c.topk < 32 * c.E;
+  GemmArgs g{};
+  g.b_tiles = x->w13_codes;
+  g.mtile_prefix = f.mtile_prefix;
+  g.counts = f.counts;
+  g.E = c.E;
+  g.K = c.H;
+  g.n_total = 2 * c.I;
+  g.status = &f.hdr->status;
+  g.I = c.I;
+  g.acc = f.acc;
+  g.row_pair = f.row_pair;
+  g.wts = f.wts;
+  g.topk = c.topk;
+  g.H = c.H;
+  g.a_scale = f.a_scale;
+  g.w_scale = x->w13_scale;
+  g.h32 = f.h32;
+  if (launch_gemm_gateup_fp8(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  Fp8RequantArgs ra{f.h32, f.rows_cap, c.I, f.row_pair, f.mtile_prefix, c.E, f.hq, f.h_scale, &f.hdr->status};
+  if (launch_fp8_requant_rows(ra, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g.b_tiles = x->wd_codes;
+  g.K = c.I;
+  g.n_total = c.H;
+  g.w_scale = x->wd_scale;
+  g.h_scale = f.h_scale;
+  if (launch_gemm_down_fp8(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, nullptr, 0.0f, 0.0f};
+  if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 4;
+
+  if (dbg != nullptr) {
+    bool ok = true;
+    if (dbg->idx) ok &= cudaMemcpyAsync(dbg->idx, f.idx, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->w) ok &= cudaMemcpyAsync(dbg->w, f.wts, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->counts) ok &= cudaMemcpyAsync(dbg->counts, f.counts, c.E * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->offsets)
+      ok &= cudaMemcpyAsync(dbg->offsets, f.offsets, (c.E + 1) * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (dbg->perm) ok &= cudaMemcpyAsync(dbg->perm, f.perm, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (!ok) return NVFP4MOE_ERR_CUDA;
+  }
+  return NVFP4MOE_OK;
 }
 
 int nvfp4moe_status_read(const void* ws, void* stream) {

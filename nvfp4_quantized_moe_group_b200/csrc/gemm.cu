@@ -54,23 +54,30 @@ constexpr int kNT = kN / 128;                       // 128-row weight tiles per 
 // frees the accumulator after its first 32-feature chunk, and the down GEMM stages 32-column
 // pieces through shared memory (whole 128-byte row pieces per reduction, 3 stages): both
 // measured faster there.
-template <bool kGateUp, bool kDecode>
+//
+// kFp8: the FP8 W8A8 variant (E4M3 x E4M3 with FP32 accumulation, kind::f8f6f4): a 128-byte
+// K block holds 128 values instead of 256, there are no block scales (per-row activation and
+// per-channel weight scales are applied in the epilogue), and gate/up writes h in FP32 for
+// the per-row requantisation that follows.
+template <bool kGateUp, bool kDecode, bool kFp8>
 struct Cfg {
   static constexpr int kStages = (kGateUp || kDecode) ? 4 : 3;
   static constexpr bool kStaging = !kGateUp && !kDecode;
   static constexpr uint32_t kSfCol0 = kN;                        // the accumulator first
-  static constexpr uint32_t kSfColsA = 16;                       // 4 K steps x 4 columns
-  static constexpr uint32_t kSfColsPerStage = kSfColsA + 16 * kNT;
+  static constexpr uint32_t kSfColsA = kFp8 ? 0 : 16;            // 4 K steps x 4 columns
+  static constexpr uint32_t kSfColsPerStage = kFp8 ? 0 : kSfColsA + 16 * kNT;
+  static constexpr int kSfaBytes = kFp8 ? 16 : 4 * kAtomBytes;
+  static constexpr int kSfbBytes = kFp8 ? 16 : kNT * 4 * kAtomBytes;
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory columns");
 };
 
-template <bool kGateUp, bool kDecode>
+template <bool kGateUp, bool kDecode, bool kFp8>
 struct __align__(1024) Smem {
-  using C = Cfg<kGateUp, kDecode>;
+  using C = Cfg<kGateUp, kDecode, kFp8>;
   uint8_t a[C::kStages][kABytes];
   uint8_t b[C::kStages][kNT * kTileBytes];
-  uint8_t sfa[C::kStages][4 * kAtomBytes];
-  uint8_t sfb[C::kStages][kNT * 4 * kAtomBytes];
+  uint8_t sfa[C::kStages][C::kSfaBytes];
+  uint8_t sfb[C::kStages][C::kSfbBytes];
   float stage_out[C::kStaging ? kEpiWarps : 1][32][33];  // down, full segments: per epilogue warp
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
@@ -100,6 +107,22 @@ __device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r)
         "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
         "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
       : "r"(taddr));
+}
+
+// tcgen05.mma kind::f8f6f4, E4M3 x E4M3 -> FP32, K = 32 (both operands K-major).
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f8f6f4: FP32 accumulator (bits 4-5 = 1), A and B formats
+// E4M3 (bits 7-9, 10-12 = 0), both K-major, N / 8 at bit 17, M / 16 (128) at bit 24.
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t n) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 __device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
@@ -181,13 +204,13 @@ __device__ __forceinline__ void quant_store32(const float* h, float gh, float r_
   }
 }
 
-template <bool kGateUp, bool kDecode>
+template <bool kGateUp, bool kDecode, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a32,
                 const GemmArgs p) {
-  using C = Cfg<kGateUp, kDecode>;
+  using C = Cfg<kGateUp, kDecode, kFp8>;
   constexpr int kStages = C::kStages;
-  using S = Smem<kGateUp, kDecode>;
+  using S = Smem<kGateUp, kDecode, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   S& s = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
@@ -220,7 +243,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   const int ntn = p.n_total / kN;           // 256-wide items per expert
   const int ntn128 = p.n_total / 128;       // 128-row weight tiles per expert
   const int total = __ldg(p.mtile_prefix + p.E) * ntn;
-  const int kb_count = (p.K + kBlockK - 1) / kBlockK;
+  const int kb_count = kFp8 ? (p.K + 127) / 128 : (p.K + kBlockK - 1) / kBlockK;   // 128-byte K blocks
   const int k64 = p.K / 64;  // scale-column tiles of A and B
 
   if (warp == 0) {
@@ -247,17 +270,18 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             break;
           }
           const int left = (p.K - kb * kBlockK) / 64;
-          const uint32_t sf_bytes = (uint32_t)(left < 4 ? left : 4) * kAtomBytes;
+          const uint32_t sf_bytes = kFp8 ? 0u : (uint32_t)(left < 4 ? left : 4) * kAtomBytes;
           mbar_arrive_expect_tx(&s.full[stage], a_bytes + kNT * (kTileBytes + sf_bytes) + sf_bytes);
           tma_load_2d(s.a[stage], a_small ? (const void*)&tma_a32 : (const void*)&tma_a, &s.full[stage],
                       kb * 128, arow, pol_a);
-          bulk_load(s.sfa[stage], sfa + kb * 4 * kAtomBytes, sf_bytes, &s.full[stage], pol_a);
+          if constexpr (!kFp8) bulk_load(s.sfa[stage], sfa + kb * 4 * kAtomBytes, sf_bytes, &s.full[stage], pol_a);
 #pragma unroll
           for (int j = 0; j < kNT; ++j) {
             bulk_load(s.b[stage] + j * kTileBytes, btile + ((int64_t)j * kb_count + kb) * kTileBytes, kTileBytes,
                       &s.full[stage], pol_w);
-            bulk_load(s.sfb[stage] + j * 4 * kAtomBytes, sfb + ((int64_t)j * k64 + kb * 4) * kAtomBytes, sf_bytes,
-                      &s.full[stage], pol_w);
+            if constexpr (!kFp8)
+              bulk_load(s.sfb[stage] + j * 4 * kAtomBytes, sfb + ((int64_t)j * k64 + kb * 4) * kAtomBytes, sf_bytes,
+                        &s.full[stage], pol_w);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -274,7 +298,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     __syncwarp();
     if (elect_one()) {
       uint32_t stage = 0, phase = 0;
-      const uint32_t idesc = idesc_nvf4(kN);
+      const uint32_t idesc = kFp8 ? idesc_f8(kN) : idesc_nvf4(kN);
       bool ok = true;
       int it = 0;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
@@ -292,6 +316,16 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             break;
           }
           tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a[stage]);
+          const uint32_t b0 = smem_u32(s.b[stage]);
+          if constexpr (kFp8) {
+            // four K = 32 instructions per 128-byte K block (32 bytes apart, like the FP4 steps)
+            for (int k = 0; k < 4; ++k)
+              mma_f8(acc, desc_k_sw128(a0 + 32 * k), desc_k_sw128(b0 + 32 * k), idesc, (kb | k) != 0 ? 1u : 0u);
+            tc_commit(&s.empty[stage]);
+            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            continue;
+          }
           const int left = (p.K - kb * kBlockK) / 64;
           const int ksteps = left < 4 ? left : 4;
           // scale atoms: A at sfa_t + 4k; B (row n at lane n % 32, column n / 32) at
@@ -306,8 +340,6 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             for (int j = 0; j < kNT; ++j)
               tc_cp_32x128b_x4(sfb_t + 4 * (kNT * k + j), desc_sf_block(sb + (j * 4 + k) * kAtomBytes));
           }
-          const uint32_t a0 = smem_u32(s.a[stage]);
-          const uint32_t b0 = smem_u32(s.b[stage]);
           for (int k = 0; k < ksteps; ++k) {
             mma_nvf4(acc, desc_k_sw128(a0 + 32 * k), desc_k_sw128(b0 + 32 * k), idesc, sfa_t + 4 * k,
                      sfb_t + 4 * kNT * k, (kb | k) != 0 ? 1u : 0u);
@@ -339,7 +371,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       float c0s = 0.f, c1s = 0.f, c2s = 0.f;
       int token = -1;
       if (warp_live) {
-        if constexpr (kGateUp) {
+        if constexpr (kGateUp && kFp8) {
+          c0s = p.a_scale[row];                       // the token's activation scale
+        } else if constexpr (kGateUp) {
           const float gx = *p.g_x;
           c0s = __fmul_rn(gx, p.g_gate[wk.e]);
           c1s = __fmul_rn(gx, p.g_up[wk.e]);
@@ -347,7 +381,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         } else {
           const int pair = valid ? p.row_pair[row] : -1;
           if (pair >= 0) {
-            c0s = __fmul_rn(p.alpha_down[wk.e], p.wts[pair]);
+            c0s = kFp8 ? __fmul_rn(p.wts[pair], p.h_scale[row]) : __fmul_rn(p.alpha_down[wk.e], p.wts[pair]);
             token = pair / p.topk;
           }
         }
@@ -368,6 +402,32 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       };
       if (!warp_live) {
         release();
+      } else if constexpr (kGateUp && kFp8) {
+        // h = silu(acc_g * sx * wg) * (acc_u * sx * wu) per feature, stored in FP32
+        const int t = wk.nt * kNT + half;             // weight tile of this warp's 64 features
+        const int tcol = half * 128;
+        const float* wsc = p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + tcol;
+        const float sx = c0s;
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+          uint32_t G[32], U[32];
+          tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
+          tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
+          tmem_ld_wait();
+          if (pr == 1) release();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gv = __fmul_rn(__fmul_rn(__uint_as_float(G[i]), sx), __ldg(wsc + 32 * pr + i));
+            const float uv = __fmul_rn(__fmul_rn(__uint_as_float(U[i]), sx), __ldg(wsc + 64 + 32 * pr + i));
+            h[i] = __fmul_rn(__fmul_rn(gv, uv), rcp_approx(__fadd_rn(1.0f, __expf(-gv))));
+          }
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(p.h32 + row * p.I + t * 64 + 32 * pr);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
+        }
       } else if constexpr (kGateUp) {
         const float sg = c0s, su = c1s, gh = c2s;
         const float r_t = __frcp_rn(__fmul_rn(6.0f, gh));
@@ -422,10 +482,18 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             const float sc = __shfl_sync(0xffffffffu, c0s, r);
             if (tok >= 0) {
               float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + half * (kN / 2) + cq;
+              const float* wsc = kFp8 ? p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + half * (kN / 2) + cq
+                                      : nullptr;
 #pragma unroll
-              for (int k = 0; k < 16; ++k)
-                red_add_v2(dst + 8 * k, __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr]), sc),
-                           __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr + 1]), sc));
+              for (int k = 0; k < 16; ++k) {
+                float v0 = __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr]), sc);
+                float v1 = __fmul_rn(__uint_as_float(V[lh][4 * k + 2 * rr + 1]), sc);
+                if constexpr (kFp8) {
+                  v0 = __fmul_rn(v0, __ldg(wsc + 8 * k));
+                  v1 = __fmul_rn(v1, __ldg(wsc + 8 * k + 1));
+                }
+                red_add_v2(dst + 8 * k, v0, v1);
+              }
             }
           }
         }
@@ -452,7 +520,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             const int tok = __shfl_sync(0xffffffffu, token, r);
             if (tok >= 0) {
               float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + c0 + col;
-              red_add_v4(dst, st[r][col], st[r][col + 1], st[r][col + 2], st[r][col + 3]);
+              if constexpr (kFp8) {
+                const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + (int64_t)wk.e * p.n_total +
+                                                                        wk.nt * kN + c0 + col));
+                red_add_v4(dst, __fmul_rn(st[r][col], w4.x), __fmul_rn(st[r][col + 1], w4.y),
+                           __fmul_rn(st[r][col + 2], w4.z), __fmul_rn(st[r][col + 3], w4.w));
+              } else {
+                red_add_v4(dst, st[r][col], st[r][col + 1], st[r][col + 2], st[r][col + 3]);
+              }
             }
           }
           __syncwarp();
@@ -469,14 +544,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   }
 }
 
-template <bool kGateUp, bool kDecode>
+template <bool kGateUp, bool kDecode, bool kFp8 = false>
 cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a, int grid,
                         cudaStream_t stream) {
-  const size_t smem = sizeof(Smem<kGateUp, kDecode>) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode>,
+  const size_t smem = sizeof(Smem<kGateUp, kDecode, kFp8>) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  moe_gemm_kernel<kGateUp, kDecode><<<grid, kThreads, smem, stream>>>(tma_a, tma_a32, a);
+  moe_gemm_kernel<kGateUp, kDecode, kFp8><<<grid, kThreads, smem, stream>>>(tma_a, tma_a32, a);
   return cudaGetLastError();
 }
 
@@ -499,10 +574,14 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-static_assert(sizeof(Smem<true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<true, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<false, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                                int grid, bool decode, cudaStream_t stream) {
@@ -514,6 +593,18 @@ cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a3
                              int grid, bool decode, cudaStream_t stream) {
   return decode ? launch_gemm<false, true>(tma_a, tma_a32, a, grid, stream)
                 : launch_gemm<false, false>(tma_a, tma_a32, a, grid, stream);
+}
+
+cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
+                                   int grid, bool decode, cudaStream_t stream) {
+  return decode ? launch_gemm<true, true, true>(tma_a, tma_a32, a, grid, stream)
+                : launch_gemm<true, false, true>(tma_a, tma_a32, a, grid, stream);
+}
+
+cudaError_t launch_gemm_down_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
+                                 int grid, bool decode, cudaStream_t stream) {
+  return decode ? launch_gemm<false, true, true>(tma_a, tma_a32, a, grid, stream)
+                : launch_gemm<false, false, true>(tma_a, tma_a32, a, grid, stream);
 }
 
 int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {

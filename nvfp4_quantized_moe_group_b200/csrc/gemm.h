@@ -37,6 +37,11 @@ struct GemmArgs {
   const float* alpha_down;     // [E] = g_h * g_down
   int topk;
   int H;
+  // FP8 variant (per-row activation scales, per-output-channel weight scales)
+  const float* a_scale;        // gate/up: [rows_cap] scale of each segment row of A
+  const float* w_scale;        // [E][n_total] weight channel scales (gate/up in packed column order)
+  float* h32;                  // gate/up: [rows_cap][I] FP32 SwiGLU product
+  const float* h_scale;        // down: [rows_cap] scale of each segment row of A (= h)
 };
 
 // gemm.cu
@@ -47,6 +52,12 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_
                                int grid, bool decode, cudaStream_t stream);
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                              int grid, bool decode, cudaStream_t stream);
+// The FP8 W8A8 variants: A and B are E4M3 rows of K bytes (tensor maps over K-byte rows), the
+// scales come from a_scale / w_scale / h_scale, and gate/up writes FP32 h to h32.
+cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
+                                   int grid, bool decode, cudaStream_t stream);
+cudaError_t launch_gemm_down_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
+                                 int grid, bool decode, cudaStream_t stream);
 // Weight codes [rows][row_bytes] -> tiled operand layout: source row r is packed row
 // (r / group) * group * mul + add * group + r % group; packed rows form 128-row tiles, each
 // split into 128-byte K blocks stored as contiguous 16 KB images of the 128-byte-swizzled

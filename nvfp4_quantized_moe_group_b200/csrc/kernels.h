@@ -166,6 +166,44 @@ struct LhArgs {
 };
 cudaError_t launch_lh_quantize(const LhArgs& a, cudaStream_t stream);
 
+// fp8.cu: per-row E4M3 quantisation for the FP8 W8A8 variant.
+struct Fp8RowsArgs {
+  const uint16_t* x;       // [rows][cols] bf16, cols % 8 == 0
+  int64_t rows, cols;
+  uint8_t* codes;          // [rows][cols]
+  float* scales;           // [rows]
+  uint32_t* status;
+};
+struct Fp8ScatterArgs {
+  const uint16_t* x;       // [T][H] bf16
+  int64_t T;
+  int H, topk;
+  const int32_t* idx;
+  const int32_t* inv;
+  const int32_t* offsets;
+  const int32_t* mtile_prefix;
+  uint8_t* seg_codes;      // [rows_cap][H]
+  float* seg_scale;        // [rows_cap]
+  float* acc;              // [T][H], zeroed
+  uint8_t* xq_codes;       // optional [T][H]
+  float* xq_scales;        // optional [T]
+  uint32_t* status;
+};
+struct Fp8RequantArgs {
+  const float* h;          // [rows][I] FP32
+  int64_t rows;            // capacity of the buffers (grid size)
+  int I;
+  const int32_t* row_pair; // rows with a pair (>= 0) are quantised
+  const int32_t* mtile_prefix;  // [E+1]: rows past mtile_prefix[E] * 128 hold no segment
+  int E;
+  uint8_t* codes;          // [rows][I]
+  float* scales;           // [rows]
+  uint32_t* status;
+};
+cudaError_t launch_fp8_quantize_rows(const Fp8RowsArgs& a, cudaStream_t stream);
+cudaError_t launch_fp8_quantize_scatter(const Fp8ScatterArgs& a, cudaStream_t stream);
+cudaError_t launch_fp8_requant_rows(const Fp8RequantArgs& a, cudaStream_t stream);
+
 // permute.cu
 // Grouping kernels: one kernel when T * topk <= kPermSmallPairs, else three.
 constexpr int kPermSmallPairs = 4096;

@@ -170,3 +170,46 @@ def requant_near_tie(h: np.ndarray, g_h: float, rel=1e-4) -> tuple[np.ndarray, n
     dv = np.min(np.abs(v[..., None] - E2M1_MIDS), axis=-1)
     elem_tie = (dv <= rel * np.maximum(v, 0.25)) | (v <= rel)
     return block_tie.reshape(h.shape[:-1] + (n // 16,)), elem_tie.reshape(h.shape)
+
+
+# ------------------------------------------------------------------ FP8 W8A8 ----
+
+def oracle_expert_fp8(shape, e: int, seed: int = 0):
+    """Expert e quantised per output channel by the oracle (FP8 W8A8 variant)."""
+    return tuple(oracle.fp8.Fp8Tensor(expert_weight(shape, e, w, seed=seed).float().numpy())
+                 for w in ("gate", "up", "down"))
+
+
+def _expert_job_fp8(args):
+    shape, e, xhat = args
+    return e, oracle.fp8.expert_mlp_fp8(xhat, *oracle_expert_fp8(shape, e))["y"]
+
+
+def oracle_layer_fp8(shape, x: np.ndarray, wr: np.ndarray, bias, tokens=None, workers=None):
+    """oracle.fp8.moe_forward_fp8 for the given tokens, its experts evaluated in a spawn
+    process pool when there are many (same steps, same functions)."""
+    cfg = cfg_ns(shape)
+    r = oracle.route(x, wr, cfg, bias)
+    xq, xs = oracle.fp8.quantize_rows(np.asarray(x, dtype=np.float32))
+    T = x.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    need = {}
+    for i, t in enumerate(tokens):
+        for j in range(cfg.topk):
+            need.setdefault(int(r.idx[t, j]), []).append((i, int(t), j))
+    jobs = []
+    for e, rows in sorted(need.items()):
+        ts = np.array([t for _, t, _ in rows])
+        jobs.append((shape, e, oracle.fp8.dequantize_rows(xq[ts], xs[ts])))
+    if workers is None:
+        workers = min(len(jobs), max(1, len(os.sched_getaffinity(0)) // 2)) if len(jobs) > 8 else 1
+    if workers > 1:
+        with mp.get_context("spawn").Pool(workers) as pool:
+            results = pool.map(_expert_job_fp8, jobs)
+    else:
+        results = [_expert_job_fp8(j) for j in jobs]
+    out = np.zeros((len(tokens), x.shape[1]))
+    for e, y in results:
+        for n, (i, t, j) in enumerate(need[e]):
+            out[i] += r.w[t, j] * y[n]
+    return {"route": r, "xq_codes": xq, "xq_scales": xs, "tokens": tokens, "out": out}
