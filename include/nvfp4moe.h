@@ -228,7 +228,11 @@ NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_
  *   logit_bias [E] FP32 or NULL;  out_bf16 [T][H] BF16 (out).
  *   dbg  NULL on the hot path.  Otherwise every non-NULL member receives a copy of that
  *        intermediate (sizes below), for checking the layer step by step.
- *   ws   workspace of nvfp4moe_forward_workspace_bytes(cfg, T_max) bytes. */
+ *   ws   workspace of nvfp4moe_forward_workspace_bytes(cfg, T_max) bytes.
+ * The grouped GEMMs and finalize are launched with programmatic stream serialization: each may
+ * be scheduled onto SMs its predecessor has left and waits on the device for that kernel's
+ * results, so a kernel's set-up overlaps the previous one's tail.  Stream order is kept:
+ * work enqueued after the call sees the finished output. */
 /* Stages of nvfp4moe_forward (for nvfp4moe_debug.events).  Launch order: ROUTE, PERMUTE,
  * QUANTIZE, GATEUP, DOWN, FINALIZE.  The input's global amax is computed inside ROUTE and
  * the rows are written into the expert segments inside QUANTIZE, so the AMAX and GATHER

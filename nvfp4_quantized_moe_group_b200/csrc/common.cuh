@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -98,6 +99,17 @@ __device__ __forceinline__ float global_scale_from_amax(float a) {
 __host__ __device__ __forceinline__ int64_t swz_offset(int64_t r, int64_t c, int64_t n_col_tiles) {
   return ((r >> 7) * n_col_tiles + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
 }
+
+// ------------------------------------------------- programmatic dependent launch ----
+// A kernel launched with programmatic stream serialization (launch_pdl) may be scheduled while
+// the previous kernel of the stream is still running.  pdl_wait() returns once that kernel has
+// completed and its memory operations are visible; such a kernel calls it before reading
+// anything the previous kernels wrote.  Without a programmatic predecessor it returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream, if launched with programmatic serialization, be scheduled
+// (onto free SM resources, where it waits in pdl_wait) once every CTA of this grid has executed
+// this or exited.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ----------------------------------------------------------------- timing ----
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -307,6 +319,24 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
                "f"(d)
                : "memory");
+}
+
+// Launches `kernel` with programmatic stream serialization: it may start while the previous
+// kernel of `stream` runs (it must call pdl_wait() before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace nvfp4moe

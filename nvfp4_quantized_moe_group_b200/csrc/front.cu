@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(FrontArgs a) {
   const int tid = threadIdx.x;
   const int nb = gridDim.x;
   const int T = (int)a.T, E = a.E, H = a.H, topk = a.topk;
+  // the gate/up GEMM that follows may take the SMs this grid leaves free and set up there
+  pdl_trigger();
 
   // ---------------------------------------------------------------- phase 1: logits --
   // CTA b: experts [64 * (b % n_etiles), +64), K slice b / n_etiles.  Thread (ts, eq, kq):

@@ -238,6 +238,11 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched programmatically: everything above overlapped the previous kernel's tail; the
+  // routing tables and the A operand are read only after it has completed.  The next kernel
+  // may then be scheduled onto SMs as this grid's CTAs exit.
+  pdl_wait();
+  pdl_trigger();
 
   const uint32_t tmem = s.tmem_base;
   const int ntn = p.n_total / kN;           // 256-wide items per expert
@@ -551,8 +556,8 @@ cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, co
   cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  moe_gemm_kernel<kGateUp, kDecode, kFp8><<<grid, kThreads, smem, stream>>>(tma_a, tma_a32, a);
-  return cudaGetLastError();
+  return launch_pdl(moe_gemm_kernel<kGateUp, kDecode, kFp8>, dim3(grid), dim3(kThreads), smem, stream, tma_a,
+                    tma_a32, a);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

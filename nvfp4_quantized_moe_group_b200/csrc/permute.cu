@@ -177,6 +177,7 @@ cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream, int* launches
 // numerical decisions"); 8 values per thread.  res may alias out: each thread reads its 8
 // residual values before it writes them.
 __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
+  pdl_wait();   // launched programmatically after the down GEMM
   const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8;
   if (i >= a.n) return;
   const float4 p = *reinterpret_cast<const float4*>(a.acc + i);
@@ -204,8 +205,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a) {
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream) {
   if (a.n == 0) return cudaSuccess;
   const int64_t threads = a.n / 8;
-  finalize_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(finalize_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, a);
 }
 
 // Linear [n_rows][cols16] scales from swizzled storage: row i of the output is row
