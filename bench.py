@@ -238,11 +238,13 @@ def run_fp8(moe, shape: LayerShape, cfg, x, wr, bias, T: int, steps: int, warmup
     torch.cuda.synchronize()
     barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed_fp8")
     f0.record()
     for _ in range(steps):
         moe.forward_fp8(ex, x, wr, bias, out=out, ws=ws)
     f1.record()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     barrier(world)
     ms = max_over_ranks(f0.elapsed_time(f1), world) / steps
     st = moe.status_read(ws)
