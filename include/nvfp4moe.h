@@ -151,13 +151,25 @@ NVFP4MOE_API int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, 
  *   idx  out [T][topk] int32: selected experts by score descending, equal scores by
  *        lower expert index (the same rule picks the groups).
  *   w    out [T][topk] FP32: routed_scale * s / sum(selected s).
- * Logits: FP32 products accumulated in FP32 so that every product passes through at most
- * 32 FP32 roundings (FMA chains of at most 32 products, or of at most 20 products added by
- * a 3-level FP32 tree); these partial sums, the split-K parts and the bias are added in
- * FP64 and the logit is rounded to FP32 once, so
- * |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
+ * Logits, T <= 64: FP32 products accumulated in FP32 so that every product passes through
+ * at most 32 FP32 roundings (FMA chains of at most 32 products, or of at most 20 products
+ * added by a 3-level FP32 tree); these partial sums, the split-K parts and the bias are
+ * added in FP64 and the logit is rounded to FP32 once, so
+ *   |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
+ * Logits, T > 64: exact integer arithmetic on the tensor cores.  Token row x_t and expert
+ * row W_e are scaled by powers of two to 30-bit fixed point (e_x, e_W: the binary exponents
+ * with max|x_t| < 2^e_x, max|W_e| < 2^e_W) and rounded to integers, split into four int8
+ * digits each, and the 13 most significant digit-pair products are summed in int32 (exact);
+ * the classes, split-K parts and bias are added in FP64 and the logit is rounded to FP32
+ * once, so
+ *   |logit - exact| <= 2^-24 |logit| + 2^(e_x - 31) sum_h |W_eh| + 2^(e_W - 31) sum_h |x_h|
+ *                      + H 2^(e_x + e_W - 36)
+ * (the first two terms are the fixed-point roundings; the last covers the dropped digit
+ * pairs, the product of the two roundings and the FP64 additions); for Beam's shapes this
+ * is about 200 times below the FP32 bound.  A token or expert row with a non-finite element
+ * makes its logits NaN.
  * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same arithmetic
- * and bound (for T <= 64 in its fused front-end kernel).  A NaN logit raises
+ * and bounds (for T <= 64 in its fused front-end kernel).  A NaN logit raises
  * NVFP4MOE_ERR_NONFINITE in the status word and ranks below every finite score. */
 NVFP4MOE_API size_t nvfp4moe_route_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
 NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T,
@@ -171,8 +183,10 @@ NVFP4MOE_API int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16
  * device allocation and gives the libraries it embeds no allocator.  Such a caller has no
  * workspace to pass to nvfp4moe_route.
  *
- * Same arguments and results as nvfp4moe_route (same kernels, identical idx and w), minus
- * the workspace.  The router's scratch is a fixed array of 9,699,584 bytes of device memory
+ * Same arguments and results as nvfp4moe_route, minus the workspace; for T > 64 it computes
+ * the logits with the FP32 kernel and bound of the T <= 64 path (the integer path's digit
+ * planes would not fit the fixed scratch), so idx can differ from nvfp4moe_route's where two
+ * scores lie within that bound.  The router's scratch is a fixed array of 9,699,584 bytes of device memory
  * declared by the library; every GPU that loads the library holds it until the process
  * exits.  Limit: the split-K partial sums must fit, which holds whenever T * E <= 1,212,416
  * (T <= 4736 for 256 experts); larger calls return NVFP4MOE_ERR_WORKSPACE and enqueue

@@ -82,9 +82,36 @@ QuantWs carve_quant(void* ws) {
   return q;
 }
 
+// Scratch of the integer tensor-core router (T >= kRouterTcMinT): digit planes of the expert
+// rows and the row exponents.  The token rows' planes (4 T H bytes) go to a buffer the caller
+// names (in the forward, the expert-segment input buffer, which is written only afterwards).
+struct RouterTcWs {
+  uint8_t* w_digits = nullptr;
+  int32_t* x_exp = nullptr;
+  int32_t* w_exp = nullptr;
+};
+
+RouterTcWs carve_router_tc(Carver& c, const nvfp4moe_cfg& cfg, int64_t T) {
+  RouterTcWs r;
+  if (T < kRouterTcMinT) return r;
+  r.w_digits = c.take<uint8_t>((size_t)4 * cfg.E * cfg.H);
+  r.x_exp = c.take<int32_t>(T);
+  r.w_exp = c.take<int32_t>(cfg.E);
+  return r;
+}
+
+void set_router_tc(RouterArgs& r, const RouterTcWs& w, uint8_t* x_digits) {
+  r.x_digits = w.w_digits != nullptr ? x_digits : nullptr;
+  r.w_digits = w.w_digits;
+  r.x_exp = w.x_exp;
+  r.w_exp = w.w_exp;
+}
+
 struct RouteWs {
   WsHeader* hdr;
   double* parts;
+  uint8_t* x_digits;
+  RouterTcWs tc;
   size_t bytes;
 };
 
@@ -93,6 +120,8 @@ RouteWs carve_route(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   RouteWs r;
   r.hdr = c.take<WsHeader>(1);
   r.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
+  r.x_digits = T >= kRouterTcMinT ? c.take<uint8_t>((size_t)4 * T * cfg.H) : nullptr;
+  r.tc = carve_router_tc(c, cfg, T);
   r.bytes = c.off;
   return r;
 }
@@ -126,6 +155,7 @@ struct ForwardWs {
   uint8_t* hq_codes;
   uint8_t* hq_sf;
   uint16_t* x_norm;        // residual forward: the normalised layer input
+  RouterTcWs tc;           // token-row digit planes alias a_codes (rows_cap H / 2 >= 4 T H)
   int64_t rows_cap;
   size_t bytes;
 };
@@ -164,6 +194,7 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg.I / 2);
   f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg.I / 16);
   f.x_norm = c.take<uint16_t>(T * cfg.H);
+  f.tc = carve_router_tc(c, cfg, T);
   f.bytes = c.off;
   return f;
 }
@@ -188,6 +219,7 @@ struct ForwardFp8Ws {
   float* h32;           // [rows_cap][I]
   uint8_t* hq;          // [rows_cap][I] E4M3
   float* h_scale;       // [rows_cap]
+  RouterTcWs tc;        // token-row digit planes alias a_codes (rows_cap H >= 4 T H)
   int64_t rows_cap;
   size_t bytes;
 };
@@ -218,6 +250,7 @@ ForwardFp8Ws carve_forward_fp8(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.h32 = c.take<float>(f.rows_cap * cfg.I);
   f.hq = c.take<uint8_t>(f.rows_cap * cfg.I);
   f.h_scale = c.take<float>(f.rows_cap);
+  f.tc = carve_router_tc(c, cfg, T);
   f.bytes = c.off;
   return f;
 }
@@ -396,8 +429,9 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   a.topk = cfg->topk;
   a.routed_scale = cfg->routed_scale;
   a.status = &r.hdr->status;
+  set_router_tc(a, r.tc, r.x_digits);
   if (launch_router(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  g_launches += 2;
+  g_launches += router_launch_count(a);
   return NVFP4MOE_OK;
 }
 
@@ -582,13 +616,14 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
     r.amax_partials = f.partials;
     r.status = &f.hdr->status;
+    set_router_tc(r, f.tc, f.a_codes);
     const int n_partials = router_amax_partials(T, c.E, c.H);
     ev.mark(NVFP4MOE_STAGE_AMAX, 0);
     ev.mark(NVFP4MOE_STAGE_AMAX, 1);
     ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
     if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
     ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
-    g_launches += 2;
+    g_launches += router_launch_count(r);
 
     // group the (token, slot) pairs by expert
     PermArgs pa{};
@@ -879,8 +914,9 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
   r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
   r.amax_partials = f.partials;
   r.status = &f.hdr->status;
+  set_router_tc(r, f.tc, f.a_codes);
   if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  g_launches += 2;
+  g_launches += router_launch_count(r);
 
   PermArgs pa{};
   pa.idx = f.idx;

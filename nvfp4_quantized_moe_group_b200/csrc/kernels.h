@@ -53,7 +53,14 @@ struct RouterArgs {
   uint32_t* amax_partials;  // optional: per-CTA max |x| (BF16 magnitude bits) for the global scale
   float* logits_out;        // optional [T][E]: the FP32 logits (bias included) the top-k used
   uint32_t* status;         // kStatusNonFinite is raised here for a NaN logit (may be nullptr)
+  // integer tensor-core logits (T >= kRouterTcMinT, when given; route_tc.cu)
+  uint8_t* x_digits;        // [4][T][H] int8 digit planes of the token rows
+  uint8_t* w_digits;        // [4][E][H] int8 digit planes of the expert rows
+  int32_t* x_exp;           // [T] row exponents (kExpNonFinite: the row has a non-finite value)
+  int32_t* w_exp;           // [E]
 };
+constexpr int kRouterTcMinT = 65;
+constexpr int32_t kExpNonFinite = 0x7FFFFFFF;
 
 struct PermArgs {
   const int32_t* idx;      // [T][topk]
@@ -130,12 +137,19 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 
 // route.cu
 int router_ksplit(int64_t T, int E, int H);
+// Kernels launch_router enqueues for these arguments.
+int router_launch_count(const RouterArgs& a);
 size_t router_parts_elems(int64_t T_max, int E, int H);
 // Number of amax partials the logits kernel writes for T tokens (grid x * split-K).
 int router_amax_partials(int64_t T, int E, int H);
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream);
 // The top-k stage alone (sums a.ksplit split-K parts of a.parts).
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);
+
+// route_tc.cu: logits in exact integer arithmetic on the tensor cores (digit planes, int8 MMAs)
+int router_tc_ksplit(int64_t T, int E, int H);
+int router_tc_amax_partials(int64_t T);
+cudaError_t launch_router_tc(RouterArgs a, cudaStream_t stream);
 
 
 

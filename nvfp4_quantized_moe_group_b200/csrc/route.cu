@@ -279,21 +279,32 @@ int router_ksplit(int64_t T, int E, int H) {
 
 size_t router_parts_elems(int64_t T_max, int E, int H) {
   size_t best = 0;
-  // ksplit depends on T only through the number of token tiles (64 or 128 tokens)
+  // ksplit depends on T only through the number of token tiles (64 or 128 tokens); the
+  // tensor-core path splits 128-token tiles
   for (int64_t c = 1; c <= (T_max + kTM - 1) / kTM; ++c) {
     const int64_t T = c * kTM < T_max ? c * kTM : T_max;
-    const size_t n = (size_t)router_ksplit(T, E, H) * (size_t)T * (size_t)E;
+    size_t n = (size_t)router_ksplit(T, E, H) * (size_t)T * (size_t)E;
+    if (T >= kRouterTcMinT) {
+      const size_t n_tc = (size_t)router_tc_ksplit(T, E, H) * (size_t)T * (size_t)E;
+      if (n_tc > n) n = n_tc;
+    }
     if (n > best) best = n;
   }
   return best;
 }
 
 int router_amax_partials(int64_t T, int E, int H) {
+  if (T >= kRouterTcMinT) return router_tc_amax_partials(T);
   const int tm = tile_tokens(T);
   return (int)((T + tm - 1) / tm) * router_ksplit(T, E, H);
 }
 
+int router_launch_count(const RouterArgs& a) {
+  return (a.T >= kRouterTcMinT && a.x_digits != nullptr) ? 4 : 2;
+}
+
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
+  if (a.T >= kRouterTcMinT && a.x_digits != nullptr) return launch_router_tc(a, stream);
   a.ksplit = router_ksplit(a.T, a.E, a.H);
   a.k_slice = a.H / a.ksplit;
   const int tm = tile_tokens(a.T);

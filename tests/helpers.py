@@ -34,14 +34,41 @@ def intermediate_scales(shape) -> np.ndarray:
 
 # ------------------------------------------------------------------ router ----
 
-def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
-    """Bound on |FP32 logit - exact| the library documents for nvfp4moe_route:
+def _row_exponents(v: np.ndarray) -> np.ndarray:
+    """Per row, the binary exponent e with max|v| < 2^e, at least -125 (the library's rule:
+    rows whose maximum is zero or subnormal take the smallest normal exponent)."""
+    m = np.max(np.abs(v), axis=1)
+    e = np.frexp(m)[1].astype(np.int64)
+    return np.where(m == 0, -125, np.maximum(e, -125))
+
+
+def router_logit_bound_int(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
+    """The documented bound of the integer tensor-core logits (T > 64):
+    2^-24 |logit| + 2^(e_x - 31) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 36)."""
+    ex = _row_exponents(x)[:, None].astype(np.float64)
+    ew = _row_exponents(wr)[None, :].astype(np.float64)
+    logit = x @ wr.T
+    if bias is not None:
+        logit = logit + np.asarray(bias, dtype=np.float64)[None, :]
+    sw = np.abs(wr).sum(axis=1)[None, :]
+    sx = np.abs(x).sum(axis=1)[:, None]
+    return (U * np.abs(logit) + np.exp2(ex - 31) * sw + np.exp2(ew - 31) * sx + H * np.exp2(ex + ew - 36)
+            + 2.0 ** -60)
+
+
+def router_logit_bound_fp32(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
+    """The documented bound of the FP32 logits (T <= 64, and the allocation-free router):
     32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (FP64 terms covered by a 2^-40 margin)."""
     sabs = np.abs(x) @ np.abs(wr).T
     logit = x @ wr.T
     if bias is not None:
         logit = logit + np.asarray(bias, dtype=np.float64)[None, :]
     return 32 * U * sabs + U * np.abs(logit) + 2.0 ** -40 * (sabs + 1)
+
+
+def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
+    """A bound that holds for either logits path: the larger of the two documented ones."""
+    return np.maximum(router_logit_bound_fp32(x, wr, bias, H), router_logit_bound_int(x, wr, bias, H))
 
 
 def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6):

@@ -131,12 +131,14 @@ def test_beam_skewed_layer_sampled():
     run_layer(BEAM, 16384, tokens=[3, 16383], bias=zipf_bias(256))
 
 
-@pytest.mark.parametrize("T", [16, 64, 200, 600, 4096])
+@pytest.mark.parametrize("T", [16, 64, 65, 200, 600, 4096])
 def test_router_logits_within_documented_bound(T):
-    """Every FP32 logit the selection used (fused front-end kernel for T <= 64, large-T logits
-    kernel above) lies within the documented 32 * 2^-24 * sum|x W| + 2^-24 |logit| of the
-    exact value."""
-    from tests.helpers import router_logit_bound
+    """Every FP32 logit the selection used lies within the documented bound of its path: for
+    T <= 64 (fused front-end kernel) 32 * 2^-24 * sum|x W| + 2^-24 |logit|; above, the integer
+    tensor-core bound 2^-24 |logit| + 2^(e_x-31) sum|W| + 2^(e_W-31) sum|x| + H 2^(e_x+e_W-36),
+    where the logits are, apart from near-ties of the final rounding, the exact values
+    rounded to FP32."""
+    from tests.helpers import router_logit_bound_fp32, router_logit_bound_int
     ex = gpu_experts(BEAM)
     x = activations(T, BEAM, seed=3)
     wr = router_weight(BEAM)
@@ -146,11 +148,51 @@ def test_router_logits_within_documented_bound(T):
     wn = wr.numpy().astype(np.float64)
     exact = xn @ wn.T
     got = dbg["logits"].cpu().numpy().astype(np.float64)
-    bound = router_logit_bound(xn, wn, None, BEAM.H)
+    err = np.abs(got - exact)
+    if T <= 64:
+        bound = router_logit_bound_fp32(xn, wn, None, BEAM.H)
+        assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
+        # the bound is not vacuous: errors are a small fraction of it
+        assert np.max(err / bound) < 0.5
+    else:
+        bound = router_logit_bound_int(xn, wn, None, BEAM.H)
+        assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
+        # far tighter than FP32 accumulation: most logits are the correctly rounded exact
+        # value (the rest lie within the fixed-point rounding of a rounding boundary)
+        rounded = exact.astype(np.float32).astype(np.float64)
+        frac = float(np.mean(got == rounded))
+        print(f"T={T}: correctly rounded {frac:.4f}, max err/bound {np.max(err / bound):.3g}")
+        assert frac > 0.95
+
+
+def test_integer_router_logits_extreme_rows():
+    """The tensor-core logits (T > 64) on rows that stress the fixed-point scaling: a zero row,
+    a row whose largest element is 2^40 times the others, a row of subnormal BF16 values, and
+    an expert row with the same spread: every logit within the documented integer bound."""
+    from tests.helpers import router_logit_bound_int
+    ex = gpu_experts(TINY)
+    T = 130
+    x = activations(T, TINY, seed=9).float()
+    x[0] = 0.0
+    x[1] = x[1] * 2.0 ** -20
+    x[1, 17] = 2.0 ** 20
+    x[2] = x[2] * 2.0 ** -130
+    x = x.to(torch.bfloat16)
+    assert 0 < float(x[2].float().abs().max()) < 2.0 ** -126
+    wr = router_weight(TINY).clone()
+    wr[5] = wr[5] * 2.0 ** -30
+    wr[5, 3] = 1.0e4
+    ws = torch.empty(moe.forward_workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
+    _, dbg = moe.forward(ex, x.cuda(), wr.cuda(), ws=ws, debug=True)
+    assert moe.status_read(ws) == moe.OK
+    xn = x.float().numpy().astype(np.float64)
+    wn = wr.numpy().astype(np.float64)
+    exact = xn @ wn.T
+    got = dbg["logits"].cpu().numpy().astype(np.float64)
+    bound = router_logit_bound_int(xn, wn, None, TINY.H)
     err = np.abs(got - exact)
     assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
-    # the bound is not vacuous: errors are a small fraction of it
-    assert np.max(err / bound) < 0.5
+    assert np.all(got[0] == 0.0)
 
 
 @pytest.mark.parametrize("T", [16, 130])
