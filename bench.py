@@ -570,6 +570,46 @@ def run_quantize(args, world, rank, local):
             "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
 
 
+def run_route(args, world, rank, local):
+    """Standalone route(hidden, W_router) (nvfp4moe_route) on Beam's router for T=4096 tokens:
+    for T > 64 the logits run as exact int8 digit-plane products on the tensor cores (13 digit
+    pairs), so the dominant kernel is bound by int8 tensor throughput; peak = measured BF16
+    burst x 2 (nominal INT8 : BF16 dense ratio)."""
+    import nvfp4_quantized_moe_group_b200 as moe
+    T = 4096
+    cfg = moe.cfg_default()
+    x = activations(T, BEAM, seed=rank, device="cuda")
+    wr = router_weight(BEAM).cuda()
+    ws = torch.empty(moe.route_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        moe.route(cfg, x, wr, ws=ws)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
+        start.record()
+        for _ in range(args.steps):
+            moe.route(cfg, x, wr, ws=ws)
+        stop.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    launches = moe.last_launch_count()
+    if moe.status_read(ws) != moe.OK:
+        raise RuntimeError("route status")
+    ops = 13 * 2.0 * T * BEAM.H * BEAM.E          # int8 digit-pair products, the dominant kernel
+    p = peaks()
+    i8_peak = p["bf16_tflops"] * 2
+    return {"metric": "route tokens/s (Beam router, T=4096)", "value": world * T / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x fp32 -> exact int8 digits",
+            "data": "synthetic", "config": {"workload": "route T=4096, E=256, H=5120",
+                                            "l2": "token digit planes 84 MB < 126 MB L2 (not flushed)"},
+            "roofline": {"bound": "tensor", "achieved": ops / (ms / 1e3) / 1e12, "peak": i8_peak, "unit": "TOP/s",
+                         "frac": ops / (ms / 1e3) / 1e12 / i8_peak, "traffic": None,
+                         "note": "whole call (slicing, logits, top-k) against the int8 work of the logits kernel"},
+            "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
+
+
 FP32_LANES_PER_SM = 128   # FP32 FMA lanes per B200 SM (4 partitions x 32)
 
 
@@ -678,7 +718,7 @@ def main():
                     help="NVML clock sampling period during the timed region")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize", "quantize_lh"])
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS) + ["quantize", "quantize_lh", "route"])
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 W8A8 variant's measurement")
@@ -700,6 +740,8 @@ def main():
             res = run_quantize(args, world, rank, local)
         elif args.workload == "quantize_lh":
             res = run_quantize_lh(args, world, rank, local)
+        elif args.workload == "route":
+            res = run_route(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
         if rank == 0:
