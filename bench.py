@@ -570,6 +570,83 @@ def run_quantize(args, world, rank, local):
             "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
 
 
+def run_ep(args, world, rank, local):
+    """The layer under expert parallelism (nvfp4_quantized_moe_group_b200.ep): rank r holds
+    experts [r E/G, (r+1) E/G); a step all-gathers the ranks' tokens (NCCL), runs the rank's
+    partial layer on all of them, reduce-scatters the FP32 sums (NCCL) and rounds to BF16.
+    Per-rank batch: the workload's T tokens.  Roofline: this rank's share of the weight bytes
+    of the experts hit by all gathered tokens, over the step time."""
+    import nvfp4_quantized_moe_group_b200 as moe
+    from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer
+    wl = WORKLOADS[args.workload]
+    shape = layer_shape(args.experts) if args.experts else wl.shape
+    T = wl.T
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    layer = ExpertParallelLayer(cfg)
+    ex = layer.create_experts()
+    g_h = intermediate_scales(shape)
+    for e in range(layer.e_begin, layer.e_begin + layer.e_count):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    x_cpu = activations(T, shape, seed=wl.seed + rank, rms_rows=wl.rms_rows)
+    x = x_cpu.cuda()
+    wr = router_weight(shape).cuda()
+    bias = zipf_bias(shape.E).cuda() if wl.zipf else None
+    # routing of the gathered batch: which of this rank's experts the step streams
+    x_all = layer.gather(x)
+    _, dbg = moe.forward_partial(ex, x_all, wr, bias, debug=True)
+    counts = dbg["counts"].cpu().numpy()[layer.e_begin:layer.e_begin + layer.e_count]
+    hit_local = int((counts > 0).sum())
+    launches = moe.last_launch_count() + 1          # + finalize
+    del dbg
+    for _ in range(args.warmup):
+        layer.forward(x, wr, bias)
+    torch.cuda.synchronize()
+    barrier(world)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
+        start.record()
+        for _ in range(args.steps):
+            layer.forward(x, wr, bias)
+        stop.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    # end to end: pinned host tokens in, BF16 rows out
+    x_host = x_cpu.pin_memory()
+    out_host = torch.empty((T, shape.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        out_host.copy_(layer.forward(x_dev, wr, bias), non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    p = peaks()
+    per_expert = 3 * shape.H * shape.I * (E2M1_BYTES + E4M3_PER16) + 16
+    local_bytes = hit_local * per_expert + world * T * shape.H * 2 + shape.E * shape.H * 4
+    layer.close()
+    return {"metric": METRIC, "value": tokens_per_second(world, T, 1, ms), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
+            "data": "synthetic (seeded counter-hash inputs; random-init NVFP4 weights)",
+            "config": {"workload": wl.describe() + f" per rank, expert parallel over {world} rank(s)",
+                       "T_per_rank": T, "experts_per_rank": layer.e_count, "local_experts_hit": hit_local,
+                       "parallelism": f"ep{world} (all-gather tokens, reduce-scatter FP32 sums)",
+                       "l2": "no flush: every step streams the rank's routed experts' weights"},
+            "roofline": {"bound": "hbm", "achieved": local_bytes / (ms / 1e3) / 1e9, "peak": p["hbm_gbs"],
+                         "unit": "GB/s", "frac": local_bytes / (ms / 1e3) / (p["hbm_gbs"] * 1e9), "traffic": None,
+                         "note": "whole step of this rank (partial layer + collectives) on its algorithmic bytes"},
+            "e2e": {"value": tokens_per_second(world, T, 1, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
+            "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
+
+
 def run_route(args, world, rank, local):
     """Standalone route(hidden, W_router) (nvfp4moe_route) on Beam's router for T=4096 tokens:
     for T > 64 the logits run as exact int8 digit-plane products on the tensor cores (13 digit
@@ -722,6 +799,9 @@ def main():
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 W8A8 variant's measurement")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the ranks (each holds E/N experts; NCCL all-gather and "
+                         "reduce-scatter) instead of one full replica per GPU")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -742,6 +822,8 @@ def main():
             res = run_quantize_lh(args, world, rank, local)
         elif args.workload == "route":
             res = run_route(args, world, rank, local)
+        elif args.ep:
+            res = run_ep(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
         if rank == 0:

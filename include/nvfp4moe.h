@@ -233,6 +233,16 @@ NVFP4MOE_API void nvfp4moe_experts_destroy(nvfp4moe_experts* experts);
 /* The handle's configuration (copied out). */
 NVFP4MOE_API int nvfp4moe_experts_cfg(const nvfp4moe_experts* experts, nvfp4moe_cfg* cfg);
 
+/* A handle that holds only experts e_begin .. e_begin + e_count - 1 of the layer (one rank's
+ * share under expert parallelism: the deployment on the pages spreads the experts over the
+ * GPUs of a node).  cfg describes the whole layer; 0 <= e_begin, e_begin + e_count <= E.
+ * nvfp4moe_experts_set takes the global expert index, which must lie in the range; the
+ * handle's device memory is e_count / E of a full one.  nvfp4moe_experts_create(cfg) is
+ * nvfp4moe_experts_create_local(cfg, 0, E). */
+NVFP4MOE_API int nvfp4moe_experts_create_local(const nvfp4moe_cfg* cfg, int32_t e_begin, int32_t e_count,
+                                               nvfp4moe_experts** out);
+NVFP4MOE_API int nvfp4moe_experts_range(const nvfp4moe_experts* experts, int32_t* e_begin, int32_t* e_count);
+
 /* ----------------------------------------------------------------- forward ----
  * moe_forward(hidden, experts) -> out: the whole layer (route, quantise x, group the
  * token/expert pairs by expert, gate/up GEMM + SwiGLU + requantisation of h, down GEMM
@@ -291,6 +301,29 @@ NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, in
 NVFP4MOE_API int nvfp4moe_forward(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
                      const float* w_router, const float* logit_bias, void* out_bf16,
                      const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------- forward, expert parallel ----
+ * One rank's part of the layer under expert parallelism.  Every rank holds the router and a
+ * share of the experts (nvfp4moe_experts_create_local); the ranks gather their tokens (the
+ * same hidden_all on every rank), each runs
+ *   nvfp4moe_forward_partial(its experts, hidden_all, T_all, ...) -> acc_out [T_all][H] FP32,
+ * the acc_out arrays are summed across ranks with a reduce-scatter that leaves each rank the
+ * rows of its own tokens, and nvfp4moe_finalize rounds those rows to BF16.  Routing and the
+ * input's global scale are computed from hidden_all, so every rank takes the same decisions
+ * and the ranks' sums add up to the single-GPU layer (up to the order of FP32 additions).
+ *
+ *   acc_out  [T][H] FP32 (16-byte aligned, out): the sum over the token's selected slots whose
+ *            expert the handle holds of w * y (zero for a token with none), written in full.
+ *   hidden_bf16, T, w_router, logit_bias, dbg, ws as for nvfp4moe_forward (same workspace
+ *   size); dbg->hq_codes / hq_scales are meaningful only for pairs of the handle's experts.
+ * With a full handle, acc_out is the FP32 sum nvfp4moe_forward rounds to BF16.
+ *
+ * nvfp4moe_finalize: out_bf16[i] = bf16(acc[i]) for n values (n % 8 == 0, both 16-byte
+ * aligned), the layer's output rounding. */
+NVFP4MOE_API int nvfp4moe_forward_partial(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
+                                          const float* w_router, const float* logit_bias, float* acc_out,
+                                          const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
+NVFP4MOE_API int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream);
 
 /* ------------------------------------------------------------------ status ----
  * Waits for `stream`, then returns the device-side status of the last call that used

@@ -109,6 +109,11 @@ _SIGS = {
     "nvfp4moe_experts_set": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(ExpertTensors), _P]),
     "nvfp4moe_experts_destroy": (None, [_P]),
     "nvfp4moe_experts_cfg": (ctypes.c_int, [_P, ctypes.POINTER(Cfg)]),
+    "nvfp4moe_experts_create_local": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.c_int32, ctypes.c_int32,
+                                                     ctypes.POINTER(_P)]),
+    "nvfp4moe_experts_range": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
+    "nvfp4moe_forward_partial": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_finalize": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nvfp4moe_forward_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_forward": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_forward_residual": (ctypes.c_int, [_P, _P, _I64, _P, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
@@ -270,12 +275,17 @@ def route(cfg: Cfg, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor 
 
 
 class Experts:
-    """Library-owned NVFP4 expert weights (nvfp4moe_experts_create / _set / _destroy)."""
+    """Library-owned NVFP4 expert weights (nvfp4moe_experts_create / _set / _destroy).  With
+    ``e_count`` the handle holds only experts e_begin .. e_begin + e_count - 1 (one rank's share
+    under expert parallelism, nvfp4moe_experts_create_local)."""
 
-    def __init__(self, cfg: Cfg):
+    def __init__(self, cfg: Cfg, e_begin: int = 0, e_count: int | None = None):
         self.cfg = cfg
+        self.e_begin = int(e_begin)
+        self.e_count = int(cfg.E - e_begin if e_count is None else e_count)
         h = ctypes.c_void_p()
-        _check(lib().nvfp4moe_experts_create(ctypes.byref(cfg), ctypes.byref(h)), "nvfp4moe_experts_create")
+        _check(lib().nvfp4moe_experts_create_local(ctypes.byref(cfg), self.e_begin, self.e_count, ctypes.byref(h)),
+               "nvfp4moe_experts_create_local")
         self.handle = h
 
     def set(self, e: int, gate, up, down, g_h: float, stream=None):
@@ -477,4 +487,39 @@ def forward_fp8(experts: Fp8Experts, x: torch.Tensor, w_router: torch.Tensor, bi
     _check(st, "nvfp4moe_forward_fp8")
     if debug:
         return out, tensors
+    return out
+
+
+# ------------------------------------------------------------- expert parallelism ----
+
+def forward_partial(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
+                    acc_out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False,
+                    stream=None):
+    """One rank's part of the layer (nvfp4moe_forward_partial): the FP32 sums [T, H] of the
+    contributions of the handle's experts for all T tokens of x."""
+    cfg = experts.cfg
+    T, H = x.shape
+    dev = x.device
+    if acc_out is None:
+        acc_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(cfg, T), dev)
+    tensors = _debug_tensors(cfg, T, H, dev) if debug else None
+    dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()}) if debug else None
+    st = lib().nvfp4moe_forward_partial(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(acc_out),
+                                        ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
+                                        _stream(stream))
+    _check(st, "nvfp4moe_forward_partial")
+    if debug:
+        return acc_out, tensors
+    return acc_out
+
+
+def finalize(acc: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """BF16 rounding of FP32 layer sums (nvfp4moe_finalize)."""
+    if acc.dtype != torch.float32 or not acc.is_cuda or not acc.is_contiguous():
+        raise TypeError("acc must be a contiguous float32 CUDA tensor")
+    if out is None:
+        out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
+    _check(lib().nvfp4moe_finalize(_ptr(acc), acc.numel(), _ptr(out), _stream(stream)), "nvfp4moe_finalize")
     return out

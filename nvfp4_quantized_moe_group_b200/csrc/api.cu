@@ -12,6 +12,7 @@ using namespace nvfp4moe;
 struct nvfp4moe_experts {
   nvfp4moe_cfg cfg;
   int device;
+  int e_begin, e_count;  // the experts this handle holds (all E, or one rank's share)
   uint8_t* w13_codes;   // tiled (see launch_tile_weights), gate/up rows interleaved per 64-row group
   uint8_t* w13_sf;      // swizzled, [E][2I/128 row tiles][H/64 column tiles][512]
   uint8_t* wd_codes;    // tiled, [E][H/128][ceil(I/256)][128][128]
@@ -435,18 +436,22 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   return NVFP4MOE_OK;
 }
 
-int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out) {
+int nvfp4moe_experts_create_local(const nvfp4moe_cfg* cfg, int32_t e_begin, int32_t e_count,
+                                  nvfp4moe_experts** out) {
   if (out == nullptr) return NVFP4MOE_ERR_ARG;
   *out = nullptr;
   int st = nvfp4moe_cfg_check(cfg);
   if (st != NVFP4MOE_OK) return st;
+  if (e_begin < 0 || e_count < 1 || e_begin + e_count > cfg->E) return NVFP4MOE_ERR_ARG;
   st = check_device();
   if (st != NVFP4MOE_OK) return st;
   nvfp4moe_experts* x = new nvfp4moe_experts();
   std::memset(x, 0, sizeof(*x));
   x->cfg = *cfg;
+  x->e_begin = e_begin;
+  x->e_count = e_count;
   cudaGetDevice(&x->device);
-  const int64_t E = cfg->E, H = cfg->H, I = cfg->I;
+  const int64_t E = e_count, H = cfg->H, I = cfg->I;
   // tiled codes: K padded to a multiple of 256 values (128 bytes)
   const size_t w13 = (size_t)E * 2 * I * ((H + 255) / 256 * 128), w13sf = (size_t)E * 2 * I * H / 16;
   const size_t wd = (size_t)E * H * ((I + 255) / 256 * 128), wdsf = (size_t)E * H * I / 16;
@@ -465,11 +470,24 @@ int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out) {
   return NVFP4MOE_OK;
 }
 
-int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e, const nvfp4moe_expert_tensors* t, void* stream) {
+int nvfp4moe_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_experts** out) {
+  if (cfg == nullptr) return NVFP4MOE_ERR_ARG;
+  return nvfp4moe_experts_create_local(cfg, 0, cfg->E, out);
+}
+
+int nvfp4moe_experts_range(const nvfp4moe_experts* x, int32_t* e_begin, int32_t* e_count) {
+  if (x == nullptr || e_begin == nullptr || e_count == nullptr) return NVFP4MOE_ERR_ARG;
+  *e_begin = x->e_begin;
+  *e_count = x->e_count;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e_global, const nvfp4moe_expert_tensors* t, void* stream) {
   g_launches = 0;
   if (x == nullptr || t == nullptr) return NVFP4MOE_ERR_ARG;
   const nvfp4moe_cfg& c = x->cfg;
-  if (e < 0 || e >= c.E) return NVFP4MOE_ERR_ARG;
+  if (e_global < x->e_begin || e_global >= x->e_begin + x->e_count) return NVFP4MOE_ERR_ARG;
+  const int32_t e = e_global - x->e_begin;   // slot in this handle
   if (!t->gate_codes || !t->gate_scales || !t->up_codes || !t->up_scales || !t->down_codes || !t->down_scales)
     return NVFP4MOE_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -523,18 +541,22 @@ size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) 
 }
 
 // The layer; with res, finalize adds the output into the residual stream.
+// acc_out: NULL for the whole layer (BF16 out_bf16); otherwise the FP32 sums of the handle's
+// experts' contributions are left in acc_out [T][H] and there is no finalize.
 static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
                         const float* logit_bias, void* out_bf16, const Residual* res, const nvfp4moe_debug* dbg,
-                        void* ws, size_t ws_bytes, void* stream) {
+                        void* ws, size_t ws_bytes, void* stream, float* acc_out = nullptr) {
   g_launches = 0;
   if (x == nullptr) return NVFP4MOE_ERR_ARG;
   const nvfp4moe_cfg& c = x->cfg;
   if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
-  if (hidden_bf16 == nullptr || w_router == nullptr || out_bf16 == nullptr || ws == nullptr)
+  if (hidden_bf16 == nullptr || w_router == nullptr || (out_bf16 == nullptr && acc_out == nullptr) || ws == nullptr)
     return NVFP4MOE_ERR_ARG;
-  if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(out_bf16, 16) || !aligned(ws, kAlign))
+  if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(out_bf16, 16) || !aligned(acc_out, 16) ||
+      !aligned(ws, kAlign))
     return NVFP4MOE_ERR_ARG;
-  const ForwardWs f = carve_forward(ws, c, T);
+  ForwardWs f = carve_forward(ws, c, T);
+  if (acc_out != nullptr) f.acc = acc_out;
   if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
@@ -682,9 +704,11 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
   g.sfb = x->w13_sf;
-  g.mtile_prefix = f.mtile_prefix;
-  g.counts = f.counts;
-  g.E = c.E;
+  // the handle's experts only (all of them unless it holds one rank's share): tiles of
+  // experts e_begin .. e_begin + e_count - 1, weights indexed from the handle's first expert
+  g.mtile_prefix = f.mtile_prefix + x->e_begin;
+  g.counts = f.counts + x->e_begin;
+  g.E = x->e_count;
   g.K = c.H;
   g.n_total = 2 * c.I;
   g.status = &f.hdr->status;
@@ -715,12 +739,14 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
 
-  FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,
-                  res != nullptr ? res->a : 0.0f, res != nullptr ? res->b : 0.0f};
-  ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
-  if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_FINALIZE, 1);
-  ++g_launches;
+  if (acc_out == nullptr) {
+    FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,
+                    res != nullptr ? res->a : 0.0f, res != nullptr ? res->b : 0.0f};
+    ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
+    if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_FINALIZE, 1);
+    ++g_launches;
+  }
 
   if (dbg != nullptr) {
     bool ok = true;
@@ -747,6 +773,26 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
                      const float* logit_bias, void* out_bf16, const nvfp4moe_debug* dbg, void* ws,
                      size_t ws_bytes, void* stream) {
   return forward_core(x, hidden_bf16, T, w_router, logit_bias, out_bf16, nullptr, dbg, ws, ws_bytes, stream);
+}
+
+int nvfp4moe_forward_partial(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
+                             const float* logit_bias, float* acc_out, const nvfp4moe_debug* dbg, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (acc_out == nullptr) return NVFP4MOE_ERR_ARG;
+  return forward_core(x, hidden_bf16, T, w_router, logit_bias, nullptr, nullptr, dbg, ws, ws_bytes, stream, acc_out);
+}
+
+int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream) {
+  g_launches = 0;
+  if (n < 0 || n % 8 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (n == 0) return NVFP4MOE_OK;
+  if (acc == nullptr || out_bf16 == nullptr || !aligned(acc, 16) || !aligned(out_bf16, 16)) return NVFP4MOE_ERR_ARG;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  FinalizeArgs fa{acc, static_cast<uint16_t*>(out_bf16), n, nullptr, 0.0f, 0.0f};
+  if (launch_finalize(fa, static_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches = 1;
+  return NVFP4MOE_OK;
 }
 
 int nvfp4moe_forward_residual(const nvfp4moe_experts* x, const void* h_bf16, int64_t T, const float* gamma,

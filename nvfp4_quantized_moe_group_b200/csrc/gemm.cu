@@ -247,7 +247,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   const uint32_t tmem = s.tmem_base;
   const int ntn = p.n_total / kN;           // 256-wide items per expert
   const int ntn128 = p.n_total / 128;       // 128-row weight tiles per expert
-  const int total = __ldg(p.mtile_prefix + p.E) * ntn;
+  // p.mtile_prefix may start at a later expert (a handle with one rank's share of the experts):
+  // its tiles are numbered from the first entry on
+  const int tile_base = __ldg(p.mtile_prefix);
+  const int total = (__ldg(p.mtile_prefix + p.E) - tile_base) * ntn;
   const int kb_count = kFp8 ? (p.K + 127) / 128 : (p.K + kBlockK - 1) / kBlockK;   // 128-byte K blocks
   const int k64 = p.K / 64;  // scale-column tiles of A and B
 
@@ -260,7 +263,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       const uint64_t pol_a = policy_evict_last();
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Work wk = decode_work(p.mtile_prefix, w, p.E, ntn, p.counts);
+        const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
         const int arow = wk.mtile * kBlockM;
         const bool a_small = wk.rows_valid <= 32;
         const uint32_t a_bytes = a_small ? 32u * 128u : (uint32_t)kABytes;
@@ -366,7 +369,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     const int row_l = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      const Work wk = decode_work(p.mtile_prefix, w, p.E, ntn, p.counts);
+      const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
       const uint32_t acc_par = (uint32_t)it & 1u;
       const int64_t row = (int64_t)wk.mtile * kBlockM + row_l;
       const bool valid = row_l < wk.rows_valid;

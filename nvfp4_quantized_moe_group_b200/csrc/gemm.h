@@ -16,9 +16,9 @@ struct GemmArgs {
   const uint8_t* b_tiles;      // weights, tiled: [E][n_total/128][ceil(K/256)][128 rows][128 B], swizzled
   const uint8_t* sfa;          // swizzled scales of A (padded rows)
   const uint8_t* sfb;          // swizzled scales of B, experts back to back
-  const int32_t* mtile_prefix; // [E+1]
+  const int32_t* mtile_prefix; // [E+1] (may point into a longer table: entries are global tile numbers)
   const int32_t* counts;       // [E]
-  int E;
+  int E;                       // experts of this launch (weights, scales, per-expert scalars indexed 0..E-1)
   int K;                       // reduction length
   int n_total;                 // B rows per expert (2I for gate/up, H for down)
   uint32_t* status;

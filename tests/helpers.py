@@ -122,9 +122,12 @@ def _expert_job(args):
     return e, res["y"], res["h"], res["hq_codes"], res["hq_scales"], (gate.g, up.g, down.g)
 
 
-def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, tokens=None, workers=None):
+def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, tokens=None, workers=None,
+                 expert_range=None):
     """Oracle layer output for the given tokens: routing of all tokens, expert MLPs of the
-    sampled tokens (experts evaluated in a spawn process pool when there are many)."""
+    sampled tokens (experts evaluated in a spawn process pool when there are many).  With
+    expert_range = (first, count) only those experts' contributions are summed (one rank's
+    part under expert parallelism)."""
     cfg = cfg_ns(shape)
     r = oracle.route(x, wr, cfg, bias)
     xc, xs, gx = oracle.quantize(np.asarray(x, dtype=np.float32))
@@ -133,7 +136,9 @@ def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, to
     need = {}
     for i, t in enumerate(tokens):
         for j in range(cfg.topk):
-            need.setdefault(int(r.idx[t, j]), []).append((i, int(t), j))
+            e = int(r.idx[t, j])
+            if expert_range is None or expert_range[0] <= e < expert_range[0] + expert_range[1]:
+                need.setdefault(e, []).append((i, int(t), j))
     jobs = []
     for e, rows in sorted(need.items()):
         ts = np.array([t for _, t, _ in rows])

@@ -1,0 +1,111 @@
+"""Expert parallelism on one GPU (nvfp4moe_experts_create_local, nvfp4moe_forward_partial,
+nvfp4moe_finalize): G ranks are emulated one after another on the same device, with the
+all-gather a concatenation and the reduce-scatter an FP32 sum over the ranks' partial sums.
+The ranks' sums must add up to the single-handle layer (up to the order of FP32 additions),
+a token none of whose experts a rank holds must get an exact zero row from it, and the
+rounded result must match nvfp4moe_forward within one BF16 unit."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_quantized_moe_group_b200 as moe
+from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer, expert_range
+from workloads import TINY, BEAM, activations, router_weight, expert_weight
+from tests.helpers import intermediate_scales, bf16_half_ulp
+from tests.test_gpu_forward import gpu_experts
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    moe.lib()
+
+
+def local_experts(shape, e0, n):
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    ex = moe.Experts(cfg, e0, n)
+    g_h = intermediate_scales(shape)
+    for e in range(e0, e0 + n):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    torch.cuda.synchronize()
+    return ex
+
+
+def run_emulated(shape, G, T_rank, seed=50):
+    full = gpu_experts(shape)
+    xs = [activations(T_rank, shape, seed=seed + r).cuda() for r in range(G)]
+    x_all = torch.cat(xs)
+    wr = router_weight(shape).cuda()
+    acc_full, dbg = moe.forward_partial(full, x_all, wr, debug=True)
+    out_full = moe.forward(full, x_all, wr)
+    idx = dbg["idx"].cpu().numpy()
+    accs = []
+    for r in range(G):
+        e0, n = expert_range(shape.E, r, G)
+        ex = local_experts(shape, e0, n)
+        assert (ex.e_begin, ex.e_count) == (e0, n)
+        acc_r, dbg_r = moe.forward_partial(ex, x_all, wr, debug=True)
+        # every rank routes the gathered tokens identically
+        np.testing.assert_array_equal(dbg_r["idx"].cpu().numpy(), idx)
+        # tokens with no selected expert in the rank's range get an exact zero row
+        none_local = ~((idx >= e0) & (idx < e0 + n)).any(axis=1)
+        a = acc_r.cpu().numpy()
+        assert np.all(a[none_local] == 0.0)
+        accs.append(acc_r)
+        ex.close()
+    total = accs[0].clone()
+    for acc_r in accs[1:]:
+        total += acc_r
+    af = acc_full.cpu().numpy()
+    diff = np.abs(total.cpu().numpy() - af)
+    assert np.all(diff <= 2.0 ** -20 * np.abs(af) + 1e-30 + 2.0 ** -22 * np.abs(af).max())
+    # each rank's own rows after the reduce-scatter, rounded: the single-GPU layer to one BF16 unit
+    out_ep = moe.finalize(total).float().cpu().numpy()
+    of = out_full.float().cpu().numpy()
+    assert np.all(np.abs(out_ep - of) <= 2 * bf16_half_ulp(of) + 1e-30)
+    return out_ep
+
+
+@pytest.mark.parametrize("G,T_rank", [(2, 24), (4, 24), (8, 8)])
+def test_tiny_emulated_ranks(G, T_rank):
+    run_emulated(TINY, G, T_rank)
+
+
+def test_beam_decode_eight_ranks():
+    """Beam decode on 8 emulated ranks: 16 tokens each, 128 gathered tokens."""
+    run_emulated(BEAM, 8, 16)
+
+
+def test_local_handle_rejects_foreign_experts_and_bad_ranges():
+    cfg = moe.make_cfg(TINY.E, TINY.n_groups, TINY.topk_groups, TINY.topk, TINY.H, TINY.I, TINY.routed_scale)
+    ex = moe.Experts(cfg, 8, 8)
+    w = [expert_weight(TINY, 3, n, device="cuda") for n in ("gate", "up", "down")]
+    with pytest.raises(moe.NvFp4MoeError):
+        ex.set_from_bf16(3, *w, 1.0)                    # expert 3 is not in 8 .. 15
+    ex.close()
+    for e0, n in ((-1, 4), (30, 4), (0, 0)):
+        with pytest.raises(moe.NvFp4MoeError):
+            moe.Experts(cfg, e0, n)
+
+
+def test_single_rank_layer_matches_forward():
+    """ExpertParallelLayer without a process group: the whole layer on this GPU."""
+    cfg = moe.make_cfg(TINY.E, TINY.n_groups, TINY.topk_groups, TINY.topk, TINY.H, TINY.I, TINY.routed_scale)
+    layer = ExpertParallelLayer(cfg)
+    assert (layer.world, layer.e_begin, layer.e_count) == (1, 0, TINY.E)
+    ex = layer.create_experts()
+    g_h = intermediate_scales(TINY)
+    for e in range(TINY.E):
+        ex.set_from_bf16(e, *(expert_weight(TINY, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    x = activations(40, TINY, seed=7).cuda()
+    wr = router_weight(TINY).cuda()
+    got = layer.forward(x, wr).float().cpu().numpy()
+    want = moe.forward(gpu_experts(TINY), x, wr).float().cpu().numpy()
+    assert np.all(np.abs(got - want) <= 2 * bf16_half_ulp(want) + 1e-30)
+    layer.close()
