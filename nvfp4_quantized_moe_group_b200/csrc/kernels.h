@@ -11,7 +11,7 @@
 namespace nvfp4moe {
 
 constexpr int kMaxAmaxPartials = 1024;   // blocks of the amax pass
-constexpr int kPermChunkTokens = 128;    // tokens per chunk of the grouping kernels
+constexpr int kPermChunkTokens = 32;     // tokens per chunk of the grouping kernels
 
 struct QuantizeArgs {
   const uint16_t* x;       // [rows][cols] bf16

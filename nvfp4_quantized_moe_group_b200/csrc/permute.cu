@@ -22,17 +22,23 @@ __global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
 }
 
 // One block, one thread per expert: per-chunk bases, counts, offsets (exclusive scan),
-// 128-row tile prefix, and -1 in every padding row of every segment.
+// 128-row tile prefix, and -1 in every padding row of every segment.  The per-chunk counts are
+// read in batches of independent loads (a chain of dependent loads, one per chunk, would wait
+// out the memory latency once per chunk).
 __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
   __shared__ int s_cnt[256];
   __shared__ int s_tiles[256];
+  constexpr int kBatch = 16;
   const int e = threadIdx.x;
+  const int* __restrict__ cc = a.chunk_counts;
   int running = 0;
   if (e < a.E) {
-    for (int c = 0; c < a.n_chunks; ++c) {
-      const int v = a.chunk_counts[(int64_t)c * a.E + e];
-      a.chunk_base[(int64_t)c * a.E + e] = running;
-      running += v;
+    for (int c0 = 0; c0 < a.n_chunks; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < a.n_chunks ? __ldg(cc + (int64_t)(c0 + j) * a.E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) running += v[j];
     }
   }
   const int tiles = e < a.E ? (running + kBlockM - 1) / kBlockM : 0;
@@ -58,7 +64,18 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
       a.offsets[a.E] = off + running;
       a.mtile_prefix[a.E] = tile0 + tiles;
     }
-    for (int c = 0; c < a.n_chunks; ++c) a.chunk_base[(int64_t)c * a.E + e] += off;
+    // chunk c's first position for expert e: off + the counts of the chunks before it
+    int base = off;
+    for (int c0 = 0; c0 < a.n_chunks; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < a.n_chunks ? __ldg(cc + (int64_t)(c0 + j) * a.E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (c0 + j < a.n_chunks) a.chunk_base[(int64_t)(c0 + j) * a.E + e] = base;
+        base += v[j];
+      }
+    }
     const int64_t r0 = (int64_t)tile0 * kBlockM;
     const int64_t r1 = r0 + (int64_t)tiles * kBlockM;
     for (int64_t r = r0 + running; r < r1; ++r) a.row_pair[r] = -1;

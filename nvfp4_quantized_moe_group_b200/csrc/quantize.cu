@@ -68,70 +68,80 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantizeArgs a) {
   const float g = s_g;
   const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
 
-  const int64_t chunks_per_row = a.cols >> 6;
-  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t r = idx / chunks_per_row;
-  const int64_t q = idx - r * chunks_per_row;
-  if (r >= a.rows_padded) return;
+  // one warp per (row, 512-value segment): lane l takes the 16-value block 32 seg + l, so every
+  // load, code store and accumulator store of the warp covers one contiguous span of the row;
+  // lanes 4k .. 4k+3 hold the 4 block scales of one 32-bit scale word
+  const int64_t blocks_per_row = a.cols >> 4;
+  const int64_t segs_per_row = (blocks_per_row + 31) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t r = warp / segs_per_row;
+  if (r >= a.rows_padded) return;                      // uniform over the warp
+  const int64_t b = (warp - r * segs_per_row) * 32 + lane;
+  // lanes past the row's last block stay for the shuffles; groups of 4 lanes are active or
+  // idle together (cols % 64 == 0)
+  const bool active = b < blocks_per_row;
+  const bool live = active && r < a.rows;
 
-  if (a.zero_out != nullptr && r < a.rows) {
-    float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + q * 64);
+  if (a.zero_out != nullptr && live) {
+    float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = zero;
+    for (int i = 0; i < 4; ++i) z[i] = zero;
   }
 
-  uint32_t sc = 0;
+  uint32_t s = 0, c0 = 0, c1 = 0;
+  if (live) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + b * 16);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+    uint32_t mb = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      f[2 * j] = __uint_as_float(w[j] << 16);
+      f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      mb = max(mb, w[j] & 0x7FFFu);
+      mb = max(mb, (w[j] >> 16) & 0x7FFFu);
+    }
+    float r_b;
+    s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
+    c0 = cvt_e2m1x8(f);
+    c1 = cvt_e2m1x8(f + 8);
+  }
+  // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes 4k)
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
+  const uint32_t sc = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  const bool word_lane = active && (lane & 3) == 0;
+
   if (r < a.rows) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + q * 64);
-    uint4 v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __ldg(src + i);
-    uint32_t out[8];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const uint32_t w[8] = {v[2 * b].x, v[2 * b].y, v[2 * b].z, v[2 * b].w,
-                             v[2 * b + 1].x, v[2 * b + 1].y, v[2 * b + 1].z, v[2 * b + 1].w};
-      float f[16];
-      uint32_t mb = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        f[2 * j] = __uint_as_float(w[j] << 16);
-        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        mb = max(mb, w[j] & 0x7FFFu);
-        mb = max(mb, (w[j] >> 16) & 0x7FFFu);
-      }
-      float r_b;
-      const uint32_t s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
-      sc |= s << (8 * b);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
-      out[2 * b] = cvt_e2m1x8(f);
-      out[2 * b + 1] = cvt_e2m1x8(f + 8);
-    }
-    if (a.codes != nullptr) {
-      uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + q * 32);
-      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    }
+    if (a.codes != nullptr && active)
+      reinterpret_cast<uint2*>(a.codes + r * (a.cols >> 1))[b] = make_uint2(c0, c1);
     if (a.seg_codes != nullptr) {
-      for (int j = 0; j < a.topk; ++j) {
-        const int64_t p = r * a.topk + j;
+      // lane j < topk finds pair j's segment row; every lane writes its block to all of them
+      int64_t my_row = 0;
+      if (lane < a.topk) {
+        const int64_t p = r * a.topk + lane;
         const int e = a.idx[p];
-        const int64_t row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
-        uint4* dst = reinterpret_cast<uint4*>(a.seg_codes + row * (a.cols >> 1) + q * 32);
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-        *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, q * 4, a.n_col_tiles)) = sc;
+        my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
+      }
+      for (int j = 0; j < a.topk; ++j) {
+        const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+        if (active) reinterpret_cast<uint2*>(a.seg_codes + row * (a.cols >> 1))[b] = make_uint2(c0, c1);
+        if (word_lane) *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, b, a.n_col_tiles)) = sc;
       }
     }
   }
-  if (a.scales == nullptr) return;
+  if (a.scales == nullptr || !word_lane) return;
   uint32_t* sdst;
   if (a.swizzled) {
-    sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, q * 4, a.n_col_tiles));
+    sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, b, a.n_col_tiles));
   } else {
-    sdst = reinterpret_cast<uint32_t*>(a.scales + r * (a.cols >> 4) + q * 4);
+    sdst = reinterpret_cast<uint32_t*>(a.scales + r * (a.cols >> 4) + b);
   }
   *sdst = sc;
 }
@@ -152,7 +162,7 @@ cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partia
 }
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
-  const int64_t threads = a.rows_padded * (a.cols >> 6);
+  const int64_t threads = a.rows_padded * (((a.cols >> 4) + 31) >> 5) * 32;
   const int64_t blocks = threads > 0 ? (threads + 255) / 256 : 1;  // one block still writes g_out
   quantize_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
