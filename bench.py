@@ -132,6 +132,7 @@ class ClockSampler:
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
+        self._device = device_index
         self._proc = None
         self._lines = []
         self._thread = None
@@ -163,6 +164,18 @@ class ClockSampler:
     def __exit__(self, *exc):
         t1 = time.monotonic()
         if self._proc is not None:
+            # one more sample from this process at the end of the region (a short region can
+            # fall between two of the child's samples)
+            try:
+                import pynvml
+                pynvml.nvmlInit()
+                h = pynvml.nvmlDeviceGetHandleByIndex(self._device)
+                get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+                self._lines.append(f"s {t1} {pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)} "
+                                   f"{int(get_reasons(h))}")
+            except Exception:
+                pass
             self._proc.terminate()
             self._proc.wait()
             self._thread.join()
@@ -283,7 +296,7 @@ def _oracle_experts(shape: LayerShape, experts):
                      for n in ("gate", "up", "down")) for e in experts}
 
 
-def cpu_baseline_oracle(shape: LayerShape, wl, x_cpu, wr_cpu, bias_cpu, n_tokens=2):
+def cpu_baseline_oracle(shape: LayerShape, wl, x_cpu, wr_cpu, bias_cpu, n_tokens=5):
     """The oracle on a bounded sample of the step: routing and input quantisation of every
     token, then the layer output of ``n_tokens`` tokens (their 8 experts' FP64 SwiGLU MLPs on
     dequantised weights).  Expert weights are quantised beforehand, untimed, as the library's

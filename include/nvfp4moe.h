@@ -396,8 +396,10 @@ NVFP4MOE_API void nvfp4moe_fp8_experts_destroy(nvfp4moe_fp8_experts* experts);
 
 /* The FP8 layer: arguments as nvfp4moe_forward, with its own workspace size.  dbg: idx, w,
  * counts, offsets, perm, logits, xq8_codes and xq8_scales are filled; the NVFP4-specific
- * members and events are ignored.  Launches: router (2), grouping (1 or 3), quantise-scatter,
- * gate/up GEMM, requantisation of h, down GEMM, finalize. */
+ * members and events are ignored.  Launches: routing and grouping (T <= 64: the fused
+ * front-end launch of nvfp4moe_forward without its NVFP4 quantisation; above: router 2 or 4,
+ * grouping 1 or 3), quantise-scatter, gate/up GEMM, requantisation of h, down GEMM,
+ * finalize. */
 NVFP4MOE_API size_t nvfp4moe_forward_fp8_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
 NVFP4MOE_API int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* experts, const void* hidden_bf16, int64_t T,
                                       const float* w_router, const float* logit_bias, void* out_bf16,

@@ -234,7 +234,12 @@ ForwardFp8Ws carve_forward_fp8(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.hdr = c.take<WsHeader>(1);
   const int n_part = router_amax_partials(T, cfg.E, cfg.H);
   f.partials = c.take<uint32_t>(n_part > kMaxAmaxPartials ? n_part : kMaxAmaxPartials);
-  f.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
+  size_t n_parts = router_parts_elems(T, cfg.E, cfg.H);
+  if (T <= kFrontMaxT) {
+    const size_t nf = (size_t)front_ksplit(cfg.E, cfg.H) * (size_t)T * (size_t)cfg.E;
+    if (nf > n_parts) n_parts = nf;
+  }
+  f.parts = c.take<double>(n_parts);
   f.idx = c.take<int32_t>(pairs);
   f.wts = c.take<float>(pairs);
   f.acc = c.take<float>(T * cfg.H);
@@ -943,42 +948,75 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
     return NVFP4MOE_ERR_CUDA;
   if (cudaMemsetAsync(&f.hdr->status, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
 
-  RouterArgs r{};
-  r.x = static_cast<const uint16_t*>(hidden_bf16);
-  r.w = w_router;
-  r.bias = logit_bias;
-  r.parts = f.parts;
-  r.idx = f.idx;
-  r.wts = f.wts;
-  r.T = T;
-  r.H = c.H;
-  r.E = c.E;
-  r.n_groups = c.n_groups;
-  r.topk_groups = c.topk_groups;
-  r.topk = c.topk;
-  r.routed_scale = c.routed_scale;
-  r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
-  r.amax_partials = f.partials;
-  r.status = &f.hdr->status;
-  set_router_tc(r, f.tc, f.a_codes);
-  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  g_launches += router_launch_count(r);
+  if (front_supported(T, c.E, c.H)) {
+    // small T: routing and grouping in the fused front-end launch (its NVFP4 quantisation
+    // is skipped: no segment buffers)
+    FrontArgs fa{};
+    fa.x = static_cast<const uint16_t*>(hidden_bf16);
+    fa.w = w_router;
+    fa.bias = logit_bias;
+    fa.T = T;
+    fa.H = c.H;
+    fa.E = c.E;
+    fa.n_groups = c.n_groups;
+    fa.topk_groups = c.topk_groups;
+    fa.topk = c.topk;
+    fa.routed_scale = c.routed_scale;
+    fa.parts = f.parts;
+    fa.amax_partials = f.partials;
+    fa.idx = f.idx;
+    fa.wts = f.wts;
+    fa.logits_out = dbg != nullptr ? dbg->logits : nullptr;
+    fa.counts = f.counts;
+    fa.offsets = f.offsets;
+    fa.mtile_prefix = f.mtile_prefix;
+    fa.perm = f.perm;
+    fa.inv = f.inv;
+    fa.row_pair = f.row_pair;
+    fa.n_col_tiles = c.H / 64;
+    fa.acc = f.acc;
+    fa.status = &f.hdr->status;
+    fa.barrier = &f.hdr->barrier;
+    if (launch_front(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ++g_launches;
+  } else {
+    RouterArgs r{};
+    r.x = static_cast<const uint16_t*>(hidden_bf16);
+    r.w = w_router;
+    r.bias = logit_bias;
+    r.parts = f.parts;
+    r.idx = f.idx;
+    r.wts = f.wts;
+    r.T = T;
+    r.H = c.H;
+    r.E = c.E;
+    r.n_groups = c.n_groups;
+    r.topk_groups = c.topk_groups;
+    r.topk = c.topk;
+    r.routed_scale = c.routed_scale;
+    r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
+    r.amax_partials = f.partials;
+    r.status = &f.hdr->status;
+    set_router_tc(r, f.tc, f.a_codes);
+    if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    g_launches += router_launch_count(r);
 
-  PermArgs pa{};
-  pa.idx = f.idx;
-  pa.T = T;
-  pa.topk = c.topk;
-  pa.E = c.E;
-  pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
-  pa.chunk_counts = f.chunk_counts;
-  pa.chunk_base = f.chunk_base;
-  pa.counts = f.counts;
-  pa.offsets = f.offsets;
-  pa.mtile_prefix = f.mtile_prefix;
-  pa.perm = f.perm;
-  pa.inv = f.inv;
-  pa.row_pair = f.row_pair;
-  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    PermArgs pa{};
+    pa.idx = f.idx;
+    pa.T = T;
+    pa.topk = c.topk;
+    pa.E = c.E;
+    pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
+    pa.chunk_counts = f.chunk_counts;
+    pa.chunk_base = f.chunk_base;
+    pa.counts = f.counts;
+    pa.offsets = f.offsets;
+    pa.mtile_prefix = f.mtile_prefix;
+    pa.perm = f.perm;
+    pa.inv = f.inv;
+    pa.row_pair = f.row_pair;
+    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  }
 
   Fp8ScatterArgs qa{static_cast<const uint16_t*>(hidden_bf16), T, c.H, c.topk, f.idx, f.inv, f.offsets,
                     f.mtile_prefix, f.a_codes, f.a_scale, f.acc,

@@ -328,6 +328,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(FrontArgs a) {
       a.row_pair[row] = p;
     }
   }
+  // without segment buffers (the FP8 variant quantises in its own kernel) the grouping ends it
+  if (a.seg_codes == nullptr) return;
   // global scale of x from the per-slice maxima
   __shared__ float s_g;
   __shared__ int s_nonfinite;

@@ -99,7 +99,7 @@ struct FrontArgs {
   int32_t* perm;            // [T*topk]
   int32_t* inv;             // [T*topk]
   int32_t* row_pair;        // [rows_cap]
-  uint8_t* seg_codes;       // [rows_cap][H/2]
+  uint8_t* seg_codes;       // [rows_cap][H/2]; nullptr: routing and grouping only (no quantisation)
   uint8_t* seg_sf;          // swizzled [rows_cap][H/16]
   int64_t n_col_tiles;      // H / 64
   uint8_t* xq_codes;        // optional token-major copy [T][H/2]

@@ -13,14 +13,20 @@ namespace nvfp4moe {
 __global__ void __launch_bounds__(256) amax_partial_kernel(const uint4* __restrict__ x, int64_t n_vec,
                                                            uint32_t* __restrict__ partials) {
   uint32_t m = 0;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint4 v = __ldg(x + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // four independent 16-byte loads in flight per thread and iteration
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec; i += 4 * stride) {
+    uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = max(m, w[j] & 0x7FFFu);
-      m = max(m, (w[j] >> 16) & 0x7FFFu);
+    for (int u = 0; u < 4; ++u) v[u] = i + u * stride < n_vec ? __ldg(x + i + u * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, w[j] & 0x7FFFu);
+        m = max(m, (w[j] >> 16) & 0x7FFFu);
+      }
     }
   }
 #pragma unroll
@@ -36,7 +42,7 @@ __global__ void __launch_bounds__(256) amax_partial_kernel(const uint4* __restri
   }
 }
 
-// One thread quantises 64 consecutive values of a row (4 blocks of 16).  Rows in
+// One warp quantises 512 consecutive values of a row, one 16-value block per lane.  Rows in
 // [rows, rows_padded) only write zero scales (swizzled layout padding).
 __global__ void __launch_bounds__(256) quantize_kernel(QuantizeArgs a) {
   __shared__ float s_g;
