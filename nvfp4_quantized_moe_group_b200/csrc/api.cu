@@ -71,6 +71,7 @@ int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
 struct QuantWs {
   WsHeader* hdr;
   uint32_t* partials;
+  float* g;                // the dynamic global scale when the caller asks for none back
   size_t bytes;
 };
 
@@ -79,6 +80,7 @@ QuantWs carve_quant(void* ws) {
   QuantWs q;
   q.hdr = c.take<WsHeader>(1);
   q.partials = c.take<uint32_t>(kMaxAmaxPartials);
+  q.g = c.take<float>(1);
   q.bytes = c.off;
   return q;
 }
@@ -362,10 +364,11 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   a.swizzled = scale_layout == NVFP4MOE_SCALES_SWIZZLED;
   a.n_col_tiles = cols / 64;
   a.g_out = g_out;
+  a.g_scratch = q.g;
   a.zero_out = nullptr;
   a.status = &q.hdr->status;
   if (launch_quantize(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ++g_launches;
+  g_launches += quantize_launch_count(a);
   return NVFP4MOE_OK;
 }
 
@@ -700,7 +703,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
     ev.mark(NVFP4MOE_STAGE_GATHER, 0);
     ev.mark(NVFP4MOE_STAGE_GATHER, 1);
-    ++g_launches;
+    g_launches += quantize_launch_count(q);
   }
 
   const int grid = num_sms();

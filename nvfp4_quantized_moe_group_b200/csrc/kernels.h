@@ -25,7 +25,8 @@ struct QuantizeArgs {
   uint8_t* scales;
   int swizzled;
   int64_t n_col_tiles;     // ceil(cols/16/4)
-  float* g_out;
+  float* g_out;            // the global scale used (may be nullptr)
+  float* g_scratch;        // dynamic scale with g_out == nullptr: where the scale is kept
   float* zero_out;         // optional [rows][cols] fp32 zeroed alongside (layer accumulator)
   uint32_t* status;
   // optional scatter into expert segments: row t also goes to the padded segment row of
@@ -133,7 +134,9 @@ struct RmsNormArgs {
 int amax_partial_blocks(int64_t n_elems);
 cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partials, int blocks,
                                 cudaStream_t stream);
-cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+// Dynamic scale (g_in == nullptr): a one-warp kernel reduces the amax partials first.
+cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream);
+int quantize_launch_count(const QuantizeArgs& a);
 
 // route.cu
 int router_ksplit(int64_t T, int E, int H);

@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
 __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
   __shared__ int s_cnt[256];
   __shared__ int s_tiles[256];
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 64;
   const int e = threadIdx.x;
   const int* __restrict__ cc = a.chunk_counts;
   int running = 0;

@@ -42,114 +42,113 @@ __global__ void __launch_bounds__(256) amax_partial_kernel(const uint4* __restri
   }
 }
 
-// One warp quantises 512 consecutive values of a row, one 16-value block per lane.  Rows in
-// [rows, rows_padded) only write zero scales (swizzled layout padding).
-__global__ void __launch_bounds__(256) quantize_kernel(QuantizeArgs a) {
-  __shared__ float s_g;
-  __shared__ int s_bad;
-  if (threadIdx.x < 32) {
-    float g;
-    int bad = 0;
-    if (a.g_in != nullptr) {
-      g = *a.g_in;
-    } else {
-      uint32_t m = 0;
-      for (int i = threadIdx.x; i < a.n_partials; i += 32) m = max(m, a.partials[i]);
+// The global scale from the amax partials (one warp): g = fp32(amax / 2688), 1 for amax 0;
+// a non-finite amax raises kStatusNonFinite and stores NaN, which makes the quantiser skip.
+__global__ void __launch_bounds__(32) global_scale_kernel(const uint32_t* partials, int n, float* g_out,
+                                                          uint32_t* status) {
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < n; i += 32) m = max(m, partials[i]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      bad = m >= 0x7F80u;
-      g = global_scale_from_amax(__uint_as_float(m << 16));
-    }
-    if (threadIdx.x == 0) {
-      s_g = g;
-      s_bad = bad;
-      if (blockIdx.x == 0) {
-        if (bad) raise_status(a.status, kStatusNonFinite);
-        if (a.g_out != nullptr) *a.g_out = g;
-      }
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (threadIdx.x == 0) {
+    if (m >= 0x7F80u) {
+      raise_status(status, kStatusNonFinite);
+      *g_out = __uint_as_float(0x7FC00000u);
+    } else {
+      *g_out = global_scale_from_amax(__uint_as_float(m << 16));
     }
   }
-  __syncthreads();
-  if (s_bad) return;
-  const float g = s_g;
+}
+
+// One CTA per row (rows_padded CTAs), min(segments, 32) warps: each warp quantises the row's
+// 512-value segments warp, warp + n_warps, ..., one 16-value block per lane.  Rows in
+// [rows, rows_padded) only write zero scales (swizzled layout padding).  The global scale is
+// read from g_in.
+__global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
+  const float g = __ldg(a.g_in);
+  if (!(g > 0.0f && g < __uint_as_float(0x7F800000u))) return;   // non-finite input: skipped
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.g_out != nullptr && a.g_out != a.g_in) *a.g_out = g;
   const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
 
   // one warp per (row, 512-value segment): lane l takes the 16-value block 32 seg + l, so every
   // load, code store and accumulator store of the warp covers one contiguous span of the row;
   // lanes 4k .. 4k+3 hold the 4 block scales of one 32-bit scale word
-  const int64_t blocks_per_row = a.cols >> 4;
-  const int64_t segs_per_row = (blocks_per_row + 31) >> 5;
+  const int blocks_per_row = (int)(a.cols >> 4);
+  const int segs_per_row = (blocks_per_row + 31) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t r = warp / segs_per_row;
-  if (r >= a.rows_padded) return;                      // uniform over the warp
-  const int64_t b = (warp - r * segs_per_row) * 32 + lane;
-  // lanes past the row's last block stay for the shuffles; groups of 4 lanes are active or
-  // idle together (cols % 64 == 0)
-  const bool active = b < blocks_per_row;
-  const bool live = active && r < a.rows;
-
-  if (a.zero_out != nullptr && live) {
-    float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
-    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) z[i] = zero;
+  const int n_warps = blockDim.x >> 5;
+  const int64_t r = blockIdx.x;
+  // segment rows of the token's pairs (lane j < topk holds pair j's), found once per warp
+  int64_t my_row = 0;
+  if (a.seg_codes != nullptr && r < a.rows && lane < a.topk) {
+    const int64_t p = r * a.topk + lane;
+    const int e = a.idx[p];
+    my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
   }
+  for (int seg = threadIdx.x >> 5; seg < segs_per_row; seg += n_warps) {
+    const int64_t b = (int64_t)seg * 32 + lane;
+    // lanes past the row's last block stay for the shuffles; groups of 4 lanes are active or
+    // idle together (cols % 64 == 0)
+    const bool active = b < blocks_per_row;
+    const bool live = active && r < a.rows;
 
-  uint32_t s = 0, c0 = 0, c1 = 0;
-  if (live) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + b * 16);
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float f[16];
-    uint32_t mb = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      f[2 * j] = __uint_as_float(w[j] << 16);
-      f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-      mb = max(mb, w[j] & 0x7FFFu);
-      mb = max(mb, (w[j] >> 16) & 0x7FFFu);
+    if (a.zero_out != nullptr && live) {
+      float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
+      const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  #pragma unroll
+      for (int i = 0; i < 4; ++i) z[i] = zero;
     }
-    float r_b;
-    s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
-    c0 = cvt_e2m1x8(f);
-    c1 = cvt_e2m1x8(f + 8);
-  }
-  // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes 4k)
-  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
-  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
-  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
-  const uint32_t sc = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
-  const bool word_lane = active && (lane & 3) == 0;
 
-  if (r < a.rows) {
-    if (a.codes != nullptr && active)
-      reinterpret_cast<uint2*>(a.codes + r * (a.cols >> 1))[b] = make_uint2(c0, c1);
-    if (a.seg_codes != nullptr) {
-      // lane j < topk finds pair j's segment row; every lane writes its block to all of them
-      int64_t my_row = 0;
-      if (lane < a.topk) {
-        const int64_t p = r * a.topk + lane;
-        const int e = a.idx[p];
-        my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
+    uint32_t s = 0, c0 = 0, c1 = 0;
+    if (live) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + b * 16);
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float f[16];
+      uint32_t mb = 0;
+  #pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        mb = max(mb, w[j] & 0x7FFFu);
+        mb = max(mb, (w[j] >> 16) & 0x7FFFu);
       }
-      for (int j = 0; j < a.topk; ++j) {
-        const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
-        if (active) reinterpret_cast<uint2*>(a.seg_codes + row * (a.cols >> 1))[b] = make_uint2(c0, c1);
-        if (word_lane) *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, b, a.n_col_tiles)) = sc;
+      float r_b;
+      s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
+  #pragma unroll
+      for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
+      c0 = cvt_e2m1x8(f);
+      c1 = cvt_e2m1x8(f + 8);
+    }
+    // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes 4k)
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
+    const uint32_t sc = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    const bool word_lane = active && (lane & 3) == 0;
+
+    if (r < a.rows) {
+      if (a.codes != nullptr && active)
+        reinterpret_cast<uint2*>(a.codes + r * (a.cols >> 1))[b] = make_uint2(c0, c1);
+      if (a.seg_codes != nullptr) {
+        // every lane writes its block to all of the token's segment rows
+        for (int j = 0; j < a.topk; ++j) {
+          const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+          if (active) reinterpret_cast<uint2*>(a.seg_codes + row * (a.cols >> 1))[b] = make_uint2(c0, c1);
+          if (word_lane) *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, b, a.n_col_tiles)) = sc;
+        }
       }
     }
+    if (a.scales != nullptr && word_lane) {
+      uint32_t* sdst;
+      if (a.swizzled) {
+        sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, b, a.n_col_tiles));
+      } else {
+        sdst = reinterpret_cast<uint32_t*>(a.scales + r * (a.cols >> 4) + b);
+      }
+      *sdst = sc;
+    }
   }
-  if (a.scales == nullptr || !word_lane) return;
-  uint32_t* sdst;
-  if (a.swizzled) {
-    sdst = reinterpret_cast<uint32_t*>(a.scales + swz_offset(r, b, a.n_col_tiles));
-  } else {
-    sdst = reinterpret_cast<uint32_t*>(a.scales + r * (a.cols >> 4) + b);
-  }
-  *sdst = sc;
 }
 
 int amax_partial_blocks(int64_t n_elems) {
@@ -167,11 +166,27 @@ cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partia
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
-  const int64_t threads = a.rows_padded * (((a.cols >> 4) + 31) >> 5) * 32;
-  const int64_t blocks = threads > 0 ? (threads + 255) / 256 : 1;  // one block still writes g_out
-  quantize_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream) {
+  if (a.g_in == nullptr) {
+    // dynamic scale: reduced once from the amax partials, then read by every CTA
+    float* g = a.g_out != nullptr ? a.g_out : a.g_scratch;
+    global_scale_kernel<<<1, 32, 0, stream>>>(a.partials, a.n_partials, g, a.status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    a.g_in = g;
+  }
+  if (a.rows_padded == 0) {
+    // no rows: only the scale used is reported
+    if (a.g_out != nullptr && a.g_out != a.g_in)
+      return cudaMemcpyAsync(a.g_out, a.g_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+    return cudaSuccess;
+  }
+  const int segs = (int)(((a.cols >> 4) + 31) >> 5);
+  const int warps = segs < 32 ? segs : 32;
+  quantize_kernel<<<(unsigned)a.rows_padded, 32 * warps, 0, stream>>>(a);
   return cudaGetLastError();
 }
+
+int quantize_launch_count(const QuantizeArgs& a) { return (a.g_in == nullptr ? 1 : 0) + (a.rows_padded > 0 ? 1 : 0); }
 
 }  // namespace nvfp4moe
