@@ -3,6 +3,11 @@
 // each group, keep the best topk_groups groups, pick the topk best experts inside them,
 // weights = routed_scale * s / sum(selected s).  FP32 throughout (section "Residual stream and
 // numerical decisions").
+//
+// This file holds the FP32 logits kernels (CUDA cores) and the top-k kernel.  The FP32
+// kernels serve T <= 64 when the fused front end cannot run, and every T in the
+// allocation-free router; with workspace for the digit planes, T > 64 takes the integer
+// tensor-core logits of route_tc.cu.
 #include "common.cuh"
 #include "kernels.h"
 #include "route_topk.cuh"
@@ -13,8 +18,8 @@ namespace {
 constexpr int kTM = 64;   // tokens per CTA tile (small-T kernel)
 constexpr int kTN = 64;   // experts per CTA tile
 constexpr int kTK = 32;   // K chunk; each chunk is summed into a fresh partial
-constexpr int kBigTM = 128;        // tokens per CTA tile (large-T kernel)
-constexpr int kBigMinT = 65;       // the large-T kernel runs from this many tokens on
+constexpr int kBigTM = 128;        // tokens per CTA tile (large-T FP32 kernel)
+constexpr int kBigMinT = 65;       // the large-T FP32 kernel runs from this many tokens on
 }  // namespace
 
 // Split-K logits: parts[ks][t][e] = sum over this CTA's K slice of x[t][k] * W[e][k].
