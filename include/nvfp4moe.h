@@ -112,7 +112,7 @@ NVFP4MOE_API int nvfp4moe_cfg_check(const nvfp4moe_cfg* cfg);
  *   g_out    out, device pointer to one FP32: the global scale used (may be NULL).
  *   ws       workspace of nvfp4moe_quantize_workspace_bytes(rows, cols) bytes.
  * A non-finite max|x| (dynamic scale) sets NVFP4MOE_ERR_NONFINITE in the status word;
- * codes and scales are then unspecified. */
+ * codes, scales and g_out are then unspecified.  rows < 2^31 - 128. */
 NVFP4MOE_API size_t nvfp4moe_quantize_workspace_bytes(int64_t rows, int64_t cols);
 NVFP4MOE_API size_t nvfp4moe_swizzled_scale_bytes(int64_t rows, int64_t cols16);
 NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const float* g_in,

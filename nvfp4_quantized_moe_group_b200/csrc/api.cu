@@ -332,6 +332,7 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   g_launches = 0;
   if (rows < 0 || cols <= 0 || cols % 64 != 0) return NVFP4MOE_ERR_SHAPE;
   if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (rows >= ((int64_t)1 << 31) - 128) return NVFP4MOE_ERR_SHAPE;   // one CTA per (padded) row
   if (scale_layout != NVFP4MOE_SCALES_LINEAR && scale_layout != NVFP4MOE_SCALES_SWIZZLED)
     return NVFP4MOE_ERR_ARG;
   if (ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
