@@ -87,24 +87,27 @@ QuantWs carve_quant(void* ws) {
 
 // Scratch of the integer tensor-core router (T >= kRouterTcMinT): digit planes of the expert
 // rows and the row exponents.  The token rows' planes (4 T H bytes) go to a buffer the caller
-// names (in the forward, the expert-segment input buffer, which is written only afterwards).
+// names when it is large enough (in the forward, the expert-segment input buffer, which is
+// written only afterwards), else to their own.
 struct RouterTcWs {
   uint8_t* w_digits = nullptr;
+  uint8_t* x_digits = nullptr;   // own planes, when the caller's buffer is too small
   int32_t* x_exp = nullptr;
   int32_t* w_exp = nullptr;
 };
 
-RouterTcWs carve_router_tc(Carver& c, const nvfp4moe_cfg& cfg, int64_t T) {
+RouterTcWs carve_router_tc(Carver& c, const nvfp4moe_cfg& cfg, int64_t T, size_t shared_bytes) {
   RouterTcWs r;
   if (T < kRouterTcMinT) return r;
   r.w_digits = c.take<uint8_t>((size_t)4 * cfg.E * cfg.H);
+  if (shared_bytes < (size_t)4 * T * cfg.H) r.x_digits = c.take<uint8_t>((size_t)4 * T * cfg.H);
   r.x_exp = c.take<int32_t>(T);
   r.w_exp = c.take<int32_t>(cfg.E);
   return r;
 }
 
-void set_router_tc(RouterArgs& r, const RouterTcWs& w, uint8_t* x_digits) {
-  r.x_digits = w.w_digits != nullptr ? x_digits : nullptr;
+void set_router_tc(RouterArgs& r, const RouterTcWs& w, uint8_t* shared) {
+  r.x_digits = w.w_digits == nullptr ? nullptr : (w.x_digits != nullptr ? w.x_digits : shared);
   r.w_digits = w.w_digits;
   r.x_exp = w.x_exp;
   r.w_exp = w.w_exp;
@@ -124,7 +127,7 @@ RouteWs carve_route(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   r.hdr = c.take<WsHeader>(1);
   r.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
   r.x_digits = T >= kRouterTcMinT ? c.take<uint8_t>((size_t)4 * T * cfg.H) : nullptr;
-  r.tc = carve_router_tc(c, cfg, T);
+  r.tc = carve_router_tc(c, cfg, T, T >= kRouterTcMinT ? (size_t)4 * T * cfg.H : 0);
   r.bytes = c.off;
   return r;
 }
@@ -197,7 +200,7 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg.I / 2);
   f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg.I / 16);
   f.x_norm = c.take<uint16_t>(T * cfg.H);
-  f.tc = carve_router_tc(c, cfg, T);
+  f.tc = carve_router_tc(c, cfg, T, (size_t)f.rows_cap * cfg.H / 2);
   f.bytes = c.off;
   return f;
 }
@@ -258,7 +261,7 @@ ForwardFp8Ws carve_forward_fp8(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   f.h32 = c.take<float>(f.rows_cap * cfg.I);
   f.hq = c.take<uint8_t>(f.rows_cap * cfg.I);
   f.h_scale = c.take<float>(f.rows_cap);
-  f.tc = carve_router_tc(c, cfg, T);
+  f.tc = carve_router_tc(c, cfg, T, (size_t)f.rows_cap * cfg.H);
   f.bytes = c.off;
   return f;
 }

@@ -195,6 +195,39 @@ def test_integer_router_logits_extreme_rows():
     assert np.all(got[0] == 0.0)
 
 
+def test_single_expert_per_token_large_batch():
+    """topk = 1 with few experts: the expert segments hold fewer rows than the router's four
+    digit planes of the tokens need, so the router takes its own scratch for them; routing
+    (near-tie protocol) and outputs still match the oracle."""
+    from workloads import LayerShape
+    shape = LayerShape(H=256, I=128, E=8, n_groups=2, topk_groups=1, topk=1, routed_scale=1.0,
+                       wr_std=1.0 / 16.0, w_std=0.02)
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    g_h = np.full(shape.E, np.float32(0.004), dtype=np.float32)
+    ex = moe.Experts(cfg)
+    for e in range(shape.E):
+        ex.set_from_bf16(e, *(expert_weight(shape, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    T = 600
+    x = activations(T, shape, seed=13)
+    wr = router_weight(shape)
+    ws = torch.empty(moe.forward_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    out, dbg = moe.forward(ex, x.cuda(), wr.cuda(), ws=ws, debug=True)
+    assert moe.status_read(ws) == moe.OK
+    xn = x.float().numpy()
+    toks = [0, 1, 299, 599]
+    ref = oracle_layer(shape, xn, wr.numpy(), None, g_h, tokens=toks)
+    idx = dbg["idx"].cpu().numpy()
+    check_routing(idx, dbg["w"].cpu().numpy(), ref["route"], xn.astype(np.float64),
+                  wr.numpy().astype(np.float64), None, shape)
+    check_grouping(dbg, idx, shape.E)
+    same = np.array([(idx[t] == ref["route"].idx[t]).all() for t in toks])
+    assert same.sum() >= 1
+    check_output(out.float().cpu().numpy()[np.array(toks)[same]], ref["out"][same])
+    ex.close()
+
+
 @pytest.mark.parametrize("T", [16, 130])
 def test_nonfinite_router_weight_reported(T):
     """A NaN in the router weight makes one expert's logits NaN: the forward reports
