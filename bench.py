@@ -277,6 +277,51 @@ def run_fp8(moe, shape: LayerShape, cfg, x, wr, bias, T: int, steps: int, warmup
                     "tcgen05 kind::f8f6f4 grouped GEMMs; same batch and routing as the NVFP4 line"}
 
 
+def e2e_pipelined(moe, ex, x_cpu, wr, bias, ws, T: int, H: int, warmup: int, steps: int, world: int) -> float:
+    """Device time of ``steps`` forwards fed from pinned host memory: per step one host-to-device
+    copy of the step's tokens and one device-to-host copy of its output, on a copy stream with
+    two buffers each, overlapped with the neighbouring steps' compute.  Returns the elapsed
+    milliseconds (max over ranks), from before the first copy in to after the last copy out."""
+    stream = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    x_host = x_cpu.pin_memory()
+    out_host = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    out_dev = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    h2d = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        copy.wait_stream(stream)
+        with torch.cuda.stream(copy):
+            for b in range(min(2, n)):
+                x_dev[b].copy_(x_host, non_blocking=True)
+                h2d[b].record(copy)
+        for k in range(n):
+            b = k & 1
+            stream.wait_event(h2d[b])
+            moe.forward(ex, x_dev[b], wr, bias, out=out_dev[b], ws=ws)
+            done[b].record(stream)
+            copy.wait_event(done[b])
+            with torch.cuda.stream(copy):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                if k + 2 < n:
+                    x_dev[b].copy_(x_host, non_blocking=True)
+                    h2d[b].record(copy)
+        stream.wait_stream(copy)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
 def _oracle_cfg(shape: LayerShape):
     import types
     return types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
@@ -422,26 +467,10 @@ def run_ours(args, world, rank, local):
     if st != moe.OK:
         raise RuntimeError(f"forward status {moe.status_string(st)}")
 
-    # ---- end to end: pinned host input -> device, forward, device -> pinned host output
-    x_host = x_cpu.pin_memory()
-    out_host = torch.empty((T, shape.H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(args.warmup):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.forward(ex, x_dev, wr, bias, out=out, ws=ws)
-        out_host.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.forward(ex, x_dev, wr, bias, out=out, ws=ws)
-        out_host.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # ---- end to end: pinned host input -> device, forward, device -> pinned host output.  Every
+    # step copies its tokens in and its output rows out; the copies run on a second stream,
+    # double-buffered, so that step k+1's input and step k-1's output move while step k computes
+    e2e_ms = e2e_pipelined(moe, ex, x_cpu, wr, bias, ws, T, shape.H, args.warmup, args.steps, world)
 
     # ---- the same step replayed from a CUDA graph (one capture, K replays; launch cost removed)
     graph = torch.cuda.CUDAGraph()
