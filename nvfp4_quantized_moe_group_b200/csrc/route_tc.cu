@@ -1,6 +1,7 @@
 // Router logits for T > 64 on the tensor cores, in exact integer arithmetic ("Reflection
-// releases Beam ...", section "Mixture-of-Experts details": every token scores all experts;
-// the router runs in full precision).
+// releases Beam ...", section "Mixture-of-Experts details": every token scores all 256
+// experts; section "Residual stream and numerical decisions": the router runs in FP32, and
+// these logits are more accurate than an FP32 accumulation).
 //
 // Each token row x_t (BF16) and each expert row W_e (FP32) is scaled by a power of two to
 // 30-bit fixed point: with e the binary exponent of the row's largest magnitude
@@ -9,7 +10,8 @@
 // d1..d3 in [-128, 127] and |d0| <= 64.  Then
 //     X . W = sum_{i,j} (a_i . b_j) 2^(8 (6 - i - j)),
 // and the 13 digit pairs with i + j <= 4 are multiplied by tcgen05 kind::i8 MMAs: int8 x int8
-// products accumulated in int32, which is exact (|class sum| < 5 * 2^14 * H < 2^31).  One
+// products accumulated in int32, which is exact (|class sum| < 5 * 2^14 * K < 2^31 for the
+// K <= 26,112 columns of one split).  One
 // tensor-memory accumulator per class c = i + j; the epilogue combines the five classes in
 // FP64 and scales by 2^(e_x + e_W - 60).  Error against the exact logit, before the FP32
 // rounding of the sum with the bias:
