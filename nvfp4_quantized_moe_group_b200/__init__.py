@@ -3,6 +3,22 @@
 The layer and its contracts are documented in include/nvfp4moe.h; this package is the
 thin Python binding of libnvfp4moe.so (ctypes; torch supplies device memory and
 streams).  Build the library with ``python -m nvfp4_quantized_moe_group_b200.build``.
+
+Typical use (all tensors on one CUDA device; the current stream is used)::
+
+    import nvfp4_quantized_moe_group_b200 as moe
+    cfg = moe.cfg_default()                       # 256 experts, 8 groups, top-4/top-8, x2.5
+    experts = moe.Experts(cfg)                    # library-owned NVFP4 weights
+    for e in range(cfg.E):                        # BF16 gate/up [I, H], down [H, I], static g_h
+        experts.set_from_bf16(e, gate[e], up[e], down[e], g_h[e])
+    ws = torch.empty(moe.forward_workspace_bytes(cfg, T_max), dtype=torch.uint8, device="cuda")
+    out = moe.forward(experts, x_bf16, w_router_fp32, ws=ws)    # [T, H] BF16
+    assert moe.status_read(ws) == moe.OK
+
+Also: ``quantize`` / ``route`` (the layer's steps alone), ``forward_residual`` (RMSNorm in,
+weighted residual add out), ``quantize_weights_lh`` (local-Hessian weight scales),
+``Fp8Experts`` / ``forward_fp8`` (the FP8 W8A8 variant), and ``ep.ExpertParallelLayer`` with
+``forward_partial`` / ``finalize`` (experts spread over the ranks of a process group).
 """
 from ._lib import (  # noqa: F401
     Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, forward,
