@@ -1,5 +1,5 @@
-"""Expert parallelism on the CPU: two gloo ranks (world size 2) run ExpertParallelLayer with
-the oracle standing in for each rank's partial layer (its 16 of the tiny layer's 32 experts).
+"""Expert parallelism on the CPU: gloo ranks (world size 2 and 4) run ExpertParallelLayer with
+the oracle standing in for each rank's partial layer (its share of the tiny layer's 32 experts).
 The exchange (all-gather of the tokens, reduce-scatter of the FP32 sums) must give every rank
 the oracle's whole-layer output for its own tokens ("Reflection releases Beam ...", section
 "Tool calling and multi-node setups": experts placed on the devices, the rest replicated)."""
@@ -53,8 +53,8 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_expert_parallel_layer():
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_expert_parallel_layer(world):
     with mp.Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
@@ -63,7 +63,8 @@ def test_two_gloo_ranks_expert_parallel_layer():
     from workloads import TINY, router_weight
     from tests.helpers import oracle_layer, intermediate_scales, bf16_half_ulp
     # disjoint expert shares covering all experts, each rank called once on all tokens
-    assert [(res[r][0], res[r][1]) for r in range(world)] == [(0, 16), (16, 16)]
+    n = TINY.E // world
+    assert [(res[r][0], res[r][1]) for r in range(world)] == [(r * n, n) for r in range(world)]
     assert all(res[r][2] == [(world * T_RANK, res[r][0], res[r][1])] for r in range(world))
     # every rank's output is the whole layer on its own tokens
     x_all = np.concatenate([res[r][4] for r in range(world)])
