@@ -584,7 +584,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
 
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
   // status word and grid-barrier counter
-  if (cudaMemsetAsync(&f.hdr->status, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  // status word, front-end barrier and the two GEMM work counters
+  if (cudaMemsetAsync(&f.hdr->status, 0, 4 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
 
   if (front_supported(T, c.E, c.H)) {
@@ -738,6 +739,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.topk = c.topk;
   g.H = c.H;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
+  g.work_counter = &f.hdr->work[0];
   if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
   ++g_launches;
@@ -747,6 +749,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.K = c.I;
   g.n_total = c.H;
   ev.mark(NVFP4MOE_STAGE_DOWN, 0);
+  g.work_counter = &f.hdr->work[1];
   if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_DOWN, 1);
   ++g_launches;
@@ -953,7 +956,8 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
       make_tma_2d(&tma_h, f.hq, c.I, f.rows_cap, kBlockM) != 0 ||
       make_tma_2d(&tma_h32, f.hq, c.I, f.rows_cap, 32) != 0)
     return NVFP4MOE_ERR_CUDA;
-  if (cudaMemsetAsync(&f.hdr->status, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  // status word, front-end barrier and the two GEMM work counters
+  if (cudaMemsetAsync(&f.hdr->status, 0, 4 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
 
   if (front_supported(T, c.E, c.H)) {
     // small T: routing and grouping in the fused front-end launch (its NVFP4 quantisation
@@ -1051,6 +1055,7 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
   g.a_scale = f.a_scale;
   g.w_scale = x->w13_scale;
   g.h32 = f.h32;
+  g.work_counter = &f.hdr->work[0];
   if (launch_gemm_gateup_fp8(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   Fp8RequantArgs ra{f.h32, f.rows_cap, c.I, f.row_pair, f.mtile_prefix, c.E, f.hq, f.h_scale, &f.hdr->status};
   if (launch_fp8_requant_rows(ra, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
@@ -1059,6 +1064,7 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
   g.n_total = c.H;
   g.w_scale = x->wd_scale;
   g.h_scale = f.h_scale;
+  g.work_counter = &f.hdr->work[1];
   if (launch_gemm_down_fp8(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, nullptr, 0.0f, 0.0f};
   if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;

@@ -23,7 +23,8 @@ enum : uint32_t {
 struct WsHeader {
   uint32_t status;
   uint32_t barrier;   // grid-barrier counter of the fused front kernel
-  uint32_t pad[62];
+  int32_t work[2];    // work counters of the gate/up and down GEMMs
+  uint32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

@@ -35,6 +35,7 @@ namespace {
 
 constexpr int kThreads = 320;                 // producer, MMA issuer, 8 epilogue warps
 constexpr int kEpiWarps = 8;
+constexpr int kWorkRing = 4;                  // items the producer may run ahead of the epilogue
 constexpr int kABytes = kBlockM * 128;        // 128 rows x 256 E2M1
 constexpr int kTileBytes = 128 * 128;         // one 128-row weight tile x 256 K values
 constexpr int kAtomBytes = 512;               // one 128-row block-scale atom (one 64-deep K step)
@@ -84,6 +85,9 @@ struct __align__(1024) Smem {
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
+  uint64_t work_full[kWorkRing];    // the producer published the item of this slot
+  uint64_t work_empty[kWorkRing];   // the MMA issuer and the epilogue warps have read it
+  int work[kWorkRing];              // item index, -1: no more items
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -224,6 +228,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     mbar_init(&s.acc_full, 1);
     mbar_init(&s.acc_empty, kEpiWarps);
     mbar_init(&s.drain, 1);
+    for (int i = 0; i < kWorkRing; ++i) {
+      mbar_init(&s.work_full[i], 1);
+      mbar_init(&s.work_empty[i], kEpiWarps + 1);
+    }
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -262,7 +270,19 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+      for (int it = 0; ok; ++it) {
+        // items are handed out dynamically: the first is the CTA's own index, the next ones
+        // come from a counter shared by the grid, so CTAs that run faster take more items
+        const int slot = it & (kWorkRing - 1);
+        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_empty[slot], ((uint32_t)(it / kWorkRing) & 1u) ^ 1u)) {
+          set_abort(&s.abort_flag, p.status);
+          break;
+        }
+        int w = it == 0 ? (int)blockIdx.x : atomicAdd(p.work_counter, 1) + (int)gridDim.x;
+        if (w >= total) w = -1;
+        s.work[slot] = w;
+        mbar_arrive(&s.work_full[slot]);      // releases the index to the MMA issuer and the epilogue
+        if (w < 0) break;
         const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
         const int arow = wk.mtile * kBlockM;
         const bool a_small = wk.rows_valid <= 32;
@@ -308,8 +328,15 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       uint32_t stage = 0, phase = 0;
       const uint32_t idesc = kFp8 ? idesc_f8(kN) : idesc_nvf4(kN);
       bool ok = true;
-      int it = 0;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
+      for (int it = 0; ok; ++it) {
+        const int slot = it & (kWorkRing - 1);
+        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u)) {
+          set_abort(&s.abort_flag, p.status);
+          break;
+        }
+        const int w = *reinterpret_cast<volatile int*>(&s.work[slot]);
+        mbar_arrive(&s.work_empty[slot]);
+        if (w < 0) break;
         const uint32_t acc_par = (uint32_t)it & 1u;
         if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u)) {
           set_abort(&s.abort_flag, p.status);
@@ -367,8 +394,17 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     const int q = warp & 3;              // tensor-memory lane quarter this warp may read
     const int half = (warp - 2) >> 2;    // which half of the tile's columns it handles
     const int row_l = q * 32 + lane;
-    int it = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+    for (int it = 0;; ++it) {
+      const int slot = it & (kWorkRing - 1);
+      const bool got_work = !aborted(&s.abort_flag) && mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u);
+      if (__any_sync(0xffffffffu, !got_work)) {
+        set_abort(&s.abort_flag, p.status);
+        break;
+      }
+      const int w = *reinterpret_cast<volatile int*>(&s.work[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.work_empty[slot]);
+      if (w < 0) break;
       const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
       const uint32_t acc_par = (uint32_t)it & 1u;
       const int64_t row = (int64_t)wk.mtile * kBlockM + row_l;

@@ -22,6 +22,7 @@ struct GemmArgs {
   int K;                       // reduction length
   int n_total;                 // B rows per expert (2I for gate/up, H for down)
   uint32_t* status;
+  int* work_counter;           // zero at launch: items handed out beyond the first gridDim.x
   // gate/up epilogue
   uint8_t* hq_codes;           // [rows_cap][I/2]
   uint8_t* hq_sf;              // swizzled [rows_cap][I/16]
