@@ -1,9 +1,11 @@
 // Grouped block-scaled NVFP4 GEMMs of the expert MLPs on the 5th-generation tensor cores.
 //
 // Each expert's token rows form a segment padded to 128 rows; a work item is one
-// (expert, 256-column tile, 128-row tile).  One persistent CTA per SM walks work items
-// (expert-major, then column tile, then row tile, so row tiles of one expert that share a
-// weight tile run at the same time and the second read of that tile comes from L2).
+// (expert, 256-column tile, 128-row tile).  One persistent CTA per SM takes work items in
+// index order (expert-major, then column tile, then row tile, so row tiles of one expert that
+// share a weight tile run at the same time and the second read of that tile comes from L2):
+// its first item is its own CTA index, the following ones are claimed from a grid-wide
+// counter, so faster CTAs take more items.
 //
 // Per CTA: warp 0 fills a shared-memory ring: the A tile by a TMA load with 128-byte
 // swizzle (a 32-row box when at most 32 rows of the tile hold pairs, as at decode: the
