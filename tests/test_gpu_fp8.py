@@ -57,6 +57,21 @@ def test_quantize_fp8_bit_exact(rows, cols):
     np.testing.assert_array_equal(codes.cpu().numpy(), ref_c)
 
 
+def test_quantize_fp8_division_tie_and_negative_zero():
+    """A value whose FP32 quotient v / s is exactly the E4M3 midpoint 5.25 (the tie goes to the
+    even code 0x4A; a multiply by fp32(1 / s) would land above it and give 0x4B), and signed
+    zeros (-0 keeps its sign bit, 0x80), bit-exact against the oracle."""
+    x = torch.zeros(2, 16)
+    x[0, :4] = torch.tensor([1.078125, 0.01263427734375, -0.0, 0.0])
+    x[1, :4] = torch.tensor([-1.078125, -0.01263427734375, 0.0, -0.0])
+    x = x.to(torch.bfloat16)
+    codes, scales = moe.quantize_fp8(x.cuda())
+    ref_c, ref_s = oracle.fp8.quantize_rows(x.float().numpy())
+    assert list(ref_c[0, :4]) == [0x7E, 0x4A, 0x80, 0x00]
+    np.testing.assert_array_equal(scales.cpu().numpy(), ref_s)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_c)
+
+
 def test_quantize_fp8_expert_weights_bit_exact():
     """The weights the layer uses: the GPU's per-channel codes and scales equal the oracle's."""
     for w in ("gate", "down"):

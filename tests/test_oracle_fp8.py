@@ -66,3 +66,51 @@ def test_expert_mlp_closed_form():
     np.testing.assert_array_equal(res["h"][0], h)
     hq = fp8.dequantize_rows(*fp8.quantize_rows(h[None]))[0]
     np.testing.assert_allclose(res["y"][0], 448 * hq, rtol=1e-15)
+
+
+def test_division_reading_at_an_e4m3_tie():
+    """The reading "code = E4M3_rne(fp32(v / s)) with one IEEE division" at a value where it
+    matters: for the row [1.078125, 0.01263427734375] the scale is s = fp32(1.078125 / 448) and
+    fp32(v / s) is exactly 5.25, the midpoint of E4M3 5.0 (code 0x4A) and 5.5 (0x4B), so the
+    tie goes to the even code 0x4A; multiplying by fp32(1 / s) instead lands one FP32 step above
+    the midpoint and gives 0x4B.  A negative zero keeps its sign bit (0x80), as PyTorch's cast."""
+    v = np.array([[1.078125, 0.01263427734375, -0.0, 0.0]], dtype=np.float32)
+    codes, s = fp8.quantize_rows(v)
+    assert s[0] == np.float32(v[0, 0]) / np.float32(448.0)
+    q = v / s[:, None]                                   # NumPy float32 division, IEEE RN
+    assert q[0, 1] == 5.25
+    ref = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(codes, ref)
+    assert list(codes[0]) == [0x7E, 0x4A, 0x80, 0x00]
+    q_mul = v * (np.float32(1.0) / s)[:, None]
+    assert torch.from_numpy(q_mul).to(torch.float8_e4m3fn).view(torch.uint8).numpy()[0, 1] == 0x4B
+
+
+def _tiny_fp8_layer(T):
+    from workloads import TINY, activations, router_weight, expert_weight
+    import types
+    shape = TINY
+    cfg = types.SimpleNamespace(E=shape.E, n_groups=shape.n_groups, topk_groups=shape.topk_groups,
+                                topk=shape.topk, routed_scale=shape.routed_scale)
+    x = activations(T, shape).float().numpy()
+    wr = router_weight(shape).numpy()
+    ex = {e: tuple(fp8.Fp8Tensor(expert_weight(shape, e, w).float().numpy()) for w in ("gate", "up", "down"))
+          for e in range(shape.E)}
+    return shape, cfg, x, wr, ex
+
+
+def test_fp8_layer_matches_dense_formulation():
+    """Gathered per-expert evaluation == every expert on every token weighted by a dense [T, E]
+    matrix of the router weights; the layer input is the per-token FP8 quantisation of x."""
+    shape, cfg, x, wr, ex = _tiny_fp8_layer(20)
+    res = fp8.moe_forward_fp8(x, wr, cfg, lambda e: ex[e])
+    r = res["route"]
+    xq, xs = fp8.quantize_rows(x)
+    np.testing.assert_array_equal(res["xq_codes"], xq)
+    xhat = fp8.dequantize_rows(xq, xs)
+    dense_w = np.zeros((x.shape[0], shape.E))
+    np.put_along_axis(dense_w, r.idx, r.w, axis=1)
+    y_all = np.stack([fp8.expert_mlp_fp8(xhat, *ex[e])["y"] for e in range(shape.E)], axis=1)
+    np.testing.assert_allclose(res["out"], np.einsum("te,teh->th", dense_w, y_all), rtol=1e-12, atol=1e-12)
+    part = fp8.moe_forward_fp8(x, wr, cfg, lambda e: ex[e], tokens=[7, 2, 19])
+    np.testing.assert_allclose(part["out"], res["out"][[7, 2, 19]], rtol=1e-12, atol=1e-15)

@@ -79,3 +79,48 @@ def test_zero_blocks_stay_zero():
 
 def test_candidate_order():
     assert oracle.candidate_offsets(2) == [0, -1, 1, -2, 2]
+
+
+def test_zero_hessian_keeps_the_rounding_rule():
+    """With H_b = 0 every candidate's error is 0; a candidate replaces the best only when strictly
+    better, so the search keeps the round-to-nearest scale S0 (the first visited)."""
+    w = _weights(8, 64, 8)
+    codes, S, g, errs, cands = oracle.quantize_local_hessian(w, np.zeros((4, 16, 16)), m=4)
+    assert np.all(errs == 0)
+    c_ref, s_ref, _ = oracle.quantize(w)
+    np.testing.assert_array_equal(S, s_ref)
+    np.testing.assert_array_equal(codes, c_ref)
+
+
+def test_h_weighting_decides():
+    """The block [2.75, 1.875, 0.1875, 0, ...] under tensor amax 168 (g = 1/16): S0 = code 79
+    (7.5, d = 0.46875) represents 1.875 = 4 d exactly and misses 2.75 by 0.0625; code 83 (11,
+    d = 0.6875) represents 2.75 = 4 d exactly and misses 1.875 by 0.1875 (1.875 / d = 2.73 ->
+    E2M1 3); of the codes 75 .. 83 only 76 (6, d = 0.375, below S0) represents 0.1875 = d / 2
+    exactly.  Weighting only element 0 the search must take 83, only element 2 it must take
+    76, and only element 1 it must keep 79 (code 82, d = 0.625, also represents 1.875 exactly,
+    as 3 d: that tie keeps S0, the first visited)."""
+    w = np.zeros((2, 16), dtype=np.float32)
+    w[0, 0] = 168.0
+    w[1, 0], w[1, 1], w[1, 2] = 2.75, 1.875, 0.1875
+    for k, want in ((0, 83), (1, 79), (2, 76)):
+        H = np.zeros((1, 16, 16))
+        H[0, k, k] = 1.0
+        codes, S, g, errs, cands = oracle.quantize_local_hessian(w, H, m=4)
+        assert g == np.float32(1 / 16) and cands[1, 0, 0] == 79
+        assert S[1, 0] == want, (k, S[1, 0])
+        deq = oracle.dequantize(codes, S, g)
+        assert deq[1, k] == w[1, k]
+
+
+def test_hessian_blocks_by_loops():
+    """H_b[i, j] = sum over tokens of x[n, 16 b + i] x[n, 16 b + j], by plain loops."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((5, 48))
+    H = oracle.hessian_blocks(x)
+    assert H.shape == (3, 16, 16)
+    for b in range(3):
+        for i in range(16):
+            for j in range(16):
+                want = sum(x[n, 16 * b + i] * x[n, 16 * b + j] for n in range(5))
+                assert abs(H[b, i, j] - want) <= 1e-12 * max(1.0, abs(want))

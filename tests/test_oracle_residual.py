@@ -70,3 +70,12 @@ def test_rmsnorm_scale_invariance_and_zero_rows():
     np.testing.assert_array_equal(z, np.zeros((2, 64), dtype=np.float32))
     # eps only lowers the scale
     assert np.all(oracle.rmsnorm_scale(h, 1e-2) <= oracle.rmsnorm_scale(h, 0.0))
+
+
+def test_rmsnorm_eps_inside_the_root():
+    """A constant row of ones with eps = 3: mean(h^2) + eps = 4, r = 1/2 exactly, so
+    x = gamma / 2 (BF16-exact gammas)."""
+    gamma = np.array([1.0, -2.0, 0.375, 96.0], dtype=np.float32)
+    x = oracle.rmsnorm(np.ones((1, 4), dtype=np.float32), gamma, 3.0)
+    np.testing.assert_array_equal(x[0], gamma / 2)
+    assert oracle.rmsnorm_scale(np.ones((1, 4)), 3.0)[0] == np.float32(0.5)

@@ -106,3 +106,24 @@ def test_ties_go_to_lower_index():
     wr = np.zeros((8, 4))                 # every score equal
     r = oracle.route(x, wr, _cfg(8, 4, 2, 3))
     assert list(r.groups[0]) == [0, 1] and list(r.idx[0]) == [0, 1, 2]
+
+
+def test_decision_margins_by_sorting():
+    """The margins the parity protocol uses to tell FP32 near-ties from mismatches, rebuilt with
+    Python sorts from sigmoid scores the test computes itself: the last kept group's score minus
+    the best dropped group's, the last selected expert's score minus the best unselected
+    admissible one's, and the smallest gap between consecutive selected scores."""
+    cfg = _cfg(TINY.E, TINY.n_groups, TINY.topk_groups, TINY.topk)
+    x = activations(16, TINY).float().numpy().astype(np.float64)
+    wr = router_weight(TINY).numpy().astype(np.float64)
+    r = oracle.route(x, wr, cfg)
+    s = 1 / (1 + np.exp(-(x @ wr.T)))
+    gs = TINY.E // TINY.n_groups
+    for t in range(x.shape[0]):
+        gsc = [sum(sorted(s[t, g * gs:(g + 1) * gs].tolist(), reverse=True)[:2]) for g in range(TINY.n_groups)]
+        gord = sorted(range(TINY.n_groups), key=lambda g: (-gsc[g], g))
+        np.testing.assert_allclose(r.group_margin[t], gsc[gord[3]] - gsc[gord[4]], rtol=1e-12, atol=0)
+        cand = sorted((e for g in gord[:4] for e in range(g * gs, (g + 1) * gs)), key=lambda e: (-s[t, e], e))
+        np.testing.assert_allclose(r.expert_margin[t], s[t, cand[7]] - s[t, cand[8]], rtol=1e-12, atol=0)
+        sel = [s[t, e] for e in cand[:8]]
+        np.testing.assert_allclose(r.order_margin[t], min(a - b for a, b in zip(sel, sel[1:])), rtol=1e-12, atol=0)
