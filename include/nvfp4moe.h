@@ -112,7 +112,8 @@ NVFP4MOE_API int nvfp4moe_cfg_check(const nvfp4moe_cfg* cfg);
  *   g_out    out, device pointer to one FP32: the global scale used (may be NULL).
  *   ws       workspace of nvfp4moe_quantize_workspace_bytes(rows, cols) bytes.
  * A non-finite max|x| (dynamic scale) sets NVFP4MOE_ERR_NONFINITE in the status word;
- * codes, scales and g_out are then unspecified.  rows < 2^31 - 128. */
+ * codes, scales and g_out are then unspecified.  Limits: rows < 2^31 - 128, cols < 2^31,
+ * rows * cols < 2^40; outside them NVFP4MOE_ERR_SHAPE. */
 NVFP4MOE_API size_t nvfp4moe_quantize_workspace_bytes(int64_t rows, int64_t cols);
 NVFP4MOE_API size_t nvfp4moe_swizzled_scale_bytes(int64_t rows, int64_t cols16);
 NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const float* g_in,
@@ -124,7 +125,8 @@ NVFP4MOE_API int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t col
  * "Quantization method": for each 16-value block, candidate scales are tried and the one
  * minimising the Hessian-weighted error dW^T H dW is kept.
  *
- *   w_bf16 [rows][cols] BF16 weight matrix (rows >= 1, cols % 16 == 0, 16-byte aligned);
+ *   w_bf16 [rows][cols] BF16 weight matrix (1 <= rows < 2^31, cols % 16 == 0, cols / 16 <=
+ *       65535, rows * cols < 2^40, 16-byte aligned);
  *   hess_blocks [cols/16][16][16] FP32: for each 16-column block, the 16x16 diagonal block of
  *       H = X^T X over calibration inputs X of this projection (shared by all rows);
  *   m  0..16: candidates are the E4M3 scale codes S0-m .. S0+m (clamped to 1..0x7E) around the
@@ -209,8 +211,9 @@ typedef struct nvfp4moe_experts nvfp4moe_experts;
 
 /* One expert's tensors, as nvfp4moe_quantize produces them with linear scales.
  * Device pointers: gate/up codes [I][H/2], scales [I][H/16]; down codes [H][I/2],
- * scales [H][I/16].  Global scales are host values.  g_h is the static global scale
- * of the SwiGLU intermediate (input of the down projection). */
+ * scales [H][I/16]; the three code pointers 16-byte aligned (else NVFP4MOE_ERR_ARG).
+ * Global scales are host values.  g_h is the static global scale of the SwiGLU
+ * intermediate (input of the down projection). */
 typedef struct {
   const uint8_t* gate_codes;
   const uint8_t* gate_scales;
@@ -318,8 +321,8 @@ NVFP4MOE_API int nvfp4moe_forward(const nvfp4moe_experts* experts, const void* h
  *   size); dbg->hq_codes / hq_scales are meaningful only for pairs of the handle's experts.
  * With a full handle, acc_out is the FP32 sum nvfp4moe_forward rounds to BF16.
  *
- * nvfp4moe_finalize: out_bf16[i] = bf16(acc[i]) for n values (n % 8 == 0, both 16-byte
- * aligned), the layer's output rounding. */
+ * nvfp4moe_finalize: out_bf16[i] = bf16(acc[i]) for n values (n % 8 == 0, n < 2^40, both
+ * 16-byte aligned), the layer's output rounding. */
 NVFP4MOE_API int nvfp4moe_forward_partial(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
                                           const float* w_router, const float* logit_bias, float* acc_out,
                                           const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
@@ -366,7 +369,8 @@ NVFP4MOE_API int nvfp4moe_forward_residual(const nvfp4moe_experts* experts, cons
  * NVFP4 layer's.
  *
  * nvfp4moe_quantize_fp8: x_bf16 [rows][cols] BF16 (16-byte aligned, cols % 16 == 0) ->
- *   codes [rows][cols] (8-byte aligned) and scales [rows] FP32.  Workspace:
+ *   codes [rows][cols] (8-byte aligned) and scales [rows] FP32.  Limits: 1 <= rows < 2^31,
+ *   cols < 2^31, rows * cols < 2^40; outside them NVFP4MOE_ERR_SHAPE.  Workspace:
  *   nvfp4moe_quantize_workspace_bytes.  A non-finite row raises NVFP4MOE_ERR_NONFINITE in the
  *   status word and leaves that row's outputs unwritten. */
 NVFP4MOE_API int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_t* codes,

@@ -333,9 +333,10 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
                       uint8_t* scales, int32_t scale_layout, float* g_out, void* ws, size_t ws_bytes,
                       void* stream) {
   g_launches = 0;
-  if (rows < 0 || cols <= 0 || cols % 64 != 0) return NVFP4MOE_ERR_SHAPE;
-  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  // rows and cols bounded first so that rows * cols cannot overflow
+  if (rows < 0 || cols <= 0 || cols % 64 != 0 || cols >= ((int64_t)1 << 31)) return NVFP4MOE_ERR_SHAPE;
   if (rows >= ((int64_t)1 << 31) - 128) return NVFP4MOE_ERR_SHAPE;   // one CTA per (padded) row
+  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
   if (scale_layout != NVFP4MOE_SCALES_LINEAR && scale_layout != NVFP4MOE_SCALES_SWIZZLED)
     return NVFP4MOE_ERR_ARG;
   if (ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
@@ -381,7 +382,7 @@ int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, int64_t cols,
                                  size_t ws_bytes, void* stream) {
   g_launches = 0;
   if (rows < 1 || cols <= 0 || cols % 16 != 0 || cols / 16 > 65535) return NVFP4MOE_ERR_SHAPE;
-  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (rows >= ((int64_t)1 << 31) || rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
   if (m < 0 || m > 16) return NVFP4MOE_ERR_ARG;
   if (w_bf16 == nullptr || hess_blocks == nullptr || codes == nullptr || scales == nullptr || g_out == nullptr ||
       ws == nullptr)
@@ -501,6 +502,9 @@ int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e_global, const nvfp4moe_e
   if (e_global < x->e_begin || e_global >= x->e_begin + x->e_count) return NVFP4MOE_ERR_ARG;
   const int32_t e = e_global - x->e_begin;   // slot in this handle
   if (!t->gate_codes || !t->gate_scales || !t->up_codes || !t->up_scales || !t->down_codes || !t->down_scales)
+    return NVFP4MOE_ERR_ARG;
+  // the code rows are copied 16 bytes at a time
+  if (!aligned(t->gate_codes, 16) || !aligned(t->up_codes, 16) || !aligned(t->down_codes, 16))
     return NVFP4MOE_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t H = c.H, I = c.I;
@@ -799,7 +803,7 @@ int nvfp4moe_forward_partial(const nvfp4moe_experts* x, const void* hidden_bf16,
 
 int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream) {
   g_launches = 0;
-  if (n < 0 || n % 8 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (n < 0 || n % 8 != 0 || n >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
   if (n == 0) return NVFP4MOE_OK;
   if (acc == nullptr || out_bf16 == nullptr || !aligned(acc, 16) || !aligned(out_bf16, 16)) return NVFP4MOE_ERR_ARG;
   int st = check_device();
@@ -844,8 +848,8 @@ int nvfp4moe_forward_residual(const nvfp4moe_experts* x, const void* h_bf16, int
 int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_t* codes, float* scales, void* ws,
                           size_t ws_bytes, void* stream) {
   g_launches = 0;
-  if (rows < 1 || cols <= 0 || cols % 16 != 0) return NVFP4MOE_ERR_SHAPE;
-  if (rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (rows < 1 || cols <= 0 || cols % 16 != 0 || cols >= ((int64_t)1 << 31)) return NVFP4MOE_ERR_SHAPE;
+  if (rows >= ((int64_t)1 << 31) || rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
   if (x_bf16 == nullptr || codes == nullptr || scales == nullptr || ws == nullptr) return NVFP4MOE_ERR_ARG;
   if (!aligned(x_bf16, 16) || !aligned(codes, 8) || !aligned(scales, 4) || !aligned(ws, kAlign))
     return NVFP4MOE_ERR_ARG;

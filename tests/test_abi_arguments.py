@@ -1,0 +1,207 @@
+"""Argument checking of every C-ABI entry point, on a machine without a GPU.
+
+include/nvfp4moe.h documents, per call, the shapes and pointers it accepts and the status it
+returns otherwise.  Every check below happens on the host before any CUDA call, so these
+calls return their documented status here; a call that passes every host check reaches the
+device check and fails with NVFP4MOE_ERR_DEVICE or NVFP4MOE_ERR_CUDA (the library has no CPU
+path).  The pointers passed are placeholders that are never dereferenced: the library reads
+no device pointer on the host.  The module is skipped where a GPU is present, since there a
+call that passed its checks would launch kernels on the placeholders.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import nvfp4_quantized_moe_group_b200 as moe
+from nvfp4_quantized_moe_group_b200 import build as build_mod
+from nvfp4_quantized_moe_group_b200._lib import ExpertTensors
+
+pytestmark = pytest.mark.skipif(torch.cuda.is_available(),
+                                reason="placeholder device pointers: host-only checks, no GPU")
+
+A = 1 << 20                       # a 16-byte (and 256-byte) aligned placeholder address
+MIS = A + 8                       # 8-byte aligned, not 16
+BIG = 1 << 40
+NO_DEVICE = (moe.ERR_DEVICE, moe.ERR_CUDA)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return moe.lib()
+
+
+def _cfg(**kw):
+    c = moe.cfg_default()
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value,want", [
+    ("H", 5000, "SHAPE"), ("H", 0, "SHAPE"), ("I", 2500, "SHAPE"), ("I", -128, "SHAPE"),
+    ("E", 0, "SHAPE"), ("E", 257, "SHAPE"), ("n_groups", 0, "SHAPE"), ("n_groups", 3, "SHAPE"),
+    ("n_groups", 4, "SHAPE"),         # 64 experts per group: above the 32 a group may hold
+    ("topk_groups", 0, "SHAPE"), ("topk_groups", 9, "SHAPE"),
+    ("topk", 0, "SHAPE"), ("topk", 9, "SHAPE"),
+    ("routed_scale", float("nan"), "ARG"),
+])
+def test_cfg_limits(lib, field, value, want):
+    c = _cfg(**{field: value})
+    assert lib.nvfp4moe_cfg_check(ctypes.byref(c)) == getattr(moe, f"ERR_{want}")
+    assert lib.nvfp4moe_forward_workspace_bytes(ctypes.byref(c), 16) == 0
+    assert lib.nvfp4moe_route_workspace_bytes(ctypes.byref(c), 16) == 0
+
+
+def test_cfg_small_layers_accepted(lib):
+    for kw in ({"E": 8, "n_groups": 1, "topk_groups": 1, "topk": 1},
+               {"E": 32, "n_groups": 8, "topk_groups": 4, "topk": 8, "H": 256, "I": 128}):
+        c = _cfg(**kw)
+        assert lib.nvfp4moe_cfg_check(ctypes.byref(c)) == moe.OK
+    c = _cfg(E=8, n_groups=4, topk_groups=1, topk=3)      # 3 experts from one group of 2
+    assert lib.nvfp4moe_cfg_check(ctypes.byref(c)) == moe.ERR_SHAPE
+    assert lib.nvfp4moe_cfg_check(None) == moe.ERR_ARG
+    assert lib.nvfp4moe_cfg_default(None) == moe.ERR_ARG
+
+
+def test_quantize_checks(lib):
+    q = lib.nvfp4moe_quantize
+    ws_n = moe.quantize_workspace_bytes(4, 64)
+    ok = dict(x=A, rows=4, cols=64, g_in=None, codes=A, scales=A, layout=0, g_out=None, ws=A, ws_n=ws_n)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return q(a["x"], a["rows"], a["cols"], a["g_in"], a["codes"], a["scales"], a["layout"], a["g_out"],
+                 a["ws"], a["ws_n"], None)
+
+    assert call(cols=63) == moe.ERR_SHAPE
+    assert call(cols=0) == moe.ERR_SHAPE
+    assert call(cols=1 << 31) == moe.ERR_SHAPE
+    assert call(rows=-1) == moe.ERR_SHAPE
+    assert call(rows=(1 << 31) - 128) == moe.ERR_SHAPE
+    assert call(rows=1 << 20, cols=1 << 20) == moe.ERR_SHAPE          # rows * cols = 2^40
+    assert call(rows=1 << 62, cols=1 << 30) == moe.ERR_SHAPE          # no overflow of rows * cols
+    assert call(layout=7) == moe.ERR_ARG
+    assert call(ws=None) == moe.ERR_ARG
+    assert call(ws=MIS) == moe.ERR_ARG
+    assert call(scales=None) == moe.ERR_ARG
+    assert call(scales=A + 2) == moe.ERR_ARG
+    assert call(x=None) == moe.ERR_ARG
+    assert call(x=MIS) == moe.ERR_ARG
+    assert call(codes=MIS) == moe.ERR_ARG
+    assert call(ws_n=ws_n - 1) == moe.ERR_WORKSPACE
+    assert call() in NO_DEVICE
+    assert call(rows=0, x=None, codes=None, scales=None) in NO_DEVICE   # empty input: pointers unused
+
+
+def test_quantize_weights_lh_checks(lib):
+    f = lib.nvfp4moe_quantize_weights_lh
+    ws_n = moe.quantize_workspace_bytes(4, 64)
+    ok = dict(w=A, rows=4, cols=64, h=A, m=4, codes=A, scales=A, g=A, ws=A, ws_n=ws_n)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["w"], a["rows"], a["cols"], a["h"], a["m"], a["codes"], a["scales"], a["g"], a["ws"],
+                 a["ws_n"], None)
+
+    assert call(rows=0) == moe.ERR_SHAPE
+    assert call(cols=8) == moe.ERR_SHAPE
+    assert call(cols=16 * 65536) == moe.ERR_SHAPE
+    assert call(rows=1 << 31) == moe.ERR_SHAPE
+    assert call(rows=1 << 62) == moe.ERR_SHAPE
+    assert call(m=-1) == moe.ERR_ARG
+    assert call(m=17) == moe.ERR_ARG
+    for k in ("w", "h", "codes", "scales", "g", "ws"):
+        assert call(**{k: None}) == moe.ERR_ARG, k
+    assert call(w=MIS) == moe.ERR_ARG
+    assert call(ws_n=ws_n - 1) == moe.ERR_WORKSPACE
+    assert call() in NO_DEVICE
+
+
+def test_route_checks(lib):
+    c = moe.cfg_default()
+    ws_n = moe.route_workspace_bytes(c, 16)
+    r = lib.nvfp4moe_route
+
+    def call(cfg=c, x=A, T=16, w=A, idx=A, wts=A, ws=A, n=ws_n):
+        return r(ctypes.byref(cfg) if cfg is not None else None, x, T, w, None, idx, wts, ws, n, None)
+
+    assert call(cfg=None) == moe.ERR_ARG
+    assert call(cfg=_cfg(H=100)) == moe.ERR_SHAPE
+    assert call(T=-1) == moe.ERR_SHAPE
+    assert call(T=(1 << 24) + 1) == moe.ERR_SHAPE
+    assert call(ws=None) == moe.ERR_ARG
+    for k in ("x", "w", "idx", "wts"):
+        assert call(**{k: None}) == moe.ERR_ARG, k
+    assert call(x=MIS) == moe.ERR_ARG
+    assert call(n=ws_n - 1) == moe.ERR_WORKSPACE
+    assert call() in NO_DEVICE
+    assert call(T=0, x=None, w=None, idx=None, wts=None) in NO_DEVICE
+
+
+def test_expert_handles_checks(lib):
+    c = moe.cfg_default()
+    h = ctypes.c_void_p()
+    assert lib.nvfp4moe_experts_create(ctypes.byref(c), None) == moe.ERR_ARG
+    assert lib.nvfp4moe_experts_create(ctypes.byref(_cfg(topk=0)), ctypes.byref(h)) == moe.ERR_SHAPE
+    assert h.value is None
+    for b, n in ((-1, 4), (0, 0), (250, 7), (256, 1)):
+        assert lib.nvfp4moe_experts_create_local(ctypes.byref(c), b, n, ctypes.byref(h)) == moe.ERR_ARG, (b, n)
+    assert lib.nvfp4moe_experts_create(ctypes.byref(c), ctypes.byref(h)) in NO_DEVICE
+    assert h.value is None
+    assert lib.nvfp4moe_fp8_experts_create(ctypes.byref(c), None) == moe.ERR_ARG
+    assert lib.nvfp4moe_fp8_experts_create(ctypes.byref(c), ctypes.byref(h)) in NO_DEVICE
+    t = ExpertTensors()
+    assert lib.nvfp4moe_experts_set(None, 0, ctypes.byref(t), None) == moe.ERR_ARG
+    assert lib.nvfp4moe_fp8_experts_set(None, 0, None, None) == moe.ERR_ARG
+    lo, n = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.nvfp4moe_experts_range(None, ctypes.byref(lo), ctypes.byref(n)) == moe.ERR_ARG
+    assert lib.nvfp4moe_experts_cfg(None, ctypes.byref(c)) == moe.ERR_ARG
+    lib.nvfp4moe_experts_destroy(None)
+    lib.nvfp4moe_fp8_experts_destroy(None)
+
+
+def test_forward_family_without_a_handle(lib):
+    for name in ("nvfp4moe_forward", "nvfp4moe_forward_partial", "nvfp4moe_forward_fp8"):
+        assert getattr(lib, name)(None, A, 16, A, None, A, None, A, 1 << 30, None) == moe.ERR_ARG, name
+    assert lib.nvfp4moe_forward_residual(None, A, 16, A, 1e-6, 2, A, None, A, None, A, 1 << 30, None) == moe.ERR_ARG
+
+
+def test_finalize_checks(lib):
+    f = lib.nvfp4moe_finalize
+    assert f(A, 7, A, None) == moe.ERR_SHAPE
+    assert f(A, -8, A, None) == moe.ERR_SHAPE
+    assert f(A, BIG, A, None) == moe.ERR_SHAPE
+    assert f(None, 0, None, None) == moe.OK                          # nothing to do, no device call
+    assert f(None, 8, A, None) == moe.ERR_ARG
+    assert f(A, 8, MIS, None) == moe.ERR_ARG
+    assert f(A, 8, A, None) in NO_DEVICE
+
+
+def test_quantize_fp8_checks(lib):
+    f = lib.nvfp4moe_quantize_fp8
+    ws_n = moe.quantize_workspace_bytes(4, 64)
+
+    def call(x=A, rows=4, cols=64, codes=A, scales=A, ws=A, n=ws_n):
+        return f(x, rows, cols, codes, scales, ws, n, None)
+
+    assert call(rows=0) == moe.ERR_SHAPE
+    assert call(cols=8) == moe.ERR_SHAPE
+    assert call(cols=1 << 31) == moe.ERR_SHAPE
+    assert call(rows=1 << 31) == moe.ERR_SHAPE
+    assert call(rows=1 << 62, cols=1 << 30) == moe.ERR_SHAPE
+    assert call(rows=1 << 24, cols=1 << 16) == moe.ERR_SHAPE          # rows * cols = 2^40
+    for k in ("x", "codes", "scales", "ws"):
+        assert call(**{k: None}) == moe.ERR_ARG, k
+    assert call(codes=A + 4) == moe.ERR_ARG
+    assert call(n=ws_n - 1) == moe.ERR_WORKSPACE
+    assert call() in NO_DEVICE
+
+
+def test_status_calls(lib):
+    assert lib.nvfp4moe_status_read(None, None) == moe.ERR_ARG
+    for code in (moe.OK, moe.ERR_ARG, moe.ERR_SHAPE, moe.ERR_CUDA, moe.ERR_WORKSPACE, moe.ERR_NONFINITE,
+                 moe.ERR_TIMEOUT, moe.ERR_DEVICE):
+        assert moe.status_string(code) != "unknown status"
+    assert moe.status_string(12345) == "unknown status"

@@ -308,3 +308,23 @@ def test_cuda_graph_replay_matches_eager():
         for key in ("idx", "w", "perm", "hq_codes", "hq_scales"):
             assert torch.equal(dbg[key], dbg_ref[key]), key
         del g
+
+
+def test_experts_set_rejects_misaligned_codes():
+    """nvfp4moe_experts_set copies the code rows 16 bytes at a time: a code pointer off a
+    16-byte boundary returns NVFP4MOE_ERR_ARG on the host, before anything is enqueued."""
+    import ctypes
+    from nvfp4_quantized_moe_group_b200._lib import ExpertTensors
+    cfg = moe.make_cfg(8, 1, 1, 1, 256, 128, 2.5)
+    ex = moe.Experts(cfg)
+    buf = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    base = buf.data_ptr()
+    assert base % 256 == 0
+    for which in (0, 2, 4):                       # gate, up, down codes
+        ptrs = [base] * 6
+        ptrs[which] = base + 8
+        t = ExpertTensors(*ptrs, 1.0, 1.0, 1.0, 1.0)
+        assert moe.lib().nvfp4moe_experts_set(ex.handle, 0, ctypes.byref(t), None) == moe.ERR_ARG
+        assert moe.last_launch_count() == 0
+    torch.cuda.synchronize()
+    ex.close()
