@@ -166,6 +166,41 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(*specs):
+    """Raise TypeError unless every (tensor, name, dtype, shape) of ``specs`` whose tensor is
+    not None is a contiguous tensor of that dtype and shape (shape None: any), and all of them
+    are CUDA tensors on the first one's device.  Types and shapes are checked before devices.
+    The library receives raw pointers, so a tensor of the wrong type or size would be read out
+    of bounds rather than rejected."""
+    present = [s for s in specs if s[0] is not None]
+    for t, name, dtype, shape in present:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if shape is not None and tuple(t.shape) != tuple(int(s) for s in shape):
+            raise TypeError(f"{name} must have shape {tuple(int(s) for s in shape)}, got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise TypeError(f"{name} must be contiguous")
+    for t, name, _, _ in present:
+        if not t.is_cuda or t.device != present[0][0].device:
+            raise TypeError(f"{name} must be a CUDA tensor on {present[0][0].device}, got {t.device}")
+
+
+def _rows(x, name: str, min_rows: int = 1) -> int:
+    """Rows of a 2-D tensor, at least min_rows."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2 or x.shape[0] < min_rows:
+        raise TypeError(f"{name} must be a 2-D tensor with at least {min_rows} rows")
+    return int(x.shape[0])
+
+
+def _layer_specs(cfg, x, w_router, bias, name="x") -> list:
+    """x [T, H] bf16 (T >= 1), w_router [E, H] float32, bias [E] float32 or None."""
+    T = _rows(x, name)
+    return [(x, name, torch.bfloat16, (T, cfg.H)), (w_router, "w_router", torch.float32, (cfg.E, cfg.H)),
+            (bias, "bias", torch.float32, (cfg.E,))]
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -211,10 +246,16 @@ def quantize(x: torch.Tensor, g: torch.Tensor | None = None, swizzled: bool = Fa
     ``g``: None for a dynamic global scale, else a 1-element CUDA float32 tensor.
     Scales are [rows, cols/16] (linear) or the flat swizzled array.
     """
-    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
-        raise TypeError("x must be a contiguous 2-D bfloat16 CUDA tensor")
-    rows, cols = x.shape
+    rows = _rows(x, "x", min_rows=0)
+    cols = int(x.shape[1])
     dev = x.device
+    specs = [(x, "x", torch.bfloat16, None), (g, "g", torch.float32, (1,)), (ws, "ws", torch.uint8, None)]
+    if out is not None:
+        specs += [(out[0], "codes", torch.uint8, (rows, cols // 2)),
+                  (out[1], "scales", torch.uint8,
+                   (swizzled_scale_bytes(rows, cols // 16),) if swizzled else (rows, cols // 16)),
+                  (out[2], "g_out", torch.float32, (1,))]
+    _require(*specs)
     if out is None:
         codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
         if swizzled:
@@ -237,13 +278,11 @@ def quantize_weights_lh(w: torch.Tensor, hess_blocks: torch.Tensor, m: int = 4, 
     """Weight quantisation with the local-Hessian block-scale search
     (nvfp4moe_quantize_weights_lh): w [rows, cols] bf16, hess_blocks [cols/16, 16, 16] float32
     -> (codes [rows, cols/2] u8, linear scales [rows, cols/16] u8, g [1] f32)."""
-    if w.dtype != torch.bfloat16 or not w.is_cuda or w.dim() != 2 or not w.is_contiguous():
-        raise TypeError("w must be a contiguous 2-D bfloat16 CUDA tensor")
-    rows, cols = w.shape
-    if hess_blocks.dtype != torch.float32 or tuple(hess_blocks.shape) != (cols // 16, 16, 16) \
-            or not hess_blocks.is_contiguous():
-        raise TypeError("hess_blocks must be a contiguous float32 tensor [cols/16, 16, 16]")
+    rows = _rows(w, "w", min_rows=0)
+    cols = int(w.shape[1])
     dev = w.device
+    _require((w, "w", torch.bfloat16, None), (hess_blocks, "hess_blocks", torch.float32, (cols // 16, 16, 16)),
+             (ws, "ws", torch.uint8, None))
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
     g_out = torch.empty(1, dtype=torch.float32, device=dev)
@@ -262,7 +301,11 @@ def route_workspace_bytes(cfg: Cfg, T: int) -> int:
 def route(cfg: Cfg, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None, ws=None,
           stream=None):
     """route(hidden, W_router) -> (idx [T, topk] int32, w [T, topk] float32)."""
-    T = x.shape[0]
+    T = _rows(x, "x", min_rows=0)
+    if T == 0:
+        _require((x, "x", torch.bfloat16, (0, cfg.H)), (ws, "ws", torch.uint8, None))
+    else:
+        _require(*_layer_specs(cfg, x, w_router, bias), (ws, "ws", torch.uint8, None))
     dev = x.device
     idx = torch.empty((T, cfg.topk), dtype=torch.int32, device=dev)
     w = torch.empty((T, cfg.topk), dtype=torch.float32, device=dev)
@@ -290,6 +333,12 @@ class Experts:
 
     def set(self, e: int, gate, up, down, g_h: float, stream=None):
         """gate/up/down: (codes, linear scales, global scale as float) from quantize()."""
+        H, I = self.cfg.H, self.cfg.I
+        specs = []
+        for name, (codes, scales, _), rows, cols in (("gate", gate, I, H), ("up", up, I, H), ("down", down, H, I)):
+            specs += [(codes, f"{name} codes", torch.uint8, (rows, cols // 2)),
+                      (scales, f"{name} scales", torch.uint8, (rows, cols // 16))]
+        _require(*specs)
         t = ExpertTensors(gate[0].data_ptr(), gate[1].data_ptr(), up[0].data_ptr(), up[1].data_ptr(),
                           down[0].data_ptr(), down[1].data_ptr(), float(gate[2]), float(up[2]),
                           float(down[2]), float(g_h))
@@ -349,8 +398,11 @@ def forward_residual(experts: Experts, h: torch.Tensor, gamma: torch.Tensor, eps
     h' = bf16(a h + b moe(rmsnorm(h) gamma)) for residual step ``step_k``.  ``out`` may be ``h``
     (in-place update).  Returns h' (and the intermediates, x_norm included, if debug)."""
     cfg = experts.cfg
+    specs = _layer_specs(cfg, h, w_router, bias, name="h")
     T, H = h.shape
     dev = h.device
+    _require(*specs, (gamma, "gamma", torch.float32, (H,)), (out, "out", torch.bfloat16, (T, H)),
+             (ws, "ws", torch.uint8, None))
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     if ws is None:
@@ -373,8 +425,10 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
     """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug).
     ``timer``: a StageTimer whose events are recorded around each stage."""
     cfg = experts.cfg
+    specs = _layer_specs(cfg, x, w_router, bias)
     T, H = x.shape
     dev = x.device
+    _require(*specs, (out, "out", torch.bfloat16, (T, H)), (ws, "ws", torch.uint8, None))
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     if ws is None:
@@ -402,10 +456,10 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
 def quantize_fp8(x: torch.Tensor, ws=None, stream=None):
     """Per-row FP8 quantisation (nvfp4moe_quantize_fp8): x [rows, cols] bf16 ->
     (codes [rows, cols] u8 E4M3, scales [rows] f32)."""
-    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
-        raise TypeError("x must be a contiguous 2-D bfloat16 CUDA tensor")
-    rows, cols = x.shape
+    rows = _rows(x, "x", min_rows=0)
+    cols = int(x.shape[1])
     dev = x.device
+    _require((x, "x", torch.bfloat16, None), (ws, "ws", torch.uint8, None))
     codes = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
     scales = torch.empty(rows, dtype=torch.float32, device=dev)
     if ws is None:
@@ -428,6 +482,12 @@ class Fp8Experts:
 
     def set(self, e: int, gate, up, down, stream=None):
         """gate/up/down: (codes, scales) from quantize_fp8()."""
+        H, I = self.cfg.H, self.cfg.I
+        specs = []
+        for name, (codes, scales), rows, cols in (("gate", gate, I, H), ("up", up, I, H), ("down", down, H, I)):
+            specs += [(codes, f"{name} codes", torch.uint8, (rows, cols)),
+                      (scales, f"{name} scales", torch.float32, (rows,))]
+        _require(*specs)
         t = Fp8ExpertTensors(gate[0].data_ptr(), gate[1].data_ptr(), up[0].data_ptr(), up[1].data_ptr(),
                              down[0].data_ptr(), down[1].data_ptr())
         _check(lib().nvfp4moe_fp8_experts_set(self.handle, int(e), ctypes.byref(t), _stream(stream)),
@@ -460,8 +520,10 @@ def forward_fp8(experts: Fp8Experts, x: torch.Tensor, w_router: torch.Tensor, bi
                 stream=None):
     """The FP8 W8A8 layer (nvfp4moe_forward_fp8) -> out [T, H] bf16 (and intermediates if debug)."""
     cfg = experts.cfg
+    specs = _layer_specs(cfg, x, w_router, bias)
     T, H = x.shape
     dev = x.device
+    _require(*specs, (out, "out", torch.bfloat16, (T, H)), (ws, "ws", torch.uint8, None))
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     if ws is None:
@@ -498,8 +560,10 @@ def forward_partial(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, b
     """One rank's part of the layer (nvfp4moe_forward_partial): the FP32 sums [T, H] of the
     contributions of the handle's experts for all T tokens of x."""
     cfg = experts.cfg
+    specs = _layer_specs(cfg, x, w_router, bias)
     T, H = x.shape
     dev = x.device
+    _require(*specs, (acc_out, "acc_out", torch.float32, (T, H)), (ws, "ws", torch.uint8, None))
     if acc_out is None:
         acc_out = torch.empty((T, H), dtype=torch.float32, device=dev)
     if ws is None:
@@ -517,8 +581,7 @@ def forward_partial(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, b
 
 def finalize(acc: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """BF16 rounding of FP32 layer sums (nvfp4moe_finalize)."""
-    if acc.dtype != torch.float32 or not acc.is_cuda or not acc.is_contiguous():
-        raise TypeError("acc must be a contiguous float32 CUDA tensor")
+    _require((acc, "acc", torch.float32, None), (out, "out", torch.bfloat16, acc.shape))
     if out is None:
         out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
     _check(lib().nvfp4moe_finalize(_ptr(acc), acc.numel(), _ptr(out), _stream(stream)), "nvfp4moe_finalize")
