@@ -1,4 +1,5 @@
 """Pins for the oracle's expert grouping, SwiGLU expert MLP and layer combine (CPU only)."""
+import math
 import types
 
 import numpy as np
@@ -122,3 +123,66 @@ def test_bf16_rounding_matches_torch():
     v32 = v.astype(np.float32).astype(np.float64)
     np.testing.assert_array_equal(_bf16_round(v32), torch.from_numpy(v32).to(torch.bfloat16).double().numpy())
     assert np.mean(_bf16_round(v) == ref) > 0.999
+
+
+def test_worked_layer_example():
+    """A whole layer worked by hand, with operands NVFP4 represents exactly.
+
+    Layer: E = 4 experts in 2 groups of 2, keep 1 group, top 2, routed scale 2.5; H = 32,
+    I = 16.  One token, x[3] = 2.625 and zeros elsewhere.
+
+    * Input quantisation: A = 2.625, g = 2.625 / 2688 = 2^-10; block 0 scales 2.625 * r_t to
+      448 (code 126), d = 0.4375, 2.625 / d = 6 -> code 7 (byte 1 = 0x70); block 1 is zero
+      (scale 0).  So xhat[3] = 2.625 exactly.
+    * Router (on the BF16 x): W[:, 3] = [1, -0.5, 0.25, 0.75], logits
+      l = [2.625, -1.3125, 0.65625, 1.96875].  Group sums: g0 = s(2.625) + s(-1.3125) = 1.144,
+      g1 = s(0.65625) + s(1.96875) = 1.536, so group 1 is kept and the experts are 3, 2 (score
+      order), although expert 0 has the best single score; w = 2.5 s / (s2 + s3).
+    * Experts, the same gate and up for all: gate[5, 3] = 21 = 2688 * 2^-7 and
+      up[5, 3] = 0.328125 = 2688 * 2^-13, each the maximum of its tensor, so g = 2^-7 and 2^-13,
+      block scale 448, code 6 and the values decode exactly.  gate = 2.625 * 21 = 55.125,
+      up = 2.625 * 0.328125 = 0.861328125, silu(55.125) = 55.125 in FP64 (e^-55 is below half
+      an ulp), h[5] = 194481 / 4096 = 47.480712890625 (exact in FP32).
+    * Requantisation of h with g_h = 1/8: r_t = fp32(1 / 0.75), h * r_t = 63.31 -> nearest E4M3
+      64 (code 104), d = 8, h / d = 5.94 -> E2M1 6 (code 7, byte 2 = 0x70): hhat[5] = 48.
+    * Down: expert e has down[9, 5] = 21 * 2^e (g = 2^(e-7), exact), y_e[9] = 48 * 21 * 2^e.
+    * Combine: out[9] = 1008 (8 w_3 + 4 w_2) = 15838.84..., every other output 0; BF16 (a step
+      of 64 there): 15808."""
+    H, I, E = 32, 16, 4
+    cfg = types.SimpleNamespace(E=E, n_groups=2, topk_groups=1, topk=2, routed_scale=2.5)
+    x = np.zeros((1, H), np.float32)
+    x[0, 3] = 2.625
+    wr = np.zeros((E, H), np.float32)
+    wr[:, 3] = [1.0, -0.5, 0.25, 0.75]
+    gate = np.zeros((I, H), np.float32)
+    gate[5, 3] = 21.0
+    up = np.zeros((I, H), np.float32)
+    up[5, 3] = 0.328125
+    ex = {}
+    for e in range(E):
+        down = np.zeros((H, I), np.float32)
+        down[9, 5] = 21.0 * 2 ** e
+        ex[e] = (oracle.quantize_tensor(gate), oracle.quantize_tensor(up), oracle.quantize_tensor(down))
+    res = oracle.moe_forward(x, wr, cfg, lambda e: ex[e], np.full(E, 0.125, np.float32), keep_intermediates=True)
+
+    assert res["g_x"] == np.float32(2.0 ** -10)
+    want_xq = np.zeros((1, H // 2), np.uint8)
+    want_xq[0, 1] = 0x70
+    np.testing.assert_array_equal(res["xq_codes"], want_xq)
+    np.testing.assert_array_equal(res["xq_scales"], [[126, 0]])
+    r = res["route"]
+    assert list(r.groups[0]) == [1] and list(r.idx[0]) == [3, 2]
+    l = [2.625, -1.3125, 0.65625, 1.96875]
+    s = [1.0 / (1.0 + math.exp(-v)) for v in l]
+    w3, w2 = 2.5 * s[3] / (s[2] + s[3]), 2.5 * s[2] / (s[2] + s[3])
+    np.testing.assert_allclose(r.w[0], [w3, w2], rtol=1e-15)
+    for j in (0, 1):
+        it = res["inter"][(0, j)]
+        assert it["gate"][5] == 55.125 and it["up"][5] == 0.861328125
+        assert it["h"][5] == 194481 / 4096 and np.count_nonzero(it["h"]) == 1
+        np.testing.assert_array_equal(it["hq_scales"], [104])
+        assert it["hq_codes"][2] == 0x70 and np.count_nonzero(it["hq_codes"]) == 1
+    out = res["out"][0]
+    assert np.flatnonzero(out).tolist() == [9]
+    np.testing.assert_allclose(out[9], 1008 * (8 * w3 + 4 * w2), rtol=1e-14)
+    assert res["out_bf16"][0, 9] == 15808.0
