@@ -161,6 +161,10 @@ CASES = [
     ("input-not-quantised", "moe", "moe_forward",
      "xhat = dequantize(xq_codes[ts], xq_scales[ts], g_x)", "xhat = x[ts].astype(np.float64)"),
     ("bf16-truncates", "moe", "_bf16_round", "r = np.round(scaled)", "r = np.trunc(scaled)"),
+    ("h-dynamic-scale", "moe", "expert_mlp",
+     "hq_codes, hq_scales, _ = quantize(h.astype(np.float32), g=g_h)",
+     "hq_codes, hq_scales, g_h = quantize(h.astype(np.float32))"),
+    ("weights-of-expert-0", "moe", "moe_forward", "gate, up, down = experts(e)", "gate, up, down = experts(0)"),
     # FP8 variant
     ("fp8-fnuz-max", "fp8", "row_scales", "(amax / F32(E4M3_MAX))", "(amax / F32(240.0))"),
     ("fp8-zero-row-scale", "fp8", "row_scales", "np.where(amax == 0, F32(1.0), s)", "s"),
