@@ -15,13 +15,13 @@ Typical use (all tensors on one CUDA device; the current stream is used)::
     out = moe.forward(experts, x_bf16, w_router_fp32, ws=ws)    # [T, H] BF16
     assert moe.status_read(ws) == moe.OK
 
-Also: ``quantize`` / ``route`` (the layer's steps alone), ``forward_residual`` (RMSNorm in,
+Also: ``quantize`` / ``route`` / ``route_noalloc`` (the layer's steps alone), ``forward_residual`` (RMSNorm in,
 weighted residual add out), ``quantize_weights_lh`` (local-Hessian weight scales),
 ``Fp8Experts`` / ``forward_fp8`` (the FP8 W8A8 variant), and ``ep.ExpertParallelLayer`` with
 ``forward_partial`` / ``finalize`` (experts spread over the ranks of a process group).
 """
 from ._lib import (  # noqa: F401
-    Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, forward,
+    Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, route_noalloc, forward,
     forward_residual, status_read, quantize_fp8, Fp8Experts, forward_fp8, forward_fp8_workspace_bytes,
     forward_partial, finalize,
     status_string, last_launch_count, forward_workspace_bytes, route_workspace_bytes,

@@ -105,6 +105,7 @@ _SIGS = {
     "nvfp4moe_quantize_weights_lh": (ctypes.c_int, [_P, _I64, _I64, _P, ctypes.c_int32, _P, _P, _P, _P, _SZ, _P]),
     "nvfp4moe_route_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_route": (ctypes.c_int, [ctypes.POINTER(Cfg), _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nvfp4moe_route_noalloc": (ctypes.c_int, [ctypes.POINTER(Cfg), _P, _I64, _P, _P, _P, _P, _P]),
     "nvfp4moe_experts_create": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.POINTER(_P)]),
     "nvfp4moe_experts_set": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(ExpertTensors), _P]),
     "nvfp4moe_experts_destroy": (None, [_P]),
@@ -314,6 +315,25 @@ def route(cfg: Cfg, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor 
     st = lib().nvfp4moe_route(ctypes.byref(cfg), _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(idx), _ptr(w),
                               _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "nvfp4moe_route")
+    return idx, w
+
+
+def route_noalloc(cfg: Cfg, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
+                  stream=None):
+    """route() without a workspace (nvfp4moe_route_noalloc): the router's scratch is a fixed
+    device array inside the library, so T * E is limited to 1,212,416 and calls that may
+    overlap on the GPU must be serialised.  -> (idx [T, topk] int32, w [T, topk] float32)."""
+    T = _rows(x, "x", min_rows=0)
+    if T == 0:
+        _require((x, "x", torch.bfloat16, (0, cfg.H)))
+    else:
+        _require(*_layer_specs(cfg, x, w_router, bias))
+    dev = x.device
+    idx = torch.empty((T, cfg.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.topk), dtype=torch.float32, device=dev)
+    st = lib().nvfp4moe_route_noalloc(ctypes.byref(cfg), _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(idx),
+                                      _ptr(w), _stream(stream))
+    _check(st, "nvfp4moe_route_noalloc")
     return idx, w
 
 

@@ -205,3 +205,21 @@ def test_status_calls(lib):
                  moe.ERR_TIMEOUT, moe.ERR_DEVICE):
         assert moe.status_string(code) != "unknown status"
     assert moe.status_string(12345) == "unknown status"
+
+
+def test_route_noalloc_checks(lib):
+    c = moe.cfg_default()
+    r = lib.nvfp4moe_route_noalloc
+
+    def call(cfg=c, x=A, T=16, w=A, idx=A, wts=A):
+        return r(ctypes.byref(cfg) if cfg is not None else None, x, T, w, None, idx, wts, None)
+
+    assert call(cfg=None) == moe.ERR_ARG
+    assert call(cfg=_cfg(topk=9)) == moe.ERR_SHAPE
+    assert call(T=-1) == moe.ERR_SHAPE
+    assert call(T=(1 << 24) + 1) == moe.ERR_SHAPE
+    for k in ("x", "w", "idx", "wts"):
+        assert call(**{k: None}) == moe.ERR_ARG, k
+    assert call(w=MIS) == moe.ERR_ARG
+    assert call(T=4737) == moe.ERR_WORKSPACE                   # T * E above the fixed scratch
+    assert call(T=4736) in NO_DEVICE

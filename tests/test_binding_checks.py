@@ -118,3 +118,15 @@ def test_finalize_inputs():
     _raises("acc must be torch.float32", moe.finalize, acc.double())
     _raises(r"out must have shape \(4, 256\)", moe.finalize, acc, out=_x(T=3))
     _raises("must be a CUDA tensor", moe.finalize, acc)
+
+
+def test_route_noalloc_inputs(cfg):
+    wr = torch.zeros((32, 256))
+    _raises(r"w_router must have shape \(32, 256\)", moe.route_noalloc, cfg, _x(), torch.zeros((32, 128)))
+    _raises("x must be torch.bfloat16", moe.route_noalloc, cfg, _x(dtype=torch.float16), wr)
+    _raises("must be a CUDA tensor", moe.route_noalloc, cfg, _x(), wr)
+
+
+def test_every_declared_call_is_bound():
+    from nvfp4_quantized_moe_group_b200 import _lib
+    assert set(_lib.declared_symbols()) == set(_lib._SIGS)
