@@ -409,8 +409,10 @@ NVFP4MOE_API int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* experts, const
                                       const float* w_router, const float* logit_bias, void* out_bf16,
                                       const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
 
-/* Number of kernels the last nvfp4moe_forward / _route / _quantize call on this host
- * thread enqueued (for launch accounting in benchmarks). */
+/* Number of kernels enqueued by the last call on this host thread that enqueues work
+ * (the quantize, route, experts_set, forward and finalize families; nvfp4moe_route_noalloc
+ * leaves the count unchanged), for launch accounting in benchmarks.  A call that returns an
+ * error before enqueuing anything reports 0. */
 NVFP4MOE_API int32_t nvfp4moe_last_launch_count(void);
 
 #ifdef __cplusplus

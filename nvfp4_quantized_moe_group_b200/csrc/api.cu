@@ -797,6 +797,7 @@ int nvfp4moe_forward(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t
 int nvfp4moe_forward_partial(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
                              const float* logit_bias, float* acc_out, const nvfp4moe_debug* dbg, void* ws,
                              size_t ws_bytes, void* stream) {
+  g_launches = 0;
   if (acc_out == nullptr) return NVFP4MOE_ERR_ARG;
   return forward_core(x, hidden_bf16, T, w_router, logit_bias, nullptr, nullptr, dbg, ws, ws_bytes, stream, acc_out);
 }

@@ -223,3 +223,19 @@ def test_route_noalloc_checks(lib):
     assert call(w=MIS) == moe.ERR_ARG
     assert call(T=4737) == moe.ERR_WORKSPACE                   # T * E above the fixed scratch
     assert call(T=4736) in NO_DEVICE
+
+
+def test_failed_calls_report_no_launches(lib):
+    """A call rejected on the host enqueued nothing, and the launch count says so."""
+    c = moe.cfg_default()
+    calls = [
+        lambda: lib.nvfp4moe_quantize(None, 4, 63, None, None, None, 0, None, None, 0, None),
+        lambda: lib.nvfp4moe_route(ctypes.byref(c), None, -1, None, None, None, None, None, 0, None),
+        lambda: lib.nvfp4moe_forward(None, A, 16, A, None, A, None, A, 1 << 30, None),
+        lambda: lib.nvfp4moe_forward_partial(None, A, 16, A, None, None, None, A, 1 << 30, None),
+        lambda: lib.nvfp4moe_finalize(A, 7, A, None),
+        lambda: lib.nvfp4moe_quantize_fp8(None, 0, 16, None, None, None, 0, None),
+    ]
+    for f in calls:
+        assert f() != moe.OK
+        assert lib.nvfp4moe_last_launch_count() == 0
