@@ -335,6 +335,18 @@ NVFP4MOE_API int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, 
 NVFP4MOE_API int nvfp4moe_status_read(const void* ws, void* stream);
 NVFP4MOE_API const char* nvfp4moe_status_string(int status);
 
+/* Waits for `stream`, then returns the device-side status of the last call on this host
+ * thread that enqueued work with a status word: the quantize, route, forward and FP8 calls
+ * (their workspace's word) and nvfp4moe_route_noalloc (the word of the library's fixed
+ * scratch, which only this call can read).  Same results as nvfp4moe_status_read; also
+ * NVFP4MOE_ERR_ARG when no such call has been made on this thread.  The workspace that call
+ * used must still be allocated. */
+NVFP4MOE_API int nvfp4moe_last_device_status(void* stream);
+
+/* Workspace bytes of nvfp4moe_forward for up to T_max tokens (the value of
+ * nvfp4moe_forward_workspace_bytes; 0 for an invalid cfg or T_max < 1). */
+NVFP4MOE_API size_t nvfp4moe_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);
+
 /* ------------------------------------------------------- forward, residual ----
  * The layer with its neighbours on the residual stream fused in ("Reflection releases Beam
  * ...", section "Residual stream and numerical decisions": at step k a sublayer output is

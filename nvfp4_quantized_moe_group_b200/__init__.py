@@ -22,7 +22,7 @@ weighted residual add out), ``quantize_weights_lh`` (local-Hessian weight scales
 """
 from ._lib import (  # noqa: F401
     Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, route_noalloc, forward,
-    forward_residual, status_read, quantize_fp8, Fp8Experts, forward_fp8, forward_fp8_workspace_bytes,
+    forward_residual, status_read, last_device_status, workspace_bytes, quantize_fp8, Fp8Experts, forward_fp8, forward_fp8_workspace_bytes,
     forward_partial, finalize,
     status_string, last_launch_count, forward_workspace_bytes, route_workspace_bytes,
     quantize_workspace_bytes, swizzled_scale_bytes, declared_symbols, lib, LIB_PATH, StageTimer, STAGES,

@@ -126,6 +126,8 @@ _SIGS = {
     "nvfp4moe_forward_fp8_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_forward_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_status_read": (ctypes.c_int, [_P, _P]),
+    "nvfp4moe_last_device_status": (ctypes.c_int, [_P]),
+    "nvfp4moe_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nvfp4moe_last_launch_count": (ctypes.c_int32, []),
 }
@@ -230,6 +232,17 @@ def last_launch_count() -> int:
 
 def status_read(ws: torch.Tensor, stream=None) -> int:
     return int(lib().nvfp4moe_status_read(_ptr(ws), _stream(stream)))
+
+
+def last_device_status(stream=None) -> int:
+    """Device-side status of this thread's latest call that had a status word (waits for the
+    stream); the only way to read nvfp4moe_route_noalloc's."""
+    return int(lib().nvfp4moe_last_device_status(_stream(stream)))
+
+
+def workspace_bytes(cfg: Cfg, T_max: int) -> int:
+    """Workspace bytes of forward() for up to T_max tokens (= forward_workspace_bytes)."""
+    return int(lib().nvfp4moe_workspace_bytes(ctypes.byref(cfg), T_max))
 
 
 def swizzled_scale_bytes(rows: int, cols16: int) -> int:

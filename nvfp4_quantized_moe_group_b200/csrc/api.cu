@@ -36,6 +36,7 @@ struct nvfp4moe_fp8_experts {
 namespace {
 
 thread_local int32_t g_launches = 0;
+thread_local const void* g_last_status = nullptr;   // status word of this thread's latest call
 
 constexpr size_t kAlign = 256;
 
@@ -291,6 +292,11 @@ struct StageEvents {
 
 }  // namespace
 
+cudaError_t nvfp4moe::reset_status(void* header, int words, cudaStream_t stream) {
+  g_last_status = header;
+  return cudaMemsetAsync(header, 0, (size_t)words * sizeof(uint32_t), stream);
+}
+
 extern "C" {
 
 int nvfp4moe_cfg_default(nvfp4moe_cfg* cfg) {
@@ -348,7 +354,7 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   int blocks = 0;
   if (g_in == nullptr) {
     blocks = amax_partial_blocks(rows * cols);
@@ -395,7 +401,7 @@ int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, int64_t cols,
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   const int blocks = amax_partial_blocks(rows * cols);
   if (launch_amax_partial(w_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   LhArgs la{static_cast<const uint16_t*>(w_bf16), rows, cols, hess_blocks, m, q.partials, blocks, codes, scales,
@@ -426,7 +432,7 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(&r.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(r.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   if (T == 0) return NVFP4MOE_OK;
   RouterArgs a{};
   a.x = static_cast<const uint16_t*>(hidden_bf16);
@@ -589,7 +595,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
   // status word and grid-barrier counter
   // status word, front-end barrier and the two GEMM work counters
-  if (cudaMemsetAsync(&f.hdr->status, 0, 4 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
 
   if (front_supported(T, c.E, c.H)) {
@@ -859,7 +865,7 @@ int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(&q.hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   Fp8RowsArgs fa{static_cast<const uint16_t*>(x_bf16), rows, cols, codes, scales, &q.hdr->status};
   if (launch_fp8_quantize_rows(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   g_launches = 1;
@@ -962,7 +968,7 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
       make_tma_2d(&tma_h32, f.hq, c.I, f.rows_cap, 32) != 0)
     return NVFP4MOE_ERR_CUDA;
   // status word, front-end barrier and the two GEMM work counters
-  if (cudaMemsetAsync(&f.hdr->status, 0, 4 * sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
 
   if (front_supported(T, c.E, c.H)) {
     // small T: routing and grouping in the fused front-end launch (its NVFP4 quantisation
@@ -1096,6 +1102,15 @@ int nvfp4moe_status_read(const void* ws, void* stream) {
   if (v & kStatusTimeout) return NVFP4MOE_ERR_TIMEOUT;
   if (v & kStatusNonFinite) return NVFP4MOE_ERR_NONFINITE;
   return NVFP4MOE_OK;
+}
+
+int nvfp4moe_last_device_status(void* stream) {
+  if (g_last_status == nullptr) return NVFP4MOE_ERR_ARG;
+  return nvfp4moe_status_read(g_last_status, stream);
+}
+
+size_t nvfp4moe_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) {
+  return nvfp4moe_forward_workspace_bytes(cfg, T_max);
 }
 
 const char* nvfp4moe_status_string(int status) {

@@ -238,4 +238,8 @@ cudaError_t launch_repack_sf(const uint8_t* linear, int rows, int cols16, uint8_
 
 int num_sms();
 
+// Zeroes the first `words` 32-bit words of a call's status header on the stream and records
+// the status word as this host thread's latest (read by nvfp4moe_last_device_status).
+cudaError_t reset_status(void* header, int words, cudaStream_t stream);
+
 }  // namespace nvfp4moe

@@ -75,7 +75,7 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
   WsHeader* hdr = static_cast<WsHeader*>(scratch);
   // the array keeps the previous call's contents: the status word starts at zero; the
   // partial sums are overwritten before they are read
-  if (cudaMemsetAsync(&hdr->status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   if (T == 0) return NVFP4MOE_OK;
   RouterArgs a{};
   a.x = static_cast<const uint16_t*>(hidden_bf16);

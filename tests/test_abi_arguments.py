@@ -239,3 +239,13 @@ def test_failed_calls_report_no_launches(lib):
     for f in calls:
         assert f() != moe.OK
         assert lib.nvfp4moe_last_launch_count() == 0
+
+
+def test_status_and_workspace_aliases(lib):
+    # no call on this thread has reached the device, so no status word has been recorded
+    assert lib.nvfp4moe_last_device_status(None) == moe.ERR_ARG
+    c = moe.cfg_default()
+    for T in (1, 16, 4096):
+        assert lib.nvfp4moe_workspace_bytes(ctypes.byref(c), T) == moe.forward_workspace_bytes(c, T) > 0
+    assert lib.nvfp4moe_workspace_bytes(ctypes.byref(c), 0) == 0
+    assert lib.nvfp4moe_workspace_bytes(ctypes.byref(_cfg(H=100)), 16) == 0

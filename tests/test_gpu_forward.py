@@ -328,3 +328,23 @@ def test_experts_set_rejects_misaligned_codes():
         assert moe.last_launch_count() == 0
     torch.cuda.synchronize()
     ex.close()
+
+
+def test_last_device_status_follows_the_latest_call():
+    """nvfp4moe_last_device_status reads the status word of this thread's latest call: clean
+    after a clean forward, NONFINITE after a forward whose router weight holds a NaN, while
+    the first workspace keeps its own clean word."""
+    ex = gpu_experts(BEAM)
+    T = 16
+    x = activations(T, BEAM, seed=5).cuda()
+    wr = router_weight(BEAM).cuda()
+    ws = torch.empty(moe.workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
+    assert ws.numel() == moe.forward_workspace_bytes(ex.cfg, T)
+    moe.forward(ex, x, wr, ws=ws)
+    assert moe.last_device_status() == moe.OK
+    bad = wr.clone()
+    bad[3, 7] = float("nan")
+    ws2 = torch.empty_like(ws)
+    moe.forward(ex, x, bad, ws=ws2)
+    assert moe.last_device_status() == moe.ERR_NONFINITE
+    assert moe.status_read(ws) == moe.OK and moe.status_read(ws2) == moe.ERR_NONFINITE

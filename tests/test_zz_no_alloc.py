@@ -74,3 +74,22 @@ def test_refuses_calls_beyond_capacity():
     ref_idx, _ = moe.route(cfg, x, wr)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(idx[:4736].cpu().numpy(), ref_idx.cpu().numpy())
+
+
+def test_status_of_the_fixed_scratch():
+    """The call's device status (here a NaN router row) is read through
+    nvfp4moe_last_device_status, the one reader of the fixed scratch's status word; the
+    selection still holds topk distinct in-range experts, the NaN expert ranked last."""
+    cfg = _cfg(BEAM)
+    x = activations(16, BEAM, seed=5).cuda()
+    wr = router_weight(BEAM).cuda()
+    idx = torch.empty((16, 8), dtype=torch.int32, device="cuda")
+    w = torch.empty((16, 8), dtype=torch.float32, device="cuda")
+    assert _route_noalloc(cfg, x, wr, None, idx, w) == moe.OK
+    assert moe.last_device_status() == moe.OK
+    wr[3, 7] = float("nan")
+    assert _route_noalloc(cfg, x, wr, None, idx, w) == moe.OK
+    assert moe.last_device_status() == moe.ERR_NONFINITE
+    got = idx.cpu().numpy()
+    assert ((got >= 0) & (got < BEAM.E)).all() and not (got == 3).any()
+    assert all(len(set(row.tolist())) == 8 for row in got)
