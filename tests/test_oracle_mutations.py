@@ -168,6 +168,8 @@ CASES = [
     # FP8 variant
     ("fp8-fnuz-max", "fp8", "row_scales", "(amax / F32(E4M3_MAX))", "(amax / F32(240.0))"),
     ("fp8-zero-row-scale", "fp8", "row_scales", "np.where(amax == 0, F32(1.0), s)", "s"),
+    ("fp8-per-tensor-scale", "fp8", "quantize_rows",
+     "s = row_scales(v)", "s = np.full(v.shape[0], row_scales(v).max(), dtype=F32)"),
     ("fp8-reciprocal-multiply", "fp8", "quantize_rows",
      "q = (v / s[:, None]).astype(F32)", "q = (v * (F32(1.0) / s)[:, None]).astype(F32)"),
     ("fp8-loses-negative-zero", "fp8", "e4m3_encode_signed", "np.where(np.signbit(q),", "np.where(q < 0,"),
