@@ -25,7 +25,7 @@ def _cuda():
 
 
 def _stream_and_gamma(shape, T, seed):
-    """A residual stream of RMS about 3 and a BF16-valued norm weight around 1 (seeded)."""
+    """A residual stream of RMS about 3 and a BF16-valued norm weight near 1 (seeded)."""
     h = (activations(T, shape, seed=seed).float() * 3.0).to(torch.bfloat16)
     gen = torch.Generator().manual_seed(1000 + seed)
     gamma = (1.0 + 0.1 * torch.randn(shape.H, generator=gen)).to(torch.bfloat16).float()
