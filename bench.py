@@ -740,7 +740,6 @@ def run_quantize_lh(args, world, rank, local):
     operations; the roofline counts 2 x 272 FLOP per block-candidate against the FP32 FMA peak
     of the SMs at the maximum SM clock."""
     import nvfp4_quantized_moe_group_b200 as moe
-    import oracle
     H, I, m = BEAM.H, BEAM.I, 4
     shapes = [(I, H), (I, H), (H, I)]
     mats, hess = [], []
@@ -748,7 +747,9 @@ def run_quantize_lh(args, world, rank, local):
         mats.append(expert_weight(BEAM, j, ("gate", "up", "down")[j], device="cuda"))
         x = activations(256, LayerShape(H=cols, I=I, E=1, n_groups=1, topk_groups=1, topk=1, routed_scale=1.0,
                                         wr_std=1.0, w_std=0.02), seed=70 + j + rank)
-        hess.append(torch.from_numpy(oracle.hessian_blocks(x.float().numpy()).astype(np.float32)).cuda())
+        # the caller's calibration statistics: the 16x16 diagonal blocks of X^T X (FP64, then FP32)
+        xb = x.double().reshape(x.shape[0], cols // 16, 16)
+        hess.append(torch.einsum("nbi,nbj->bij", xb, xb).float().contiguous().cuda())
     ws = torch.empty(moe.quantize_workspace_bytes(H, H), dtype=torch.uint8, device="cuda")
 
     def step():
