@@ -186,3 +186,17 @@ def test_worked_layer_example():
     assert np.flatnonzero(out).tolist() == [9]
     np.testing.assert_allclose(out[9], 1008 * (8 * w3 + 4 * w2), rtol=1e-14)
     assert res["out_bf16"][0, 9] == 15808.0
+
+
+def test_stored_intermediate_scales_are_reproducible():
+    """The stored static scales g_h of the tiny layer are what the committed calibration
+    script computes from the oracle today."""
+    import importlib.util
+    import os
+    from tests.helpers import intermediate_scales
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location(
+        "make_intermediate_scales", os.path.join(root, "tests", "golden", "make_intermediate_scales.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    np.testing.assert_array_equal(mod.calibrate(TINY), intermediate_scales(TINY))
