@@ -56,9 +56,13 @@ def test_stored_traffic_applies_only_to_its_sources_and_workload(monkeypatch):
     assert bench.stored_traffic("decode", 99) is None
 
 
-def test_peaks_are_the_measured_file():
+def test_peaks_are_the_measured_file_else_the_fallback():
     p = bench.peaks()
-    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(path):
+        assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16_tflops"] == 1590.0
+        return
+    with open(path) as f:
         m = json.load(f)
     assert p["source"] == "measured" and p["hbm_gbs"] == m["hbm_gbs"] and p["bf16_tflops"] == m["bf16_tflops"]
 
