@@ -46,3 +46,15 @@ def test_zipf_bias_range():
     p = np.arange(1, 257) ** -1.1
     p /= p.sum()
     assert abs(b.max().item() - 0.5 * np.log(p[0])) < 1e-6 and abs(b.min().item() - 0.5 * np.log(p[-1])) < 1e-6
+
+
+def test_hash_follows_the_published_fmix32():
+    """Both backends' hash is MurmurHash3's 32-bit finaliser: the torch one (int64 with emulated
+    32-bit products) equals the plain Python-integer statement of it on edge and random words;
+    fmix32(1) = 0x514E28B7 and fmix32(0) = 0, values the finaliser is commonly checked with."""
+    from workloads.synthetic import _fmix32, _fmix32_int
+    assert _fmix32_int(0) == 0 and _fmix32_int(1) == 0x514E28B7
+    words = [0, 1, 2, 0x7FFFFFFF, 0x80000000, 0xFFFFFFFF, 0xDEADBEEF]
+    words += np.random.default_rng(0).integers(0, 1 << 32, 2000, dtype=np.uint64).tolist()
+    got = _fmix32(torch.tensor(words, dtype=torch.int64)).tolist()
+    assert got == [_fmix32_int(w) for w in words]
