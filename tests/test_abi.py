@@ -49,3 +49,41 @@ def test_argument_errors_return_without_gpu(lib):
     c = moe.cfg_default()
     assert lib.nvfp4moe_route(ctypes.byref(c), None, 4, None, None, None, None, None, 0, None) == moe.ERR_ARG
     assert lib.nvfp4moe_forward(None, None, 4, None, None, None, None, None, 0, None) == moe.ERR_ARG
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "nvfp4moe.h"
+int main(void) {
+  nvfp4moe_cfg c;
+  if (nvfp4moe_cfg_default(&c) != NVFP4MOE_OK) return 1;
+  if (nvfp4moe_cfg_check(&c) != NVFP4MOE_OK) return 2;
+  size_t ws = nvfp4moe_workspace_bytes(&c, 16);
+  if (ws == 0 || ws != nvfp4moe_forward_workspace_bytes(&c, 16)) return 3;
+  if (nvfp4moe_quantize(NULL, 4, 63, NULL, NULL, NULL, 0, NULL, NULL, 0, NULL) != NVFP4MOE_ERR_SHAPE) return 4;
+  printf("%d %d %d %d %d %d %s\n", c.E, c.n_groups, c.topk_groups, c.topk, c.H, c.I,
+         nvfp4moe_status_string(NVFP4MOE_ERR_SHAPE));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/nvfp4moe.h compiles as C99 and C++17, and a C program links against the library
+    and calls its host-only entry points."""
+    import os
+    inc = os.path.join(os.path.dirname(moe.LIB_PATH), "..", "include")
+    hdr = os.path.join(inc, "nvfp4moe.h")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-x", "c", hdr],
+                   check=True)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Werror", "-fsyntax-only", "-x", "c++", hdr], check=True)
+    src = tmp_path / "main.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "main"
+    libdir = os.path.dirname(moe.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-L", libdir, "-lnvfp4moe",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out
+    assert out.stdout.split()[:6] == ["256", "8", "4", "8", "5120", "2560"]
+    assert "unsupported shape" in out.stdout
