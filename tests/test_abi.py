@@ -68,11 +68,15 @@ int main(void) {
 """
 
 
-def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+def test_header_is_plain_c_and_links_from_c(lib):
     """include/nvfp4moe.h compiles as C99 and C++17, and a C program links against the library
-    and calls its host-only entry points."""
+    and calls its host-only entry points (built under the git-ignored _build/)."""
     import os
-    inc = os.path.join(os.path.dirname(moe.LIB_PATH), "..", "include")
+    import pathlib
+    root = os.path.dirname(os.path.dirname(moe.LIB_PATH))
+    inc = os.path.join(root, "include")
+    tmp_path = pathlib.Path(root, "_build", "abi_c")
+    tmp_path.mkdir(parents=True, exist_ok=True)
     hdr = os.path.join(inc, "nvfp4moe.h")
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-x", "c", hdr],
                    check=True)
