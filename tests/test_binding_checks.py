@@ -130,3 +130,14 @@ def test_route_noalloc_inputs(cfg):
 def test_every_declared_call_is_bound():
     from nvfp4_quantized_moe_group_b200 import _lib
     assert set(_lib.declared_symbols()) == set(_lib._SIGS)
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No CPU fallback: without the built library every call raises instead of computing."""
+    from nvfp4_quantized_moe_group_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libnvfp4moe.so")
+    with pytest.raises(ImportError, match="is missing"):
+        _lib.lib()
+    with pytest.raises(ImportError):
+        _lib.cfg_default()
