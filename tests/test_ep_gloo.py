@@ -55,7 +55,7 @@ def _rank_main(rank, world, port, out):
 
 @pytest.mark.parametrize("world", [2, 4])
 def test_gloo_ranks_expert_parallel_layer(world):
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)

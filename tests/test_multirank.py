@@ -38,7 +38,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_time_and_sum_tokens():
     world = 2
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
