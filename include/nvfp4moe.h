@@ -35,7 +35,8 @@
  *   * Argument and shape errors are reported synchronously by the return code and
  *     nothing is enqueued.  Errors found on the device (non-finite input, a bounded
  *     wait that ran out) are OR-ed into a status word at the start of the caller's
- *     workspace; nvfp4moe_status_read() returns it once the stream has finished.
+ *     workspace; nvfp4moe_status_read() (or nvfp4moe_last_device_status() for the
+ *     thread's latest call) returns it once the stream has finished.
  *   * Workspaces are caller-allocated device memory, 256-byte aligned, of at least the
  *     size the matching *_workspace_bytes() function returns.  A workspace must not be
  *     used by two calls that can run at the same time.
