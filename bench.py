@@ -39,7 +39,6 @@ E2M1_BYTES = 0.5                    # per value
 E4M3_PER16 = 1.0 / 16.0             # block-scale bytes per value
 
 
-GATEUP_SAMPLE = 8    # every 8th timed step carries the gate/up duration events
 RESIDUAL_STEP = 30   # residual step k of the timed fused-residual forward (a mid-depth MoE block)
 
 
@@ -215,7 +214,10 @@ def build_layer(moe, shape: LayerShape):
 
 
 def algorithmic(shape: LayerShape, T: int, counts: np.ndarray):
-    """Algorithmic bytes / FLOPs of one step, from the routing the step actually produced."""
+    """Algorithmic bytes / FLOPs of one step, from the routing the step actually produced.
+    Per GEMM: its weights (codes, E4M3 scales, FP32 globals) of the experts hit plus its NVFP4
+    A operand (gate/up also the requantised h it writes); the down GEMM's FP32 combine into the
+    accumulator is implementation traffic and not counted."""
     H, I, k = shape.H, shape.I, shape.topk
     hit = int((counts > 0).sum())
     pairs = T * k
@@ -223,11 +225,40 @@ def algorithmic(shape: LayerShape, T: int, counts: np.ndarray):
     w13 = 2 * I * H * per_val + 8                          # gate + up codes, scales, globals
     wd = H * I * per_val + 8
     gateup_bytes = hit * w13 + pairs * H * per_val + pairs * I * per_val
+    down_bytes = hit * wd + pairs * I * per_val
     layer_bytes = hit * (w13 + wd) + T * H * 2 + T * H * 2 + shape.E * H * 4
     flops = 2.0 * pairs * (2 * I * H + H * I)
     gateup_flops = 2.0 * pairs * 2 * I * H
-    return {"experts_hit": hit, "gateup_bytes": gateup_bytes, "layer_bytes": layer_bytes, "flops": flops,
-            "gateup_flops": gateup_flops}
+    down_flops = 2.0 * pairs * H * I
+    return {"experts_hit": hit, "gateup_bytes": gateup_bytes, "down_bytes": down_bytes, "layer_bytes": layer_bytes,
+            "flops": flops, "gateup_flops": gateup_flops, "down_flops": down_flops}
+
+
+def fp4_peaks(p: dict) -> tuple[float, float]:
+    """Dense FP4 tensor peak in TFLOP/s: the measured BF16 GEMM peak times the nominal
+    FP4 : BF16 ratio, burst (a kernel timed alone or a step of milliseconds) and sustained (a
+    seconds-long loop under the power cap)."""
+    return p["bf16_tflops"] * FP4_OVER_BF16, p["bf16_tflops_sustained"] * FP4_OVER_BF16
+
+
+def kernel_roofline(nbytes: float, flops: float, ms: float, p: dict) -> dict:
+    """One kernel against the roofline that binds it: HBM (bytes over the measured copy
+    bandwidth) or FP4 tensor (FLOPs over the burst FP4 peak), whichever takes longer; both
+    fractions are given, and the FP4 one also against the sustained peak."""
+    burst, sustained = fp4_peaks(p)
+    s = ms / 1e3
+    t_bytes = nbytes / (p["hbm_gbs"] * 1e9)
+    t_flops = flops / (burst * 1e12)
+    gbs = nbytes / s / 1e9
+    tflops = flops / s / 1e12
+    out = {"ms": ms, "bytes": nbytes, "flops": flops, "gbs": gbs, "tflops": tflops,
+           "hbm_frac": gbs / p["hbm_gbs"], "fp4_frac": tflops / burst, "fp4_frac_sustained": tflops / sustained}
+    if t_bytes >= t_flops:
+        out.update({"bound": "hbm", "achieved": gbs, "peak": p["hbm_gbs"], "unit": "GB/s"})
+    else:
+        out.update({"bound": "tensor", "achieved": tflops, "peak": burst, "unit": "TFLOP/s"})
+    out["frac"] = out["achieved"] / out["peak"]
+    return out
 
 
 def run_fp8(moe, shape: LayerShape, cfg, x, wr, bias, T: int, steps: int, warmup: int, world: int) -> dict:
@@ -407,6 +438,96 @@ def barrier(world: int):
         dist.barrier()
 
 
+CONFIG_WORKLOADS = ("prefill", "skewed", "sweep32768")   # the compute-heavy configs beside the headline
+
+
+def timed_steps(fn, steps: int, world: int, stream=None) -> float:
+    """Device time of ``steps`` calls of fn (CUDA events on the launching stream, a barrier and a
+    synchronize on both sides), max over ranks, in milliseconds."""
+    stream = stream if stream is not None else torch.cuda.current_stream()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for k in range(steps):
+        fn(k)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(start.elapsed_time(stop), world)
+
+
+def measure_workload(moe, ex, shape: LayerShape, wl, x, wr, bias, steps: int, warmup: int, world: int,
+                     clock=None) -> dict:
+    """One workload on the layer: K device-timed forwards with nothing recorded between their
+    launches (the figure the line reports), then K more with CUDA events around each
+    grouped GEMM (their durations, for the kernel rooflines), then a stage breakdown from
+    steps with every stage bracketed.  ``clock``: a ClockSampler to run over the first region."""
+    import contextlib
+    T = wl.T
+    out = torch.empty((T, shape.H), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(moe.forward_workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
+    _, dbg = moe.forward(ex, x, wr, bias, out=out, ws=ws, debug=True)
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"{wl.name}: forward status {moe.status_string(st)}")
+    alg = algorithmic(shape, T, dbg["counts"].cpu().numpy())
+    launches = moe.last_launch_count()
+    del dbg
+    for _ in range(warmup):
+        moe.forward(ex, x, wr, bias, out=out, ws=ws)
+    torch.cuda.synchronize()
+    with (clock if clock is not None else contextlib.nullcontext()):
+        torch.cuda.nvtx.range_push("timed")
+        elapsed = timed_steps(lambda k: moe.forward(ex, x, wr, bias, out=out, ws=ws), steps, world)
+        torch.cuda.nvtx.range_pop()
+    # the GEMM durations, from a second region of the same steps with events around both GEMMs
+    timers = [moe.StageTimer(("gateup", "down")) for _ in range(steps)]
+    ev_elapsed = timed_steps(lambda k: moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=timers[k]), steps, world)
+    gemm_ms = {n: max_over_ranks(statistics.mean(t.stage_ms()[n] for t in timers), world) for n in ("gateup", "down")}
+    full = [moe.StageTimer() for _ in range(min(steps, 20))]
+    for t in full:
+        moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=t)
+    torch.cuda.synchronize()
+    stage = {n: statistics.mean(t.stage_ms()[n] for t in full) for n in moe.STAGES if n not in ("amax", "gather")}
+    st = moe.status_read(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"{wl.name}: forward status {moe.status_string(st)}")
+    p = peaks()
+    ms = elapsed / steps
+    burst, sustained = fp4_peaks(p)
+    layer_s = ms / 1e3
+    return {
+        "workload": wl.describe(), "T_per_rank": T, "experts_hit": alg["experts_hit"], "ms_per_step": ms,
+        "value": tokens_per_second(world, T, steps, elapsed), "unit": "tokens/s",
+        "gpu_launches_per_step": launches, "alg": alg, "stage_ms": stage,
+        "gemms": {"gateup": kernel_roofline(alg["gateup_bytes"], alg["gateup_flops"], gemm_ms["gateup"], p),
+                  "down": kernel_roofline(alg["down_bytes"], alg["down_flops"], gemm_ms["down"], p)},
+        "gemm_region_ms_per_step": ev_elapsed / steps,
+        "layer_roofline": {"bytes_per_step": alg["layer_bytes"], "flops_per_step": alg["flops"],
+                           "hbm_frac": alg["layer_bytes"] / layer_s / (p["hbm_gbs"] * 1e9),
+                           "fp4_frac": alg["flops"] / layer_s / (burst * 1e12),
+                           "fp4_frac_sustained": alg["flops"] / layer_s / (sustained * 1e12),
+                           "tflops": alg["flops"] / layer_s / 1e12},
+        "_ws": ws, "_out": out,
+    }
+
+
+def config_entry(m: dict, wl) -> dict:
+    """The JSON object of one compute-heavy config: its step time and throughput, stage times,
+    the roofline of its dominant kernel (the gate/up GEMM, two thirds of the FLOPs and weight
+    bytes) and of the down GEMM, and the whole layer against both rooflines."""
+    g = m["gemms"]
+    return {"workload": m["workload"], "T_per_rank": m["T_per_rank"], "experts_hit": m["experts_hit"],
+            "ms_per_step": m["ms_per_step"], "value": m["value"], "unit": "tokens/s",
+            "stage_ms": m["stage_ms"], "roofline": {**{k: g["gateup"][k] for k in
+                                                       ("bound", "achieved", "peak", "unit", "frac")},
+                                                    "kernel": "moe_gemm_kernel<gate/up>", "traffic": None},
+            "gemms": g, "layer_roofline": m["layer_roofline"],
+            "l2": "no flush: every step streams the routed experts' weights "
+                  f"({m['alg']['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"}
+
+
 def run_ours(args, world, rank, local):
     import nvfp4_quantized_moe_group_b200 as moe
     wl = WORKLOADS[args.workload]
@@ -419,53 +540,14 @@ def run_ours(args, world, rank, local):
     x = x_cpu.cuda()
     wr = wr_cpu.cuda()
     bias = None if bias_cpu is None else bias_cpu.cuda()
-    out = torch.empty((T, shape.H), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(moe.forward_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    # routing of this batch (for the algorithmic byte count) and a status check
-    _, dbg = moe.forward(ex, x, wr, bias, out=out, ws=ws, debug=True)
-    st = moe.status_read(ws)
-    if st != moe.OK:
-        raise RuntimeError(f"forward status {moe.status_string(st)}")
-    alg = algorithmic(shape, T, dbg["counts"].cpu().numpy())
-    launches_per_step = moe.last_launch_count()
-    del dbg
-
-    # inside the timed region only the dominant kernel is bracketed by events
-    # The GEMMs are launched programmatically (each may start while its predecessor drains); an
-    # event recorded between two kernels serialises them, so only every GATEUP_SAMPLE-th step
-    # brackets its gate/up launch with events.
-    timers = {k: moe.StageTimer(("gateup",)) for k in range(0, args.steps, GATEUP_SAMPLE)}
-    for _ in range(args.warmup):
-        moe.forward(ex, x, wr, bias, out=out, ws=ws)
-    torch.cuda.synchronize()
-
-    # ---- device-timed region: K back-to-back steps, inputs resident in HBM
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
-        torch.cuda.nvtx.range_push("timed")
-        start.record(stream)
-        for k in range(args.steps):
-            moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=timers.get(k))
-        stop.record(stream)
-        torch.cuda.synchronize()
-        torch.cuda.nvtx.range_pop()
-    barrier(world)
-    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
-    gateup_ms = statistics.mean(t.stage_ms()["gateup"] for t in timers.values())
-    # stage breakdown from separate (untimed) steps with every stage bracketed
-    full = [moe.StageTimer() for _ in range(min(args.steps, 20))]
-    for t in full:
-        moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=t)
-    torch.cuda.synchronize()
-    stage = {n: statistics.mean(t.stage_ms()[n] for t in full) for n in moe.STAGES
-             if n not in ("amax", "gather")}
-    st = moe.status_read(ws)
-    if st != moe.OK:
-        raise RuntimeError(f"forward status {moe.status_string(st)}")
+    # ---- the headline workload: device-timed steps with inputs resident in HBM and nothing
+    # recorded between launches, then the GEMMs' durations and the stage breakdown
+    clocks = ClockSampler(local, args.clock_period_ms / 1000.0)
+    m = measure_workload(moe, ex, shape, wl, x, wr, bias, args.steps, args.warmup, world, clock=clocks)
+    ws, out = m.pop("_ws"), m.pop("_out")
+    alg = m["alg"]
 
     # ---- end to end: pinned host input -> device, forward, device -> pinned host output.  Every
     # step copies its tokens in and its output rows out; the copies run on a second stream,
@@ -481,15 +563,7 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
-    barrier(world)
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record()
-    for _ in range(args.steps):
-        graph.replay()
-    g1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    graph_ms = max_over_ranks(g0.elapsed_time(g1), world)
+    graph_ms = timed_steps(lambda k: graph.replay(), args.steps, world)
     del graph
     st = moe.status_read(ws)
     if st != moe.OK:
@@ -502,60 +576,59 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         moe.forward_residual(ex, h_res, gamma, 1e-6, RESIDUAL_STEP, wr, bias, out=h_out, ws=ws)
     torch.cuda.synchronize()
-    barrier(world)
-    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    r0.record()
-    for _ in range(args.steps):
-        moe.forward_residual(ex, h_res, gamma, 1e-6, RESIDUAL_STEP, wr, bias, out=h_out, ws=ws)
-    r1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    residual_ms = max_over_ranks(r0.elapsed_time(r1), world)
+    residual_ms = timed_steps(lambda k: moe.forward_residual(ex, h_res, gamma, 1e-6, RESIDUAL_STEP, wr, bias,
+                                                             out=h_out, ws=ws), args.steps, world)
     st = moe.status_read(ws)
     if st != moe.OK:
         raise RuntimeError(f"residual forward status {moe.status_string(st)}")
+    del ws, out
 
     fp8 = None if args.no_fp8 else run_fp8(moe, shape, cfg, x, wr, bias, T, args.steps, args.warmup, world)
 
+    # ---- the compute-heavy configs on the same layer (prefill, skewed routing, the largest
+    # token count of the sweep) and the standalone activation quantisation
+    configs = {}
+    if not args.no_configs and not args.experts and wl.shape == BEAM:
+        for name in CONFIG_WORKLOADS:
+            cw = WORKLOADS[name]
+            xc = activations(cw.T, shape, seed=cw.seed + rank, device="cuda")
+            bc = zipf_bias(shape.E).cuda() if cw.zipf else None
+            cclk = ClockSampler(local, args.clock_period_ms / 1000.0)
+            cm = measure_workload(moe, ex, shape, cw, xc, wr, bc, args.steps, args.warmup, world, clock=cclk)
+            cm.pop("_ws"), cm.pop("_out")
+            configs[name] = {**config_entry(cm, cw), "clocks": cclk.summary()}
+            del xc
+            torch.cuda.empty_cache()
+        qclk = ClockSampler(local, args.clock_period_ms / 1000.0)
+        q = measure_quantize(moe, args.steps, args.warmup, world, rank, clock=qclk)
+        configs["quantize"] = {**{k: q[k] for k in ("workload", "ms_per_step", "value", "unit", "roofline")},
+                               "clocks": qclk.summary()}
+
     p = peaks()
-    ms_step = elapsed_ms / args.steps
-    tokens_per_s = tokens_per_second(world, T, args.steps, elapsed_ms)
-    # dominant kernel: the gate/up grouped GEMM (2/3 of the weight bytes and FLOPs)
-    gu_s = gateup_ms / 1e3
-    t_bytes = alg["gateup_bytes"] / (p["hbm_gbs"] * 1e9)
-    fp4_peak = p["bf16_tflops_sustained"] * FP4_OVER_BF16
-    t_flops = alg["gateup_flops"] / (fp4_peak * 1e12)
-    if t_bytes >= t_flops:
-        roof = {"bound": "hbm", "achieved": alg["gateup_bytes"] / gu_s / 1e9, "peak": p["hbm_gbs"], "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": alg["gateup_flops"] / gu_s / 1e12, "peak": fp4_peak,
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    gu = m["gemms"]["gateup"]
+    roof = {k: gu[k] for k in ("bound", "achieved", "peak", "unit", "frac")}
     roof["traffic"] = stored_traffic(args.workload if not args.experts else f"{args.workload}-e{shape.E}",
                                      alg["experts_hit"])
     roof["kernel"] = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
-    roof["duration_source"] = (f"CUDA events around the gate/up launch of every {GATEUP_SAMPLE}th step of the "
-                               f"timed region ({len(timers)} launches), on the launching stream")
-    roof["peak_source"] = (f"{p['source']} hbm_gbs" if roof["bound"] == "hbm"
-                           else f"{p['source']} bf16_tflops_sustained x {FP4_OVER_BF16:g} (nominal FP4:BF16)")
-    layer_s = ms_step / 1e3
-    layer_roof = {"bytes_per_step": alg["layer_bytes"], "flops_per_step": alg["flops"],
-                  "hbm_frac": alg["layer_bytes"] / layer_s / (p["hbm_gbs"] * 1e9),
-                  "fp4_frac": alg["flops"] / layer_s / (fp4_peak * 1e12)}
+    roof["duration_source"] = (f"CUDA events around the gate/up launch of each of {args.steps} steps of a second "
+                               "timed region right after the headline one (same inputs), on the launching stream")
+    roof["peak_source"] = (f"{p['source']} hbm_gbs (a copy bandwidth: a read-only stream can exceed it slightly)"
+                           if roof["bound"] == "hbm"
+                           else f"{p['source']} bf16_tflops (burst) x {FP4_OVER_BF16:g} (nominal FP4:BF16)")
     res = {
-        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate)",
         "data": "synthetic (seeded counter-hash inputs; random-init NVFP4 weights)",
         "config": {"workload": wl.describe() if not args.experts else wl.describe() + f" (E={shape.E} variant)",
                    "T_per_rank": T, "experts_hit": alg["experts_hit"], "parallelism": f"dp{world} (replicas)",
                    "l2": "no flush: every step streams the routed experts' weights "
                          f"({alg['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"},
-        "roofline": roof, "layer_roofline": layer_roof,
-        "stage_ms": stage,
+        "roofline": roof, "layer_roofline": m["layer_roofline"], "gemms": m["gemms"],
+        "stage_ms": m["stage_ms"],
         "e2e": {"value": tokens_per_second(world, T, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": m["gpu_launches_per_step"] * args.steps,
         "clocks": clocks.summary(),
         "residual": {"value": tokens_per_second(world, T, args.steps, residual_ms), "unit": "tokens/s",
                      "ms_per_step": residual_ms / args.steps, "step_k": RESIDUAL_STEP,
@@ -565,6 +638,8 @@ def run_ours(args, world, rank, local):
                   "ms_per_step": graph_ms / args.steps,
                   "note": "the same forward captured once in a CUDA graph and replayed K times"},
     }
+    if configs:
+        res["configs"] = configs
     if fp8 is not None:
         res["fp8"] = fp8
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -573,43 +648,50 @@ def run_ours(args, world, rank, local):
     return res
 
 
-def run_quantize(args, world, rank, local):
+QUANT_ROWS = 32768
+
+
+def measure_quantize(moe, steps: int, warmup: int, world: int, rank: int, clock=None) -> dict:
     """Standalone quantize_nvfp4 on 32768 x 5120 BF16 activations with a dynamic global scale
     and swizzled scales: the amax pass reads x once, the quantise pass reads it again and
     writes codes + scales, so the algorithmic bytes are 2 * 2 * rows * cols + rows * cols * 9/16."""
-    import nvfp4_quantized_moe_group_b200 as moe
-    rows, cols = 32768, BEAM.H
+    import contextlib
+    rows, cols = QUANT_ROWS, BEAM.H
     x = activations(rows, BEAM, seed=rank, device="cuda")
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
     scales = torch.empty(moe.swizzled_scale_bytes(rows, cols // 16), dtype=torch.uint8, device="cuda")
     g = torch.empty(1, dtype=torch.float32, device="cuda")
     ws = torch.empty(moe.quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g))
     torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    with ClockSampler(local, args.clock_period_ms / 1000.0) as clocks:
-        start.record()
-        for _ in range(args.steps):
-            moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g))
-        stop.record()
-        torch.cuda.synchronize()
-    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    with (clock if clock is not None else contextlib.nullcontext()):
+        elapsed = timed_steps(lambda k: moe.quantize(x, swizzled=True, ws=ws, out=(codes, scales, g)), steps, world)
+    ms = elapsed / steps
     launches = moe.last_launch_count()
     if moe.status_read(ws) != moe.OK:
         raise RuntimeError("quantize status")
     nbytes = 2 * rows * cols * 2 + rows * cols // 2 + rows * cols // 16
     p = peaks()
     gbs = world * nbytes / (ms / 1e3) / 1e9
-    return {"metric": "quantize_nvfp4 HBM GB/s (32768x5120 BF16, dynamic global scale, swizzled scales)",
-            "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e2m1",
-            "data": "synthetic", "config": {"workload": "quantize 32768x5120", "bytes_per_step": nbytes,
-                                            "l2": "input 335 MB > 126 MB L2 (no flush)"},
+    return {"workload": f"quantize {rows}x{cols} (dynamic global scale, swizzled scales)", "ms_per_step": ms,
+            "value": gbs, "unit": "GB/s", "bytes_per_step": nbytes, "launches": launches,
             "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": p["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / world / p["hbm_gbs"], "traffic": None},
-            "gpu_launches": launches * args.steps, "clocks": clocks.summary()}
+                         "frac": gbs / world / p["hbm_gbs"], "traffic": None}}
+
+
+def run_quantize(args, world, rank, local):
+    """The standalone quantisation as its own bench line (``--workload quantize``)."""
+    import nvfp4_quantized_moe_group_b200 as moe
+    clocks = ClockSampler(local, args.clock_period_ms / 1000.0)
+    q = measure_quantize(moe, args.steps, args.warmup, world, rank, clock=clocks)
+    return {"metric": "quantize_nvfp4 HBM GB/s (32768x5120 BF16, dynamic global scale, swizzled scales)",
+            "value": q["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": q["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16->e2m1", "data": "synthetic",
+            "config": {"workload": "quantize 32768x5120", "bytes_per_step": q["bytes_per_step"],
+                       "l2": "input 335 MB > 126 MB L2 (no flush)"},
+            "roofline": q["roofline"], "gpu_launches": q["launches"] * args.steps, "clocks": clocks.summary()}
 
 
 def run_ep(args, world, rank, local):
@@ -842,6 +924,8 @@ def main():
     ap.add_argument("--experts", type=int, default=None, help="smaller layer with this many experts (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 W8A8 variant's measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the compute-heavy configs (prefill, skewed, 32768 tokens, quantise) of the line")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the ranks (each holds E/N experts; NCCL all-gather and "
                          "reduce-scatter) instead of one full replica per GPU")

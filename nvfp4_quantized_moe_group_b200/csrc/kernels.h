@@ -143,6 +143,9 @@ int router_ksplit(int64_t T, int E, int H);
 // Kernels launch_router enqueues for these arguments.
 int router_launch_count(const RouterArgs& a);
 size_t router_parts_elems(int64_t T_max, int E, int H);
+// The same bound for the FP32 logits kernels alone (what launch_router uses when it is given
+// no digit-plane buffers, as the allocation-free router is).
+size_t router_fp32_parts_elems(int64_t T_max, int E, int H);
 // Number of amax partials the logits kernel writes for T tokens (grid x * split-K).
 int router_amax_partials(int64_t T, int E, int H);
 cudaError_t launch_router(RouterArgs a, cudaStream_t stream);

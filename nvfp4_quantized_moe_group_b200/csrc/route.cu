@@ -298,6 +298,16 @@ size_t router_parts_elems(int64_t T_max, int E, int H) {
   return best;
 }
 
+size_t router_fp32_parts_elems(int64_t T_max, int E, int H) {
+  size_t best = 0;
+  for (int64_t c = 1; c <= (T_max + kTM - 1) / kTM; ++c) {
+    const int64_t T = c * kTM < T_max ? c * kTM : T_max;
+    const size_t n = (size_t)router_ksplit(T, E, H) * (size_t)T * (size_t)E;
+    if (n > best) best = n;
+  }
+  return best;
+}
+
 int router_amax_partials(int64_t T, int E, int H) {
   if (T >= kRouterTcMinT) return router_tc_amax_partials(T);
   const int tm = tile_tokens(T);

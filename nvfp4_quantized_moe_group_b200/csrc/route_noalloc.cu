@@ -61,7 +61,9 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
                 reinterpret_cast<uintptr_t>(hidden_bf16) % 16 != 0 ||
                 reinterpret_cast<uintptr_t>(w_router) % 16 != 0))
     return NVFP4MOE_ERR_ARG;
-  if (T > 0 && router_parts_elems(T, cfg->E, cfg->H) > kNoAllocParts) return NVFP4MOE_ERR_WORKSPACE;
+  // this call runs the FP32 logits kernels only (no digit-plane buffers), so only their
+  // split-K partials have to fit
+  if (T > 0 && router_fp32_parts_elems(T, cfg->E, cfg->H) > kNoAllocParts) return NVFP4MOE_ERR_WORKSPACE;
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||

@@ -10,9 +10,9 @@ quantisation rule is stated in FP32.
 Sources followed (page titles of the pages describing the method):
 
 * "NVFP4 quantization" (Reflection developer docs), section "Quantization
-  scheme": weights and input activations are 4-bit E2M1 values, each block of
-  16 values shares one FP8 E4M3 scale, and each tensor has one more global
-  scale; the routed-expert gate/up/down projections are the quantised tensors.
+  scheme": the format (E2M1 codes, an E4M3 scale for every 16-value block and
+  an FP32 scale for the whole tensor) and which tensors carry it (the routed
+  experts' gate, up and down projections and their input activations).
 * "Reflection releases Beam, a 501B-parameter MoE model ..." (bpdata news),
   section "Mixture-of-Experts details": sigmoid scores over 256 experts,
   8 groups of 32, keep 4 groups by the sum of each group's top two scores,

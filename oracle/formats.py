@@ -1,8 +1,8 @@
 """NVFP4 number formats and the quantisation rule, written out plainly.  TEST INFRASTRUCTURE ONLY.
 
-Format ("NVFP4 quantization", section "Quantization scheme"): every value is a
-4-bit E2M1 number; every block of 16 consecutive values along a row shares one
-FP8 E4M3 scale; every tensor carries one FP32 global scale.  A stored value
+Format ("NVFP4 quantization", section "Quantization scheme"): 4-bit E2M1 codes,
+an E4M3 scale for each run of 16 consecutive values along a row, and an FP32
+scale for the whole tensor.  A stored value
 decodes to ``E2M1[c] * E4M3[S_b] * g``.
 
 The pages do not say how the scales are chosen.  Reading used here (a block

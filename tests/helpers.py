@@ -71,16 +71,18 @@ def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarra
     return np.maximum(router_logit_bound_fp32(x, wr, bias, H), router_logit_bound_int(x, wr, bias, H))
 
 
-def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6):
+def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6,
+                  bound=router_logit_bound):
     """Near-tie protocol.  A token is clean when every routing decision has a margin larger
     than the FP32 error bound; clean tokens must match the oracle bit for bit (experts and
     their order).  Other tokens must pick an admissible selection: experts from groups and
     scores within the error bound of the exact choice.  Weights are compared (relative
-    tolerance) against the oracle's weights of the GPU's own selection.
+    tolerance) against the oracle's weights of the GPU's own selection.  ``bound`` gives the
+    logit error bound of the path under test (default: the larger of the two documented ones).
     Returns (clean token mask, number of flagged tokens)."""
     T, K = gpu_idx.shape
     gs = shape.E // shape.n_groups
-    bl = router_logit_bound(x, wr, bias, shape.H)
+    bl = bound(x, wr, bias, shape.H)
     s = r.scores
     eps_s = bl * s * (1 - s) + 8 * U                       # sigmoid: Lipschitz s(1-s) + its own rounding
     eps = eps_s.max(axis=1)                                # per token
@@ -120,6 +122,43 @@ def _expert_job(args):
     gate, up, down = oracle_expert(shape, e)
     res = oracle.expert_mlp(xhat, gate, up, down, np.float32(g_h))
     return e, res["y"], res["h"], res["hq_codes"], res["hq_scales"], (gate.g, up.g, down.g)
+
+
+def _init_single_thread():
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+
+
+def _expert_rows_job(args):
+    """One expert on a batch of dequantised input rows (possibly from several layer calls):
+    the oracle's SwiGLU MLP and requantised h, plus the down projection of the GPU's own
+    requantised h of the same rows (the oracle run on the same quantised operands)."""
+    shape, e, xhat, g_h, gpu_hq_codes, gpu_hq_scales = args
+    gate, up, down = oracle_expert(shape, e)
+    res = oracle.expert_mlp(xhat, gate, up, down, np.float32(g_h))
+    y_gpu_hq = res["y"].copy()
+    if gpu_hq_codes is None:
+        return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"]
+    same = (np.all(gpu_hq_codes == res["hq_codes"], axis=1) & np.all(gpu_hq_scales == res["hq_scales"], axis=1))
+    if not same.all():
+        hhat = oracle.dequantize(gpu_hq_codes[~same], gpu_hq_scales[~same], np.float32(g_h))
+        y_gpu_hq[~same] = hhat @ down.dequant().T
+    return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"]
+
+
+def oracle_expert_pass(shape, jobs: dict, workers=None) -> dict:
+    """Runs _expert_rows_job for every expert of ``jobs`` (e -> (xhat, g_h, gpu hq codes,
+    gpu hq scales), the last two None when there is no GPU intermediate to reuse) in a spawn
+    process pool, one BLAS thread per worker."""
+    args = [(shape, e, *v) for e, v in sorted(jobs.items())]
+    if workers is None:
+        workers = max(1, min(len(args), len(os.sched_getaffinity(0)) - 1))
+    if workers > 1:
+        with mp.get_context("spawn").Pool(workers, initializer=_init_single_thread) as pool:
+            results = pool.map(_expert_rows_job, args, chunksize=1)
+    else:
+        results = [_expert_rows_job(a) for a in args]
+    return {r[0]: r[1:] for r in results}
 
 
 def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, tokens=None, workers=None,
@@ -167,11 +206,14 @@ def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
 
 
 def check_output(gpu_out: np.ndarray, ref: np.ndarray, max_abs=2e-2, rel_fro=5e-3):
-    """Layer output tolerance: max-abs 2e-2 (plus the BF16 output rounding of each value)
-    and relative Frobenius 5e-3 against the oracle's FP64 output."""
+    """Layer output tolerance: max-abs 2e-2 and relative Frobenius 5e-3 of the BF16 output
+    against the oracle's FP64 output.  The BF16 rounding of the output is part of the error
+    (half a unit in the last place is below 2e-2 for every |value| < 8, which every output
+    checked here is)."""
+    assert np.all(np.abs(ref) < 8.0), f"an output of magnitude {np.abs(ref).max():.3g} is beyond the range " \
+                                      "where the BF16 rounding alone stays below the limit"
     err = np.abs(gpu_out - ref)
-    lim = max_abs + bf16_half_ulp(ref)
-    bad = err > lim
+    bad = err > max_abs
     assert not bad.any(), f"{int(bad.sum())} outputs beyond tolerance; worst {err.max():.4g}"
     fro = np.linalg.norm(gpu_out - ref) / max(np.linalg.norm(ref), 1e-30)
     assert fro <= rel_fro, f"relative Frobenius error {fro:.3g}"

@@ -34,6 +34,10 @@ def test_per_unit_figures_of_the_beam_layer():
     gu = 3 * (2 * BEAM.I * BEAM.H * 9 // 16 + 8) + 8 * BEAM.H * 9 // 16 + 8 * BEAM.I * 9 // 16
     assert a1["gateup_bytes"] == gu
     assert a1["gateup_flops"] == 2 * 8 * 2 * BEAM.I * BEAM.H
+    # down: its weights (1/3 of the codes and scales, two globals) and its A operand (the h rows)
+    assert a1["down_bytes"] == 3 * (BEAM.I * BEAM.H * 9 // 16 + 8) + 8 * BEAM.I * 9 // 16
+    assert a1["down_flops"] == 2 * 8 * BEAM.H * BEAM.I
+    assert a1["gateup_flops"] + a1["down_flops"] == a1["flops"]
 
 
 def test_decode_step_bytes_match_the_stated_figure():
@@ -78,3 +82,42 @@ def test_small_layer_accounting_scales_with_the_shape():
     a = bench.algorithmic(TINY, 4, counts)
     assert a["experts_hit"] == TINY.E
     assert a["flops"] == 2 * 4 * TINY.topk * 3 * TINY.H * TINY.I
+
+
+def test_prefill_down_bytes_match_the_stated_figure():
+    """At T = 4096 with every expert hit the down GEMM moves 1.934 GB: 256 experts x 7,372,808
+    bytes of weights plus 32,768 pairs x 1,440 bytes of requantised h."""
+    counts = np.full(BEAM.E, 128, dtype=np.int64)
+    a = bench.algorithmic(BEAM, 4096, counts)
+    assert a["down_bytes"] == 256 * 7_372_808 + 32_768 * 1_440
+    assert abs(a["down_bytes"] / 1e9 - 1.9346) < 0.0001
+
+
+def test_kernel_roofline_takes_the_binding_bound_and_the_burst_fp4_peak():
+    p = {"hbm_gbs": 6546.2, "bf16_tflops": 1615.2, "bf16_tflops_sustained": 1365.0, "source": "measured"}
+    burst, sustained = bench.fp4_peaks(p)
+    assert burst == pytest.approx(6460.8) and sustained == pytest.approx(5460.0)
+    # decode gate/up: 1.46 GB, 5.2 GFLOP in 0.2157 ms -> HBM bound
+    r = bench.kernel_roofline(1_460_368_152, 5.2e9, 0.2157, p)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(1_460_368_152 / 0.2157e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6546.2)
+    # T = 32768 gate/up: 13.7 TFLOP in 3.30 ms -> tensor bound, scored against the burst peak
+    r = bench.kernel_roofline(6.4e9, 13.74e12, 3.30, p)
+    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(burst)
+    assert r["frac"] == pytest.approx(13.74e12 / 3.30e-3 / 1e12 / burst)
+    assert r["fp4_frac_sustained"] == pytest.approx(13.74e12 / 3.30e-3 / 1e12 / sustained)
+    assert r["fp4_frac"] == r["frac"] and r["hbm_frac"] == pytest.approx(6.4e9 / 3.30e-3 / 1e9 / 6546.2)
+
+
+def test_config_entry_reports_the_dominant_kernel():
+    p = {"hbm_gbs": 6546.2, "bf16_tflops": 1615.2, "bf16_tflops_sustained": 1365.0, "source": "measured"}
+    counts = np.full(BEAM.E, 1024, dtype=np.int64)
+    alg = bench.algorithmic(BEAM, 32768, counts)
+    m = {"workload": "w", "T_per_rank": 32768, "experts_hit": 256, "ms_per_step": 8.0, "value": 1.0,
+         "stage_ms": {}, "alg": alg, "layer_roofline": {},
+         "gemms": {"gateup": bench.kernel_roofline(alg["gateup_bytes"], alg["gateup_flops"], 3.3, p),
+                   "down": bench.kernel_roofline(alg["down_bytes"], alg["down_flops"], 3.3, p)}}
+    e = bench.config_entry(m, None)
+    assert e["roofline"]["bound"] == "tensor" and e["roofline"]["frac"] == m["gemms"]["gateup"]["frac"]
+    assert e["gemms"]["down"]["bound"] == "tensor"

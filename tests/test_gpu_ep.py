@@ -1,9 +1,11 @@
 """Expert parallelism on one GPU (nvfp4moe_experts_create_local, nvfp4moe_forward_partial,
 nvfp4moe_finalize): G ranks are emulated one after another on the same device, with the
 all-gather a concatenation and the reduce-scatter an FP32 sum over the ranks' partial sums.
-The ranks' sums must add up to the single-handle layer (up to the order of FP32 additions),
-a token none of whose experts a rank holds must get an exact zero row from it, and the
-rounded result must match nvfp4moe_forward within one BF16 unit."""
+Each rank's FP32 sums are judged against the oracle's sum of that rank's experts'
+contributions (max-abs 2e-2, relative Frobenius 5e-3, on tokens the GPU routes as the oracle
+does); the ranks' sums must add up to the single-handle layer (up to the order of FP32
+additions), a token none of whose experts a rank holds must get an exact zero row from it,
+and the rounded result must match nvfp4moe_forward within one BF16 unit."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +13,8 @@ import torch
 import nvfp4_quantized_moe_group_b200 as moe
 from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer, expert_range
 from workloads import TINY, BEAM, activations, router_weight, expert_weight
-from tests.helpers import intermediate_scales, bf16_half_ulp
+import oracle
+from tests.helpers import intermediate_scales, bf16_half_ulp, cfg_ns, oracle_expert_pass, check_output
 from tests.test_gpu_forward import gpu_experts
 
 pytestmark = pytest.mark.gpu
@@ -36,14 +39,34 @@ def local_experts(shape, e0, n):
     return ex
 
 
-def run_emulated(shape, G, T_rank, seed=50):
+def run_emulated(shape, G, T_rank, seed=50, sample=None):
+    """``sample``: gathered token indices whose per-rank sums are compared with the oracle
+    (default: all)."""
     full = gpu_experts(shape)
-    xs = [activations(T_rank, shape, seed=seed + r).cuda() for r in range(G)]
-    x_all = torch.cat(xs)
-    wr = router_weight(shape).cuda()
+    xs_cpu = [activations(T_rank, shape, seed=seed + r) for r in range(G)]
+    x_all_cpu = torch.cat(xs_cpu)
+    x_all = x_all_cpu.cuda()
+    wr_cpu = router_weight(shape)
+    wr = wr_cpu.cuda()
+    g_h = intermediate_scales(shape)
+    sample = np.arange(G * T_rank) if sample is None else np.asarray(sample)
     acc_full, dbg = moe.forward_partial(full, x_all, wr, debug=True)
     out_full = moe.forward(full, x_all, wr)
     idx = dbg["idx"].cpu().numpy()
+    # the oracle: routing of all gathered tokens, every sampled pair's expert evaluated once
+    xn = x_all_cpu.float().numpy()
+    r_or = oracle.route(xn.astype(np.float64), wr_cpu.numpy().astype(np.float64), cfg_ns(shape), None)
+    xc, xsc, gx = oracle.quantize(xn)
+    same = (idx[sample] == r_or.idx[sample]).all(axis=1)
+    assert same.mean() > 0.9
+    checked = sample[same]
+    rows = {}
+    for i, t in enumerate(checked):
+        for j in range(shape.topk):
+            rows.setdefault(int(r_or.idx[t, j]), []).append((i, int(t), j))
+    xhat = oracle.dequantize(xc[checked], xsc[checked], gx)
+    ys = oracle_expert_pass(shape, {e: (xhat[[i for i, _, _ in v]], float(g_h[e]), None, None)
+                                    for e, v in rows.items()})
     accs = []
     for r in range(G):
         e0, n = expert_range(shape.E, r, G)
@@ -57,6 +80,13 @@ def run_emulated(shape, G, T_rank, seed=50):
         a = acc_r.cpu().numpy()
         assert np.all(a[none_local] == 0.0), f"rank {r}: non-zero rows for tokens without a local expert"
         assert not np.any(np.all(a[~none_local] == 0.0, axis=1)), f"rank {r}: a token's local experts added nothing"
+        # the rank's sums against the oracle's sum over the rank's experts
+        ref = np.zeros((len(checked), shape.H))
+        for e, v in rows.items():
+            if e0 <= e < e0 + n:
+                for m, (i, t, j) in enumerate(v):
+                    ref[i] += r_or.w[t, j] * ys[e][0][m]
+        check_output(a[checked], ref)
         accs.append(acc_r)
         ex.close()
     total = accs[0].clone()
@@ -86,7 +116,7 @@ def test_tiny_emulated_ranks(G, T_rank):
 
 def test_beam_decode_eight_ranks():
     """Beam decode on 8 emulated ranks: 16 tokens each, 128 gathered tokens."""
-    run_emulated(BEAM, 8, 16)
+    run_emulated(BEAM, 8, 16, sample=[0, 21, 47, 70, 101, 127])
 
 
 def test_local_handle_rejects_foreign_experts_and_bad_ranges():
