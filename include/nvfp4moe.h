@@ -299,6 +299,19 @@ typedef struct {
   uint16_t* x_norm;    /* [T][H] BF16 layer input computed by nvfp4moe_forward_residual */
   uint8_t* xq8_codes;  /* [T][H] E4M3 layer input of nvfp4moe_forward_fp8 */
   float* xq8_scales;   /* [T] its per-token scales */
+  /* Failure detection (nvfp4moe_forward, nvfp4moe_forward_residual, nvfp4moe_forward_partial;
+   * the other calls ignore these two fields).  Every wait of the call's kernels on another
+   * CTA or on the tensor cores is bounded: when one runs out, the kernel raises
+   * NVFP4MOE_ERR_TIMEOUT in the status word and returns, and the later kernels of the call
+   * (the grouped GEMMs) find the timeout in the status word and do no work, so the call ends
+   * with its outputs unspecified but finite work, no access outside its buffers, and the
+   * device context usable. */
+  uint32_t wait_limit_us;      /* limit of each bounded wait in microseconds; 0: 1.5 s */
+  int32_t inject_skip_arrive;  /* test hook, 0 in normal use: c > 0 makes CTA c - 1 of the fused
+                                  front-end kernel (T <= 64) skip its arrival at the first grid
+                                  barrier, so every CTA's wait there runs out (a timeout that
+                                  needs no fault); NVFP4MOE_ERR_ARG when the call does not take
+                                  the fused front end, or c < 0 */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);

@@ -580,6 +580,10 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   ForwardWs f = carve_forward(ws, c, T);
   if (acc_out != nullptr) f.acc = acc_out;
   if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  // the bounded waits' limit and the front-end test hook (nvfp4moe_debug)
+  const uint64_t wait_ns = dbg != nullptr ? (uint64_t)dbg->wait_limit_us * 1000ull : 0ull;
+  const int32_t skip_arrive = dbg != nullptr ? dbg->inject_skip_arrive : 0;
+  if (skip_arrive < 0 || (skip_arrive > 0 && !front_supported(T, c.E, c.H))) return NVFP4MOE_ERR_ARG;
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -631,6 +635,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     fa.acc = f.acc;
     fa.status = &f.hdr->status;
     fa.barrier = &f.hdr->barrier;
+    fa.wait_ns = wait_ns;
+    fa.skip_arrive = skip_arrive;
     ev.mark(NVFP4MOE_STAGE_AMAX, 0);
     ev.mark(NVFP4MOE_STAGE_AMAX, 1);
     ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
@@ -661,6 +667,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     r.logits_out = dbg != nullptr ? dbg->logits : nullptr;
     r.amax_partials = f.partials;
     r.status = &f.hdr->status;
+    r.wait_ns = wait_ns;
     set_router_tc(r, f.tc, f.a_codes);
     const int n_partials = router_amax_partials(T, c.E, c.H);
     ev.mark(NVFP4MOE_STAGE_AMAX, 0);
@@ -742,6 +749,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.g_up = x->g_up;
   g.g_h = x->g_h;
   g.I = c.I;
+  g.wait_ns = wait_ns;
   g.acc = f.acc;
   g.row_pair = f.row_pair;
   g.wts = f.wts;

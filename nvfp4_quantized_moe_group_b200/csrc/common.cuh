@@ -119,8 +119,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// A bounded wait gives up after this long (a correct kernel never waits this long).
+// A bounded wait gives up after this long (a correct kernel never waits this long), unless
+// the call sets another limit (nvfp4moe_debug.wait_limit_us; kernels receive it as wait_ns,
+// 0 meaning this default).
 constexpr uint64_t kWaitLimitNs = 1500ull * 1000ull * 1000ull;
+
+__host__ __device__ __forceinline__ uint64_t wait_limit(uint64_t wait_ns) {
+  return wait_ns != 0 ? wait_ns : kWaitLimitNs;
+}
 
 // --------------------------------------------------------------- mbarriers ----
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -158,13 +164,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and leaves the
-// caller to record a timeout) if it does not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// caller to record a timeout) if it does not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++n & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((++n & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
   }
   return true;
 }

@@ -38,21 +38,23 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 // launch starts; every barrier adds 0x80000000 in total (CTA 0 adds 0x80000000 - (nb - 1),
 // every other CTA 1), so the top bit takes the value `top` (0x80000000 after the first
 // barrier, 0 after the second) exactly when the last CTA arrives, and the low bits are 0
-// again.  The arrival is a release reduction (no round trip); the wait is bounded: on
-// timeout kStatusTimeout is raised and false returned (the caller stops).
-__device__ bool grid_barrier(uint32_t* bar, uint32_t top, uint32_t* status) {
+// again.  The arrival is a release reduction (no round trip); the wait is bounded by limit_ns:
+// on timeout kStatusTimeout is raised and false returned (the caller stops).  With
+// arrive == false the CTA only waits (a test hook: the other CTAs' waits then run out too).
+__device__ bool grid_barrier(uint32_t* bar, uint32_t top, uint32_t* status, uint64_t limit_ns, bool arrive = true) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t nb = gridDim.x;
     const uint32_t add = blockIdx.x == 0 ? 0x80000000u - (nb - 1u) : 1u;
-    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(bar), "r"(add)
-                 : "memory");
+    if (arrive)
+      asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(bar), "r"(add)
+                   : "memory");
     int ok = 1;
     const uint64_t t0 = globaltimer_ns();
     uint32_t n = 0;
     while ((ld_acquire_u32(bar) & 0x80000000u) != top) {
-      if ((++n & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      if ((++n & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) {
         raise_status(status, kStatusTimeout);
         ok = 0;
         break;
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(FrontArgs a) {
       }
     }
   }
-  if (!grid_barrier(a.barrier, 0x80000000u, a.status)) return;
+  const uint64_t wait_ns = wait_limit(a.wait_ns);
+  if (!grid_barrier(a.barrier, 0x80000000u, a.status, wait_ns, (int)blockIdx.x + 1 != a.skip_arrive)) return;
 
   // ------------------------------------------------------------ phase 2: top-k ---------
   for (int t = blockIdx.x; t < T; t += nb) {
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(FrontArgs a) {
     route_topk_block(s_sc, E, a.n_groups, a.topk_groups, topk, a.routed_scale, a.idx + (int64_t)t * topk,
                      a.wts + (int64_t)t * topk, a.status);
   }
-  if (!grid_barrier(a.barrier, 0u, a.status)) return;
+  if (!grid_barrier(a.barrier, 0u, a.status, wait_ns)) return;
 
   // ------------------------------------------- phase 3: grouping + quantise-scatter --
   // Every CTA rebuilds the grouping from idx (at most 512 pairs) in shared memory; CTA 0

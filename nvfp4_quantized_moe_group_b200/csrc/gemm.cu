@@ -254,13 +254,16 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   pdl_wait();
   pdl_trigger();
 
+  const uint64_t wait_ns = wait_limit(p.wait_ns);
   const uint32_t tmem = s.tmem_base;
   const int ntn = p.n_total / kN;           // 256-wide items per expert
   const int ntn128 = p.n_total / 128;       // 128-row weight tiles per expert
   // p.mtile_prefix may start at a later expert (a handle with one rank's share of the experts):
-  // its tiles are numbered from the first entry on
-  const int tile_base = __ldg(p.mtile_prefix);
-  const int total = (__ldg(p.mtile_prefix + p.E) - tile_base) * ntn;
+  // its tiles are numbered from the first entry on.  When an earlier kernel of the call has
+  // timed out, the grouping tables may be incomplete: no work items then.
+  const bool upstream_timeout = (*reinterpret_cast<const volatile uint32_t*>(p.status) & kStatusTimeout) != 0;
+  const int tile_base = upstream_timeout ? 0 : __ldg(p.mtile_prefix);
+  const int total = upstream_timeout ? 0 : (__ldg(p.mtile_prefix + p.E) - tile_base) * ntn;
   const int kb_count = kFp8 ? (p.K + 127) / 128 : (p.K + kBlockK - 1) / kBlockK;   // 128-byte K blocks
   const int k64 = p.K / 64;  // scale-column tiles of A and B
 
@@ -276,7 +279,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         // items are handed out dynamically: the first is the CTA's own index, the next ones
         // come from a counter shared by the grid, so CTAs that run faster take more items
         const int slot = it & (kWorkRing - 1);
-        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_empty[slot], ((uint32_t)(it / kWorkRing) & 1u) ^ 1u)) {
+        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_empty[slot], ((uint32_t)(it / kWorkRing) & 1u) ^ 1u, wait_ns)) {
           set_abort(&s.abort_flag, p.status);
           break;
         }
@@ -294,7 +297,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         const uint8_t* sfa = p.sfa + (int64_t)wk.mtile * k64 * kAtomBytes;
         const uint8_t* sfb = p.sfb + ((int64_t)wk.e * ntn128 + t0) * k64 * kAtomBytes;
         for (int kb = 0; kb < kb_count; ++kb) {
-          if (aborted(&s.abort_flag) || !mbar_wait(&s.empty[stage], phase ^ 1u)) {
+          if (aborted(&s.abort_flag) || !mbar_wait(&s.empty[stage], phase ^ 1u, wait_ns)) {
             set_abort(&s.abort_flag, p.status);
             ok = false;
             break;
@@ -321,7 +324,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       // wait for every copy this thread started before the CTA can exit
       for (int st = 0; st < kStages; ++st)
         if ((issued >> st) & 1u)
-          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u)) set_abort(&s.abort_flag, p.status);
+          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u, wait_ns)) set_abort(&s.abort_flag, p.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer ----
@@ -332,7 +335,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int slot = it & (kWorkRing - 1);
-        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u)) {
+        if (aborted(&s.abort_flag) || !mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u, wait_ns)) {
           set_abort(&s.abort_flag, p.status);
           break;
         }
@@ -340,14 +343,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         mbar_arrive(&s.work_empty[slot]);
         if (w < 0) break;
         const uint32_t acc_par = (uint32_t)it & 1u;
-        if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u)) {
+        if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u, wait_ns)) {
           set_abort(&s.abort_flag, p.status);
           break;
         }
         tc_fence_after();
         const uint32_t acc = tmem;
         for (int kb = 0; kb < kb_count; ++kb) {
-          if (aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase)) {
+          if (aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase, wait_ns)) {
             set_abort(&s.abort_flag, p.status);
             ok = false;
             break;
@@ -389,7 +392,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       }
       // every tensor-core operation of this thread is done before the memory is freed
       tc_commit(&s.drain);
-      if (!mbar_wait(&s.drain, 0)) set_abort(&s.abort_flag, p.status);
+      if (!mbar_wait(&s.drain, 0, wait_ns)) set_abort(&s.abort_flag, p.status);
     }
   } else {
     // ------------------------------------------------------------ epilogue ----
@@ -398,7 +401,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     const int row_l = q * 32 + lane;
     for (int it = 0;; ++it) {
       const int slot = it & (kWorkRing - 1);
-      const bool got_work = !aborted(&s.abort_flag) && mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u);
+      const bool got_work = !aborted(&s.abort_flag) && mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u, wait_ns);
       if (__any_sync(0xffffffffu, !got_work)) {
         set_abort(&s.abort_flag, p.status);
         break;
@@ -432,7 +435,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           }
         }
       }
-      const bool got = !aborted(&s.abort_flag) && mbar_wait(&s.acc_full, acc_par);
+      const bool got = !aborted(&s.abort_flag) && mbar_wait(&s.acc_full, acc_par, wait_ns);
       if (__any_sync(0xffffffffu, !got)) {
         set_abort(&s.abort_flag, p.status);
         break;

@@ -21,7 +21,9 @@ struct GemmArgs {
   int E;                       // experts of this launch (weights, scales, per-expert scalars indexed 0..E-1)
   int K;                       // reduction length
   int n_total;                 // B rows per expert (2I for gate/up, H for down)
-  uint32_t* status;
+  uint32_t* status;            // the call's status word; a timeout already raised in it (by an
+                               // earlier kernel of the call) makes the GEMM do no work
+  uint64_t wait_ns;            // limit of each bounded wait (0: kWaitLimitNs)
   int* work_counter;           // zero at launch: items handed out beyond the first gridDim.x
   // gate/up epilogue
   uint8_t* hq_codes;           // [rows_cap][I/2]

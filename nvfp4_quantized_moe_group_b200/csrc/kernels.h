@@ -54,6 +54,7 @@ struct RouterArgs {
   uint32_t* amax_partials;  // optional: per-CTA max |x| (BF16 magnitude bits) for the global scale
   float* logits_out;        // optional [T][E]: the FP32 logits (bias included) the top-k used
   uint32_t* status;         // kStatusNonFinite is raised here for a NaN logit (may be nullptr)
+  uint64_t wait_ns;         // limit of each bounded wait of the tensor-core logits (0: kWaitLimitNs)
   // integer tensor-core logits (T >= kRouterTcMinT, when given; route_tc.cu)
   uint8_t* x_digits;        // [4][T][H] int8 digit planes of the token rows
   uint8_t* w_digits;        // [4][E][H] int8 digit planes of the expert rows
@@ -109,6 +110,9 @@ struct FrontArgs {
   float* acc;               // [T][H] FP32, zeroed
   uint32_t* status;
   uint32_t* barrier;        // zero at launch
+  uint64_t wait_ns;         // limit of each grid-barrier wait (0: kWaitLimitNs)
+  int skip_arrive;          // test hook: CTA skip_arrive - 1 does not arrive at the first grid
+                            // barrier (0: every CTA arrives)
 };
 
 struct FinalizeArgs {

@@ -227,6 +227,7 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  const uint64_t wait_ns = wait_limit(a.wait_ns);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
@@ -235,7 +236,7 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
       const uint64_t pol = policy_evict_last();
       uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (tc_aborted(&s.abort_flag) || !mbar_wait(&s.empty[stage], phase ^ 1u)) {
+        if (tc_aborted(&s.abort_flag) || !mbar_wait(&s.empty[stage], phase ^ 1u, wait_ns)) {
           tc_set_abort(&s.abort_flag, a.status);
           break;
         }
@@ -251,7 +252,7 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
       }
       for (int st = 0; st < kTcStages; ++st)
         if ((issued >> st) & 1u)
-          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u)) tc_set_abort(&s.abort_flag, a.status);
+          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u, wait_ns)) tc_set_abort(&s.abort_flag, a.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer ----
@@ -261,7 +262,7 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
       uint32_t stage = 0, phase = 0;
       uint32_t started = 0;   // bit c: class c has its first product
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (tc_aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase)) {
+        if (tc_aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase, wait_ns)) {
           tc_set_abort(&s.abort_flag, a.status);
           break;
         }
@@ -289,7 +290,7 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
     // ------------------------------------------------------------ epilogue ----
     const int q = warp & 3;                       // tensor-memory lane quarter of this warp
     const int64_t t = t0 + q * 32 + lane;
-    const bool got = mbar_wait(&s.acc_full, 0);
+    const bool got = mbar_wait(&s.acc_full, 0, wait_ns);
     if (__any_sync(0xffffffffu, !got)) {
       tc_set_abort(&s.abort_flag, a.status);
     } else if (!tc_aborted(&s.abort_flag)) {
