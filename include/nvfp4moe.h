@@ -299,6 +299,8 @@ typedef struct {
   uint16_t* x_norm;    /* [T][H] BF16 layer input computed by nvfp4moe_forward_residual */
   uint8_t* xq8_codes;  /* [T][H] E4M3 layer input of nvfp4moe_forward_fp8 */
   float* xq8_scales;   /* [T] its per-token scales */
+  float* acc;          /* [T][H] FP32 sums of the weighted expert rows, the values the BF16 output
+                          rounds (to nearest, ties to even); nvfp4moe_forward and _residual */
   /* Failure detection (nvfp4moe_forward, nvfp4moe_forward_residual, nvfp4moe_forward_partial;
    * the other calls ignore these two fields).  Every wait of the call's kernels on another
    * CTA or on the tensor cores is bounded: when one runs out, the kernel raises

@@ -53,7 +53,7 @@ STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "f
 class Debug(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
                 + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p), ("xq8_codes", ctypes.c_void_p),
-                   ("xq8_scales", ctypes.c_void_p), ("wait_limit_us", ctypes.c_uint32),
+                   ("xq8_scales", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("wait_limit_us", ctypes.c_uint32),
                    ("inject_skip_arrive", ctypes.c_int32)])
 
 
@@ -419,6 +419,7 @@ def _debug_tensors(cfg: Cfg, T: int, H: int, dev, x_norm: bool = False) -> dict:
         "hq_codes": torch.empty((T * k, I // 2), dtype=torch.uint8, device=dev),
         "hq_scales": torch.empty((T * k, I // 16), dtype=torch.uint8, device=dev),
         "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
+        "acc": torch.empty((T, H), dtype=torch.float32, device=dev),
     }
     if x_norm:
         tensors["x_norm"] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)

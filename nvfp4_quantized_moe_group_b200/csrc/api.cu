@@ -797,6 +797,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     if (dbg->hq_codes && dbg->hq_scales)
       ok &= launch_export_hq(f.hq_codes, f.hq_sf, f.perm, f.idx, f.offsets, f.mtile_prefix, pairs, c.I,
                              dbg->hq_codes, dbg->hq_scales, s) == cudaSuccess;
+    if (dbg->acc && dbg->acc != f.acc)
+      ok &= cudaMemcpyAsync(dbg->acc, f.acc, T * c.H * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
     if (!ok) return NVFP4MOE_ERR_CUDA;
   }
   return NVFP4MOE_OK;
