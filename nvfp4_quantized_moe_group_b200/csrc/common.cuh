@@ -322,11 +322,6 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
 
 // Launches `kernel` with programmatic stream serialization: it may start while the previous
 // kernel of `stream` runs (it must call pdl_wait() before reading that kernel's results).

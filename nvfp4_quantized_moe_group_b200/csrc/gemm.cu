@@ -19,9 +19,11 @@
 //   gate/up:  each 128-column half holds 64 gate and 64 up columns of the same features:
 //             h = silu(g_x g_gate acc_gate) * (g_x g_up acc_up) in FP32, requantised to
 //             NVFP4 with the expert's static scale g_h (the down GEMM's A operand);
-//   down:     acc_out[token] += w * g_h * g_down * acc by FP32 vector reductions, each adding
-//             whole row pieces (staged through shared memory, or straight from the 16x256b
-//             register layout when segments hold few rows).
+//   down:     acc_out[token] += w * g_h * g_down * acc, FP32 additions into the token's row:
+//             with full segments each lane stages its row's 32-column piece in shared memory
+//             and adds it with one bulk reduction (cp.reduce.async.bulk .add.f32, 128 bytes);
+//             when segments hold few rows, vector reductions straight from the 16x256b register
+//             layout.
 // Every wait is bounded; a wait that runs out sets the timeout bit of the status word and
 // the CTA winds down (waits for its own copies and tensor-core work, frees tensor memory).
 //
@@ -55,8 +57,7 @@ constexpr int kNT = kN / 128;                       // 128-row weight tiles per 
 // accumulator before any arithmetic (gate/up) and reduce straight from the 16x256b register
 // layout (down), and the down GEMM keeps 4 stages.  With full segments the gate/up epilogue
 // frees the accumulator after its first 32-feature chunk, and the down GEMM stages 32-column
-// pieces through shared memory (whole 128-byte row pieces per reduction, 3 stages): both
-// measured faster there.
+// row pieces in shared memory for bulk reductions (3 stages): both measured faster there.
 //
 // kFp8: the FP8 W8A8 variant (E4M3 x E4M3 with FP32 accumulation, kind::f8f6f4): a 128-byte
 // K block holds 128 values instead of 256, there are no block scales (per-row activation and
@@ -81,7 +82,10 @@ struct __align__(1024) Smem {
   uint8_t b[C::kStages][kNT * kTileBytes];
   uint8_t sfa[C::kStages][C::kSfaBytes];
   uint8_t sfb[C::kStages][C::kSfbBytes];
-  float stage_out[C::kStaging ? kEpiWarps : 1][32][33];  // down, full segments: per epilogue warp
+  // down, full segments: per epilogue warp, 32 staged row pieces of 32 FP32 values, 144 bytes
+  // apart (16-byte aligned for the bulk reductions; the float4 stores of 8 consecutive lanes
+  // fall in 8 different bank groups)
+  alignas(16) float stage_rows[C::kStaging ? kEpiWarps : 1][32 * 36];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
   uint64_t acc_full;
@@ -134,6 +138,22 @@ __host__ __device__ constexpr uint32_t idesc_f8(uint32_t n) {
 __device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
 }
+
+// Orders this thread's earlier shared-memory writes before its later bulk (async-proxy) reads.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// gdst[i] += ssrc[i] for bytes / 4 FP32 values (both 16-byte aligned, bytes a multiple of 16),
+// performed by the bulk-copy unit; completion tracked in this thread's bulk group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const float* ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk operations have read their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until they have completed (their global writes done).
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct Work {
   int e;          // expert
@@ -552,37 +572,42 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + half * (kN / 2) + c * 32, R[c]);
         tmem_ld_wait();
         release();
-        // staged through shared memory: each reduction instruction adds 4 rows x 128 bytes
+        // each lane's row piece (32 columns, 128 bytes) staged in shared memory and added to the
+        // token's accumulator row by one bulk reduction (async proxy)
         const float scale = c0s;
-        float (*st)[33] = s.stage_out[warp - 2];
-        const int sub = lane >> 3;        // which of the 4 rows this lane writes per pass
-        const int col = (lane & 7) * 4;   // its 4 columns inside the 32-column chunk
+        float* mine = s.stage_rows[warp - 2] + lane * 36;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int c0 = half * (kN / 2) + c * 32;
+          if (c > 0) bulk_wait_read0();
+          if constexpr (kFp8) {
+            const float* wsc = p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + c0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) st[lane][j] = __fmul_rn(__uint_as_float(R[c][j]), scale);
-          __syncwarp();
-#pragma unroll
-          for (int pass = 0; pass < 8; ++pass) {
-            const int r = pass * 4 + sub;
-            const int tok = __shfl_sync(0xffffffffu, token, r);
-            if (tok >= 0) {
-              float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + c0 + col;
-              if constexpr (kFp8) {
-                const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + (int64_t)wk.e * p.n_total +
-                                                                        wk.nt * kN + c0 + col));
-                red_add_v4(dst, __fmul_rn(st[r][col], w4.x), __fmul_rn(st[r][col + 1], w4.y),
-                           __fmul_rn(st[r][col + 2], w4.z), __fmul_rn(st[r][col + 3], w4.w));
-              } else {
-                red_add_v4(dst, st[r][col], st[r][col + 1], st[r][col + 2], st[r][col + 3]);
-              }
+            for (int i = 0; i < 8; ++i) {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(wsc) + i);
+              *reinterpret_cast<float4*>(mine + 4 * i) =
+                  make_float4(__fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i]), scale), w4.x),
+                              __fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i + 1]), scale), w4.y),
+                              __fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i + 2]), scale), w4.z),
+                              __fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i + 3]), scale), w4.w));
             }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4*>(mine + 4 * i) =
+                  make_float4(__fmul_rn(__uint_as_float(R[c][4 * i]), scale), __fmul_rn(__uint_as_float(R[c][4 * i + 1]), scale),
+                              __fmul_rn(__uint_as_float(R[c][4 * i + 2]), scale), __fmul_rn(__uint_as_float(R[c][4 * i + 3]), scale));
           }
-          __syncwarp();
+          if (token >= 0) {
+            fence_proxy_async_smem();
+            bulk_reduce_add_f32(p.acc + (int64_t)token * p.H + wk.nt * kN + c0, mine, 128u);
+            bulk_commit();
+          }
         }
+        bulk_wait_read0();
       }
     }
+    bulk_wait_all0();
   }
 
   __syncthreads();

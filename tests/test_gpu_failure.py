@@ -33,9 +33,13 @@ def _cuda():
 
 def _within_one_bf16_unit(a: torch.Tensor, b: torch.Tensor) -> bool:
     """The 8 weighted expert rows of a token are added with FP32 atomics in no fixed order, so
-    two clean calls agree to one BF16 unit in the last place."""
+    two clean calls agree to one BF16 unit in the last place, except where the rows cancel:
+    there the FP32 sums differ by a few units of 2^-24 of the rows' own magnitude, which can
+    exceed a BF16 unit of the small result (bounded here by 2^-16 of the token row's largest
+    output)."""
     a, b = a.float().cpu().numpy(), b.float().cpu().numpy()
-    return bool(np.all(np.abs(a - b) <= 2 * bf16_half_ulp(b) + 1e-30))
+    row = np.abs(b).max(axis=1, keepdims=True)
+    return bool(np.all(np.abs(a - b) <= 2 * bf16_half_ulp(b) + 2.0 ** -16 * row + 1e-30))
 
 
 @pytest.mark.parametrize("shape,cta", [(TINY, 1), (BEAM, 1), (BEAM, 2)])
