@@ -344,10 +344,69 @@ NVFP4MOE_API int nvfp4moe_forward_partial(const nvfp4moe_experts* experts, const
                                           const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
 NVFP4MOE_API int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream);
 
+/* ------------------------------- expert parallelism, all-to-all exchange of quantised rows ----
+ * The exchange of the experts' placement across devices ("Reflection releases Beam ...",
+ * section "Tool calling and multi-node setups": experts on the devices, a device count that
+ * divides the 256 experts) in which each token's pairs travel to the experts, for batches where
+ * gathering every rank's tokens costs more than sending the pairs.  Rank d of G (G divides E)
+ * holds experts d E/G .. (d+1) E/G - 1 (nvfp4moe_experts_create_local) and the whole router;
+ * every rank passes the same T.  One step on rank d:
+ *   1. nvfp4moe_amax(x_d) -> amax_d; the ranks' values are combined with a maximum (an
+ *      all-reduce over int32, the values being below 2^15).
+ *   2. nvfp4moe_ep_dispatch(x_d, amax): routes the rank's tokens, groups their T*topk pairs by
+ *      expert (stable: expert, then token, then slot), quantises the tokens with the global
+ *      scale g = A / 2688 of the combined amax A (so every code and scale equals the
+ *      single-GPU layer's on the concatenated batch), and writes the pairs in that order:
+ *      send_codes [P][H/2], send_scales [P][H/16] (linear), send_expert [P] (the expert's index
+ *      on its rank), send_w [P] (routing weight), send_pos [T*topk] (position of pair t*topk+j
+ *      in the send order) and rank_counts [G] (pairs for each rank, in rank order), P = T*topk.
+ *   3. the caller's all-to-all sends rank_counts[e] consecutive rows (and their expert and
+ *      weight entries) to rank e.
+ *   4. nvfp4moe_ep_experts(local handle, received rows) -> out_rows [n][H] FP32: row i is
+ *      w_i * (the expert's SwiGLU MLP of the row), through the layer's grouped GEMMs.
+ *   5. the caller's all-to-all returns those rows (the reverse split).
+ *   6. nvfp4moe_ep_combine(returned rows, send_pos) -> out [T][H] BF16: for each token the
+ *      FP32 sum of its topk rows in slot order, rounded to nearest even.
+ * The result equals nvfp4moe_forward on the concatenated batch up to the order of the FP32
+ * additions of a token's rows (fixed here, atomic there).
+ *
+ * nvfp4moe_amax: amax_bits[0] = max over the rows x cols BF16 values of (bits & 0x7FFF) (the
+ *   magnitude's bit pattern: 0x7F80 and above mean Inf or NaN; 0 for no rows).  cols % 8 == 0;
+ *   workspace nvfp4moe_quantize_workspace_bytes(rows, cols).  amax_bits: device, 4-byte aligned.
+ * nvfp4moe_ep_dispatch: cfg of the whole layer; n_ranks divides cfg->E; amax_bits (device) the
+ *   combined amax; send buffers device, send_codes 16-byte and send_scales 4-byte aligned;
+ *   rank_counts device [n_ranks].  A non-finite amax raises NVFP4MOE_ERR_NONFINITE in the
+ *   status word and leaves the codes unwritten.
+ * nvfp4moe_ep_experts: the rank's handle; codes [n][H/2] (16-byte aligned), scales [n][H/16]
+ *   (4-byte aligned), expert [n] (0 <= expert < the handle's count), w [n] (device), amax_bits
+ *   as for dispatch; out_rows [n][H] FP32 (16-byte aligned, written in full).  n from 0 to
+ *   2^23; the workspace of nvfp4moe_ep_experts_workspace_bytes(cfg, handle's count, n).  The
+ *   expert indices arrive from other ranks and are checked on the device: one out of range is
+ *   replaced by 0 (so every access stays inside the buffers) and the status word reports
+ *   NVFP4MOE_ERR_ARG.
+ * nvfp4moe_ep_combine: rows [T*topk][H] FP32 in send order (16-byte aligned), send_pos from
+ *   dispatch, out_bf16 [T][H] (16-byte aligned); topk <= 8, H % 64 == 0.
+ * All arguments on the device are owned by the caller; all calls are asynchronous on `stream`. */
+NVFP4MOE_API int nvfp4moe_amax(const void* x_bf16, int64_t rows, int64_t cols, uint32_t* amax_bits, void* ws,
+                               size_t ws_bytes, void* stream);
+NVFP4MOE_API size_t nvfp4moe_ep_dispatch_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T);
+NVFP4MOE_API int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* hidden_bf16, int64_t T,
+                                      const float* w_router, const float* logit_bias, const uint32_t* amax_bits,
+                                      uint8_t* send_codes, uint8_t* send_scales, int32_t* send_expert, float* send_w,
+                                      int32_t* send_pos, int32_t* rank_counts, void* ws, size_t ws_bytes,
+                                      void* stream);
+NVFP4MOE_API size_t nvfp4moe_ep_experts_workspace_bytes(const nvfp4moe_cfg* cfg, int32_t e_count, int64_t n_rows_max);
+NVFP4MOE_API int nvfp4moe_ep_experts(const nvfp4moe_experts* experts, const uint8_t* codes, const uint8_t* scales,
+                                     const int32_t* expert, const float* w, int64_t n_rows,
+                                     const uint32_t* amax_bits, float* out_rows, void* ws, size_t ws_bytes,
+                                     void* stream);
+NVFP4MOE_API int nvfp4moe_ep_combine(const float* rows, const int32_t* send_pos, int64_t T, int32_t topk, int32_t H,
+                                     void* out_bf16, void* stream);
+
 /* ------------------------------------------------------------------ status ----
  * Waits for `stream`, then returns the device-side status of the last call that used
- * workspace `ws` (NVFP4MOE_OK, _ERR_NONFINITE or _ERR_TIMEOUT; _ERR_CUDA if the wait or
- * the read failed). */
+ * workspace `ws` (NVFP4MOE_OK, _ERR_NONFINITE, _ERR_TIMEOUT, or _ERR_ARG for an argument the
+ * device found out of range; _ERR_CUDA if the wait or the read failed). */
 NVFP4MOE_API int nvfp4moe_status_read(const void* ws, void* stream);
 NVFP4MOE_API const char* nvfp4moe_status_string(int status);
 

@@ -126,6 +126,13 @@ _SIGS = {
     "nvfp4moe_fp8_experts_destroy": (None, [_P]),
     "nvfp4moe_forward_fp8_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_forward_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_amax": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _SZ, _P]),
+    "nvfp4moe_ep_dispatch_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
+    "nvfp4moe_ep_dispatch": (ctypes.c_int, [ctypes.POINTER(Cfg), ctypes.c_int32, _P, _I64, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _SZ, _P]),
+    "nvfp4moe_ep_experts_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), ctypes.c_int32, _I64]),
+    "nvfp4moe_ep_experts": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
+    "nvfp4moe_ep_combine": (ctypes.c_int, [_P, _P, _I64, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "nvfp4moe_status_read": (ctypes.c_int, [_P, _P]),
     "nvfp4moe_last_device_status": (ctypes.c_int, [_P]),
     "nvfp4moe_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
@@ -627,4 +634,88 @@ def finalize(acc: torch.Tensor, out: torch.Tensor | None = None, stream=None) ->
     if out is None:
         out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
     _check(lib().nvfp4moe_finalize(_ptr(acc), acc.numel(), _ptr(out), _stream(stream)), "nvfp4moe_finalize")
+    return out
+
+
+# ------------------------------------------------- expert parallelism, all-to-all exchange ----
+
+def amax(x: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """max |x| of a BF16 tensor as its magnitude bit pattern (nvfp4moe_amax) -> int32 [1] on the
+    device (below 2^15, so a maximum over int32 combines the ranks' values)."""
+    rows = _rows(x, "x", min_rows=0)
+    cols = int(x.shape[1])
+    _require((x, "x", torch.bfloat16, None), (ws, "ws", torch.uint8, None))
+    out = torch.empty(1, dtype=torch.int32, device=x.device)
+    if ws is None:
+        ws = _workspace(quantize_workspace_bytes(rows, cols), x.device)
+    _check(lib().nvfp4moe_amax(_ptr(x), rows, cols, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "nvfp4moe_amax")
+    return out
+
+
+def ep_dispatch_workspace_bytes(cfg: Cfg, T: int) -> int:
+    return int(lib().nvfp4moe_ep_dispatch_workspace_bytes(ctypes.byref(cfg), T))
+
+
+def ep_dispatch(cfg: Cfg, n_ranks: int, x: torch.Tensor, w_router: torch.Tensor, bias, amax_bits: torch.Tensor,
+                ws=None, stream=None) -> dict:
+    """nvfp4moe_ep_dispatch: this rank's pairs in send order.  Returns a dict of device tensors:
+    codes [P, H/2] u8, scales [P, H/16] u8, expert [P] i32 (destination-local), w [P] f32,
+    pos [T*topk] i32 (send position of each pair), rank_counts [n_ranks] i32."""
+    specs = _layer_specs(cfg, x, w_router, bias)
+    T, H = x.shape
+    dev = x.device
+    _require(*specs, (amax_bits, "amax_bits", torch.int32, (1,)), (ws, "ws", torch.uint8, None))
+    P = T * cfg.topk
+    out = {"codes": torch.empty((P, H // 2), dtype=torch.uint8, device=dev),
+           "scales": torch.empty((P, H // 16), dtype=torch.uint8, device=dev),
+           "expert": torch.empty(P, dtype=torch.int32, device=dev),
+           "w": torch.empty(P, dtype=torch.float32, device=dev),
+           "pos": torch.empty(P, dtype=torch.int32, device=dev),
+           "rank_counts": torch.empty(int(n_ranks), dtype=torch.int32, device=dev)}
+    if ws is None:
+        ws = _workspace(ep_dispatch_workspace_bytes(cfg, T), dev)
+    st = lib().nvfp4moe_ep_dispatch(ctypes.byref(cfg), int(n_ranks), _ptr(x), T, _ptr(w_router), _ptr(bias),
+                                    _ptr(amax_bits), _ptr(out["codes"]), _ptr(out["scales"]), _ptr(out["expert"]),
+                                    _ptr(out["w"]), _ptr(out["pos"]), _ptr(out["rank_counts"]), _ptr(ws),
+                                    ws.numel(), _stream(stream))
+    _check(st, "nvfp4moe_ep_dispatch")
+    return out
+
+
+def ep_experts_workspace_bytes(cfg: Cfg, e_count: int, n_rows_max: int) -> int:
+    return int(lib().nvfp4moe_ep_experts_workspace_bytes(ctypes.byref(cfg), int(e_count), int(n_rows_max)))
+
+
+def ep_experts(experts: Experts, codes: torch.Tensor, scales: torch.Tensor, expert: torch.Tensor, w: torch.Tensor,
+               amax_bits: torch.Tensor, out: torch.Tensor | None = None, ws=None, stream=None) -> torch.Tensor:
+    """nvfp4moe_ep_experts: the handle's experts on received rows -> weighted FP32 rows [n, H]."""
+    cfg = experts.cfg
+    n = _rows(codes, "codes", min_rows=0)
+    H = cfg.H
+    _require((codes, "codes", torch.uint8, (n, H // 2)), (scales, "scales", torch.uint8, (n, H // 16)),
+             (expert, "expert", torch.int32, (n,)), (w, "w", torch.float32, (n,)),
+             (amax_bits, "amax_bits", torch.int32, (1,)), (out, "out", torch.float32, (n, H)),
+             (ws, "ws", torch.uint8, None))
+    dev = amax_bits.device
+    if out is None:
+        out = torch.empty((n, H), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(ep_experts_workspace_bytes(cfg, experts.e_count, max(n, 1)), dev)
+    st = lib().nvfp4moe_ep_experts(experts.handle, _ptr(codes), _ptr(scales), _ptr(expert), _ptr(w), n,
+                                   _ptr(amax_bits), _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "nvfp4moe_ep_experts")
+    return out
+
+
+def ep_combine(rows: torch.Tensor, pos: torch.Tensor, T: int, topk: int, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """nvfp4moe_ep_combine: out [T, H] BF16, each token's topk returned rows added in slot order."""
+    H = int(rows.shape[1])
+    _require((rows, "rows", torch.float32, (T * topk, H)), (pos, "pos", torch.int32, (T * topk,)),
+             (out, "out", torch.bfloat16, (T, H)))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=rows.device)
+    _check(lib().nvfp4moe_ep_combine(_ptr(rows), _ptr(pos), int(T), int(topk), H, _ptr(out), _stream(stream)),
+           "nvfp4moe_ep_combine")
     return out

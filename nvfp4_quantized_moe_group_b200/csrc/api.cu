@@ -267,6 +267,100 @@ ForwardFp8Ws carve_forward_fp8(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   return f;
 }
 
+// Expert parallelism, all-to-all exchange: the dispatching rank's scratch (routing of its own
+// tokens, their grouping by expert, the global scale, the tokens quantised token-major).
+struct EpDispatchWs {
+  WsHeader* hdr;
+  double* parts;
+  RouterTcWs tc;
+  int32_t* idx;
+  float* wts;
+  int32_t* chunk_counts;
+  int32_t* chunk_base;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile_prefix;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* row_pair;
+  float* g;
+  uint8_t* xq_codes;
+  uint8_t* xq_scales;
+  size_t bytes;
+};
+
+EpDispatchWs carve_ep_dispatch(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
+  Carver c(ws);
+  EpDispatchWs d;
+  const int64_t pairs = T * cfg.topk;
+  const int64_t n_chunks = (T + kPermChunkTokens - 1) / kPermChunkTokens;
+  d.hdr = c.take<WsHeader>(1);
+  d.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
+  d.tc = carve_router_tc(c, cfg, T, 0);
+  d.idx = c.take<int32_t>(pairs);
+  d.wts = c.take<float>(pairs);
+  d.chunk_counts = c.take<int32_t>(n_chunks * cfg.E);
+  d.chunk_base = c.take<int32_t>(n_chunks * cfg.E);
+  d.counts = c.take<int32_t>(cfg.E);
+  d.offsets = c.take<int32_t>(cfg.E + 1);
+  d.mtile_prefix = c.take<int32_t>(cfg.E + 1);
+  d.perm = c.take<int32_t>(pairs);
+  d.inv = c.take<int32_t>(pairs);
+  d.row_pair = c.take<int32_t>(rows_capacity(cfg, T));
+  d.g = c.take<float>(1);
+  d.xq_codes = c.take<uint8_t>(T * cfg.H / 2);
+  d.xq_scales = c.take<uint8_t>(T * cfg.H / 16);
+  d.bytes = c.off;
+  return d;
+}
+
+// The receiving rank's scratch: the grouping of the received rows by local expert (one slot
+// per row), the global scale, the rows in padded expert segments and the requantised h.
+struct EpExpertsWs {
+  WsHeader* hdr;
+  float* g_x;
+  int32_t* chunk_counts;
+  int32_t* chunk_base;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile_prefix;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* row_pair;
+  int32_t* expert;         // the received rows' expert indices, checked
+  uint8_t* a_codes;
+  uint8_t* a_sf;
+  uint8_t* hq_codes;
+  uint8_t* hq_sf;
+  int64_t rows_cap;
+  size_t bytes;
+};
+
+// cfg_local: the layer's cfg with E = the handle's expert count and topk = 1.
+EpExpertsWs carve_ep_experts(void* ws, const nvfp4moe_cfg& cfg_local, int64_t n) {
+  Carver c(ws);
+  EpExpertsWs f;
+  const int64_t n_chunks = (n + kPermChunkTokens - 1) / kPermChunkTokens;
+  f.rows_cap = rows_capacity(cfg_local, n);
+  f.hdr = c.take<WsHeader>(1);
+  f.g_x = c.take<float>(1);
+  f.chunk_counts = c.take<int32_t>(n_chunks * cfg_local.E);
+  f.chunk_base = c.take<int32_t>(n_chunks * cfg_local.E);
+  f.counts = c.take<int32_t>(cfg_local.E);
+  f.offsets = c.take<int32_t>(cfg_local.E + 1);
+  f.mtile_prefix = c.take<int32_t>(cfg_local.E + 1);
+  f.perm = c.take<int32_t>(n);
+  f.inv = c.take<int32_t>(n);
+  f.row_pair = c.take<int32_t>(f.rows_cap);
+  f.expert = c.take<int32_t>(n);
+  f.a_codes = c.take<uint8_t>(f.rows_cap * cfg_local.H / 2);
+  f.a_sf = c.take<uint8_t>(f.rows_cap * cfg_local.H / 16);
+  f.hq_codes = c.take<uint8_t>(f.rows_cap * cfg_local.I / 2);
+  f.hq_sf = c.take<uint8_t>(f.rows_cap * cfg_local.I / 16);
+  f.bytes = c.off;
+  return f;
+}
+
 __global__ void set_expert_scalars_kernel(float* g_gate, float* g_up, float* g_h, float* alpha, int e,
                                           float gg, float gu, float gh, float gd) {
   g_gate[e] = gg;
@@ -1110,6 +1204,7 @@ int nvfp4moe_status_read(const void* ws, void* stream) {
   uint32_t v = 0;
   if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   if (v & kStatusTimeout) return NVFP4MOE_ERR_TIMEOUT;
+  if (v & kStatusBadInput) return NVFP4MOE_ERR_ARG;
   if (v & kStatusNonFinite) return NVFP4MOE_ERR_NONFINITE;
   return NVFP4MOE_OK;
 }
@@ -1135,6 +1230,247 @@ const char* nvfp4moe_status_string(int status) {
     case NVFP4MOE_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
     default: return "unknown status";
   }
+}
+
+/* ------------------------------------------ expert parallelism, all-to-all exchange ---- */
+
+int nvfp4moe_amax(const void* x_bf16, int64_t rows, int64_t cols, uint32_t* amax_bits, void* ws, size_t ws_bytes,
+                  void* stream) {
+  g_launches = 0;
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || rows * cols >= ((int64_t)1 << 40)) return NVFP4MOE_ERR_SHAPE;
+  if (amax_bits == nullptr || ws == nullptr || !aligned(ws, kAlign) || !aligned(amax_bits, 4)) return NVFP4MOE_ERR_ARG;
+  if (rows > 0 && (x_bf16 == nullptr || !aligned(x_bf16, 16))) return NVFP4MOE_ERR_ARG;
+  const QuantWs q = carve_quant(ws);
+  if (ws_bytes < q.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rows == 0) return cudaMemsetAsync(amax_bits, 0, 4, s) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
+  const int blocks = amax_partial_blocks(rows * cols);
+  if (launch_amax_partial(x_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_amax_reduce(q.partials, blocks, amax_bits, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches = 2;
+  return NVFP4MOE_OK;
+}
+
+size_t nvfp4moe_ep_dispatch_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T) {
+  if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || T < 1) return 0;
+  return carve_ep_dispatch(nullptr, *cfg, T).bytes;
+}
+
+int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* hidden_bf16, int64_t T,
+                         const float* w_router, const float* logit_bias, const uint32_t* amax_bits,
+                         uint8_t* send_codes, uint8_t* send_scales, int32_t* send_expert, float* send_w,
+                         int32_t* send_pos, int32_t* rank_counts, void* ws, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  int st = nvfp4moe_cfg_check(cfg);
+  if (st != NVFP4MOE_OK) return st;
+  if (n_ranks < 1 || cfg->E % n_ranks != 0) return NVFP4MOE_ERR_ARG;
+  if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
+  if (hidden_bf16 == nullptr || w_router == nullptr || amax_bits == nullptr || send_codes == nullptr ||
+      send_scales == nullptr || send_expert == nullptr || send_w == nullptr || send_pos == nullptr ||
+      rank_counts == nullptr || ws == nullptr)
+    return NVFP4MOE_ERR_ARG;
+  if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(send_codes, 16) || !aligned(send_scales, 4) ||
+      !aligned(ws, kAlign))
+    return NVFP4MOE_ERR_ARG;
+  const nvfp4moe_cfg& c = *cfg;
+  const EpDispatchWs d = carve_ep_dispatch(ws, c, T);
+  if (ws_bytes < d.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (reset_status(d.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  // route this rank's tokens
+  RouterArgs r{};
+  r.x = static_cast<const uint16_t*>(hidden_bf16);
+  r.w = w_router;
+  r.bias = logit_bias;
+  r.parts = d.parts;
+  r.idx = d.idx;
+  r.wts = d.wts;
+  r.T = T;
+  r.H = c.H;
+  r.E = c.E;
+  r.n_groups = c.n_groups;
+  r.topk_groups = c.topk_groups;
+  r.topk = c.topk;
+  r.routed_scale = c.routed_scale;
+  r.status = &d.hdr->status;
+  set_router_tc(r, d.tc, nullptr);
+  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += router_launch_count(r);
+  // group its pairs by expert: the stable expert-major order is also destination-rank order
+  PermArgs pa{};
+  pa.idx = d.idx;
+  pa.T = T;
+  pa.topk = c.topk;
+  pa.E = c.E;
+  pa.n_chunks = (int)((T + kPermChunkTokens - 1) / kPermChunkTokens);
+  pa.chunk_counts = d.chunk_counts;
+  pa.chunk_base = d.chunk_base;
+  pa.counts = d.counts;
+  pa.offsets = d.offsets;
+  pa.mtile_prefix = d.mtile_prefix;
+  pa.perm = d.perm;
+  pa.inv = d.inv;
+  pa.row_pair = d.row_pair;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  // quantise the tokens with the global scale of all ranks' tokens (from their amax)
+  QuantizeArgs q{};
+  q.x = static_cast<const uint16_t*>(hidden_bf16);
+  q.rows = T;
+  q.rows_padded = T;
+  q.cols = c.H;
+  q.g_in = nullptr;
+  q.partials = amax_bits;
+  q.n_partials = 1;
+  q.codes = d.xq_codes;
+  q.scales = d.xq_scales;
+  q.swizzled = 0;
+  q.n_col_tiles = c.H / 64;
+  q.g_out = d.g;
+  q.status = &d.hdr->status;
+  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += quantize_launch_count(q);
+  // pack the pairs' rows in send order, with their metadata and the per-rank counts
+  EpPackArgs pk{};
+  pk.perm = d.perm;
+  pk.idx = d.idx;
+  pk.wts = d.wts;
+  pk.xq_codes = d.xq_codes;
+  pk.xq_scales = d.xq_scales;
+  pk.counts = d.counts;
+  pk.n_pairs = T * c.topk;
+  pk.topk = c.topk;
+  pk.H = c.H;
+  pk.E = c.E;
+  pk.experts_per_rank = c.E / n_ranks;
+  pk.send_codes = send_codes;
+  pk.send_scales = send_scales;
+  pk.send_expert = send_expert;
+  pk.send_w = send_w;
+  pk.send_pos = send_pos;
+  pk.rank_counts = rank_counts;
+  if (launch_ep_pack(pk, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  g_launches += 2;
+  return NVFP4MOE_OK;
+}
+
+size_t nvfp4moe_ep_experts_workspace_bytes(const nvfp4moe_cfg* cfg, int32_t e_count, int64_t n_rows_max) {
+  if (nvfp4moe_cfg_check(cfg) != NVFP4MOE_OK || e_count < 1 || e_count > cfg->E || n_rows_max < 1) return 0;
+  nvfp4moe_cfg cl = *cfg;
+  cl.E = e_count;
+  cl.topk = 1;
+  return carve_ep_experts(nullptr, cl, n_rows_max).bytes;
+}
+
+int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const uint8_t* scales,
+                        const int32_t* expert, const float* w, int64_t n_rows, const uint32_t* amax_bits,
+                        float* out_rows, void* ws, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (x == nullptr) return NVFP4MOE_ERR_ARG;
+  if (n_rows < 0 || n_rows > ((int64_t)1 << 23)) return NVFP4MOE_ERR_SHAPE;
+  if (amax_bits == nullptr || ws == nullptr || !aligned(ws, kAlign)) return NVFP4MOE_ERR_ARG;
+  if (n_rows > 0 && (codes == nullptr || scales == nullptr || expert == nullptr || w == nullptr ||
+                     out_rows == nullptr || !aligned(codes, 16) || !aligned(scales, 4) || !aligned(out_rows, 16)))
+    return NVFP4MOE_ERR_ARG;
+  nvfp4moe_cfg cl = x->cfg;
+  cl.E = x->e_count;
+  cl.topk = 1;
+  const EpExpertsWs f = carve_ep_experts(ws, cl, n_rows > 0 ? n_rows : 1);
+  if (ws_bytes < f.bytes) return NVFP4MOE_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (n_rows == 0) return NVFP4MOE_OK;
+  CUtensorMap tma_a, tma_a32, tma_h, tma_h32;
+  if (make_tma_2d(&tma_a, f.a_codes, cl.H / 2, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_a32, f.a_codes, cl.H / 2, f.rows_cap, 32) != 0 ||
+      make_tma_2d(&tma_h, f.hq_codes, cl.I / 2, f.rows_cap, kBlockM) != 0 ||
+      make_tma_2d(&tma_h32, f.hq_codes, cl.I / 2, f.rows_cap, 32) != 0)
+    return NVFP4MOE_ERR_CUDA;
+  // the expert indices come from other ranks: checked on the device (an index outside the
+  // handle's experts is replaced by 0 and raises NVFP4MOE_ERR_ARG in the status word)
+  if (launch_check_indices(expert, n_rows, cl.E, f.expert, &f.hdr->status, s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  // group the received rows by local expert (stable: source rank, then its order)
+  PermArgs pa{};
+  pa.idx = f.expert;
+  pa.T = n_rows;
+  pa.topk = 1;
+  pa.E = cl.E;
+  pa.n_chunks = (int)((n_rows + kPermChunkTokens - 1) / kPermChunkTokens);
+  pa.chunk_counts = f.chunk_counts;
+  pa.chunk_base = f.chunk_base;
+  pa.counts = f.counts;
+  pa.offsets = f.offsets;
+  pa.mtile_prefix = f.mtile_prefix;
+  pa.perm = f.perm;
+  pa.inv = f.inv;
+  pa.row_pair = f.row_pair;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_global_scale(amax_bits, 1, f.g_x, &f.hdr->status, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  RowsToSegmentsArgs ra{codes, scales, f.expert, f.inv, f.offsets, f.mtile_prefix, n_rows, cl.H, cl.H / 64,
+                        f.a_codes, f.a_sf, out_rows};
+  if (launch_rows_to_segments(ra, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  const int grid = num_sms();
+  const bool decode_cfg = n_rows < 32 * (int64_t)cl.E;
+  GemmArgs g{};
+  g.b_tiles = x->w13_codes;
+  g.sfa = f.a_sf;
+  g.sfb = x->w13_sf;
+  g.mtile_prefix = f.mtile_prefix;
+  g.counts = f.counts;
+  g.E = cl.E;
+  g.K = cl.H;
+  g.n_total = 2 * cl.I;
+  g.status = &f.hdr->status;
+  g.hq_codes = f.hq_codes;
+  g.hq_sf = f.hq_sf;
+  g.g_x = f.g_x;
+  g.g_gate = x->g_gate;
+  g.g_up = x->g_up;
+  g.g_h = x->g_h;
+  g.I = cl.I;
+  g.acc = out_rows;          // one received row per slot: the reduction writes it once
+  g.row_pair = f.row_pair;
+  g.wts = w;
+  g.alpha_down = x->alpha_down;
+  g.topk = 1;
+  g.H = cl.H;
+  g.work_counter = &f.hdr->work[0];
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  g.b_tiles = x->wd_codes;
+  g.sfa = f.hq_sf;
+  g.sfb = x->wd_sf;
+  g.K = cl.I;
+  g.n_total = cl.H;
+  g.work_counter = &f.hdr->work[1];
+  if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  ++g_launches;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_ep_combine(const float* rows, const int32_t* send_pos, int64_t T, int32_t topk, int32_t H, void* out_bf16,
+                        void* stream) {
+  g_launches = 0;
+  if (T < 0 || T > (1 << 20) || topk < 1 || topk > 8 || H < 64 || H % 64 != 0) return NVFP4MOE_ERR_SHAPE;
+  if (T == 0) return NVFP4MOE_OK;
+  if (rows == nullptr || send_pos == nullptr || out_bf16 == nullptr || !aligned(rows, 16) || !aligned(out_bf16, 16))
+    return NVFP4MOE_ERR_ARG;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  if (launch_ep_combine(rows, send_pos, T, topk, H, static_cast<uint16_t*>(out_bf16), static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
+  g_launches = 1;
+  return NVFP4MOE_OK;
 }
 
 int32_t nvfp4moe_last_launch_count(void) { return g_launches; }

@@ -17,6 +17,7 @@ namespace nvfp4moe {
 enum : uint32_t {
   kStatusNonFinite = 1u,
   kStatusTimeout = 2u,
+  kStatusBadInput = 4u,   // a device-side argument out of range (replaced by a valid one)
 };
 
 // Every workspace starts with this header.

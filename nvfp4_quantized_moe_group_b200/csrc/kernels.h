@@ -140,6 +140,11 @@ cudaError_t launch_amax_partial(const void* x, int64_t n_elems, uint32_t* partia
                                 cudaStream_t stream);
 // Dynamic scale (g_in == nullptr): a one-warp kernel reduces the amax partials first.
 cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream);
+// g = A / 2688 (1 for A = 0) from BF16 magnitude-bit partials; NaN and kStatusNonFinite for a
+// non-finite amax (the kernel the dynamic quantisation runs first).
+cudaError_t launch_global_scale(const uint32_t* partials, int n, float* g_out, uint32_t* status, cudaStream_t stream);
+// The maximum of n amax partials (BF16 magnitude bits) into *amax_bits.
+cudaError_t launch_amax_reduce(const uint32_t* partials, int n, uint32_t* amax_bits, cudaStream_t stream);
 int quantize_launch_count(const QuantizeArgs& a);
 
 // route.cu
@@ -162,6 +167,47 @@ int router_tc_amax_partials(int64_t T);
 cudaError_t launch_router_tc(RouterArgs a, cudaStream_t stream);
 
 
+
+// ep.cu: expert parallelism with an all-to-all exchange of quantised rows
+struct EpPackArgs {
+  const int32_t* perm;       // [n_pairs] pair ids in stable expert-major order
+  const int32_t* idx;        // [T][topk] experts (global indices)
+  const float* wts;          // [T][topk] routing weights
+  const uint8_t* xq_codes;   // [T][H/2] the tokens' codes (quantised with the global scale)
+  const uint8_t* xq_scales;  // [T][H/16] their block scales, linear
+  const int32_t* counts;     // [E] pairs per expert
+  int64_t n_pairs;           // T * topk
+  int topk, H, E, experts_per_rank;
+  uint8_t* send_codes;       // [n_pairs][H/2]
+  uint8_t* send_scales;      // [n_pairs][H/16]
+  int32_t* send_expert;      // [n_pairs] expert index local to the destination rank
+  float* send_w;             // [n_pairs]
+  int32_t* send_pos;         // [n_pairs] position of pair p in the send order
+  int32_t* rank_counts;      // [E / experts_per_rank] pairs sent to each rank
+};
+cudaError_t launch_ep_pack(const EpPackArgs& a, cudaStream_t stream);
+
+struct RowsToSegmentsArgs {
+  const uint8_t* codes;      // [n_rows][H/2]
+  const uint8_t* scales;     // [n_rows][H/16] linear
+  const int32_t* expert;     // [n_rows] local expert of each row
+  const int32_t* inv;        // [n_rows] position of row i in the grouping (topk = 1)
+  const int32_t* offsets;    // [E_local + 1]
+  const int32_t* mtile_prefix;  // [E_local + 1]
+  int64_t n_rows;
+  int H;
+  int64_t n_col_tiles;       // H / 64
+  uint8_t* seg_codes;        // [rows_cap][H/2]
+  uint8_t* seg_sf;           // swizzled
+  float* out_rows;           // [n_rows][H] FP32, zeroed
+};
+cudaError_t launch_rows_to_segments(const RowsToSegmentsArgs& a, cudaStream_t stream);
+// out[i] = idx[i] if 0 <= idx[i] < n, else 0 and kStatusBadInput raised (indices from another rank).
+cudaError_t launch_check_indices(const int32_t* idx, int64_t count, int n, int32_t* out, uint32_t* status,
+                                 cudaStream_t stream);
+// out[t] = bf16(sum_j rows[send_pos[t topk + j]]), slots in order.
+cudaError_t launch_ep_combine(const float* rows, const int32_t* send_pos, int64_t T, int topk, int H, uint16_t* out,
+                              cudaStream_t stream);
 
 // front.cu
 // True when the fused front end runs for T tokens on the current device (T <= kFrontMaxT and

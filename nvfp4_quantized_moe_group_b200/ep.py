@@ -17,6 +17,21 @@ equals the single-GPU layer up to the order of the FP32 additions.  Per GPU the 
 weights streamed at decode fall from the experts hit by its own tokens to its share of the
 experts hit by all tokens.  The two collectives are NCCL's (all_gather_into_tensor,
 reduce_scatter_tensor); every rank passes the same number of tokens.
+
+With ``exchange="all_to_all"`` (large batches) the pairs travel instead of the tokens:
+
+  1. nvfp4moe_amax of the rank's tokens, all-reduced with a maximum (the global scale of the
+     concatenated batch, so every rank quantises as the single-GPU layer would);
+  2. nvfp4moe_ep_dispatch: the rank routes and quantises its own tokens and lays out its
+     T * topk pairs' quantised rows (2,880 bytes each for Beam) in destination-rank order;
+  3. an all-to-all of the per-rank counts, then of the rows, their local expert and weight;
+  4. nvfp4moe_ep_experts on the received rows: weighted FP32 output rows;
+  5. an all-to-all returns the rows to their tokens' ranks;
+  6. nvfp4moe_ep_combine adds each token's topk rows in slot order and rounds to BF16.
+
+Per step and rank that moves T topk (H/2 + H/16 + 8) bytes out and T topk H 4 bytes back,
+against G T H 2 gathered and G T H 4 reduce-scattered bytes for the gather exchange, and each
+rank routes and quantises T tokens instead of G T.
 """
 from __future__ import annotations
 
@@ -45,9 +60,21 @@ class ExpertParallelLayer:
 
     def __init__(self, cfg: _lib.Cfg, group=None,
                  partial: Callable[[torch.Tensor, torch.Tensor, torch.Tensor | None], torch.Tensor] | None = None,
-                 finalize: Callable[[torch.Tensor], torch.Tensor] | None = None):
+                 finalize: Callable[[torch.Tensor], torch.Tensor] | None = None,
+                 exchange: str = "gather", a2a_ops: dict | None = None):
+        """``exchange``: "gather" (all-gather the tokens, reduce-scatter FP32 sums) or
+        "all_to_all" (send each pair's quantised row to its expert's rank and its weighted
+        output row back).  ``a2a_ops`` replaces the all-to-all path's library calls (keys
+        amax, dispatch, experts, combine; the signatures of the default methods below), to
+        exercise the exchange without a GPU."""
+        if exchange not in ("gather", "all_to_all"):
+            raise ValueError(f"unknown exchange {exchange!r}")
         self.cfg = cfg
         self.group = group
+        self.exchange = exchange
+        self._a2a = {"amax": self._amax_cuda, "dispatch": self._dispatch_cuda, "experts": self._experts_cuda,
+                     "combine": self._combine_cuda}
+        self._a2a.update(a2a_ops or {})
         initialized = dist.is_available() and dist.is_initialized()
         self.world = dist.get_world_size(group) if initialized else 1
         self.rank = dist.get_rank(group) if initialized else 0
@@ -89,8 +116,55 @@ class ExpertParallelLayer:
         dist.reduce_scatter_tensor(mine, acc.contiguous(), op=dist.ReduceOp.SUM, group=self.group)
         return mine
 
+    # ------------------------------------------------------ all-to-all library calls ----
+    def _amax_cuda(self, x: torch.Tensor) -> torch.Tensor:
+        return _lib.amax(x)
+
+    def _dispatch_cuda(self, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None,
+                       amax_bits: torch.Tensor) -> dict:
+        return _lib.ep_dispatch(self.cfg, self.world, x, w_router, bias, amax_bits)
+
+    def _experts_cuda(self, codes, scales, expert, w, amax_bits) -> torch.Tensor:
+        return _lib.ep_experts(self.create_experts(), codes, scales, expert, w, amax_bits)
+
+    def _combine_cuda(self, rows: torch.Tensor, pos: torch.Tensor, T: int) -> torch.Tensor:
+        return _lib.ep_combine(rows, pos, T, self.cfg.topk)
+
+    def _all_to_all(self, out: torch.Tensor, inp: torch.Tensor, out_splits: list, in_splits: list):
+        if self.world == 1:
+            out.copy_(inp)
+            return
+        dist.all_to_all_single(out, inp, output_split_sizes=out_splits, input_split_sizes=in_splits,
+                               group=self.group)
+
+    def forward_all_to_all(self, x: torch.Tensor, w_router: torch.Tensor,
+                           bias: torch.Tensor | None = None) -> torch.Tensor:
+        """The all-to-all exchange: x [T, H] BF16 (T equal on every rank) -> out [T, H] BF16."""
+        T, H = x.shape
+        amax_bits = self._a2a["amax"](x)
+        if self.world > 1:
+            dist.all_reduce(amax_bits, op=dist.ReduceOp.MAX, group=self.group)
+        send = self._a2a["dispatch"](x, w_router, bias, amax_bits)
+        send_counts = send["rank_counts"]
+        recv_counts = torch.empty_like(send_counts)
+        self._all_to_all(recv_counts, send_counts, [1] * self.world, [1] * self.world)
+        sc = [int(v) for v in send_counts.cpu().tolist()]
+        rc = [int(v) for v in recv_counts.cpu().tolist()]
+        n = sum(rc)
+        recv = {}
+        for key in ("codes", "scales", "expert", "w"):
+            t = send[key]
+            recv[key] = torch.empty((n,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            self._all_to_all(recv[key], t, rc, sc)
+        rows = self._a2a["experts"](recv["codes"], recv["scales"], recv["expert"], recv["w"], amax_bits)
+        back = torch.empty((T * self.cfg.topk, rows.shape[1]), dtype=rows.dtype, device=rows.device)
+        self._all_to_all(back, rows, sc, rc)
+        return self._a2a["combine"](back, send["pos"], T)
+
     def forward(self, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None) -> torch.Tensor:
         """x [T, H] BF16: this rank's tokens (T equal on every rank) -> out [T, H] BF16."""
+        if self.exchange == "all_to_all":
+            return self.forward_all_to_all(x, w_router, bias)
         x_all = self.gather(x)
         partial = self._partial if self._partial is not None else self._partial_cuda
         acc = partial(x_all, w_router, bias)

@@ -249,3 +249,42 @@ def test_status_and_workspace_aliases(lib):
         assert lib.nvfp4moe_workspace_bytes(ctypes.byref(c), T) == moe.forward_workspace_bytes(c, T) > 0
     assert lib.nvfp4moe_workspace_bytes(ctypes.byref(c), 0) == 0
     assert lib.nvfp4moe_workspace_bytes(ctypes.byref(_cfg(H=100)), 16) == 0
+
+
+def test_expert_parallel_exchange_checks(lib):
+    """nvfp4moe_amax, _ep_dispatch, _ep_experts and _ep_combine: the documented host-side checks."""
+    c = moe.cfg_default()
+    ws_q = moe.quantize_workspace_bytes(16, 5120)
+    assert lib.nvfp4moe_amax(A, 16, 5120, None, A, ws_q, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_amax(A, 16, 5121, A, A, ws_q, None) == moe.ERR_SHAPE
+    assert lib.nvfp4moe_amax(MIS, 16, 5120, A, A, ws_q, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_amax(A, 16, 5120, A, A, 8, None) == moe.ERR_WORKSPACE
+    assert lib.nvfp4moe_amax(A, 16, 5120, A, A, ws_q, None) in NO_DEVICE
+
+    wsd = moe.ep_dispatch_workspace_bytes(c, 16)
+    assert wsd > 0 and moe.ep_dispatch_workspace_bytes(_cfg(H=100), 16) == 0
+
+    def dispatch(cfg=c, G=8, x=A, T=16, w=A, amax=A, codes=A, scales=A, ws_bytes=wsd):
+        return lib.nvfp4moe_ep_dispatch(ctypes.byref(cfg), G, x, T, w, None, amax, codes, scales, A, A, A, A, A,
+                                        ws_bytes, None)
+
+    assert dispatch(G=3) == moe.ERR_ARG                 # 256 experts do not split over 3 ranks
+    assert dispatch(G=0) == moe.ERR_ARG
+    assert dispatch(T=0) == moe.ERR_SHAPE
+    for k in ("x", "w", "amax", "codes", "scales"):
+        assert dispatch(**{k: None}) == moe.ERR_ARG, k
+    assert dispatch(codes=MIS) == moe.ERR_ARG
+    assert dispatch(ws_bytes=wsd - 1) == moe.ERR_WORKSPACE
+    assert dispatch() in NO_DEVICE
+
+    assert moe.ep_experts_workspace_bytes(c, 32, 4096) > 0
+    assert moe.ep_experts_workspace_bytes(c, 0, 4096) == 0
+    assert moe.ep_experts_workspace_bytes(c, 257, 4096) == 0
+    assert lib.nvfp4moe_ep_experts(None, A, A, A, A, 16, A, A, A, 1 << 30, None) == moe.ERR_ARG
+
+    assert lib.nvfp4moe_ep_combine(A, A, 16, 9, 5120, A, None) == moe.ERR_SHAPE
+    assert lib.nvfp4moe_ep_combine(A, A, 16, 8, 5000, A, None) == moe.ERR_SHAPE
+    assert lib.nvfp4moe_ep_combine(None, A, 16, 8, 5120, A, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_ep_combine(MIS, A, 16, 8, 5120, A, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_ep_combine(A, A, 0, 8, 5120, A, None) == moe.OK
+    assert lib.nvfp4moe_ep_combine(A, A, 16, 8, 5120, A, None) in NO_DEVICE

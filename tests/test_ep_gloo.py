@@ -1,7 +1,8 @@
 """Expert parallelism on the CPU: gloo ranks (world size 2 and 4) run ExpertParallelLayer with
-the oracle standing in for each rank's partial layer (its share of the tiny layer's 32 experts).
-The exchange (all-gather of the tokens, reduce-scatter of the FP32 sums) must give every rank
-the oracle's whole-layer output for its own tokens ("Reflection releases Beam ...", section
+the oracle standing in for the library's calls (each rank's share of the tiny layer's 32
+experts).  Both exchanges (all-gather of the tokens with a reduce-scatter of the FP32 sums;
+all-to-all of the pairs' quantised rows and of their weighted output rows) must give every
+rank the oracle's whole-layer output for its own tokens ("Reflection releases Beam ...", section
 "Tool calling and multi-node setups": experts placed on the devices, the rest replicated)."""
 import os
 import socket
@@ -74,6 +75,104 @@ def test_gloo_ranks_expert_parallel_layer(world):
         got = res[r][3]
         # FP32 partial sums added across ranks, then BF16: within one BF16 unit of the oracle
         assert np.all(np.abs(got - want) <= 2 * bf16_half_ulp(want) + 1e-30)
+
+
+def _rank_main_a2a(rank, world, port, out):
+    """One gloo rank of the all-to-all exchange, the library's four calls replaced by oracle
+    stand-ins (routing, quantisation with the global scale, grouping, expert MLPs, slot-order
+    combine), kept in FP64 so the exchange itself is what the comparison checks."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import oracle
+    import nvfp4_quantized_moe_group_b200 as moe
+    from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer
+    from workloads import TINY, activations, router_weight
+    from tests.helpers import cfg_ns, intermediate_scales, oracle_expert
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        s = TINY
+        cfg = moe.Cfg(s.E, s.n_groups, s.topk_groups, s.topk, s.H, s.I, s.routed_scale)
+        g_h = intermediate_scales(s)
+        k = s.topk
+        seen = {}
+
+        def g_of(amax_bits):
+            a = np.array([int(amax_bits.item()) << 16], dtype=np.uint32).view(np.float32)[0]
+            return oracle.global_scale(a)
+
+        def amax(x):
+            return (x.view(torch.int16).to(torch.int32) & 0x7FFF).max().reshape(1)
+
+        def dispatch(x, wr, bias, amax_bits):
+            xn = x.float().numpy()
+            r = oracle.route(xn.astype(np.float64), wr.numpy().astype(np.float64), cfg_ns(s), None)
+            codes, scales, _ = oracle.quantize(xn, g=g_of(amax_bits))
+            counts, _, perm, inv = oracle.permutation(r.idx, s.E)
+            epr = s.E // world
+            seen["send_counts"] = counts.reshape(world, epr).sum(axis=1).tolist()
+            return {"codes": torch.from_numpy(codes[perm // k]), "scales": torch.from_numpy(scales[perm // k]),
+                    "expert": torch.from_numpy((r.idx.reshape(-1)[perm] % epr).astype(np.int32)),
+                    "w": torch.from_numpy(r.w.reshape(-1)[perm].astype(np.float64)),
+                    "pos": torch.from_numpy(inv.reshape(-1).astype(np.int32)),
+                    "rank_counts": torch.from_numpy(counts.reshape(world, epr).sum(axis=1).astype(np.int32))}
+
+        def experts(codes, scales, expert, w, amax_bits):
+            seen["recv_rows"] = int(codes.shape[0])
+            xhat = oracle.dequantize(codes.numpy(), scales.numpy(), g_of(amax_bits))
+            rows = np.zeros((codes.shape[0], s.H))
+            e_loc = expert.numpy()
+            for e in np.unique(e_loc):
+                sel = np.flatnonzero(e_loc == e)
+                eg = int(e) + layer.e_begin
+                y = oracle.expert_mlp(xhat[sel], *oracle_expert(s, eg), np.float32(g_h[eg]))["y"]
+                rows[sel] = w.numpy()[sel][:, None] * y
+            return torch.from_numpy(rows)
+
+        def combine(back, pos, T):
+            b = back.numpy()
+            p = pos.numpy().reshape(T, k)
+            outv = np.zeros((T, s.H))
+            for j in range(k):
+                outv += b[p[:, j]]
+            return torch.from_numpy(outv)
+
+        layer = ExpertParallelLayer(cfg, exchange="all_to_all",
+                                    a2a_ops={"amax": amax, "dispatch": dispatch, "experts": experts,
+                                             "combine": combine})
+        wr = router_weight(s)
+        x = activations(T_RANK, s, seed=60 + rank)
+        y = layer.forward(x, wr)
+        out[rank] = (layer.e_begin, layer.e_count, seen, y.numpy(), x.float().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_all_to_all_exchange(world):
+    """The all-to-all exchange on gloo ranks: uneven per-rank counts, rows and their metadata
+    out, weighted output rows back, each token's rows added in slot order.  Every rank must get
+    the oracle's whole layer on the concatenated batch for its own tokens (the global scale of
+    all ranks' tokens included), and the rows each rank receives must be the pairs routed to
+    its experts."""
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main_a2a, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    sys.path.insert(0, ROOT)
+    from workloads import TINY, router_weight
+    from tests.helpers import oracle_layer, intermediate_scales
+    x_all = np.concatenate([res[r][4] for r in range(world)])
+    ref = oracle_layer(TINY, x_all, router_weight(TINY).numpy(), None, intermediate_scales(TINY), workers=1)
+    n = TINY.E // world
+    sent = np.array([res[r][2]["send_counts"] for r in range(world)])      # [source, destination]
+    for r in range(world):
+        assert (res[r][0], res[r][1]) == (r * n, n)
+        assert res[r][2]["recv_rows"] == int(sent[:, r].sum())
+        assert int(((ref["route"].idx >= r * n) & (ref["route"].idx < (r + 1) * n)).sum()) == int(sent[:, r].sum())
+        want = ref["out"][r * T_RANK:(r + 1) * T_RANK]
+        np.testing.assert_allclose(res[r][3], want, rtol=1e-12, atol=1e-12)
 
 
 def test_expert_range_split():

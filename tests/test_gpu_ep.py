@@ -14,7 +14,8 @@ import nvfp4_quantized_moe_group_b200 as moe
 from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer, expert_range
 from workloads import TINY, BEAM, activations, router_weight, expert_weight
 import oracle
-from tests.helpers import intermediate_scales, bf16_half_ulp, cfg_ns, oracle_expert_pass, check_output
+from tests.helpers import (intermediate_scales, bf16_half_ulp, cfg_ns, oracle_expert_pass, check_output,
+                           check_routing)
 from tests.test_gpu_forward import gpu_experts
 
 pytestmark = pytest.mark.gpu
@@ -147,3 +148,140 @@ def test_single_rank_layer_matches_forward():
     want = moe.forward(gpu_experts(TINY), x, wr).float().cpu().numpy()
     assert np.all(np.abs(got - want) <= 2 * bf16_half_ulp(want) + 1e-30)
     layer.close()
+
+
+def run_all_to_all_emulated(shape, G, T_rank, seed=70, sample=None):
+    """The all-to-all exchange (nvfp4moe_amax, _ep_dispatch, _ep_experts, _ep_combine) with G ranks
+    emulated one after another on this GPU, each collective a host-side concatenation of the
+    ranks' buffers.  Checked: every rank's dispatched rows are the oracle's quantisation of its
+    tokens with the global scale of all ranks' tokens, in the oracle's expert-major order, with
+    the oracle's per-rank counts (bit-exact, where the GPU routes as the oracle does); every
+    rank's output equals nvfp4moe_forward on the concatenated batch up to the order of the FP32
+    additions; the sampled tokens' FP32 sums are within the layer tolerance of the oracle, and
+    the BF16 output is their exact rounding."""
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I, shape.routed_scale)
+    k, H = shape.topk, shape.H
+    xs_cpu = [activations(T_rank, shape, seed=seed + r) for r in range(G)]
+    xs = [x.cuda() for x in xs_cpu]
+    wr_cpu = router_weight(shape)
+    wr = wr_cpu.cuda()
+    g_h = intermediate_scales(shape)
+    # 1. the global amax
+    amax = torch.stack([moe.amax(x) for x in xs]).max(dim=0).values
+    x_all_cpu = torch.cat(xs_cpu)
+    ref_bits = int((x_all_cpu.view(torch.int16).to(torch.int32) & 0x7FFF).max())
+    assert int(amax.item()) == ref_bits
+    # 2. dispatch on every rank
+    sends = [moe.ep_dispatch(cfg, G, x, wr, None, amax) for x in xs]
+    torch.cuda.synchronize()
+    g_glob = oracle.global_scale(np.array([ref_bits << 16], dtype=np.uint32).view(np.float32)[0])
+    epr = shape.E // G
+    idx_gpu = []
+    for r, sd in enumerate(sends):
+        xn = xs_cpu[r].float().numpy()
+        ro = oracle.route(xn.astype(np.float64), wr_cpu.numpy().astype(np.float64), cfg_ns(shape), None)
+        # the rank's routing (the kernels nvfp4moe_route runs) under the near-tie protocol; the
+        # layout is then fixed by it
+        gi, gw = moe.route(cfg, xs[r], wr)
+        gi, gw = gi.cpu().numpy(), gw.cpu().numpy()
+        check_routing(gi, gw, ro, xn.astype(np.float64), wr_cpu.numpy().astype(np.float64), None, shape)
+        idx_gpu.append(gi)
+        codes, scales, _ = oracle.quantize(xn, g=g_glob)
+        counts, _, perm, inv = oracle.permutation(gi, shape.E)
+        np.testing.assert_array_equal(sd["rank_counts"].cpu().numpy(), counts.reshape(G, epr).sum(axis=1))
+        np.testing.assert_array_equal(sd["codes"].cpu().numpy(), codes[perm // k])
+        np.testing.assert_array_equal(sd["scales"].cpu().numpy(), scales[perm // k])
+        np.testing.assert_array_equal(sd["expert"].cpu().numpy(), gi.reshape(-1)[perm] % epr)
+        np.testing.assert_array_equal(sd["pos"].cpu().numpy(), inv.reshape(-1))
+        np.testing.assert_array_equal(sd["w"].cpu().numpy(), gw.reshape(-1)[perm])
+    # 3. rows to their experts' ranks
+    counts = [sd["rank_counts"].cpu().tolist() for sd in sends]
+    offs = [np.concatenate([[0], np.cumsum(c)]) for c in counts]
+    rows_back = [[None] * G for _ in range(G)]
+    for d in range(G):
+        recv = {key: torch.cat([sends[src][key][offs[src][d]:offs[src][d + 1]] for src in range(G)])
+                for key in ("codes", "scales", "expert", "w")}
+        ex = local_experts(shape, d * epr, epr)
+        rows = moe.ep_experts(ex, recv["codes"], recv["scales"], recv["expert"], recv["w"], amax)
+        torch.cuda.synchronize()
+        ex.close()
+        o = 0
+        for src in range(G):
+            n = counts[src][d]
+            rows_back[src][d] = rows[o:o + n]
+            o += n
+    # 4. rows back and the combine
+    outs, accs = [], []
+    for src in range(G):
+        back = torch.cat(rows_back[src])
+        out = moe.ep_combine(back, sends[src]["pos"], T_rank, k)
+        b = back.cpu().numpy()
+        p = sends[src]["pos"].cpu().numpy().reshape(T_rank, k)
+        acc = np.zeros((T_rank, H), dtype=np.float32)
+        for j in range(k):
+            acc = (acc + b[p[:, j]]).astype(np.float32)
+        assert torch.equal(out.cpu(), torch.from_numpy(acc).to(torch.bfloat16)), "combine is not the slot-order sum"
+        outs.append(out.float().cpu().numpy())
+        accs.append(acc)
+    # the single-GPU layer on the concatenated batch, same routing and codes
+    full = gpu_experts(shape)
+    single = moe.forward(full, torch.cat(xs), wr).float().cpu().numpy()
+    got = np.concatenate(outs)
+    row = np.abs(single).max(axis=1, keepdims=True)
+    assert np.all(np.abs(got - single) <= 2 * bf16_half_ulp(single) + 2.0 ** -16 * row + 1e-30)
+    # sampled tokens against the oracle (FP32 sums)
+    acc_all = np.concatenate(accs)
+    T_all = G * T_rank
+    sample = np.arange(T_all) if sample is None else np.asarray(sample)
+    xn = x_all_cpu.float().numpy()
+    r_or = oracle.route(xn.astype(np.float64), wr_cpu.numpy().astype(np.float64), cfg_ns(shape), None)
+    xc, xsc, gx = oracle.quantize(xn)
+    assert gx == g_glob
+    same = (np.concatenate(idx_gpu)[sample] == r_or.idx[sample]).all(axis=1)
+    assert same.mean() > 0.9
+    sample = sample[same]
+    need = {}
+    for i, t in enumerate(sample):
+        for j in range(k):
+            need.setdefault(int(r_or.idx[t, j]), []).append((i, int(t), j))
+    xhat = oracle.dequantize(xc[sample], xsc[sample], gx)
+    ys = oracle_expert_pass(shape, {e: (xhat[[i for i, _, _ in v]], float(g_h[e]), None, None) for e, v in need.items()})
+    ref = np.zeros((len(sample), H))
+    for e, v in need.items():
+        for m, (i, t, j) in enumerate(v):
+            ref[i] += r_or.w[t, j] * ys[e][0][m]
+    check_output(acc_all[sample], ref)
+
+
+@pytest.mark.parametrize("G,T_rank", [(2, 24), (4, 40)])
+def test_tiny_all_to_all_emulated(G, T_rank):
+    run_all_to_all_emulated(TINY, G, T_rank)
+
+
+def test_beam_all_to_all_eight_ranks_full_segments():
+    """Beam prefill on 8 emulated ranks of 512 tokens: every receiving rank groups about 4096
+    rows over its 32 experts (the full-segment GEMM epilogues)."""
+    run_all_to_all_emulated(BEAM, 8, 512, sample=[0, 700, 1500, 2222, 3000, 4095])
+
+
+def test_ep_experts_checks_received_expert_indices_on_the_device():
+    """Expert indices arrive from other ranks: one outside the handle's experts is replaced on
+    the device (every access stays in bounds) and reported as NVFP4MOE_ERR_ARG."""
+    shape = TINY
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I, shape.routed_scale)
+    ex = local_experts(shape, 0, 16)
+    x = activations(4, shape, seed=90).cuda()
+    amax = moe.amax(x)
+    codes, scales, _ = moe.quantize(x)
+    w = torch.ones(4, dtype=torch.float32, device="cuda")
+    good = torch.tensor([3, 0, 15, 5], dtype=torch.int32, device="cuda")
+    rows = moe.ep_experts(ex, codes, scales, good, w, amax)
+    assert moe.last_device_status() == moe.OK
+    bad = torch.tensor([3, -1, 16, 5], dtype=torch.int32, device="cuda")
+    rows_bad = moe.ep_experts(ex, codes, scales, bad, w, amax)
+    assert moe.last_device_status() == moe.ERR_ARG
+    assert bool(torch.isfinite(rows_bad).all())
+    # the rows with valid indices are unchanged by the bad ones
+    for i in (0, 3):
+        assert torch.equal(rows_bad[i], rows[i])
+    ex.close()
