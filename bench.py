@@ -707,7 +707,7 @@ def run_ep(args, world, rank, local):
     T = wl.T
     cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
                        shape.routed_scale)
-    layer = ExpertParallelLayer(cfg)
+    layer = ExpertParallelLayer(cfg, exchange=args.exchange)
     ex = layer.create_experts()
     g_h = intermediate_scales(shape)
     for e in range(layer.e_begin, layer.e_begin + layer.e_count):
@@ -724,6 +724,23 @@ def run_ep(args, world, rank, local):
     hit_local = int((counts > 0).sum())
     launches = moe.last_launch_count() + 1          # + finalize
     del dbg
+    if args.exchange == "all_to_all":
+        # one step with every library call's launch count added up
+        counted = []
+
+        def counting(fn):
+            def call(*a, **kw):
+                r = fn(*a, **kw)
+                counted.append(moe.last_launch_count())
+                return r
+            return call
+
+        ops = dict(layer._a2a)
+        layer._a2a = {k: counting(v) for k, v in ops.items()}
+        layer.forward(x, wr, bias)
+        layer._a2a = ops
+        launches = sum(counted)
+
     for _ in range(args.warmup):
         layer.forward(x, wr, bias)
     torch.cuda.synchronize()
@@ -761,7 +778,9 @@ def run_ep(args, world, rank, local):
             "data": "synthetic (seeded counter-hash inputs; random-init NVFP4 weights)",
             "config": {"workload": wl.describe() + f" per rank, expert parallel over {world} rank(s)",
                        "T_per_rank": T, "experts_per_rank": layer.e_count, "local_experts_hit": hit_local,
-                       "parallelism": f"ep{world} (all-gather tokens, reduce-scatter FP32 sums)",
+                       "parallelism": f"ep{world} " + ("(all-gather tokens, reduce-scatter FP32 sums)"
+                                                      if args.exchange == "gather" else
+                                                      "(all-to-all of quantised pair rows and weighted output rows)"),
                        "l2": "no flush: every step streams the rank's routed experts' weights"},
             "roofline": {"bound": "hbm", "achieved": local_bytes / (ms / 1e3) / 1e9, "peak": p["hbm_gbs"],
                          "unit": "GB/s", "frac": local_bytes / (ms / 1e3) / (p["hbm_gbs"] * 1e9), "traffic": None,
@@ -927,8 +946,11 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the compute-heavy configs (prefill, skewed, 32768 tokens, quantise) of the line")
     ap.add_argument("--ep", action="store_true",
-                    help="expert parallelism over the ranks (each holds E/N experts; NCCL all-gather and "
-                         "reduce-scatter) instead of one full replica per GPU")
+                    help="expert parallelism over the ranks (each holds E/N experts) instead of one full replica "
+                         "per GPU")
+    ap.add_argument("--exchange", choices=["gather", "all_to_all"], default="gather",
+                    help="with --ep: all-gather the tokens and reduce-scatter FP32 sums, or send each pair's "
+                         "quantised row to its expert's rank and its output row back (NCCL all-to-all)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -301,6 +301,9 @@ typedef struct {
   float* xq8_scales;   /* [T] its per-token scales */
   float* acc;          /* [T][H] FP32 sums of the weighted expert rows, the values the BF16 output
                           rounds (to nearest, ties to even); nvfp4moe_forward and _residual */
+  float* h_f32;        /* [T*topk][I] FP32 SwiGLU product of every pair, rows in perm order, as
+                          the gate/up epilogue computes it before requantising it (NVFP4 forward
+                          calls); pairs of experts a local handle does not hold are not written */
   /* Failure detection (nvfp4moe_forward, nvfp4moe_forward_residual, nvfp4moe_forward_partial;
    * the other calls ignore these two fields).  Every wait of the call's kernels on another
    * CTA or on the tensor cores is bounded: when one runs out, the kernel raises

@@ -53,7 +53,8 @@ STAGES = ("amax", "route", "quantize", "permute", "gather", "gateup", "down", "f
 class Debug(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_void_p) for n in DEBUG_FIELDS] + [("events", ctypes.POINTER(ctypes.c_void_p))]
                 + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p), ("xq8_codes", ctypes.c_void_p),
-                   ("xq8_scales", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("wait_limit_us", ctypes.c_uint32),
+                   ("xq8_scales", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("h_f32", ctypes.c_void_p),
+                   ("wait_limit_us", ctypes.c_uint32),
                    ("inject_skip_arrive", ctypes.c_int32)])
 
 
@@ -412,7 +413,7 @@ def forward_workspace_bytes(cfg: Cfg, T_max: int) -> int:
     return int(lib().nvfp4moe_forward_workspace_bytes(ctypes.byref(cfg), T_max))
 
 
-def _debug_tensors(cfg: Cfg, T: int, H: int, dev, x_norm: bool = False) -> dict:
+def _debug_tensors(cfg: Cfg, T: int, H: int, dev, x_norm: bool = False, h_f32: bool = False) -> dict:
     k, E, I = cfg.topk, cfg.E, cfg.I
     tensors = {
         "idx": torch.empty((T, k), dtype=torch.int32, device=dev),
@@ -430,6 +431,8 @@ def _debug_tensors(cfg: Cfg, T: int, H: int, dev, x_norm: bool = False) -> dict:
     }
     if x_norm:
         tensors["x_norm"] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if h_f32:
+        tensors["h_f32"] = torch.empty((T * k, I), dtype=torch.float32, device=dev)
     return tensors
 
 
@@ -463,11 +466,13 @@ def forward_residual(experts: Experts, h: torch.Tensor, gamma: torch.Tensor, eps
 
 def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
             out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None,
-            timer: StageTimer | None = None, wait_limit_us: int = 0, inject_skip_arrive: int = 0):
+            timer: StageTimer | None = None, wait_limit_us: int = 0, inject_skip_arrive: int = 0,
+            debug_h: bool = False):
     """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug).
     ``timer``: a StageTimer whose events are recorded around each stage.  ``wait_limit_us``
     and ``inject_skip_arrive``: the failure-detection fields of nvfp4moe_debug (a bounded-wait
-    limit, and the test hook that makes one front-end CTA skip a grid-barrier arrival)."""
+    limit, and the test hook that makes one front-end CTA skip a grid-barrier arrival).
+    ``debug_h``: with debug, also the FP32 SwiGLU product of every pair (h_f32, [T*topk, I])."""
     cfg = experts.cfg
     specs = _layer_specs(cfg, x, w_router, bias)
     T, H = x.shape
@@ -480,7 +485,7 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
     dbg = None
     tensors = None
     if debug:
-        tensors = _debug_tensors(cfg, T, H, dev)
+        tensors = _debug_tensors(cfg, T, H, dev, h_f32=debug_h)
         dbg = Debug(**{n: t.data_ptr() for n, t in tensors.items()})
     if timer is not None:
         if dbg is None:

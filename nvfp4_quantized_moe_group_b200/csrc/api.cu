@@ -844,6 +844,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.g_h = x->g_h;
   g.I = c.I;
   g.wait_ns = wait_ns;
+  g.h_dbg = dbg != nullptr ? dbg->h_f32 : nullptr;
+  g.dbg_offsets = f.offsets + x->e_begin;
   g.acc = f.acc;
   g.row_pair = f.row_pair;
   g.wts = f.wts;
@@ -860,6 +862,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.sfb = x->wd_sf;
   g.K = c.I;
   g.n_total = c.H;
+  g.h_dbg = nullptr;
   ev.mark(NVFP4MOE_STAGE_DOWN, 0);
   g.work_counter = &f.hdr->work[1];
   if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;

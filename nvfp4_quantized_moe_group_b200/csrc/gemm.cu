@@ -204,6 +204,14 @@ __device__ __forceinline__ void swiglu32(const uint32_t* G, const uint32_t* U, f
   }
 }
 
+// Debug export of 32 features of one pair's FP32 h (feature f0 on).
+__device__ __forceinline__ void store_h_dbg(const GemmArgs& p, const Work& wk, int row_l, int f0, const float* h) {
+  const int64_t pos = (int64_t)__ldg(p.dbg_offsets + wk.e) + (int64_t)wk.mt_local * kBlockM + row_l;
+  float4* dst = reinterpret_cast<float4*>(p.h_dbg + pos * p.I + f0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+}
+
 // NVFP4 requantisation of 32 features with the expert's static scale gh: 16 code bytes and
 // 2 scale bytes stored at feature f0 of the row.
 __device__ __forceinline__ void quant_store32(const float* h, float gh, float r_t, bool valid, int64_t row, int f0,
@@ -516,8 +524,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           release();
           float h[32];
           swiglu32(G0, U0, sg, su, h);
+          if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64, h);
           quant_store32(h, gh, r_t, valid, row, t * 64, p, n_ct);
           swiglu32(G1, U1, sg, su, h);
+          if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64 + 32, h);
           quant_store32(h, gh, r_t, valid, row, t * 64 + 32, p, n_ct);
         } else {
 #pragma unroll
@@ -529,6 +539,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             if (pr == 1) release();
             float h[32];
             swiglu32(G, U, sg, su, h);
+            if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64 + 32 * pr, h);
             quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, p, n_ct);
           }
         }

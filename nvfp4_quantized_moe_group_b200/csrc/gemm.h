@@ -45,6 +45,11 @@ struct GemmArgs {
   const float* w_scale;        // [E][n_total] weight channel scales (gate/up in packed column order)
   float* h32;                  // gate/up: [rows_cap][I] FP32 SwiGLU product
   const float* h_scale;        // down: [rows_cap] scale of each segment row of A (= h)
+  // debug (NVFP4 gate/up): the FP32 SwiGLU product h of every pair before its requantisation,
+  // [pairs][I] in grouping order (pair position = dbg_offsets[e] + row in the expert's
+  // segment); nullptr on the hot path
+  float* h_dbg;
+  const int32_t* dbg_offsets;  // [E + 1], with h_dbg
 };
 
 // gemm.cu

@@ -69,9 +69,6 @@ __global__ void __launch_bounds__(32) amax_reduce_kernel(const uint32_t* partial
   if (threadIdx.x == 0) *amax_bits = m;
 }
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantCtasPerSm = 8;
-
 // Per-halfword unsigned maximum of two packed pairs.
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -79,45 +76,43 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Persistent: gridDim.x CTAs of 8 warps; a work unit is one (row, 512-value segment) and a
-// warp takes units warp, warp + all warps, ..., one 16-value block per lane, so every load,
-// code store and accumulator store of the warp covers one contiguous span of the row; lanes
-// 4k .. 4k+3 hold the 4 block scales of one 32-bit scale word.  Each CTA first tabulates the
-// block reciprocal r_b = 1 / (E4M3(S) g) for the 128 non-negative E4M3 codes S (0 where the
-// scale decodes to 0): the same operations as the block rule, once per code instead of once
-// per block.  Rows in [rows, rows_padded) only write zero scales (swizzled-layout padding).
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantizeArgs a) {
-  __shared__ float s_rb[128];
+// One CTA per row (rows_padded CTAs), min(segments, 32) warps: each warp quantises the row's
+// 512-value segments warp, warp + n_warps, ..., one 16-value block per lane.  Rows in
+// [rows, rows_padded) only write zero scales (swizzled layout padding).  The global scale is
+// read from g_in.
+__global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
   const float g = __ldg(a.g_in);
   if (!(g > 0.0f && g < __uint_as_float(0x7F800000u))) return;   // non-finite input: skipped
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.g_out != nullptr && a.g_out != a.g_in) *a.g_out = g;
   const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
-  if (threadIdx.x < 128) {
-    const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
-    s_rb[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-  }
-  __syncthreads();
 
+  // one warp per (row, 512-value segment): lane l takes the 16-value block 32 seg + l, so every
+  // load, code store and accumulator store of the warp covers one contiguous span of the row;
+  // lanes 4k .. 4k+3 hold the 4 block scales of one 32-bit scale word
   const int blocks_per_row = (int)(a.cols >> 4);
   const int segs_per_row = (blocks_per_row + 31) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t n_units = a.rows_padded * segs_per_row;
-  const int64_t warp0 = (int64_t)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
-  const int64_t n_warps = (int64_t)gridDim.x * (kQuantThreads / 32);
-  for (int64_t u = warp0; u < n_units; u += n_warps) {
-    const int64_t r = u / segs_per_row;
-    const int seg = (int)(u - r * segs_per_row);
+  const int n_warps = blockDim.x >> 5;
+  const int64_t r = blockIdx.x;
+  // segment rows of the token's pairs (lane j < topk holds pair j's), found once per warp
+  int64_t my_row = 0;
+  if (a.seg_codes != nullptr && r < a.rows && lane < a.topk) {
+    const int64_t p = r * a.topk + lane;
+    const int e = a.idx[p];
+    my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
+  }
+  for (int seg = threadIdx.x >> 5; seg < segs_per_row; seg += n_warps) {
     const int64_t b = (int64_t)seg * 32 + lane;
     // lanes past the row's last block stay for the shuffles; groups of 4 lanes are active or
     // idle together (cols % 64 == 0)
     const bool active = b < blocks_per_row;
     const bool live = active && r < a.rows;
-    // segment rows of the token's pairs (lane j < topk holds pair j's)
-    int64_t my_row = 0;
-    if (a.seg_codes != nullptr && r < a.rows && lane < a.topk) {
-      const int64_t p = r * a.topk + lane;
-      const int e = __ldg(a.idx + p);
-      my_row = (int64_t)__ldg(a.mtile_prefix + e) * kBlockM + (__ldg(a.inv + p) - __ldg(a.offsets + e));
+
+    if (a.zero_out != nullptr && live) {
+      float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
+      const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  #pragma unroll
+      for (int i = 0; i < 4; ++i) z[i] = zero;
     }
 
     uint32_t s = 0, c0 = 0, c1 = 0;
@@ -125,27 +120,24 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantizeArgs a)
       const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + b * 16);
       const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
       const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      // block maximum of |x| on the BF16 magnitude bits (exact; >= 0x7F80: Inf or NaN)
+      float f[16];
+      // block maximum of |x| on the BF16 magnitude bits, two halves per instruction (exact;
+      // >= 0x7F80: Inf or NaN)
       uint32_t m2 = w[0] & 0x7FFF7FFFu;
-#pragma unroll
+  #pragma unroll
       for (int j = 1; j < 8; ++j) m2 = max_u16x2(m2, w[j] & 0x7FFF7FFFu);
       const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
-      s = cvt_e4m3(__fmul_rn(__uint_as_float(mb << 16), r_t));
-      const float r_b = s_rb[s & 127u];   // a non-negative input gives a code below 128
-      float f[16];
-#pragma unroll
+  #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        f[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), r_b);
-        f[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), r_b);
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
       }
+      float r_b;
+      s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
+  #pragma unroll
+      for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
       c0 = cvt_e2m1x8(f);
       c1 = cvt_e2m1x8(f + 8);
-    }
-    if (a.zero_out != nullptr && live) {
-      float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
-      const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) z[i] = zero;
     }
     // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes 4k)
     const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
@@ -208,13 +200,9 @@ cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream) {
       return cudaMemcpyAsync(a.g_out, a.g_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
     return cudaSuccess;
   }
-  const int64_t segs = ((a.cols >> 4) + 31) >> 5;
-  const int64_t units = a.rows_padded * segs;
-  const int64_t warps_per_cta = kQuantThreads / 32;
-  int64_t grid = (units + warps_per_cta - 1) / warps_per_cta;
-  const int64_t cap = (int64_t)num_sms() * kQuantCtasPerSm;
-  if (grid > cap) grid = cap;
-  quantize_kernel<<<(unsigned)grid, kQuantThreads, 0, stream>>>(a);
+  const int segs = (int)(((a.cols >> 4) + 31) >> 5);
+  const int warps = segs < 32 ? segs : 32;
+  quantize_kernel<<<(unsigned)a.rows_padded, 32 * warps, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -117,11 +117,35 @@ def oracle_expert(shape, e: int, seed: int = 0):
                  for w in ("gate", "up", "down"))
 
 
+def _abs_sums(xhat, t: "oracle.QuantTensor") -> np.ndarray:
+    """sum_k |x_k w_k| of every (row, output) of a product with dequantised operands (the scale of
+    the FP32 accumulation error of that output)."""
+    return np.abs(xhat) @ np.abs(t.dequant()).T
+
+
+def accumulation_bound(xhat, t: "oracle.QuantTensor", step: int = 64) -> np.ndarray:
+    """Bound on |acc - exact| of every (row, output) of x W^T accumulated as the grouped GEMM
+    issues it: K in ascending order, one tensor-core instruction per ``step`` values, each adding
+    its exact products into the FP32 accumulator.  Per instruction i at most one rounding of the
+    running sum P_i (2^-23 |P_i|) and an internal error of at most 2^-23 sum|products of i|:
+    2^-23 (sum_i |P_i| + sum_k |x_k w_k|)."""
+    W = t.dequant()
+    K = xhat.shape[1]
+    P = np.zeros((xhat.shape[0], W.shape[0]))
+    total = np.zeros_like(P)
+    for k0 in range(0, K, step):
+        xs, ws = xhat[:, k0:k0 + step], W[:, k0:k0 + step]
+        P += xs @ ws.T
+        total += np.abs(P) + np.abs(xs) @ np.abs(ws).T
+    return U23 * total
+
+
 def _expert_job(args):
     shape, e, xhat, g_h = args
     gate, up, down = oracle_expert(shape, e)
     res = oracle.expert_mlp(xhat, gate, up, down, np.float32(g_h))
-    return e, res["y"], res["h"], res["hq_codes"], res["hq_scales"], (gate.g, up.g, down.g)
+    dh = h_error_bound(res["gate"], res["up"], accumulation_bound(xhat, gate), accumulation_bound(xhat, up))
+    return e, res["y"], res["h"], res["hq_codes"], res["hq_scales"], dh
 
 
 def _init_single_thread():
@@ -138,12 +162,13 @@ def _expert_rows_job(args):
     res = oracle.expert_mlp(xhat, gate, up, down, np.float32(g_h))
     y_gpu_hq = res["y"].copy()
     if gpu_hq_codes is None:
-        return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"]
+        return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"], None
+    dh = h_error_bound(res["gate"], res["up"], accumulation_bound(xhat, gate), accumulation_bound(xhat, up))
     same = (np.all(gpu_hq_codes == res["hq_codes"], axis=1) & np.all(gpu_hq_scales == res["hq_scales"], axis=1))
     if not same.all():
         hhat = oracle.dequantize(gpu_hq_codes[~same], gpu_hq_scales[~same], np.float32(g_h))
         y_gpu_hq[~same] = hhat @ down.dequant().T
-    return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"]
+    return e, res["y"], y_gpu_hq, res["h"], res["hq_codes"], res["hq_scales"], dh
 
 
 def oracle_expert_pass(shape, jobs: dict, workers=None) -> dict:
@@ -191,10 +216,10 @@ def oracle_layer(shape, x: np.ndarray, wr: np.ndarray, bias, g_h: np.ndarray, to
         results = [_expert_job(j) for j in jobs]
     out = np.zeros((len(tokens), x.shape[1]))
     inter = {}
-    for e, y, h, hc, hs, _ in results:
+    for e, y, h, hc, hs, dh in results:
         for n, (i, t, j) in enumerate(need[e]):
             out[i] += r.w[t, j] * y[n]
-            inter[(t, j)] = (h[n], hc[n], hs[n])
+            inter[(t, j)] = (h[n], hc[n], hs[n], dh[n])
     return {"route": r, "xq_codes": xc, "xq_scales": xs, "g_x": gx, "tokens": tokens, "out": out,
             "inter": inter}
 
@@ -222,28 +247,54 @@ def check_output(gpu_out: np.ndarray, ref: np.ndarray, max_abs=2e-2, rel_fro=5e-
 
 
 E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+U23 = 2.0 ** -23
 
 
-def requant_near_tie(h: np.ndarray, g_h: float, rel=1e-4) -> tuple[np.ndarray, np.ndarray]:
-    """Where the requantisation of h (FP64) sits within a relative ``rel`` of a rounding
-    boundary: per block (E4M3 scale) and per element (E2M1 code).  A kernel whose FP32 h
-    differs from the exact value by less than that may round the other way there.  An
-    element whose scaled value is within ``rel`` of zero has an ambiguous sign: +0 and -0
-    (codes 0x0 and 0x8) both decode to zero."""
+def h_error_bound(gate: np.ndarray, up: np.ndarray, acc_gate: np.ndarray, acc_up: np.ndarray) -> np.ndarray:
+    """Bound on |h_gpu - h| for every element of the SwiGLU product as the gate/up epilogue
+    computes it, from the oracle's exact gate and up values and the bounds on their FP32
+    accumulation errors (accumulation_bound; the block-scaled products themselves are exact in
+    FP32: E2M1 x E2M1 x two E4M3 scales).
+
+    * The global-scale multiply rounds once more: dg = acc_gate + 2^-24 |g| (du alike).
+    * h = fl(fl(g u) rcp(fl(1 + e))), e = __expf(-g): __expf within (2 + 1.173 |g|) ulp, entering
+      1 / (1 + e) with weight e / (1 + e) = 1 - s(g); the sum, the two products and the
+      approximate reciprocal (1 ulp) add 3 2^-24 + 2^-23 relative.
+    * Propagation to first order, doubled: dh = 2 (|u| |silu'(g)| dg + |silu(g)| du) + |h| eps_f."""
+    g = np.asarray(gate, dtype=np.float64)
+    u = np.asarray(up, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-g))
+    dg = acc_gate + 2.0 ** -24 * np.abs(g)
+    du = acc_up + 2.0 ** -24 * np.abs(u)
+    dsilu = s * (1.0 + g * (1.0 - s))
+    h = g * s * u
+    eps_f = 3 * 2.0 ** -24 + U23 + (2.0 + 1.173 * np.abs(g)) * U23 * (1.0 - s)
+    return 2.0 * (np.abs(u) * np.abs(dsilu) * dg + np.abs(g * s) * du) + np.abs(h) * eps_f
+
+
+def requant_near_tie(h: np.ndarray, g_h: float, dh: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Where the requantisation of h (exact, FP64) can round the other way for a value within
+    dh (h_error_bound) of it: per block, the E4M3 scale of amax / (6 g_h) lies within the
+    propagated bound (plus the FP32 roundings of h and of the scaled amax) of an E4M3
+    rounding boundary; per element, the scaled value h / d_b lies within its bound of an E2M1
+    boundary, or of zero (the sign of zero: codes 0x0 and 0x8 both decode to zero)."""
     h = np.asarray(h, dtype=np.float64)
     n = h.shape[-1]
     hb = h.reshape(-1, n // 16, 16)
+    db = np.asarray(dh, dtype=np.float64).reshape(hb.shape) + 2.0 ** -24 * np.abs(hb)
     r_t = 1.0 / (6.0 * g_h)
-    q = np.abs(hb).max(axis=2) * r_t
+    amax = np.abs(hb).max(axis=2)
+    q = amax * r_t
+    dq = r_t * db.max(axis=2) + 2 * U23 * q
     grid = oracle.e4m3_table()[:127]
     mids = (grid[:-1] + grid[1:]) / 2
-    dq = np.min(np.abs(q[..., None] - mids[None, None, :]), axis=-1)
-    block_tie = dq <= rel * np.maximum(q, 2.0 ** -9)
+    block_tie = np.min(np.abs(q[..., None] - mids[None, None, :]), axis=-1) <= dq
     S = oracle.e4m3_encode(q.astype(np.float32))
     d = oracle.e4m3_decode(S) * g_h
-    v = np.abs(hb) / np.where(d == 0, np.inf, d)[..., None]
-    dv = np.min(np.abs(v[..., None] - E2M1_MIDS), axis=-1)
-    elem_tie = (dv <= rel * np.maximum(v, 0.25)) | (v <= rel)
+    rb = 1.0 / np.where(d == 0, np.inf, d)[..., None]
+    v = np.abs(hb) * rb
+    dv = db * rb + 2 * U23 * v
+    elem_tie = (np.min(np.abs(v[..., None] - E2M1_MIDS), axis=-1) <= dv) | (v <= dv)
     return block_tie.reshape(h.shape[:-1] + (n // 16,)), elem_tie.reshape(h.shape)
 
 

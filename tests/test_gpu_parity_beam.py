@@ -20,8 +20,9 @@ holding one or two rows, and seeded random tokens.
 
 For every case: routing of all tokens under the near-tie protocol; the input's global scale,
 codes and scales bit-exact; the grouping exactly the oracle's stable sort of the GPU routing;
-the requantised SwiGLU intermediate of every sampled pair equal to the oracle's except at
-FP32 near-ties of the rounding; the FP32 sums of the sampled tokens within max-abs 2e-2 and
+the FP32 SwiGLU product of every sampled pair (exported by the epilogue) within the derived
+error bound of that epilogue (h_error_bound) of the exact value, and its requantisation equal
+to the oracle's except where the exact value lies within that bound of a rounding boundary; the FP32 sums of the sampled tokens within max-abs 2e-2 and
 relative Frobenius 5e-3 of the oracle run on the same quantised operands (the GPU's own
 requantised intermediate, where it differs at a near-tie), the fully independent oracle
 output reported beside it, and the BF16 output exactly the round-to-nearest-even of the FP32
@@ -116,7 +117,8 @@ def gpu_run(ex, case: Case, x, wr, bias, tokens):
     requantised intermediate ([tokens, topk, ...]), and the status word."""
     T, k = case.T, BEAM.topk
     ws = torch.empty(moe.forward_workspace_bytes(ex.cfg, T), dtype=torch.uint8, device="cuda")
-    out, dbg = moe.forward(ex, x.cuda(), wr.cuda(), None if bias is None else bias.cuda(), ws=ws, debug=True)
+    out, dbg = moe.forward(ex, x.cuda(), wr.cuda(), None if bias is None else bias.cuda(), ws=ws, debug=True,
+                           debug_h=True)
     status = moe.status_read(ws)
     g = {n: dbg[n].cpu().numpy() for n in ("idx", "w", "counts", "offsets", "perm", "xq_codes", "xq_scales")}
     g["g_x"] = np.float32(dbg["g_x"].item())
@@ -131,6 +133,7 @@ def gpu_run(ex, case: Case, x, wr, bias, tokens):
     sel = torch.from_numpy(pos[pairs]).cuda()
     hq_c = dbg["hq_codes"][sel].cpu().numpy().reshape(len(tokens), k, -1)
     hq_s = dbg["hq_scales"][sel].cpu().numpy().reshape(len(tokens), k, -1)
+    g["h_f32"] = dbg["h_f32"][sel].cpu().numpy().reshape(len(tokens), k, -1)
     del out, dbg, ws
     torch.cuda.empty_cache()
     return g, hq_c, hq_s, status
@@ -168,15 +171,16 @@ def collect(ex, cases=CASES):
             for j in range(BEAM.topk):
                 e = int(r.idx[t, j])
                 jobs.setdefault(e, []).append((case.name, int(t), j, xhat[i], hq_c[i, j], hq_s[i, j]))
+                rec["pairs"][(int(t), j)] = {"h_gpu": g["h_f32"][i, j]}
         res[case.name] = rec
     packed = {e: (np.stack([v[3] for v in rows]), float(g_h[e]), np.stack([v[4] for v in rows]),
                   np.stack([v[5] for v in rows])) for e, rows in jobs.items()}
     out = oracle_expert_pass(BEAM, packed)
     for e, rows in jobs.items():
-        y, y_g, h, hc, hs = out[e]
+        y, y_g, h, hc, hs, dh = out[e]
         for n, (name, t, j, _, gc, gs) in enumerate(rows):
-            res[name]["pairs"][(t, j)] = {"e": e, "y": y[n], "y_gpu_hq": y_g[n], "h": h[n], "hq_codes": hc[n],
-                                          "hq_scales": hs[n], "gpu_codes": gc, "gpu_scales": gs}
+            res[name]["pairs"][(t, j)].update({"e": e, "y": y[n], "y_gpu_hq": y_g[n], "h": h[n], "hq_codes": hc[n],
+                                               "hq_scales": hs[n], "gpu_codes": gc, "gpu_scales": gs, "dh": dh[n]})
     return res
 
 
@@ -199,9 +203,16 @@ def test_beam_layer(runs, name):
     assert counts.sum() == case.T * BEAM.topk
     # requantised intermediate: equal except at near-ties of the FP32 rounding
     g_h = intermediate_scales(BEAM)
+    # the FP32 SwiGLU product of every sampled pair within the derived bound of the epilogue
+    worst = 0.0
+    for (t, j), p in rec["pairs"].items():
+        err = np.abs(p["h_gpu"].astype(np.float64) - p["h"])
+        ratio = float(np.max(err / p["dh"]))
+        worst = max(worst, ratio)
+        assert ratio <= 1.0, f"{name}: pair ({t},{j}) h off by {ratio:.3g} of its bound"
     n_el = n_diff = 0
     for (t, j), p in rec["pairs"].items():
-        block_tie, elem_tie = requant_near_tie(p["h"], float(g_h[p["e"]]))
+        block_tie, elem_tie = requant_near_tie(p["h"], float(g_h[p["e"]]), p["dh"])
         sb = p["gpu_scales"] != p["hq_scales"]
         assert not (sb & ~block_tie).any(), f"{name}: pair ({t},{j}) block scale differs away from a near-tie"
         gc = oracle.formats.unpack_codes(p["gpu_codes"][None])[0]
@@ -229,7 +240,8 @@ def test_beam_layer(runs, name):
     err_ind = float(np.abs(got - ref_ind).max())
     fro_ind = float(np.linalg.norm(got - ref_ind) / np.linalg.norm(ref_ind))
     print(f"{name}: T={case.T}, {len(tokens)} sampled tokens ({int(same.sum())} routed as the oracle), "
-          f"{n_flag} near-tie tokens, {n_diff}/{n_el} intermediate codes at near-ties; max |out| "
+          f"{n_flag} near-tie tokens, h error at most {worst:.3g} of its bound, "
+          f"{n_diff}/{n_el} intermediate codes at near-ties; max |out| "
           f"{np.abs(ref_ops).max():.3f}; same operands: max-abs {err:.3g}, rel-Frobenius {fro:.3g}; "
           f"independent oracle: max-abs {err_ind:.3g}, rel-Frobenius {fro_ind:.3g}")
 
