@@ -35,6 +35,7 @@ from workloads import WORKLOADS, BEAM, LayerShape, activations, router_weight, e
 
 METRIC = "NVFP4 MoE-layer tokens/s; % of FP4 tensor peak (prefill) / HBM BW (decode)"
 FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense FP4 : BF16 tensor ratio
+HBM_SPEC_GBS = 7700.0               # nominal HBM3e bandwidth of a B200 (HGX figure), a second reference
 E2M1_BYTES = 0.5                    # per value
 E4M3_PER16 = 1.0 / 16.0             # block-scale bytes per value
 
@@ -254,7 +255,8 @@ def kernel_roofline(nbytes: float, flops: float, ms: float, p: dict) -> dict:
     out = {"ms": ms, "bytes": nbytes, "flops": flops, "gbs": gbs, "tflops": tflops,
            "hbm_frac": gbs / p["hbm_gbs"], "fp4_frac": tflops / burst, "fp4_frac_sustained": tflops / sustained}
     if t_bytes >= t_flops:
-        out.update({"bound": "hbm", "achieved": gbs, "peak": p["hbm_gbs"], "unit": "GB/s"})
+        out.update({"bound": "hbm", "achieved": gbs, "peak": p["hbm_gbs"], "unit": "GB/s",
+                    "frac_of_spec": gbs / HBM_SPEC_GBS})
     else:
         out.update({"bound": "tensor", "achieved": tflops, "peak": burst, "unit": "TFLOP/s"})
     out["frac"] = out["achieved"] / out["peak"]
@@ -607,6 +609,9 @@ def run_ours(args, world, rank, local):
     p = peaks()
     gu = m["gemms"]["gateup"]
     roof = {k: gu[k] for k in ("bound", "achieved", "peak", "unit", "frac")}
+    if roof["bound"] == "hbm":
+        roof["frac_of_spec"] = gu["frac_of_spec"]
+        roof["spec_peak"] = HBM_SPEC_GBS
     roof["traffic"] = stored_traffic(args.workload if not args.experts else f"{args.workload}-e{shape.E}",
                                      alg["experts_hit"])
     roof["kernel"] = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
@@ -624,7 +629,10 @@ def run_ours(args, world, rank, local):
                    "T_per_rank": T, "experts_hit": alg["experts_hit"], "parallelism": f"dp{world} (replicas)",
                    "l2": "no flush: every step streams the routed experts' weights "
                          f"({alg['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"},
-        "roofline": roof, "layer_roofline": m["layer_roofline"], "gemms": m["gemms"],
+        "roofline": roof, "layer_roofline": {**m["layer_roofline"],
+                                             "hbm_frac_of_spec": m["layer_roofline"]["hbm_frac"] * peaks()["hbm_gbs"]
+                                             / HBM_SPEC_GBS},
+        "gemms": m["gemms"],
         "stage_ms": m["stage_ms"],
         "e2e": {"value": tokens_per_second(world, T, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},

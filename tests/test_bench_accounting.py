@@ -105,6 +105,7 @@ def test_kernel_roofline_takes_the_binding_bound_and_the_burst_fp4_peak():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(1_460_368_152 / 0.2157e-3 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6546.2)
+    assert r["frac_of_spec"] == pytest.approx(r["achieved"] / bench.HBM_SPEC_GBS)
     # T = 32768 gate/up: 13.7 TFLOP in 3.30 ms -> tensor bound, scored against the burst peak
     r = bench.kernel_roofline(6.4e9, 13.74e12, 3.30, p)
     assert r["bound"] == "tensor" and r["peak"] == pytest.approx(burst)
