@@ -39,8 +39,6 @@ thread_local int32_t g_launches = 0;
 thread_local const void* g_last_status = nullptr;   // status word of this thread's latest call
 
 constexpr size_t kAlign = 256;
-// Average rows per expert segment from which the gate/up GEMM loads replicated block scales.
-constexpr int64_t kRepSfMinRows = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -826,9 +824,6 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
 
   const int grid = num_sms();
   const bool decode_cfg = T * c.topk < 32 * c.E;   // segments average fewer than 32 rows
-  // segments averaging 256 rows or more: the gate/up main loop is bound by the block-scale
-  // copies into tensor memory, which the replicated-scale variant halves
-  const bool rep_sf = T * c.topk >= kRepSfMinRows * (int64_t)c.E;
   GemmArgs g{};
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
@@ -859,7 +854,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.H = c.H;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
   g.work_counter = &f.hdr->work[0];
-  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s, rep_sf) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
   ++g_launches;
   g.b_tiles = x->wd_codes;
@@ -1428,7 +1423,6 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   ++g_launches;
   const int grid = num_sms();
   const bool decode_cfg = n_rows < 32 * (int64_t)cl.E;
-  const bool rep_sf = n_rows >= kRepSfMinRows * (int64_t)cl.E;
   GemmArgs g{};
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
@@ -1453,7 +1447,7 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   g.topk = 1;
   g.H = cl.H;
   g.work_counter = &f.hdr->work[0];
-  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s, rep_sf) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
   ++g_launches;
   g.b_tiles = x->wd_codes;
   g.sfa = f.hq_sf;

@@ -308,19 +308,6 @@ __device__ __forceinline__ uint64_t desc_sf_block(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
-// Descriptor of a 128-row x 32-byte block, no swizzle, as two 2 KB halves (bytes 0-15 of row r
-// at 16 r, bytes 16-31 at 2048 + 16 r): the tcgen05.cp.128x256b source.
-__device__ __forceinline__ uint64_t desc_sf_pair(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(2048 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
-         ((uint64_t)1 << 46);
-}
-
-// Copies a 128-row x 32-byte shared-memory block into tensor memory: lane r gets row r,
-// columns taddr .. taddr+7.
-__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t src_desc) {
-  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
-}
-
 // Instruction descriptor of kind::mxf4nvf4: A and B E2M1, UE4M3 scales, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t n) {
   return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (0u << 23) | ((128u >> 4) << 24);

@@ -63,30 +63,21 @@ constexpr int kNT = kN / 128;                       // 128-row weight tiles per 
 // K block holds 128 values instead of 256, there are no block scales (per-row activation and
 // per-channel weight scales are applied in the epilogue), and gate/up writes h in FP32 for
 // the per-row requantisation that follows.
-//
-// kRepSf (gate/up with full segments, NVFP4): every block-scale atom is loaded four times into
-// shared memory, so one 128-row source of a tcgen05.cp.128x256b holds the atom in each 32-row
-// quarter: the copy then writes tensor memory exactly as 32x128b.warpx4 copies of the same
-// atoms do (lane 32q + i gets atom row i), two atoms per instruction.  Per K block that is 6
-// copies instead of 12 (the copies bound the main loop), for 18 KB more of scale bytes from
-// L2 and 3 stages instead of 4.
-template <bool kGateUp, bool kDecode, bool kFp8, bool kRepSf = false>
+template <bool kGateUp, bool kDecode, bool kFp8>
 struct Cfg {
-  static_assert(!kRepSf || (kGateUp && !kDecode && !kFp8), "replicated scales: NVFP4 gate/up, full segments");
-  static constexpr int kStages = kRepSf ? 3 : ((kGateUp || kDecode) ? 4 : 3);
+  static constexpr int kStages = (kGateUp || kDecode) ? 4 : 3;
   static constexpr bool kStaging = !kGateUp && !kDecode;
   static constexpr uint32_t kSfCol0 = kN;                        // the accumulator first
   static constexpr uint32_t kSfColsA = kFp8 ? 0 : 16;            // 4 K steps x 4 columns
   static constexpr uint32_t kSfColsPerStage = kFp8 ? 0 : kSfColsA + 16 * kNT;
-  static constexpr int kRep = kRepSf ? 4 : 1;                    // copies of each atom in shared memory
-  static constexpr int kSfaBytes = kFp8 ? 16 : kRep * 4 * kAtomBytes;
-  static constexpr int kSfbBytes = kFp8 ? 16 : kRep * kNT * 4 * kAtomBytes;
+  static constexpr int kSfaBytes = kFp8 ? 16 : 4 * kAtomBytes;
+  static constexpr int kSfbBytes = kFp8 ? 16 : kNT * 4 * kAtomBytes;
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory columns");
 };
 
-template <bool kGateUp, bool kDecode, bool kFp8, bool kRepSf = false>
+template <bool kGateUp, bool kDecode, bool kFp8>
 struct __align__(1024) Smem {
-  using C = Cfg<kGateUp, kDecode, kFp8, kRepSf>;
+  using C = Cfg<kGateUp, kDecode, kFp8>;
   uint8_t a[C::kStages][kABytes];
   uint8_t b[C::kStages][kNT * kTileBytes];
   uint8_t sfa[C::kStages][C::kSfaBytes];
@@ -247,13 +238,13 @@ __device__ __forceinline__ void quant_store32(const float* h, float gh, float r_
   }
 }
 
-template <bool kGateUp, bool kDecode, bool kFp8, bool kRepSf = false>
+template <bool kGateUp, bool kDecode, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a32,
                 const GemmArgs p) {
-  using C = Cfg<kGateUp, kDecode, kFp8, kRepSf>;
+  using C = Cfg<kGateUp, kDecode, kFp8>;
   constexpr int kStages = C::kStages;
-  using S = Smem<kGateUp, kDecode, kFp8, kRepSf>;
+  using S = Smem<kGateUp, kDecode, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   S& s = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
@@ -340,36 +331,18 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             break;
           }
           const int left = (p.K - kb * kBlockK) / 64;
-          const int ksteps = left < 4 ? left : 4;
-          const uint32_t sf_bytes = kFp8 ? 0u : (uint32_t)ksteps * kAtomBytes;
-          mbar_arrive_expect_tx(&s.full[stage], a_bytes + kNT * (kTileBytes + C::kRep * sf_bytes) + C::kRep * sf_bytes);
+          const uint32_t sf_bytes = kFp8 ? 0u : (uint32_t)(left < 4 ? left : 4) * kAtomBytes;
+          mbar_arrive_expect_tx(&s.full[stage], a_bytes + kNT * (kTileBytes + sf_bytes) + sf_bytes);
           tma_load_2d(s.a[stage], a_small ? (const void*)&tma_a32 : (const void*)&tma_a, &s.full[stage],
                       kb * 128, arow, pol_a);
-          if constexpr (kRepSf) {
-            // A atom of K step k, copy r at (k / 2) 4 KB + (k % 2) 2 KB + r 512; B atom of tile j
-            // and K step k, copy r at k 4 KB + j 2 KB + r 512 (the 128x256b sources)
-            for (int k = 0; k < ksteps; ++k)
-#pragma unroll
-              for (int r = 0; r < 4; ++r)
-                bulk_load(s.sfa[stage] + (k >> 1) * 4096 + (k & 1) * 2048 + r * kAtomBytes,
-                          sfa + (kb * 4 + k) * kAtomBytes, kAtomBytes, &s.full[stage], pol_a);
-          } else if constexpr (!kFp8) {
-            bulk_load(s.sfa[stage], sfa + kb * 4 * kAtomBytes, sf_bytes, &s.full[stage], pol_a);
-          }
+          if constexpr (!kFp8) bulk_load(s.sfa[stage], sfa + kb * 4 * kAtomBytes, sf_bytes, &s.full[stage], pol_a);
 #pragma unroll
           for (int j = 0; j < kNT; ++j) {
             bulk_load(s.b[stage] + j * kTileBytes, btile + ((int64_t)j * kb_count + kb) * kTileBytes, kTileBytes,
                       &s.full[stage], pol_w);
-            if constexpr (kRepSf) {
-              for (int k = 0; k < ksteps; ++k)
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                  bulk_load(s.sfb[stage] + k * 4096 + j * 2048 + r * kAtomBytes,
-                            sfb + ((int64_t)j * k64 + kb * 4 + k) * kAtomBytes, kAtomBytes, &s.full[stage], pol_w);
-            } else if constexpr (!kFp8) {
+            if constexpr (!kFp8)
               bulk_load(s.sfb[stage] + j * 4 * kAtomBytes, sfb + ((int64_t)j * k64 + kb * 4) * kAtomBytes, sf_bytes,
                         &s.full[stage], pol_w);
-            }
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -429,18 +402,11 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           const uint32_t sfb_t = sfa_t + C::kSfColsA;
           const uint32_t sa = smem_u32(s.sfa[stage]);
           const uint32_t sb = smem_u32(s.sfb[stage]);
-          if constexpr (kRepSf) {
-            // A: K steps 2c and 2c + 1 in one copy (columns 8c .. 8c + 7); B: both weight
-            // tiles of K step k in one copy (columns 8k .. 8k + 7)
-            for (int c = 0; c < (ksteps + 1) / 2; ++c) tc_cp_128x256b(sfa_t + 8 * c, desc_sf_pair(sa + c * 4096));
-            for (int k = 0; k < ksteps; ++k) tc_cp_128x256b(sfb_t + 4 * kNT * k, desc_sf_pair(sb + k * 4096));
-          } else {
-            for (int k = 0; k < ksteps; ++k) {
-              tc_cp_32x128b_x4(sfa_t + 4 * k, desc_sf_block(sa + kAtomBytes * k));
+          for (int k = 0; k < ksteps; ++k) {
+            tc_cp_32x128b_x4(sfa_t + 4 * k, desc_sf_block(sa + kAtomBytes * k));
 #pragma unroll
-              for (int j = 0; j < kNT; ++j)
-                tc_cp_32x128b_x4(sfb_t + 4 * (kNT * k + j), desc_sf_block(sb + (j * 4 + k) * kAtomBytes));
-            }
+            for (int j = 0; j < kNT; ++j)
+              tc_cp_32x128b_x4(sfb_t + 4 * (kNT * k + j), desc_sf_block(sb + (j * 4 + k) * kAtomBytes));
           }
           for (int k = 0; k < ksteps; ++k) {
             mma_nvf4(acc, desc_k_sw128(a0 + 32 * k), desc_k_sw128(b0 + 32 * k), idesc, sfa_t + 4 * k,
@@ -663,15 +629,15 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   }
 }
 
-template <bool kGateUp, bool kDecode, bool kFp8 = false, bool kRepSf = false>
+template <bool kGateUp, bool kDecode, bool kFp8 = false>
 cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a, int grid,
                         cudaStream_t stream) {
-  const size_t smem = sizeof(Smem<kGateUp, kDecode, kFp8, kRepSf>) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode, kFp8, kRepSf>,
+  const size_t smem = sizeof(Smem<kGateUp, kDecode, kFp8>) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(moe_gemm_kernel<kGateUp, kDecode, kFp8, kRepSf>, dim3(grid), dim3(kThreads), smem, stream,
-                    tma_a, tma_a32, a);
+  return launch_pdl(moe_gemm_kernel<kGateUp, kDecode, kFp8>, dim3(grid), dim3(kThreads), smem, stream, tma_a,
+                    tma_a32, a);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -701,13 +667,11 @@ static_assert(sizeof(Smem<true, true, true>) + 1024 <= 232448, "GEMM shared memo
 static_assert(sizeof(Smem<true, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 static_assert(sizeof(Smem<false, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 static_assert(sizeof(Smem<false, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<true, false, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                               int grid, bool decode, cudaStream_t stream, bool replicated_scales) {
-  if (decode) return launch_gemm<true, true>(tma_a, tma_a32, a, grid, stream);
-  return replicated_scales ? launch_gemm<true, false, false, true>(tma_a, tma_a32, a, grid, stream)
-                           : launch_gemm<true, false>(tma_a, tma_a32, a, grid, stream);
+                               int grid, bool decode, cudaStream_t stream) {
+  return decode ? launch_gemm<true, true>(tma_a, tma_a32, a, grid, stream)
+                : launch_gemm<true, false>(tma_a, tma_a32, a, grid, stream);
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,

@@ -56,10 +56,8 @@ struct GemmArgs {
 // tma_a / tma_a32: the A rows with a 128-row / 32-row box (both 128 bytes wide).  Work items
 // are 256 output columns wide: n_total (2I, H) must be a multiple of 256.
 // decode: the configuration for segments that average fewer than 32 rows.
-// replicated_scales (with decode false): the block scales reach tensor memory through
-// 128x256b copies of atoms loaded four times (fewer copy instructions, more scale bytes).
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
-                               int grid, bool decode, cudaStream_t stream, bool replicated_scales = false);
+                               int grid, bool decode, cudaStream_t stream);
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                              int grid, bool decode, cudaStream_t stream);
 // The FP8 W8A8 variants: A and B are E4M3 rows of K bytes (tensor maps over K-byte rows), the
