@@ -268,6 +268,138 @@ __global__ void __launch_bounds__(kTopkThreads) router_topk_kernel(RouterArgs a)
                    a.wts + t * a.topk, a.status);
 }
 
+constexpr int kTopkWarpTokens = 8;   // tokens per CTA of the warp-per-token top-k
+
+// The group-limited top-k of one token per warp, for layouts whose groups are whole lanes
+// (group size a multiple of 8, at most 32, so E <= 256): lane l holds experts 8l .. 8l + 7.
+// The arithmetic and the tie rules are route_topk_block's: the logit is the FP64 sum of the
+// split-K parts in split order (plus the bias) rounded to FP32, the score its sigmoid, a NaN
+// score becomes -1 (raising kStatusNonFinite), a group's score is fp32(top1 + top2) of its
+// scores, equal values go to the lower group / expert index, the selected experts are listed
+// by score, and the weights divide routed_scale * s by the sum of the selected scores in slot
+// order.  No shared memory and no block barrier: 8 tokens per 256-thread CTA.
+__global__ void __launch_bounds__(256) router_topk_warp_kernel(RouterArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kTopkWarpTokens + (threadIdx.x >> 5);
+  if (t >= a.T) return;
+  const int E = a.E, G = a.n_groups, gs = E / G, L = gs / 8;   // lanes per group
+  const int e0 = lane * 8;
+  const bool valid = e0 < E;
+  float v[8];
+  bool nan = false;
+  {
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    if (valid) {
+      const int64_t step = a.T * E;
+      const double2* src = reinterpret_cast<const double2*>(a.parts + t * E + e0);
+      for (int ks = 0; ks < a.ksplit; ++ks) {
+        const double2* q = src + (int64_t)ks * (step / 2);
+        const double2 q0 = __ldcg(q), q1 = __ldcg(q + 1), q2 = __ldcg(q + 2), q3 = __ldcg(q + 3);
+        acc[0] = __dadd_rn(acc[0], q0.x);
+        acc[1] = __dadd_rn(acc[1], q0.y);
+        acc[2] = __dadd_rn(acc[2], q1.x);
+        acc[3] = __dadd_rn(acc[3], q1.y);
+        acc[4] = __dadd_rn(acc[4], q2.x);
+        acc[5] = __dadd_rn(acc[5], q2.y);
+        acc[6] = __dadd_rn(acc[6], q3.x);
+        acc[7] = __dadd_rn(acc[7], q3.y);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = -3.0f;
+      if (valid) {
+        double d = acc[i];
+        if (a.bias != nullptr) d = __dadd_rn(d, (double)a.bias[e0 + i]);
+        const float l = __double2float_rn(d);
+        if (a.logits_out != nullptr) a.logits_out[t * E + e0 + i] = l;
+        float sc = router_sigmoid(l);
+        if (sc != sc) {
+          sc = -1.0f;
+          nan = true;
+        }
+        v[i] = sc;
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, nan) && lane == 0 && a.status != nullptr) raise_status(a.status, kStatusNonFinite);
+  // the two best scores of the lane, then of its group (values only: equal values count twice)
+  float t1 = v[0], t2 = -4.0f;
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    if (v[i] > t1) {
+      t2 = t1;
+      t1 = v[i];
+    } else if (v[i] > t2) {
+      t2 = v[i];
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
+    const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
+    if (off < L) {
+      const float n2 = fmaxf(fminf(t1, o1), fmaxf(t2, o2));
+      t1 = fmaxf(t1, o1);
+      t2 = n2;
+    }
+  }
+  const int g = e0 / gs;
+  const float gscore = __fadd_rn(t1, t2);
+  // rank of the lane's group among the G groups (lane h L holds group h's score)
+  int grank = 0;
+#pragma unroll
+  for (int h = 0; h < 32; ++h) {
+    const float o = __shfl_sync(0xffffffffu, gscore, (h * L) & 31);
+    grank += (int)((h < G) & ((o > gscore) | ((o == gscore) & (h < g))));
+  }
+  const bool keep = valid && g < G && grank < a.topk_groups;
+  // the topk best experts of the kept groups, one per round (max score, then lower index)
+  uint32_t cand = keep ? 0xFFu : 0u;
+  float sum = 0.0f, my_s = 0.0f;
+  int my_e = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r < a.topk) {
+      float bv = -5.0f;
+      int be = 0x7FFFFFFF;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (((cand >> i) & 1u) && v[i] > bv) {
+          bv = v[i];
+          be = e0 + i;
+        }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be >> 3) == lane) cand &= ~(1u << (be & 7));
+      sum = __fadd_rn(sum, bv);
+      if (lane == r) {
+        my_s = bv;
+        my_e = be;
+      }
+    }
+  }
+  if (lane < a.topk) {
+    a.idx[t * a.topk + lane] = my_e;
+    a.wts[t * a.topk + lane] = __fdiv_rn(__fmul_rn(a.routed_scale, my_s), sum);
+  }
+}
+
+// The warp-per-token top-k handles layouts whose groups are whole lanes.
+static bool topk_warp_layout(const RouterArgs& a) {
+  const int gs = a.E / a.n_groups;
+  return a.E <= 256 && gs % 8 == 0 && gs <= 32;
+}
+
 static int tile_tokens(int64_t T) { return T >= kBigMinT ? kBigTM : kTM; }
 
 // K split: doubled while the grid stays within about two CTAs per SM; the cap is chosen so
@@ -334,7 +466,12 @@ cudaError_t launch_router(RouterArgs a, cudaStream_t stream) {
 }
 
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
-  router_topk_kernel<<<(unsigned)a.T, kTopkThreads, 0, stream>>>(a);
+  if (topk_warp_layout(a)) {
+    router_topk_warp_kernel<<<(unsigned)((a.T + kTopkWarpTokens - 1) / kTopkWarpTokens), 32 * kTopkWarpTokens, 0,
+                              stream>>>(a);
+  } else {
+    router_topk_kernel<<<(unsigned)a.T, kTopkThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

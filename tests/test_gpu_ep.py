@@ -285,3 +285,21 @@ def test_ep_experts_checks_received_expert_indices_on_the_device():
     for i in (0, 3):
         assert torch.equal(rows_bad[i], rows[i])
     ex.close()
+
+
+def test_ep_experts_and_combine_with_nothing_to_do():
+    """A rank that receives no row (every pair routed elsewhere) runs nvfp4moe_ep_experts on zero
+    rows: status clean, nothing written; a combine of zero tokens enqueues nothing."""
+    shape = TINY
+    ex = local_experts(shape, 16, 16)
+    amax = moe.amax(activations(4, shape, seed=91).cuda())
+    empty_codes = torch.empty((0, shape.H // 2), dtype=torch.uint8, device="cuda")
+    empty_scales = torch.empty((0, shape.H // 16), dtype=torch.uint8, device="cuda")
+    rows = moe.ep_experts(ex, empty_codes, empty_scales, torch.empty(0, dtype=torch.int32, device="cuda"),
+                          torch.empty(0, dtype=torch.float32, device="cuda"), amax)
+    assert tuple(rows.shape) == (0, shape.H)
+    assert moe.last_device_status() == moe.OK
+    out = moe.ep_combine(torch.empty((0, shape.H), dtype=torch.float32, device="cuda"),
+                         torch.empty(0, dtype=torch.int32, device="cuda"), 0, shape.topk)
+    assert tuple(out.shape) == (0, shape.H)
+    ex.close()
