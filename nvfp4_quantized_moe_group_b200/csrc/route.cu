@@ -270,8 +270,8 @@ __global__ void __launch_bounds__(kTopkThreads) router_topk_kernel(RouterArgs a)
 
 constexpr int kTopkWarpTokens = 8;   // tokens per CTA of the warp-per-token top-k
 
-// The group-limited top-k of one token per warp, for layouts whose groups are whole lanes
-// (group size a multiple of 8, at most 32, so E <= 256): lane l holds experts 8l .. 8l + 7.
+// The group-limited top-k of one token per warp, for layouts whose groups are 1, 2 or 4 whole
+// lanes (group size 8, 16 or 32, E <= 256): lane l holds experts 8l .. 8l + 7.
 // The arithmetic and the tie rules are route_topk_block's: the logit is the FP64 sum of the
 // split-K parts in split order (plus the bias) rounded to FP32, the score its sigmoid, a NaN
 // score becomes -1 (raising kStatusNonFinite), a group's score is fp32(top1 + top2) of its
@@ -394,10 +394,11 @@ __global__ void __launch_bounds__(256) router_topk_warp_kernel(RouterArgs a) {
   }
 }
 
-// The warp-per-token top-k handles layouts whose groups are whole lanes.
+// The warp-per-token top-k handles layouts whose groups are 1, 2 or 4 whole lanes (the
+// group's top-2 merge is an xor butterfly inside aligned lane groups).
 static bool topk_warp_layout(const RouterArgs& a) {
   const int gs = a.E / a.n_groups;
-  return a.E <= 256 && gs % 8 == 0 && gs <= 32;
+  return a.E <= 256 && (gs == 8 || gs == 16 || gs == 32);
 }
 
 static int tile_tokens(int64_t T) { return T >= kBigMinT ? kBigTM : kTM; }

@@ -64,7 +64,7 @@ def test_ragged_token_counts():
         _run(BEAM, T)
 
 
-# Group layouts beyond Beam's: a group size that is not a power of two (the in-group ranks
+# Group layouts beyond Beam's: group sizes that are not a power of two (the in-group ranks
 # go through shared memory instead of shuffles), one expert per group (the group score is
 # its single score), every group kept, and more than 32 selection candidates.
 ODD_SHAPES = {
@@ -76,6 +76,14 @@ ODD_SHAPES = {
                              wr_std=1.0 / 16.0, w_std=0.02),
     "64_candidates": LayerShape(H=512, I=128, E=256, n_groups=8, topk_groups=8, topk=8, routed_scale=2.5,
                                 wr_std=512 ** -0.5, w_std=0.02),
+    # groups of one and two lanes of the warp-per-token top-k, and a group of 24 experts
+    # (three lanes: not a butterfly, so the block top-k takes it)
+    "gs8": LayerShape(H=256, I=128, E=64, n_groups=8, topk_groups=3, topk=8, routed_scale=2.5,
+                      wr_std=1.0 / 16.0, w_std=0.02),
+    "gs16": LayerShape(H=256, I=128, E=128, n_groups=8, topk_groups=2, topk=6, routed_scale=2.5,
+                       wr_std=1.0 / 16.0, w_std=0.02),
+    "gs24": LayerShape(H=256, I=128, E=96, n_groups=4, topk_groups=2, topk=8, routed_scale=2.5,
+                       wr_std=1.0 / 16.0, w_std=0.02),
 }
 
 
@@ -83,3 +91,47 @@ ODD_SHAPES = {
 @pytest.mark.parametrize("T", [16, 100])
 def test_group_layouts(name, T):
     _run(ODD_SHAPES[name], T)
+
+
+@pytest.mark.parametrize("T", [16, 512])
+def test_exact_ties_go_to_the_lower_index(T):
+    """Router rows duplicated on purpose (expert 5 = expert 4; every expert of group 3 = its
+    counterpart in group 2) give bit-identical logits on every path, so the tie rules decide:
+    a token never takes expert 5 without expert 4, nor group 3 without group 2, equal experts
+    are listed lower index first, and their weights are equal.  nvfp4moe_route (FP32 logits at
+    T = 16, tensor-core logits at T = 512, both with the warp-per-token top-k), the
+    allocation-free router (FP32 logits) and, at T = 16, the forward's fused front end (its
+    block top-k) are checked on the same rows."""
+    shape = BEAM
+    cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
+                       shape.routed_scale)
+    wr = router_weight(shape).clone()
+    wr[5] = wr[4]
+    wr[96:128] = wr[64:96]
+    x = activations(T, shape, seed=17).cuda()
+    runs = {"route": moe.route(cfg, x, wr.cuda()), "route_noalloc": moe.route_noalloc(cfg, x, wr.cuda())}
+    if T <= 64:
+        from tests.test_gpu_forward import gpu_experts
+        _, dbg = moe.forward(gpu_experts(shape), x, wr.cuda(), debug=True)
+        runs["forward front end"] = (dbg["idx"], dbg["w"])
+    torch.cuda.synchronize()
+    n_tie_decided = n_pair = n_group = 0
+    for name, (idx, w) in runs.items():
+        idx, w = idx.cpu().numpy(), w.cpu().numpy()
+        for t in range(T):
+            sel = list(idx[t])
+            n_pair += 4 in sel
+            n_group += any(64 <= e < 128 for e in sel)
+            if 5 in sel:
+                assert 4 in sel, f"{name} token {t}: expert 5 without expert 4"
+                i4, i5 = sel.index(4), sel.index(5)
+                assert i5 == i4 + 1, f"{name} token {t}: equal experts 4, 5 not adjacent in index order"
+                assert w[t, i4] == w[t, i5]
+            elif 4 in sel:
+                n_tie_decided += 1
+            g3 = [e for e in sel if 96 <= e < 128]
+            for e in g3:
+                assert e - 32 in sel, f"{name} token {t}: expert {e} of group 3 without its twin {e - 32}"
+                assert sel.index(e - 32) < sel.index(e)
+    print(f"T={T}: expert 4 selected {n_pair} times ({n_tie_decided} without its twin), groups 2/3 in {n_group}")
+    assert n_pair > 0 and n_group > 0
