@@ -95,8 +95,9 @@ def test_group_layouts(name, T):
 
 @pytest.mark.parametrize("T", [16, 512])
 def test_exact_ties_go_to_the_lower_index(T):
-    """Router rows duplicated on purpose (expert 5 = expert 4; every expert of group 3 = its
-    counterpart in group 2) give bit-identical logits on every path, so the tie rules decide:
+    """Router rows duplicated on purpose (expert 5 = expert 4, scaled up so that the pair is
+    often selected; every expert of group 3 = its counterpart in group 2) give bit-identical
+    logits on every path, so the tie rules decide:
     a token never takes expert 5 without expert 4, nor group 3 without group 2, equal experts
     are listed lower index first, and their weights are equal.  nvfp4moe_route (FP32 logits at
     T = 16, tensor-core logits at T = 512, both with the warp-per-token top-k), the
@@ -106,6 +107,7 @@ def test_exact_ties_go_to_the_lower_index(T):
     cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
                        shape.routed_scale)
     wr = router_weight(shape).clone()
+    wr[4] = 3.0 * wr[4]                     # a larger logit spread: expert 4 is picked often
     wr[5] = wr[4]
     wr[96:128] = wr[64:96]
     x = activations(T, shape, seed=17).cuda()
