@@ -76,21 +76,44 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// The E2M1 codes and E4M3 scale of one 16-value block held as 8 BF16 pairs in w: 8 code
+// bytes in *c0, *c1, the scale byte returned.
+__device__ __forceinline__ uint32_t quantize_block(const uint32_t* w, float r_t, float g, uint32_t* c0,
+                                                   uint32_t* c1) {
+  // block maximum of |x| on the BF16 magnitude bits, two halves per instruction (exact)
+  uint32_t m2 = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+  for (int j = 1; j < 8; ++j) m2 = max_u16x2(m2, w[j] & 0x7FFF7FFFu);
+  const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+  float f[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    f[2 * j] = __uint_as_float(w[j] << 16);
+    f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+  float r_b;
+  const uint32_t s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
+  *c0 = cvt_e2m1x8(f);
+  *c1 = cvt_e2m1x8(f + 8);
+  return s;
+}
+
 // One CTA per row (rows_padded CTAs), min(segments, 32) warps: each warp quantises the row's
-// 512-value segments warp, warp + n_warps, ..., one 16-value block per lane.  Rows in
-// [rows, rows_padded) only write zero scales (swizzled layout padding).  The global scale is
-// read from g_in.
+// 1024-value segments warp, warp + n_warps, ..., two consecutive 16-value blocks per lane, so
+// every load and store of the warp covers one contiguous span of the row (16 code bytes per
+// lane).  Rows in [rows, rows_padded) only write zero scales (swizzled layout padding).  The
+// global scale is read from g_in.
 __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
   const float g = __ldg(a.g_in);
   if (!(g > 0.0f && g < __uint_as_float(0x7F800000u))) return;   // non-finite input: skipped
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.g_out != nullptr && a.g_out != a.g_in) *a.g_out = g;
   const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
 
-  // one warp per (row, 512-value segment): lane l takes the 16-value block 32 seg + l, so every
-  // load, code store and accumulator store of the warp covers one contiguous span of the row;
-  // lanes 4k .. 4k+3 hold the 4 block scales of one 32-bit scale word
+  // lanes 2k, 2k+1 hold the 4 block scales of one 32-bit scale word
   const int blocks_per_row = (int)(a.cols >> 4);
-  const int segs_per_row = (blocks_per_row + 31) >> 5;
+  const int segs_per_row = (blocks_per_row + 63) >> 6;
   const int lane = threadIdx.x & 31;
   const int n_warps = blockDim.x >> 5;
   const int64_t r = blockIdx.x;
@@ -102,58 +125,41 @@ __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
     my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
   }
   for (int seg = threadIdx.x >> 5; seg < segs_per_row; seg += n_warps) {
-    const int64_t b = (int64_t)seg * 32 + lane;
-    // lanes past the row's last block stay for the shuffles; groups of 4 lanes are active or
-    // idle together (cols % 64 == 0)
+    const int b = seg * 64 + 2 * lane;          // first of the lane's two blocks
+    // lanes past the row's last block stay for the shuffle; lane pairs are active or idle
+    // together (cols % 64 == 0)
     const bool active = b < blocks_per_row;
     const bool live = active && r < a.rows;
 
     if (a.zero_out != nullptr && live) {
-      float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + b * 16);
+      float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + (int64_t)b * 16);
       const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-  #pragma unroll
-      for (int i = 0; i < 4; ++i) z[i] = zero;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) z[i] = zero;
     }
 
-    uint32_t s = 0, c0 = 0, c1 = 0;
+    uint32_t s2 = 0;                            // the two scale bytes of the lane
+    uint4 codes = make_uint4(0, 0, 0, 0);
     if (live) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + b * 16);
-      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float f[16];
-      // block maximum of |x| on the BF16 magnitude bits, two halves per instruction (exact;
-      // >= 0x7F80: Inf or NaN)
-      uint32_t m2 = w[0] & 0x7FFF7FFFu;
-  #pragma unroll
-      for (int j = 1; j < 8; ++j) m2 = max_u16x2(m2, w[j] & 0x7FFF7FFFu);
-      const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
-  #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        f[2 * j] = __uint_as_float(w[j] << 16);
-        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-      }
-      float r_b;
-      s = block_scale(__uint_as_float(mb << 16), r_t, g, &r_b);
-  #pragma unroll
-      for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], r_b);
-      c0 = cvt_e2m1x8(f);
-      c1 = cvt_e2m1x8(f + 8);
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + (int64_t)b * 16);
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1), v2 = __ldg(src + 2), v3 = __ldg(src + 3);
+      const uint32_t w0[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      const uint32_t w1[8] = {v2.x, v2.y, v2.z, v2.w, v3.x, v3.y, v3.z, v3.w};
+      const uint32_t sa = quantize_block(w0, r_t, g, &codes.x, &codes.y);
+      const uint32_t sb = quantize_block(w1, r_t, g, &codes.z, &codes.w);
+      s2 = sa | (sb << 8);
     }
-    // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes 4k)
-    const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
-    const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
-    const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
-    const uint32_t sc = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
-    const bool word_lane = active && (lane & 3) == 0;
+    // the 32-bit scale word of this lane's group of 4 blocks (valid in even lanes)
+    const uint32_t sc = s2 | (__shfl_down_sync(0xffffffffu, s2, 1) << 16);
+    const bool word_lane = active && (lane & 1) == 0;
 
     if (r < a.rows) {
-      if (a.codes != nullptr && active)
-        reinterpret_cast<uint2*>(a.codes + r * (a.cols >> 1))[b] = make_uint2(c0, c1);
+      if (a.codes != nullptr && active) reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1))[b >> 1] = codes;
       if (a.seg_codes != nullptr) {
-        // every lane writes its block to all of the token's segment rows
+        // every lane writes its blocks to all of the token's segment rows
         for (int j = 0; j < a.topk; ++j) {
           const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
-          if (active) reinterpret_cast<uint2*>(a.seg_codes + row * (a.cols >> 1))[b] = make_uint2(c0, c1);
+          if (active) reinterpret_cast<uint4*>(a.seg_codes + row * (a.cols >> 1))[b >> 1] = codes;
           if (word_lane) *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, b, a.n_col_tiles)) = sc;
         }
       }
@@ -200,7 +206,7 @@ cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream) {
       return cudaMemcpyAsync(a.g_out, a.g_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
     return cudaSuccess;
   }
-  const int segs = (int)(((a.cols >> 4) + 31) >> 5);
+  const int segs = (int)(((a.cols >> 4) + 63) >> 6);
   const int warps = segs < 32 ? segs : 32;
   quantize_kernel<<<(unsigned)a.rows_padded, 32 * warps, 0, stream>>>(a);
   return cudaGetLastError();
