@@ -54,11 +54,15 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_experts_decode_traffic.txt")
+
+
 def stored_traffic(workload: str, experts_hit: int):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary, scaled to
-    this run's experts hit (traffic is proportional to the weight tiles streamed); None when
-    the summary was taken on other kernel sources or another workload."""
-    path = os.path.join(ROOT, "profiles", "gemm_gateup_traffic.txt")
+    """DRAM bytes per launch of the decode layer's grouped-GEMM launch (both GEMMs) from the
+    committed ncu summary, scaled to this run's experts hit (traffic is proportional to the
+    weight tiles streamed); None when the summary was taken on other kernel sources or another
+    workload."""
+    path = TRAFFIC_FILE
     if not os.path.exists(path):
         return None
     vals = {}
@@ -483,10 +487,24 @@ def measure_workload(moe, ex, shape: LayerShape, wl, x, wr, bias, steps: int, wa
         torch.cuda.nvtx.range_push("timed")
         elapsed = timed_steps(lambda k: moe.forward(ex, x, wr, bias, out=out, ws=ws), steps, world)
         torch.cuda.nvtx.range_pop()
-    # the GEMM durations, from a second region of the same steps with events around both GEMMs
+    # the grouped GEMMs' durations, from a second region of the same steps with events around
+    # them: with short segments one launch runs both (the GATEUP events bracket it, DOWN is
+    # empty), else two launches, each bracketed
+    one_launch = T * shape.topk < 32 * shape.E          # the library's rule (nvfp4moe_debug.separate_gemms)
     timers = [moe.StageTimer(("gateup", "down")) for _ in range(steps)]
     ev_elapsed = timed_steps(lambda k: moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=timers[k]), steps, world)
     gemm_ms = {n: max_over_ranks(statistics.mean(t.stage_ms()[n] for t in timers), world) for n in ("gateup", "down")}
+    sep_elapsed = None
+    if one_launch:
+        experts_ms = gemm_ms["gateup"] + gemm_ms["down"]
+        # for context: the same GEMMs as two launches, each timed
+        timers = [moe.StageTimer(("gateup", "down")) for _ in range(steps)]
+        for k in range(warmup):
+            moe.forward(ex, x, wr, bias, out=out, ws=ws, separate_gemms=True)
+        sep_elapsed = timed_steps(lambda k: moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=timers[k],
+                                                        separate_gemms=True), steps, world)
+        gemm_ms = {n: max_over_ranks(statistics.mean(t.stage_ms()[n] for t in timers), world)
+                   for n in ("gateup", "down")}
     full = [moe.StageTimer() for _ in range(min(steps, 20))]
     for t in full:
         moe.forward(ex, x, wr, bias, out=out, ws=ws, timer=t)
@@ -499,33 +517,49 @@ def measure_workload(moe, ex, shape: LayerShape, wl, x, wr, bias, steps: int, wa
     ms = elapsed / steps
     burst, sustained = fp4_peaks(p)
     layer_s = ms / 1e3
-    return {
+    res = {
         "workload": wl.describe(), "T_per_rank": T, "experts_hit": alg["experts_hit"], "ms_per_step": ms,
         "value": tokens_per_second(world, T, steps, elapsed), "unit": "tokens/s",
         "gpu_launches_per_step": launches, "alg": alg, "stage_ms": stage,
+        "gemm_region_ms_per_step": ev_elapsed / steps,
         "gemms": {"gateup": kernel_roofline(alg["gateup_bytes"], alg["gateup_flops"], gemm_ms["gateup"], p),
                   "down": kernel_roofline(alg["down_bytes"], alg["down_flops"], gemm_ms["down"], p)},
-        "gemm_region_ms_per_step": ev_elapsed / steps,
+    }
+    if one_launch:
+        res["experts_kernel"] = kernel_roofline(alg["gateup_bytes"] + alg["down_bytes"],
+                                                alg["gateup_flops"] + alg["down_flops"], experts_ms, p)
+        res["dominant"] = {**res["experts_kernel"], "kernel": EXPERTS_KERNEL}
+        res["gemms"]["note"] = (f"the same step with the two GEMMs as two launches (nvfp4moe_debug.separate_gemms), "
+                                f"each timed with CUDA events: {sep_elapsed / steps:.4f} ms per step")
+    else:
+        res["dominant"] = {**res["gemms"]["gateup"], "kernel": GATEUP_KERNEL}
+    res.update({
         "layer_roofline": {"bytes_per_step": alg["layer_bytes"], "flops_per_step": alg["flops"],
                            "hbm_frac": alg["layer_bytes"] / layer_s / (p["hbm_gbs"] * 1e9),
                            "fp4_frac": alg["flops"] / layer_s / (burst * 1e12),
                            "fp4_frac_sustained": alg["flops"] / layer_s / (sustained * 1e12),
                            "tflops": alg["flops"] / layer_s / 1e12},
         "_ws": ws, "_out": out,
-    }
+    })
+    return res
+
+
+EXPERTS_KERNEL = ("moe_gemm_kernel<fused, decode> (one persistent launch of both tcgen05 mxf4nvf4 grouped GEMMs: "
+                  "gate/up + SwiGLU + requant, down + combine)")
+GATEUP_KERNEL = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
 
 
 def config_entry(m: dict, wl) -> dict:
     """The JSON object of one compute-heavy config: its step time and throughput, stage times,
-    the roofline of its dominant kernel (the gate/up GEMM, two thirds of the FLOPs and weight
-    bytes) and of the down GEMM, and the whole layer against both rooflines."""
-    g = m["gemms"]
+    the roofline of its dominant kernel (with full segments the gate/up GEMM, two thirds of the
+    FLOPs and weight bytes; with short ones the launch that runs both GEMMs), both GEMMs'
+    rooflines, and the whole layer against both rooflines."""
+    k = m["dominant"]
     return {"workload": m["workload"], "T_per_rank": m["T_per_rank"], "experts_hit": m["experts_hit"],
             "ms_per_step": m["ms_per_step"], "value": m["value"], "unit": "tokens/s",
-            "stage_ms": m["stage_ms"], "roofline": {**{k: g["gateup"][k] for k in
-                                                       ("bound", "achieved", "peak", "unit", "frac")},
-                                                    "kernel": "moe_gemm_kernel<gate/up>", "traffic": None},
-            "gemms": g, "layer_roofline": m["layer_roofline"],
+            "stage_ms": m["stage_ms"], "roofline": {**{n: k[n] for n in ("bound", "achieved", "peak", "unit", "frac")},
+                                                    "kernel": k["kernel"], "traffic": None},
+            "gemms": m["gemms"], "layer_roofline": m["layer_roofline"],
             "l2": "no flush: every step streams the routed experts' weights "
                   f"({m['alg']['layer_bytes'] / 1e9:.2f} GB > 126 MB L2)"}
 
@@ -607,15 +641,15 @@ def run_ours(args, world, rank, local):
                                "clocks": qclk.summary()}
 
     p = peaks()
-    gu = m["gemms"]["gateup"]
+    gu = m["dominant"]
     roof = {k: gu[k] for k in ("bound", "achieved", "peak", "unit", "frac")}
     if roof["bound"] == "hbm":
         roof["frac_of_spec"] = gu["frac_of_spec"]
         roof["spec_peak"] = HBM_SPEC_GBS
     roof["traffic"] = stored_traffic(args.workload if not args.experts else f"{args.workload}-e{shape.E}",
                                      alg["experts_hit"])
-    roof["kernel"] = "moe_gemm_kernel<gate/up> (tcgen05 mxf4nvf4 grouped GEMM + SwiGLU + requant)"
-    roof["duration_source"] = (f"CUDA events around the gate/up launch of each of {args.steps} steps of a second "
+    roof["kernel"] = gu["kernel"]
+    roof["duration_source"] = (f"CUDA events around the GEMM launch of each of {args.steps} steps of a second "
                                "timed region right after the headline one (same inputs), on the launching stream")
     roof["peak_source"] = (f"{p['source']} hbm_gbs (a copy bandwidth: a read-only stream can exceed it slightly)"
                            if roof["bound"] == "hbm"
@@ -633,6 +667,7 @@ def run_ours(args, world, rank, local):
                                              "hbm_frac_of_spec": m["layer_roofline"]["hbm_frac"] * peaks()["hbm_gbs"]
                                              / HBM_SPEC_GBS},
         "gemms": m["gemms"],
+        **({"experts_kernel": m["experts_kernel"]} if "experts_kernel" in m else {}),
         "stage_ms": m["stage_ms"],
         "e2e": {"value": tokens_per_second(world, T, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2},

@@ -159,18 +159,18 @@ NVFP4MOE_API int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, 
  * added by a 3-level FP32 tree); these partial sums, the split-K parts and the bias are
  * added in FP64 and the logit is rounded to FP32 once, so
  *   |logit - exact| <= 32 * 2^-24 * sum_h |x_h W_eh| + 2^-24 |logit| (+ FP64 rounding).
- * Logits, T > 64: exact integer arithmetic on the tensor cores.  Token row x_t and expert
- * row W_e are scaled by powers of two to 30-bit fixed point (e_x, e_W: the binary exponents
- * with max|x_t| < 2^e_x, max|W_e| < 2^e_W) and rounded to integers, split into four int8
- * digits each, and the 13 most significant digit-pair products are summed in int32 (exact);
- * the classes, split-K parts and bias are added in FP64 and the logit is rounded to FP32
- * once, so
- *   |logit - exact| <= 2^-24 |logit| + 2^(e_x - 31) sum_h |W_eh| + 2^(e_W - 31) sum_h |x_h|
- *                      + H 2^(e_x + e_W - 36)
- * (the first two terms are the fixed-point roundings; the last covers the dropped digit
- * pairs, the product of the two roundings and the FP64 additions); for Beam's shapes this
- * is about 200 times below the FP32 bound.  A token or expert row with a non-finite element
- * makes its logits NaN.
+ * Logits, T > 64: integer arithmetic on the tensor cores.  Token row x_t is scaled by a
+ * power of two to 22-bit fixed point and expert row W_e to 30-bit fixed point (e_x, e_W: the
+ * binary exponents with max|x_t| < 2^e_x, max|W_e| < 2^e_W) and rounded to integers (a BF16
+ * element within 2^14 of its row's largest is exact), split into three and four int8 digits,
+ * and the 9 most significant digit-pair products are summed in int32 (exact); the classes,
+ * split-K parts and bias are added in FP64 and the logit is rounded to FP32 once, so
+ *   |logit - exact| <= 2^-24 |logit| + sum_h |x_h - x'_h| |W_eh| + sum_h |x_h| |W_eh - W'_eh|
+ *                      + H 2^(e_x + e_W - 28)
+ * where x', W' are the fixed-point values (the two sums are at most 2^(e_x - 23) sum_h |W_eh|
+ * and 2^(e_W - 31) sum_h |x_h|; the last term covers the dropped digit pairs, the product of
+ * the two roundings and the FP64 additions); for Beam's shapes this is below the FP32 bound.
+ * A token or expert row with a non-finite element makes its logits NaN.
  * Scores are 1 / (1 + expf(-logit)) in FP32.  nvfp4moe_forward uses the same arithmetic
  * and bounds (for T <= 64 in its fused front-end kernel).  A NaN logit raises
  * NVFP4MOE_ERR_NONFINITE in the status word and ranks below every finite score. */
@@ -317,6 +317,13 @@ typedef struct {
                                   barrier, so every CTA's wait there runs out (a timeout that
                                   needs no fault); NVFP4MOE_ERR_ARG when the call does not take
                                   the fused front end, or c < 0 */
+  int32_t separate_gemms;      /* 0 (normal use): when the expert segments average fewer than
+                                  32 rows (T * topk < 32 * E), the NVFP4 forward calls run the
+                                  gate/up and the down GEMM in one persistent launch (each down
+                                  tile starts once the gate/up tiles of its rows are done),
+                                  bracketed by the GATEUP stage events, DOWN empty; otherwise
+                                  two launches.  Nonzero: always two launches, which the GATEUP
+                                  and DOWN events time apart */
 } nvfp4moe_debug;
 
 NVFP4MOE_API size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max);

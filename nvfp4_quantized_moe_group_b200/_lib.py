@@ -55,7 +55,8 @@ class Debug(ctypes.Structure):
                 + [("logits", ctypes.c_void_p), ("x_norm", ctypes.c_void_p), ("xq8_codes", ctypes.c_void_p),
                    ("xq8_scales", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("h_f32", ctypes.c_void_p),
                    ("wait_limit_us", ctypes.c_uint32),
-                   ("inject_skip_arrive", ctypes.c_int32)])
+                   ("inject_skip_arrive", ctypes.c_int32),
+                   ("separate_gemms", ctypes.c_int32)])
 
 
 class Fp8ExpertTensors(ctypes.Structure):
@@ -467,12 +468,13 @@ def forward_residual(experts: Experts, h: torch.Tensor, gamma: torch.Tensor, eps
 def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None,
             out: torch.Tensor | None = None, ws: torch.Tensor | None = None, debug: bool = False, stream=None,
             timer: StageTimer | None = None, wait_limit_us: int = 0, inject_skip_arrive: int = 0,
-            debug_h: bool = False):
+            debug_h: bool = False, separate_gemms: bool = False):
     """moe_forward(hidden, experts) -> out [T, H] bf16 (and a dict of intermediates if debug).
     ``timer``: a StageTimer whose events are recorded around each stage.  ``wait_limit_us``
     and ``inject_skip_arrive``: the failure-detection fields of nvfp4moe_debug (a bounded-wait
     limit, and the test hook that makes one front-end CTA skip a grid-barrier arrival).
-    ``debug_h``: with debug, also the FP32 SwiGLU product of every pair (h_f32, [T*topk, I])."""
+    ``debug_h``: with debug, also the FP32 SwiGLU product of every pair (h_f32, [T*topk, I]).
+    ``separate_gemms``: run the gate/up and down GEMMs as two launches instead of one."""
     cfg = experts.cfg
     specs = _layer_specs(cfg, x, w_router, bias)
     T, H = x.shape
@@ -491,11 +493,12 @@ def forward(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: tor
         if dbg is None:
             dbg = Debug()
         dbg.events = ctypes.cast(timer.array, ctypes.POINTER(ctypes.c_void_p))
-    if wait_limit_us or inject_skip_arrive:
+    if wait_limit_us or inject_skip_arrive or separate_gemms:
         if dbg is None:
             dbg = Debug()
         dbg.wait_limit_us = int(wait_limit_us)
         dbg.inject_skip_arrive = int(inject_skip_arrive)
+        dbg.separate_gemms = int(bool(separate_gemms))
     st = lib().nvfp4moe_forward(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(out),
                                 ctypes.byref(dbg) if dbg is not None else None, _ptr(ws), ws.numel(),
                                 _stream(stream))

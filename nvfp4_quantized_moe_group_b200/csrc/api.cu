@@ -39,6 +39,10 @@ thread_local int32_t g_launches = 0;
 thread_local const void* g_last_status = nullptr;   // status word of this thread's latest call
 
 constexpr size_t kAlign = 256;
+// Fused GEMM launch: gate/up items claimed between an expert's last gate/up item and its first
+// down item, per SM of the grid (about the items a CTA has in flight, so that the down items
+// rarely wait for h).
+constexpr int kFusedLagPerSm = 4;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -87,7 +91,7 @@ QuantWs carve_quant(void* ws) {
 }
 
 // Scratch of the integer tensor-core router (T >= kRouterTcMinT): digit planes of the expert
-// rows and the row exponents.  The token rows' planes (4 T H bytes) go to a buffer the caller
+// rows and the row exponents.  The token rows' planes (3 T H bytes) go to a buffer the caller
 // names when it is large enough (in the forward, the expert-segment input buffer, which is
 // written only afterwards), else to their own.
 struct RouterTcWs {
@@ -100,8 +104,9 @@ struct RouterTcWs {
 RouterTcWs carve_router_tc(Carver& c, const nvfp4moe_cfg& cfg, int64_t T, size_t shared_bytes) {
   RouterTcWs r;
   if (T < kRouterTcMinT) return r;
-  r.w_digits = c.take<uint8_t>((size_t)4 * cfg.E * cfg.H);
-  if (shared_bytes < (size_t)4 * T * cfg.H) r.x_digits = c.take<uint8_t>((size_t)4 * T * cfg.H);
+  r.w_digits = c.take<uint8_t>((size_t)kRouterWDigits * cfg.E * cfg.H);
+  if (shared_bytes < (size_t)kRouterXDigits * T * cfg.H)
+    r.x_digits = c.take<uint8_t>((size_t)kRouterXDigits * T * cfg.H);
   r.x_exp = c.take<int32_t>(T);
   r.w_exp = c.take<int32_t>(cfg.E);
   return r;
@@ -127,8 +132,8 @@ RouteWs carve_route(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   RouteWs r;
   r.hdr = c.take<WsHeader>(1);
   r.parts = c.take<double>(router_parts_elems(T, cfg.E, cfg.H));
-  r.x_digits = T >= kRouterTcMinT ? c.take<uint8_t>((size_t)4 * T * cfg.H) : nullptr;
-  r.tc = carve_router_tc(c, cfg, T, T >= kRouterTcMinT ? (size_t)4 * T * cfg.H : 0);
+  r.x_digits = T >= kRouterTcMinT ? c.take<uint8_t>((size_t)kRouterXDigits * T * cfg.H) : nullptr;
+  r.tc = carve_router_tc(c, cfg, T, T >= kRouterTcMinT ? (size_t)kRouterXDigits * T * cfg.H : 0);
   r.bytes = c.off;
   return r;
 }
@@ -141,6 +146,7 @@ int64_t rows_capacity(const nvfp4moe_cfg& cfg, int64_t T) {
 
 struct ForwardWs {
   WsHeader* hdr;
+  int32_t* dep;            // per 128-row tile: gate/up epilogue warps done (fused GEMM launch)
   uint32_t* partials;
   float* g_x;
   double* parts;
@@ -162,7 +168,7 @@ struct ForwardWs {
   uint8_t* hq_codes;
   uint8_t* hq_sf;
   uint16_t* x_norm;        // residual forward: the normalised layer input
-  RouterTcWs tc;           // token-row digit planes alias a_codes (rows_cap H / 2 >= 4 T H)
+  RouterTcWs tc;           // token-row digit planes alias a_codes (when rows_cap H / 2 >= 3 T H)
   int64_t rows_cap;
   size_t bytes;
 };
@@ -174,6 +180,7 @@ ForwardWs carve_forward(void* ws, const nvfp4moe_cfg& cfg, int64_t T) {
   const int64_t n_chunks = (T + kPermChunkTokens - 1) / kPermChunkTokens;
   f.rows_cap = rows_capacity(cfg, T);
   f.hdr = c.take<WsHeader>(1);
+  f.dep = c.take<int32_t>(f.rows_cap / kBlockM);   // right after the header: zeroed with it
   const int n_part = router_amax_partials(T, cfg.E, cfg.H);
   f.partials = c.take<uint32_t>(n_part > kMaxAmaxPartials ? n_part : kMaxAmaxPartials);
   f.g_x = c.take<float>(1);
@@ -226,7 +233,7 @@ struct ForwardFp8Ws {
   float* h32;           // [rows_cap][I]
   uint8_t* hq;          // [rows_cap][I] E4M3
   float* h_scale;       // [rows_cap]
-  RouterTcWs tc;        // token-row digit planes alias a_codes (rows_cap H >= 4 T H)
+  RouterTcWs tc;        // token-row digit planes alias a_codes (when rows_cap H >= 3 T H)
   int64_t rows_cap;
   size_t bytes;
 };
@@ -691,10 +698,16 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     return NVFP4MOE_ERR_CUDA;
 
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
-  // status word and grid-barrier counter
-  // status word, front-end barrier and the two GEMM work counters
-  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  // status word, front-end barrier, the GEMM work counters and the row-tile counters that follow
+  // the header
+  if (reset_status(f.hdr, (int)(sizeof(WsHeader) / 4 + f.rows_cap / kBlockM), s) != cudaSuccess)
+    return NVFP4MOE_ERR_CUDA;
   const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
+  const bool decode_cfg = T * c.topk < 32 * c.E;   // segments average fewer than 32 rows
+  // two GEMM launches (else one for both, see below); the gate/up launch then zeroes the FP32
+  // accumulator beside its work (its HBM traffic leaves room at large T), else the quantiser
+  // or the front end does
+  const bool separate = !decode_cfg || (dbg != nullptr && dbg->separate_gemms != 0);
 
   if (front_supported(T, c.E, c.H)) {
     // small T: route, amax, grouping and quantise-scatter in one cooperative launch
@@ -791,7 +804,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
 
     // quantise x and write each token's row into its expert-segment rows (zeroes the
-    // accumulator alongside); the token-major copy is only kept for the debug export
+    // accumulator alongside when one launch runs both GEMMs); the token-major copy is only
+    // kept for the debug export
     QuantizeArgs q{};
     q.x = static_cast<const uint16_t*>(hidden_bf16);
     q.rows = T;
@@ -805,7 +819,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     q.swizzled = 1;
     q.n_col_tiles = c.H / 64;
     q.g_out = f.g_x;
-    q.zero_out = f.acc;
+    q.zero_out = separate ? nullptr : f.acc;
     q.status = &f.hdr->status;
     q.idx = f.idx;
     q.inv = f.inv;
@@ -823,7 +837,6 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   }
 
   const int grid = num_sms();
-  const bool decode_cfg = T * c.topk < 32 * c.E;   // segments average fewer than 32 rows
   GemmArgs g{};
   g.b_tiles = x->w13_codes;
   g.sfa = f.a_sf;
@@ -852,22 +865,45 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   g.alpha_down = x->alpha_down;
   g.topk = c.topk;
   g.H = c.H;
-  ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
   g.work_counter = &f.hdr->work[0];
-  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
-  ++g_launches;
-  g.b_tiles = x->wd_codes;
-  g.sfa = f.hq_sf;
-  g.sfb = x->wd_sf;
-  g.K = c.I;
-  g.n_total = c.H;
-  g.h_dbg = nullptr;
-  ev.mark(NVFP4MOE_STAGE_DOWN, 0);
-  g.work_counter = &f.hdr->work[1];
-  if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  ev.mark(NVFP4MOE_STAGE_DOWN, 1);
-  ++g_launches;
+  GemmArgs gd = g;
+  gd.b_tiles = x->wd_codes;
+  gd.sfa = f.hq_sf;
+  gd.sfb = x->wd_sf;
+  gd.K = c.I;
+  gd.n_total = c.H;
+  gd.h_dbg = nullptr;
+  // one launch for both GEMMs when segments are short (weight streaming dominates and the
+  // boundary between two launches costs a few per cent); with full segments the down GEMM's
+  // FP32 reductions, bound by the L2's reduction rate, slow the gate/up loads they would run
+  // beside, and two launches are faster
+  if (separate) {
+    ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
+    GemmArgs gz = g;
+    if (!front_supported(T, c.E, c.H)) {
+      gz.zero_acc = f.acc;
+      gz.zero_acc_elems = T * c.H;
+    }
+    if (launch_gemm_gateup(tma_a, tma_a32, gz, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
+    ++g_launches;
+    ev.mark(NVFP4MOE_STAGE_DOWN, 0);
+    gd.work_counter = &f.hdr->work[1];
+    if (launch_gemm_down(tma_h, tma_h32, gd, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_DOWN, 1);
+    ++g_launches;
+  } else {
+    // both GEMMs in one launch: an expert's down items are claimed kFusedLagPerSm * grid
+    // gate/up items after its last gate/up item
+    ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
+    if (launch_gemm_fused(tma_a, tma_a32, tma_h, tma_h32, g, gd, f.dep, kFusedLagPerSm * grid, grid, s) !=
+        cudaSuccess)
+      return NVFP4MOE_ERR_CUDA;
+    ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
+    ev.mark(NVFP4MOE_STAGE_DOWN, 0);
+    ev.mark(NVFP4MOE_STAGE_DOWN, 1);
+    ++g_launches;
+  }
 
   if (acc_out == nullptr) {
     FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,

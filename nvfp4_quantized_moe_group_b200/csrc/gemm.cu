@@ -53,20 +53,27 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kN = 256;
 constexpr int kNT = kN / 128;                       // 128-row weight tiles per item
 
+// kMode: which GEMM the launch runs.  kModeFused runs both in one persistent launch (used
+// with short segments): the gate/up items and the down items share the work counter, and a
+// down item waits until every gate/up item of its 128-row tile has stored its part of h
+// (per-tile counters), so no CTA idles at a boundary between two launches.
+enum : int { kModeDown = 0, kModeGateUp = 1, kModeFused = 2 };
+
 // kDecode: segments average fewer than 32 rows.  The epilogues then read the whole
 // accumulator before any arithmetic (gate/up) and reduce straight from the 16x256b register
 // layout (down), and the down GEMM keeps 4 stages.  With full segments the gate/up epilogue
 // frees the accumulator after its first 32-feature chunk, and the down GEMM stages 32-column
 // row pieces in shared memory for bulk reductions (3 stages): both measured faster there.
+// The fused launch keeps 4 stages and reduces from registers in both regimes.
 //
 // kFp8: the FP8 W8A8 variant (E4M3 x E4M3 with FP32 accumulation, kind::f8f6f4): a 128-byte
 // K block holds 128 values instead of 256, there are no block scales (per-row activation and
 // per-channel weight scales are applied in the epilogue), and gate/up writes h in FP32 for
 // the per-row requantisation that follows.
-template <bool kGateUp, bool kDecode, bool kFp8>
+template <int kMode, bool kDecode, bool kFp8>
 struct Cfg {
-  static constexpr int kStages = (kGateUp || kDecode) ? 4 : 3;
-  static constexpr bool kStaging = !kGateUp && !kDecode;
+  static constexpr int kStages = (kMode != kModeDown || kDecode) ? 4 : 3;
+  static constexpr bool kStaging = kMode == kModeDown && !kDecode;
   static constexpr uint32_t kSfCol0 = kN;                        // the accumulator first
   static constexpr uint32_t kSfColsA = kFp8 ? 0 : 16;            // 4 K steps x 4 columns
   static constexpr uint32_t kSfColsPerStage = kFp8 ? 0 : kSfColsA + 16 * kNT;
@@ -75,9 +82,9 @@ struct Cfg {
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory columns");
 };
 
-template <bool kGateUp, bool kDecode, bool kFp8>
+template <int kMode, bool kDecode, bool kFp8>
 struct __align__(1024) Smem {
-  using C = Cfg<kGateUp, kDecode, kFp8>;
+  using C = Cfg<kMode, kDecode, kFp8>;
   uint8_t a[C::kStages][kABytes];
   uint8_t b[C::kStages][kNT * kTileBytes];
   uint8_t sfa[C::kStages][C::kSfaBytes];
@@ -183,6 +190,59 @@ __device__ __forceinline__ Work decode_work(const int* prefix, int w, int E, int
   return k;
 }
 
+// The fused schedule.  The gate/up items keep their order (expert-major, then column tile,
+// then row tile); expert e's down items (same order) follow as one block after the first
+// min(G(e + 1) + lag, NG) gate/up items, G(e) counting the gate/up items of the experts before
+// e and NG all of them.  Every gate/up item of an expert thus precedes its down items by at
+// least lag claims (except for the last experts, whose down items close the list), so the
+// dependency waits stay rare.  (Spreading the down items evenly among the gate/up items
+// measured 6 % slower at decode.)
+struct Sched {
+  int base;      // global tile number of the launch's first row tile
+  int ntn_g;     // gate/up items per row tile
+  int ntn_d;     // down items per row tile
+  int NG;        // gate/up items
+  int lag;
+  int E;
+};
+
+__device__ __forceinline__ Work decode_fused(const int* prefix, const int* counts, const Sched& sc, int w,
+                                             bool* gu) {
+  // start of expert e's down block: min(G(e + 1) + lag, NG) + D(e)
+  auto start = [&](int e) {
+    const int g1 = (__ldg(prefix + e + 1) - sc.base) * sc.ntn_g + sc.lag;
+    return (g1 < sc.NG ? g1 : sc.NG) + (__ldg(prefix + e) - sc.base) * sc.ntn_d;
+  };
+  int lo = -1, hi = sc.E;     // start(lo) <= w < start(hi); lo = -1: before every down block
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (start(mid) <= w) lo = mid; else hi = mid;
+  }
+  int g = w;
+  if (lo >= 0) {
+    const int s0 = start(lo);
+    const int p_lo = __ldg(prefix + lo);
+    const int mt_e = __ldg(prefix + lo + 1) - p_lo;
+    if (w < s0 + mt_e * sc.ntn_d) {
+      *gu = false;
+      return decode_work(prefix, (p_lo - sc.base) * sc.ntn_d + (w - s0) + sc.base * sc.ntn_d, sc.E, sc.ntn_d,
+                         counts);
+    }
+    g = w - (p_lo + mt_e - sc.base) * sc.ntn_d;   // the down items before w: experts 0 .. lo
+  }
+  *gu = true;
+  return decode_work(prefix, g + sc.base * sc.ntn_g, sc.E, sc.ntn_g, counts);
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Orders this thread's generic-proxy global accesses with its async-proxy (TMA, bulk copy) ones.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 __device__ __forceinline__ void set_abort(int* flag, uint32_t* status) {
   raise_status(status, kStatusTimeout);
   *reinterpret_cast<volatile int*>(flag) = 1;
@@ -238,17 +298,20 @@ __device__ __forceinline__ void quant_store32(const float* h, float gh, float r_
   }
 }
 
-template <bool kGateUp, bool kDecode, bool kFp8>
+template <int kMode, bool kDecode, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a32,
-                const GemmArgs p) {
-  using C = Cfg<kGateUp, kDecode, kFp8>;
+                const __grid_constant__ CUtensorMap tma_h, const __grid_constant__ CUtensorMap tma_h32,
+                const __grid_constant__ GemmArgs pg, const __grid_constant__ GemmArgs pd, int* dep, int lag) {
+  using C = Cfg<kMode, kDecode, kFp8>;
   constexpr int kStages = C::kStages;
-  using S = Smem<kGateUp, kDecode, kFp8>;
+  using S = Smem<kMode, kDecode, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   S& s = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the fields every item shares (status, grouping tables, work counter)
+  const GemmArgs& P0 = kMode == kModeDown ? pd : pg;
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
@@ -266,8 +329,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tma_a);
-    prefetch_tmap(&tma_a32);
+    if (kMode != kModeDown) {
+      prefetch_tmap(&tma_a);
+      prefetch_tmap(&tma_a32);
+    }
+    if (kMode != kModeGateUp) {
+      prefetch_tmap(&tma_h);
+      prefetch_tmap(&tma_h32);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&s.tmem_base, kTmemCols);
@@ -282,18 +351,29 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   pdl_wait();
   pdl_trigger();
 
-  const uint64_t wait_ns = wait_limit(p.wait_ns);
+  const uint64_t wait_ns = wait_limit(P0.wait_ns);
   const uint32_t tmem = s.tmem_base;
-  const int ntn = p.n_total / kN;           // 256-wide items per expert
-  const int ntn128 = p.n_total / 128;       // 128-row weight tiles per expert
-  // p.mtile_prefix may start at a later expert (a handle with one rank's share of the experts):
+  // P0.mtile_prefix may start at a later expert (a handle with one rank's share of the experts):
   // its tiles are numbered from the first entry on.  When an earlier kernel of the call has
   // timed out, the grouping tables may be incomplete: no work items then.
-  const bool upstream_timeout = (*reinterpret_cast<const volatile uint32_t*>(p.status) & kStatusTimeout) != 0;
-  const int tile_base = upstream_timeout ? 0 : __ldg(p.mtile_prefix);
-  const int total = upstream_timeout ? 0 : (__ldg(p.mtile_prefix + p.E) - tile_base) * ntn;
-  const int kb_count = kFp8 ? (p.K + 127) / 128 : (p.K + kBlockK - 1) / kBlockK;   // 128-byte K blocks
-  const int k64 = p.K / 64;  // scale-column tiles of A and B
+  const bool upstream_timeout = (*reinterpret_cast<const volatile uint32_t*>(P0.status) & kStatusTimeout) != 0;
+  const int tile_base = upstream_timeout ? 0 : __ldg(P0.mtile_prefix);
+  const int m_total = upstream_timeout ? 0 : __ldg(P0.mtile_prefix + P0.E) - tile_base;
+  const int ntn_g = pg.n_total / kN;        // 256-wide items per row tile: gate/up
+  const int ntn_d = pd.n_total / kN;        // and down
+  const Sched sc{tile_base, ntn_g, ntn_d, m_total * ntn_g, lag, P0.E};
+  const int total = kMode == kModeFused ? m_total * (ntn_g + ntn_d) : m_total * (kMode == kModeGateUp ? ntn_g : ntn_d);
+  // item w of the schedule; *gu: a gate/up item (else down)
+  auto item = [&](int w, bool* gu) -> Work {
+    if constexpr (kMode == kModeFused) {
+      return decode_fused(P0.mtile_prefix, P0.counts, sc, w, gu);
+    } else {
+      *gu = kMode == kModeGateUp;
+      const int ntn = kMode == kModeGateUp ? ntn_g : ntn_d;
+      return decode_work(P0.mtile_prefix, w + tile_base * ntn, P0.E, ntn, P0.counts);
+    }
+  };
+  auto k_blocks = [](int K) { return kFp8 ? (K + 127) / 128 : (K + kBlockK - 1) / kBlockK; };   // 128-byte K blocks
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
@@ -308,33 +388,61 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         // come from a counter shared by the grid, so CTAs that run faster take more items
         const int slot = it & (kWorkRing - 1);
         if (aborted(&s.abort_flag) || !mbar_wait(&s.work_empty[slot], ((uint32_t)(it / kWorkRing) & 1u) ^ 1u, wait_ns)) {
-          set_abort(&s.abort_flag, p.status);
+          set_abort(&s.abort_flag, P0.status);
           break;
         }
-        int w = it == 0 ? (int)blockIdx.x : atomicAdd(p.work_counter, 1) + (int)gridDim.x;
+        int w = it == 0 ? (int)blockIdx.x : atomicAdd(P0.work_counter, 1) + (int)gridDim.x;
         if (w >= total) w = -1;
         s.work[slot] = w;
         mbar_arrive(&s.work_full[slot]);      // releases the index to the MMA issuer and the epilogue
         if (w < 0) break;
-        const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
+        bool gu;
+        const Work wk = item(w, &gu);
+        const GemmArgs& P = gu ? pg : pd;
+        if constexpr (kMode == kModeFused) {
+          if (!gu) {
+            // h of this row tile is complete once all gate/up items of the tile have signalled
+            const int* d = dep + (wk.mtile - tile_base);
+            const int need = kEpiWarps * ntn_g;
+            if (ld_acquire_gpu(d) < need) {
+              const uint64_t t_start = globaltimer_ns();
+              while (ld_acquire_gpu(d) < need) {
+                if (aborted(&s.abort_flag) || globaltimer_ns() - t_start > wait_ns) {
+                  ok = false;
+                  break;
+                }
+                __nanosleep(256);
+              }
+              if (!ok) {
+                set_abort(&s.abort_flag, P0.status);
+                break;
+              }
+            }
+            fence_proxy_async_global();
+          }
+        }
+        const int kb_count = k_blocks(P.K);
+        const int k64 = P.K / 64;               // scale-column tiles of A and B
+        const int ntn128 = P.n_total / 128;     // 128-row weight tiles per expert
         const int arow = wk.mtile * kBlockM;
         const bool a_small = wk.rows_valid <= 32;
         const uint32_t a_bytes = a_small ? 32u * 128u : (uint32_t)kABytes;
+        const void* amap = gu ? (a_small ? (const void*)&tma_a32 : (const void*)&tma_a)
+                              : (a_small ? (const void*)&tma_h32 : (const void*)&tma_h);
         const int t0 = wk.nt * kNT;           // first 128-row weight tile of the item
-        const uint8_t* btile = p.b_tiles + ((int64_t)wk.e * ntn128 + t0) * kb_count * (int64_t)kTileBytes;
-        const uint8_t* sfa = p.sfa + (int64_t)wk.mtile * k64 * kAtomBytes;
-        const uint8_t* sfb = p.sfb + ((int64_t)wk.e * ntn128 + t0) * k64 * kAtomBytes;
+        const uint8_t* btile = P.b_tiles + ((int64_t)wk.e * ntn128 + t0) * kb_count * (int64_t)kTileBytes;
+        const uint8_t* sfa = P.sfa + (int64_t)wk.mtile * k64 * kAtomBytes;
+        const uint8_t* sfb = P.sfb + ((int64_t)wk.e * ntn128 + t0) * k64 * kAtomBytes;
         for (int kb = 0; kb < kb_count; ++kb) {
           if (aborted(&s.abort_flag) || !mbar_wait(&s.empty[stage], phase ^ 1u, wait_ns)) {
-            set_abort(&s.abort_flag, p.status);
+            set_abort(&s.abort_flag, P0.status);
             ok = false;
             break;
           }
-          const int left = (p.K - kb * kBlockK) / 64;
+          const int left = (P.K - kb * kBlockK) / 64;
           const uint32_t sf_bytes = kFp8 ? 0u : (uint32_t)(left < 4 ? left : 4) * kAtomBytes;
           mbar_arrive_expect_tx(&s.full[stage], a_bytes + kNT * (kTileBytes + sf_bytes) + sf_bytes);
-          tma_load_2d(s.a[stage], a_small ? (const void*)&tma_a32 : (const void*)&tma_a, &s.full[stage],
-                      kb * 128, arow, pol_a);
+          tma_load_2d(s.a[stage], amap, &s.full[stage], kb * 128, arow, pol_a);
           if constexpr (!kFp8) bulk_load(s.sfa[stage], sfa + kb * 4 * kAtomBytes, sf_bytes, &s.full[stage], pol_a);
 #pragma unroll
           for (int j = 0; j < kNT; ++j) {
@@ -352,7 +460,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       // wait for every copy this thread started before the CTA can exit
       for (int st = 0; st < kStages; ++st)
         if ((issued >> st) & 1u)
-          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u, wait_ns)) set_abort(&s.abort_flag, p.status);
+          if (!mbar_wait(&s.full[st], (issued_par >> st) & 1u, wait_ns)) set_abort(&s.abort_flag, P0.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer ----
@@ -364,22 +472,26 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       for (int it = 0; ok; ++it) {
         const int slot = it & (kWorkRing - 1);
         if (aborted(&s.abort_flag) || !mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u, wait_ns)) {
-          set_abort(&s.abort_flag, p.status);
+          set_abort(&s.abort_flag, P0.status);
           break;
         }
         const int w = *reinterpret_cast<volatile int*>(&s.work[slot]);
         mbar_arrive(&s.work_empty[slot]);
         if (w < 0) break;
+        bool gu = kMode == kModeGateUp;
+        if constexpr (kMode == kModeFused) item(w, &gu);
+        const int K = gu ? pg.K : pd.K;
+        const int kb_count = k_blocks(K);
         const uint32_t acc_par = (uint32_t)it & 1u;
         if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u, wait_ns)) {
-          set_abort(&s.abort_flag, p.status);
+          set_abort(&s.abort_flag, P0.status);
           break;
         }
         tc_fence_after();
         const uint32_t acc = tmem;
         for (int kb = 0; kb < kb_count; ++kb) {
           if (aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase, wait_ns)) {
-            set_abort(&s.abort_flag, p.status);
+            set_abort(&s.abort_flag, P0.status);
             ok = false;
             break;
           }
@@ -394,7 +506,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             if (++stage == kStages) { stage = 0; phase ^= 1u; }
             continue;
           }
-          const int left = (p.K - kb * kBlockK) / 64;
+          const int left = (K - kb * kBlockK) / 64;
           const int ksteps = left < 4 ? left : 4;
           // scale atoms: A at sfa_t + 4k; B (row n at lane n % 32, column n / 32) at
           // sfb_t + 4 (kNT k + j) for its 128-row tile j
@@ -420,7 +532,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       }
       // every tensor-core operation of this thread is done before the memory is freed
       tc_commit(&s.drain);
-      if (!mbar_wait(&s.drain, 0, wait_ns)) set_abort(&s.abort_flag, p.status);
+      if (!mbar_wait(&s.drain, 0, wait_ns)) set_abort(&s.abort_flag, P0.status);
     }
   } else {
     // ------------------------------------------------------------ epilogue ----
@@ -431,14 +543,28 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       const int slot = it & (kWorkRing - 1);
       const bool got_work = !aborted(&s.abort_flag) && mbar_wait(&s.work_full[slot], (uint32_t)(it / kWorkRing) & 1u, wait_ns);
       if (__any_sync(0xffffffffu, !got_work)) {
-        set_abort(&s.abort_flag, p.status);
+        set_abort(&s.abort_flag, P0.status);
         break;
       }
       const int w = *reinterpret_cast<volatile int*>(&s.work[slot]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.work_empty[slot]);
       if (w < 0) break;
-      const Work wk = decode_work(p.mtile_prefix, w + tile_base * ntn, p.E, ntn, p.counts);
+      bool gu;
+      const Work wk = item(w, &gu);
+      const GemmArgs& P = gu ? pg : pd;
+      if constexpr (kMode == kModeGateUp) {
+        // the launch's share of zeroing the down GEMM's accumulator, item w's slice, while the
+        // tensor cores work on the item
+        if (P.zero_acc != nullptr) {
+          const int64_t n = P.zero_acc_elems;
+          const int64_t per = ((n + total - 1) / total + 3) & ~(int64_t)3;
+          const int64_t z1 = min((int64_t)(w + 1) * per, n);
+          const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int64_t i = (int64_t)w * per + 4 * ((warp - 2) * 32 + lane); i < z1; i += 4 * 32 * kEpiWarps)
+            *reinterpret_cast<float4*>(P.zero_acc + i) = zero;
+        }
+      }
       const uint32_t acc_par = (uint32_t)it & 1u;
       const int64_t row = (int64_t)wk.mtile * kBlockM + row_l;
       const bool valid = row_l < wk.rows_valid;
@@ -448,24 +574,26 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       float c0s = 0.f, c1s = 0.f, c2s = 0.f;
       int token = -1;
       if (warp_live) {
-        if constexpr (kGateUp && kFp8) {
-          c0s = p.a_scale[row];                       // the token's activation scale
-        } else if constexpr (kGateUp) {
-          const float gx = *p.g_x;
-          c0s = __fmul_rn(gx, p.g_gate[wk.e]);
-          c1s = __fmul_rn(gx, p.g_up[wk.e]);
-          c2s = p.g_h[wk.e];
+        if (gu) {
+          if constexpr (kFp8) {
+            c0s = P.a_scale[row];                     // the token's activation scale
+          } else {
+            const float gx = *P.g_x;
+            c0s = __fmul_rn(gx, P.g_gate[wk.e]);
+            c1s = __fmul_rn(gx, P.g_up[wk.e]);
+            c2s = P.g_h[wk.e];
+          }
         } else {
-          const int pair = valid ? p.row_pair[row] : -1;
+          const int pair = valid ? P.row_pair[row] : -1;
           if (pair >= 0) {
-            c0s = kFp8 ? __fmul_rn(p.wts[pair], p.h_scale[row]) : __fmul_rn(p.alpha_down[wk.e], p.wts[pair]);
-            token = pair / p.topk;
+            c0s = kFp8 ? __fmul_rn(P.wts[pair], P.h_scale[row]) : __fmul_rn(P.alpha_down[wk.e], P.wts[pair]);
+            token = pair / P.topk;
           }
         }
       }
       const bool got = !aborted(&s.abort_flag) && mbar_wait(&s.acc_full, acc_par, wait_ns);
       if (__any_sync(0xffffffffu, !got)) {
-        set_abort(&s.abort_flag, p.status);
+        set_abort(&s.abort_flag, P0.status);
         break;
       }
       __syncwarp();
@@ -479,57 +607,13 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
       };
       if (!warp_live) {
         release();
-      } else if constexpr (kGateUp && kFp8) {
-        // h = silu(acc_g * sx * wg) * (acc_u * sx * wu) per feature, stored in FP32
-        const int t = wk.nt * kNT + half;             // weight tile of this warp's 64 features
-        const int tcol = half * 128;
-        const float* wsc = p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + tcol;
-        const float sx = c0s;
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          uint32_t G[32], U[32];
-          tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
-          tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
-          tmem_ld_wait();
-          if (pr == 1) release();
-          float h[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gv = __fmul_rn(__fmul_rn(__uint_as_float(G[i]), sx), __ldg(wsc + 32 * pr + i));
-            const float uv = __fmul_rn(__fmul_rn(__uint_as_float(U[i]), sx), __ldg(wsc + 64 + 32 * pr + i));
-            h[i] = __fmul_rn(__fmul_rn(gv, uv), rcp_approx(__fadd_rn(1.0f, __expf(-gv))));
-          }
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(p.h32 + row * p.I + t * 64 + 32 * pr);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
-          }
-        }
-      } else if constexpr (kGateUp) {
-        const float sg = c0s, su = c1s, gh = c2s;
-        const float r_t = __frcp_rn(__fmul_rn(6.0f, gh));
-        const int64_t n_ct = p.I / 64;
-        // weight tile t = 2 nt + half holds this warp's 64 features: accumulator columns
-        // [128 half, +64) are their gate, [128 half + 64, +64) their up projections
-        const int t = wk.nt * kNT + half;
-        const int tcol = half * 128;
-        if constexpr (kDecode) {
-          // all four 32-column chunks into registers first, then the accumulator is released
-          uint32_t G0[32], U0[32], G1[32], U1[32];
-          tmem_ld_32x32b_x32(t_row + tcol, G0);
-          tmem_ld_32x32b_x32(t_row + tcol + 64, U0);
-          tmem_ld_32x32b_x32(t_row + tcol + 32, G1);
-          tmem_ld_32x32b_x32(t_row + tcol + 96, U1);
-          tmem_ld_wait();
-          release();
-          float h[32];
-          swiglu32(G0, U0, sg, su, h);
-          if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64, h);
-          quant_store32(h, gh, r_t, valid, row, t * 64, p, n_ct);
-          swiglu32(G1, U1, sg, su, h);
-          if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64 + 32, h);
-          quant_store32(h, gh, r_t, valid, row, t * 64 + 32, p, n_ct);
-        } else {
+      } else if (gu) {
+        if constexpr (kFp8) {
+          // h = silu(acc_g * sx * wg) * (acc_u * sx * wu) per feature, stored in FP32
+          const int t = wk.nt * kNT + half;           // weight tile of this warp's 64 features
+          const int tcol = half * 128;
+          const float* wsc = P.w_scale + (int64_t)wk.e * P.n_total + wk.nt * kN + tcol;
+          const float sx = c0s;
 #pragma unroll
           for (int pr = 0; pr < 2; ++pr) {
             uint32_t G[32], U[32];
@@ -538,12 +622,58 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             tmem_ld_wait();
             if (pr == 1) release();
             float h[32];
-            swiglu32(G, U, sg, su, h);
-            if (p.h_dbg != nullptr && valid) store_h_dbg(p, wk, row_l, t * 64 + 32 * pr, h);
-            quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, p, n_ct);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float gv = __fmul_rn(__fmul_rn(__uint_as_float(G[i]), sx), __ldg(wsc + 32 * pr + i));
+              const float uv = __fmul_rn(__fmul_rn(__uint_as_float(U[i]), sx), __ldg(wsc + 64 + 32 * pr + i));
+              h[i] = __fmul_rn(__fmul_rn(gv, uv), rcp_approx(__fadd_rn(1.0f, __expf(-gv))));
+            }
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(P.h32 + row * P.I + t * 64 + 32 * pr);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+            }
+          }
+        } else {
+          const float sg = c0s, su = c1s, gh = c2s;
+          const float r_t = __frcp_rn(__fmul_rn(6.0f, gh));
+          const int64_t n_ct = P.I / 64;
+          // weight tile t = 2 nt + half holds this warp's 64 features: accumulator columns
+          // [128 half, +64) are their gate, [128 half + 64, +64) their up projections
+          const int t = wk.nt * kNT + half;
+          const int tcol = half * 128;
+          if constexpr (kDecode) {
+            // all four 32-column chunks into registers first, then the accumulator is released
+            uint32_t G0[32], U0[32], G1[32], U1[32];
+            tmem_ld_32x32b_x32(t_row + tcol, G0);
+            tmem_ld_32x32b_x32(t_row + tcol + 64, U0);
+            tmem_ld_32x32b_x32(t_row + tcol + 32, G1);
+            tmem_ld_32x32b_x32(t_row + tcol + 96, U1);
+            tmem_ld_wait();
+            release();
+            float h[32];
+            swiglu32(G0, U0, sg, su, h);
+            if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64, h);
+            quant_store32(h, gh, r_t, valid, row, t * 64, P, n_ct);
+            swiglu32(G1, U1, sg, su, h);
+            if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64 + 32, h);
+            quant_store32(h, gh, r_t, valid, row, t * 64 + 32, P, n_ct);
+          } else {
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {
+              uint32_t G[32], U[32];
+              tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
+              tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
+              tmem_ld_wait();
+              if (pr == 1) release();
+              float h[32];
+              swiglu32(G, U, sg, su, h);
+              if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64 + 32 * pr, h);
+              quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, P, n_ct);
+            }
           }
         }
-      } else if constexpr (kDecode) {
+      } else if constexpr (!C::kStaging) {
         // two 16-lane blocks of this warp's rows, 128 columns each, in the 16x256b layout:
         // four consecutive threads hold one row's 8 consecutive columns, so every reduction
         // instruction adds whole 32-byte sectors of 8 token rows
@@ -561,8 +691,8 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             const int tok = __shfl_sync(0xffffffffu, token, r);
             const float sc = __shfl_sync(0xffffffffu, c0s, r);
             if (tok >= 0) {
-              float* dst = p.acc + (int64_t)tok * p.H + wk.nt * kN + half * (kN / 2) + cq;
-              const float* wsc = kFp8 ? p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + half * (kN / 2) + cq
+              float* dst = P.acc + (int64_t)tok * P.H + wk.nt * kN + half * (kN / 2) + cq;
+              const float* wsc = kFp8 ? P.w_scale + (int64_t)wk.e * P.n_total + wk.nt * kN + half * (kN / 2) + cq
                                       : nullptr;
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
@@ -592,7 +722,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           const int c0 = half * (kN / 2) + c * 32;
           if (c > 0) bulk_wait_read0();
           if constexpr (kFp8) {
-            const float* wsc = p.w_scale + (int64_t)wk.e * p.n_total + wk.nt * kN + c0;
+            const float* wsc = P.w_scale + (int64_t)wk.e * P.n_total + wk.nt * kN + c0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float4 w4 = __ldg(reinterpret_cast<const float4*>(wsc) + i);
@@ -611,11 +741,21 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           }
           if (token >= 0) {
             fence_proxy_async_smem();
-            bulk_reduce_add_f32(p.acc + (int64_t)token * p.H + wk.nt * kN + c0, mine, 128u);
+            bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, mine, 128u);
             bulk_commit();
           }
         }
         bulk_wait_read0();
+      }
+      if constexpr (kMode == kModeFused) {
+        if (gu) {
+          // this warp's share of the tile's h is stored: make it visible to the TMA and bulk
+          // loads of the down items, then count it
+          fence_proxy_async_global();
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(dep + (wk.mtile - tile_base), 1);
+        }
       }
     }
     bulk_wait_all0();
@@ -629,15 +769,16 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
   }
 }
 
-template <bool kGateUp, bool kDecode, bool kFp8 = false>
-cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a, int grid,
-                        cudaStream_t stream) {
-  const size_t smem = sizeof(Smem<kGateUp, kDecode, kFp8>) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kGateUp, kDecode, kFp8>,
+template <int kMode, bool kDecode, bool kFp8 = false>
+cudaError_t launch_gemm(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const CUtensorMap& tma_h,
+                        const CUtensorMap& tma_h32, const GemmArgs& pg, const GemmArgs& pd, int* dep, int lag,
+                        int grid, cudaStream_t stream) {
+  const size_t smem = sizeof(Smem<kMode, kDecode, kFp8>) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(moe_gemm_kernel<kMode, kDecode, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(moe_gemm_kernel<kGateUp, kDecode, kFp8>, dim3(grid), dim3(kThreads), smem, stream, tma_a,
-                    tma_a32, a);
+  return launch_pdl(moe_gemm_kernel<kMode, kDecode, kFp8>, dim3(grid), dim3(kThreads), smem, stream, tma_a,
+                    tma_a32, tma_h, tma_h32, pg, pd, dep, lag);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -659,37 +800,44 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-static_assert(sizeof(Smem<true, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<true, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<true, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<true, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
-static_assert(sizeof(Smem<false, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeGateUp, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeGateUp, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeDown, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeDown, false, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeFused, true, false>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeGateUp, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeGateUp, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeDown, true, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
+static_assert(sizeof(Smem<kModeDown, false, true>) + 1024 <= 232448, "GEMM shared memory exceeds the per-block limit");
 
 cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                                int grid, bool decode, cudaStream_t stream) {
-  return decode ? launch_gemm<true, true>(tma_a, tma_a32, a, grid, stream)
-                : launch_gemm<true, false>(tma_a, tma_a32, a, grid, stream);
+  return decode ? launch_gemm<kModeGateUp, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream)
+                : launch_gemm<kModeGateUp, false>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream);
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                              int grid, bool decode, cudaStream_t stream) {
-  return decode ? launch_gemm<false, true>(tma_a, tma_a32, a, grid, stream)
-                : launch_gemm<false, false>(tma_a, tma_a32, a, grid, stream);
+  return decode ? launch_gemm<kModeDown, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream)
+                : launch_gemm<kModeDown, false>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream);
+}
+
+cudaError_t launch_gemm_fused(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const CUtensorMap& tma_h,
+                              const CUtensorMap& tma_h32, const GemmArgs& gate_up, const GemmArgs& down, int* dep,
+                              int lag, int grid, cudaStream_t stream) {
+  return launch_gemm<kModeFused, true>(tma_a, tma_a32, tma_h, tma_h32, gate_up, down, dep, lag, grid, stream);
 }
 
 cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                                    int grid, bool decode, cudaStream_t stream) {
-  return decode ? launch_gemm<true, true, true>(tma_a, tma_a32, a, grid, stream)
-                : launch_gemm<true, false, true>(tma_a, tma_a32, a, grid, stream);
+  return decode ? launch_gemm<kModeGateUp, true, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream)
+                : launch_gemm<kModeGateUp, false, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream);
 }
 
 cudaError_t launch_gemm_down_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                                  int grid, bool decode, cudaStream_t stream) {
-  return decode ? launch_gemm<false, true, true>(tma_a, tma_a32, a, grid, stream)
-                : launch_gemm<false, false, true>(tma_a, tma_a32, a, grid, stream);
+  return decode ? launch_gemm<kModeDown, true, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream)
+                : launch_gemm<kModeDown, false, true>(tma_a, tma_a32, tma_a, tma_a32, a, a, nullptr, 0, grid, stream);
 }
 
 int make_tma_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {

@@ -33,6 +33,8 @@ struct GemmArgs {
   const float* g_up;           // [E]
   const float* g_h;            // [E]
   int I;
+  float* zero_acc;             // optional [zero_acc_elems] FP32 zeroed by the launch's epilogue
+  int64_t zero_acc_elems;      // warps (a slice per work item; gate/up launch only)
   // down epilogue
   float* acc;                  // [T][H]
   const int32_t* row_pair;     // [rows_cap]
@@ -60,6 +62,15 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tma_a, const CUtensorMap& tma_
                                int grid, bool decode, cudaStream_t stream);
 cudaError_t launch_gemm_down(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,
                              int grid, bool decode, cudaStream_t stream);
+// Both GEMMs in one persistent launch (NVFP4, the configuration for segments that average
+// fewer than 32 rows): gate_up and down as for the two launches above (the same grouping
+// tables, status and work counter: gate_up's), tma_h / tma_h32 the maps of the down GEMM's A
+// rows (h).  dep: one zeroed counter per 128-row tile of the launch; a down item starts once its
+// tile's counter reaches 8 per gate/up column tile.  lag: gate/up items claimed, beyond the
+// largest expert's, between an expert's last gate/up item and its first down item.
+cudaError_t launch_gemm_fused(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const CUtensorMap& tma_h,
+                              const CUtensorMap& tma_h32, const GemmArgs& gate_up, const GemmArgs& down, int* dep,
+                              int lag, int grid, cudaStream_t stream);
 // The FP8 W8A8 variants: A and B are E4M3 rows of K bytes (tensor maps over K-byte rows), the
 // scales come from a_scale / w_scale / h_scale, and gate/up writes FP32 h to h32.
 cudaError_t launch_gemm_gateup_fp8(const CUtensorMap& tma_a, const CUtensorMap& tma_a32, const GemmArgs& a,

@@ -56,12 +56,14 @@ struct RouterArgs {
   uint32_t* status;         // kStatusNonFinite is raised here for a NaN logit (may be nullptr)
   uint64_t wait_ns;         // limit of each bounded wait of the tensor-core logits (0: kWaitLimitNs)
   // integer tensor-core logits (T >= kRouterTcMinT, when given; route_tc.cu)
-  uint8_t* x_digits;        // [4][T][H] int8 digit planes of the token rows
-  uint8_t* w_digits;        // [4][E][H] int8 digit planes of the expert rows
+  uint8_t* x_digits;        // [kRouterXDigits][T][H] int8 digit planes of the token rows
+  uint8_t* w_digits;        // [kRouterWDigits][E][H] int8 digit planes of the expert rows
   int32_t* x_exp;           // [T] row exponents (kExpNonFinite: the row has a non-finite value)
   int32_t* w_exp;           // [E]
 };
 constexpr int kRouterTcMinT = 65;
+constexpr int kRouterXDigits = 3;   // int8 digit planes of a token row (22-bit fixed point)
+constexpr int kRouterWDigits = 4;   // and of an expert row (30-bit)
 constexpr int32_t kExpNonFinite = 0x7FFFFFFF;
 
 struct PermArgs {
@@ -70,7 +72,7 @@ struct PermArgs {
   int topk, E;
   int n_chunks;
   int32_t* chunk_counts;   // [n_chunks][E]
-  int32_t* chunk_base;     // [n_chunks][E]
+  int32_t* chunk_base;     // [n_chunks][E] first position of the chunk's pairs in the expert's segment
   int32_t* counts;         // [E]
   int32_t* offsets;        // [E+1]
   int32_t* mtile_prefix;   // [E+1] cumulative 128-row tiles

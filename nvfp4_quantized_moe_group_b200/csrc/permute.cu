@@ -21,28 +21,62 @@ __global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a) {
     a.chunk_counts[(int64_t)blockIdx.x * a.E + e] = hist[e];
 }
 
-// One block, one thread per expert: per-chunk bases, counts, offsets (exclusive scan),
-// 128-row tile prefix, and -1 in every padding row of every segment.  The per-chunk counts are
-// read in batches of independent loads (a chain of dependent loads, one per chunk, would wait
-// out the memory latency once per chunk).
+// Per expert, the position of each chunk's first pair inside the expert's segment (exclusive
+// prefix of the chunk counts over the chunks) and the expert's pair count.  One CTA per 32
+// experts (lane = expert), its 8 warps splitting the chunks into 8 consecutive runs: each warp
+// sums its run, the CTA turns the 8 sums into run bases, and each warp writes its run's
+// prefixes.  The chunk counts are read in batches of independent loads.
+__global__ void __launch_bounds__(256) perm_colscan_kernel(PermArgs a) {
+  __shared__ int s_sum[8][32];
+  constexpr int kBatch = 32;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const bool on = e < a.E;
+  const int per = (a.n_chunks + 7) / 8;
+  const int c0 = warp * per;
+  const int c1 = min(c0 + per, a.n_chunks);
+  const int* __restrict__ cc = a.chunk_counts;
+  int sum = 0;
+  for (int b = c0; b < c1; b += kBatch) {
+    int v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) v[j] = on && b + j < c1 ? __ldg(cc + (int64_t)(b + j) * a.E + e) : 0;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) sum += v[j];
+  }
+  s_sum[warp][lane] = sum;
+  __syncthreads();
+  int base = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int v = s_sum[w][lane];
+    base += w < warp ? v : 0;
+    total += v;
+  }
+  if (!on) return;
+  if (warp == 0) a.counts[e] = total;
+  for (int b = c0; b < c1; b += kBatch) {
+    int v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) v[j] = b + j < c1 ? __ldg(cc + (int64_t)(b + j) * a.E + e) : 0;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (b + j < c1) a.chunk_base[(int64_t)(b + j) * a.E + e] = base;
+      base += v[j];
+    }
+  }
+}
+
+// One block, one thread per expert: offsets (exclusive scan of the counts), the 128-row tile
+// prefix, and -1 in every padding row of every segment.
 __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
   __shared__ int s_cnt[256];
   __shared__ int s_tiles[256];
-  constexpr int kBatch = 64;
   const int e = threadIdx.x;
-  const int* __restrict__ cc = a.chunk_counts;
-  int running = 0;
-  if (e < a.E) {
-    for (int c0 = 0; c0 < a.n_chunks; c0 += kBatch) {
-      int v[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < a.n_chunks ? __ldg(cc + (int64_t)(c0 + j) * a.E + e) : 0;
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) running += v[j];
-    }
-  }
-  const int tiles = e < a.E ? (running + kBlockM - 1) / kBlockM : 0;
-  s_cnt[e] = e < a.E ? running : 0;
+  const int count = e < a.E ? a.counts[e] : 0;
+  const int tiles = (count + kBlockM - 1) / kBlockM;
+  s_cnt[e] = count;
   s_tiles[e] = tiles;
   __syncthreads();
   // inclusive scans (Hillis-Steele) of counts and tiles over the 256 threads
@@ -55,30 +89,17 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(PermArgs a) {
     __syncthreads();
   }
   if (e < a.E) {
-    const int off = s_cnt[e] - running;       // exclusive
+    const int off = s_cnt[e] - count;         // exclusive
     const int tile0 = s_tiles[e] - tiles;
     a.offsets[e] = off;
     a.mtile_prefix[e] = tile0;
-    a.counts[e] = running;
     if (e == a.E - 1) {
-      a.offsets[a.E] = off + running;
+      a.offsets[a.E] = off + count;
       a.mtile_prefix[a.E] = tile0 + tiles;
-    }
-    // chunk c's first position for expert e: off + the counts of the chunks before it
-    int base = off;
-    for (int c0 = 0; c0 < a.n_chunks; c0 += kBatch) {
-      int v[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < a.n_chunks ? __ldg(cc + (int64_t)(c0 + j) * a.E + e) : 0;
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        if (c0 + j < a.n_chunks) a.chunk_base[(int64_t)(c0 + j) * a.E + e] = base;
-        base += v[j];
-      }
     }
     const int64_t r0 = (int64_t)tile0 * kBlockM;
     const int64_t r1 = r0 + (int64_t)tiles * kBlockM;
-    for (int64_t r = r0 + running; r < r1; ++r) a.row_pair[r] = -1;
+    for (int64_t r = r0 + count; r < r1; ++r) a.row_pair[r] = -1;
   }
 }
 
@@ -88,7 +109,7 @@ __global__ void __launch_bounds__(32) perm_scatter_kernel(PermArgs a) {
   __shared__ int run[256];
   const int lane = threadIdx.x;
   const int c = blockIdx.x;
-  for (int e = lane; e < a.E; e += 32) run[e] = a.chunk_base[(int64_t)c * a.E + e];
+  for (int e = lane; e < a.E; e += 32) run[e] = a.offsets[e] + a.chunk_base[(int64_t)c * a.E + e];
   __syncwarp();
   const int64_t p0 = (int64_t)c * kPermChunkTokens * a.topk;
   const int64_t p1 = min(p0 + (int64_t)kPermChunkTokens * a.topk, a.T * a.topk);
@@ -178,9 +199,12 @@ cudaError_t launch_permute(const PermArgs& a, cudaStream_t stream, int* launches
     *launches += 1;
     return cudaGetLastError();
   }
-  *launches += 3;
+  *launches += 4;
   perm_count_kernel<<<a.n_chunks, 256, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  perm_colscan_kernel<<<(a.E + 31) / 32, 256, 0, stream>>>(a);
+  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   perm_scan_kernel<<<1, 256, 0, stream>>>(a);
   err = cudaGetLastError();

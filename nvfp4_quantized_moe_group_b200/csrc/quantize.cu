@@ -101,19 +101,23 @@ __device__ __forceinline__ uint32_t quantize_block(const uint32_t* w, float r_t,
 }
 
 // One CTA per row (rows_padded CTAs), min(segments, 32) warps: each warp quantises the row's
-// 1024-value segments warp, warp + n_warps, ..., two consecutive 16-value blocks per lane, so
-// every load and store of the warp covers one contiguous span of the row (16 code bytes per
-// lane).  Rows in [rows, rows_padded) only write zero scales (swizzled layout padding).  The
-// global scale is read from g_in.
+// segments of 32 kBpl blocks (warp, warp + n_warps, ...), kBpl consecutive 16-value blocks per
+// lane, so every load and store of the warp covers one contiguous span of the row.  Rows in
+// [rows, rows_padded) only write zero scales (swizzled layout padding).  The global scale is
+// read from g_in.  Two blocks per lane take fewer instructions per block (one 16-byte code
+// store, one shuffle per scale word); one block per lane keeps twice the warps in flight for
+// the forward's scatter into 8 segment rows and accumulator zeroing (measured faster there).
+template <int kBpl>
 __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
+  static_assert(kBpl == 1 || kBpl == 2, "one or two blocks per lane");
+  constexpr int kWordLanes = 4 / kBpl;          // lanes holding the 4 scales of one scale word
   const float g = __ldg(a.g_in);
   if (!(g > 0.0f && g < __uint_as_float(0x7F800000u))) return;   // non-finite input: skipped
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.g_out != nullptr && a.g_out != a.g_in) *a.g_out = g;
   const float r_t = __frcp_rn(__fmul_rn(6.0f, g));
 
-  // lanes 2k, 2k+1 hold the 4 block scales of one 32-bit scale word
   const int blocks_per_row = (int)(a.cols >> 4);
-  const int segs_per_row = (blocks_per_row + 63) >> 6;
+  const int segs_per_row = (blocks_per_row + 32 * kBpl - 1) / (32 * kBpl);
   const int lane = threadIdx.x & 31;
   const int n_warps = blockDim.x >> 5;
   const int64_t r = blockIdx.x;
@@ -125,9 +129,9 @@ __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
     my_row = (int64_t)a.mtile_prefix[e] * kBlockM + (a.inv[p] - a.offsets[e]);
   }
   for (int seg = threadIdx.x >> 5; seg < segs_per_row; seg += n_warps) {
-    const int b = seg * 64 + 2 * lane;          // first of the lane's two blocks
-    // lanes past the row's last block stay for the shuffle; lane pairs are active or idle
-    // together (cols % 64 == 0)
+    const int b = seg * 32 * kBpl + kBpl * lane;    // first of the lane's blocks
+    // lanes past the row's last block stay for the shuffles; the lanes of one scale word are
+    // active or idle together (cols % 64 == 0)
     const bool active = b < blocks_per_row;
     const bool live = active && r < a.rows;
 
@@ -135,31 +139,42 @@ __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
       float4* z = reinterpret_cast<float4*>(a.zero_out + r * a.cols + (int64_t)b * 16);
       const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) z[i] = zero;
+      for (int i = 0; i < 4 * kBpl; ++i) z[i] = zero;
     }
 
-    uint32_t s2 = 0;                            // the two scale bytes of the lane
-    uint4 codes = make_uint4(0, 0, 0, 0);
+    uint32_t sl = 0;                            // the lane's scale bytes
+    uint32_t codes[2 * kBpl];
+#pragma unroll
+    for (int i = 0; i < 2 * kBpl; ++i) codes[i] = 0;
     if (live) {
       const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + (int64_t)b * 16);
-      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1), v2 = __ldg(src + 2), v3 = __ldg(src + 3);
-      const uint32_t w0[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      const uint32_t w1[8] = {v2.x, v2.y, v2.z, v2.w, v3.x, v3.y, v3.z, v3.w};
-      const uint32_t sa = quantize_block(w0, r_t, g, &codes.x, &codes.y);
-      const uint32_t sb = quantize_block(w1, r_t, g, &codes.z, &codes.w);
-      s2 = sa | (sb << 8);
+#pragma unroll
+      for (int k = 0; k < kBpl; ++k) {
+        const uint4 v0 = __ldg(src + 2 * k), v1 = __ldg(src + 2 * k + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        sl |= quantize_block(w, r_t, g, &codes[2 * k], &codes[2 * k + 1]) << (8 * k);
+      }
     }
-    // the 32-bit scale word of this lane's group of 4 blocks (valid in even lanes)
-    const uint32_t sc = s2 | (__shfl_down_sync(0xffffffffu, s2, 1) << 16);
-    const bool word_lane = active && (lane & 1) == 0;
+    // the 32-bit scale word of this lane's group of 4 blocks (valid in lanes kWordLanes k)
+    uint32_t sc = sl;
+#pragma unroll
+    for (int k = 1; k < kWordLanes; ++k) sc |= __shfl_down_sync(0xffffffffu, sl, k) << (8 * kBpl * k);
+    const bool word_lane = active && (lane & (kWordLanes - 1)) == 0;
 
+    auto store_codes = [&](uint8_t* row_base) {
+      if constexpr (kBpl == 2) {
+        reinterpret_cast<uint4*>(row_base)[b >> 1] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+      } else {
+        reinterpret_cast<uint2*>(row_base)[b] = make_uint2(codes[0], codes[1]);
+      }
+    };
     if (r < a.rows) {
-      if (a.codes != nullptr && active) reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1))[b >> 1] = codes;
+      if (a.codes != nullptr && active) store_codes(a.codes + r * (a.cols >> 1));
       if (a.seg_codes != nullptr) {
         // every lane writes its blocks to all of the token's segment rows
         for (int j = 0; j < a.topk; ++j) {
           const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
-          if (active) reinterpret_cast<uint4*>(a.seg_codes + row * (a.cols >> 1))[b >> 1] = codes;
+          if (active) store_codes(a.seg_codes + row * (a.cols >> 1));
           if (word_lane) *reinterpret_cast<uint32_t*>(a.seg_sf + swz_offset(row, b, a.n_col_tiles)) = sc;
         }
       }
@@ -206,9 +221,14 @@ cudaError_t launch_quantize(QuantizeArgs a, cudaStream_t stream) {
       return cudaMemcpyAsync(a.g_out, a.g_in, sizeof(float), cudaMemcpyDeviceToDevice, stream);
     return cudaSuccess;
   }
-  const int segs = (int)(((a.cols >> 4) + 63) >> 6);
-  const int warps = segs < 32 ? segs : 32;
-  quantize_kernel<<<(unsigned)a.rows_padded, 32 * warps, 0, stream>>>(a);
+  // the scatter into expert segments (the forward) keeps one block per lane
+  if (a.seg_codes != nullptr || a.zero_out != nullptr) {
+    const int segs = (int)(((a.cols >> 4) + 31) >> 5);
+    quantize_kernel<1><<<(unsigned)a.rows_padded, 32 * (segs < 32 ? segs : 32), 0, stream>>>(a);
+  } else {
+    const int segs = (int)(((a.cols >> 4) + 63) >> 6);
+    quantize_kernel<2><<<(unsigned)a.rows_padded, 32 * (segs < 32 ? segs : 32), 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -1,24 +1,26 @@
-// Router logits for T > 64 on the tensor cores, in exact integer arithmetic ("Reflection
-// releases Beam ...", section "Mixture-of-Experts details": every token scores all 256
-// experts; section "Residual stream and numerical decisions": the router runs in FP32, and
-// these logits are more accurate than an FP32 accumulation).
+// Router logits for T > 64 on the tensor cores, in integer arithmetic ("Reflection releases
+// Beam ...", section "Mixture-of-Experts details": every token scores all 256 experts; section
+// "Residual stream and numerical decisions": the router runs in FP32, and these logits are
+// more accurate than an FP32 accumulation).
 //
-// Each token row x_t (BF16) and each expert row W_e (FP32) is scaled by a power of two to
-// 30-bit fixed point: with e the binary exponent of the row's largest magnitude
-// (max |v| < 2^e), V = RNE(v * 2^(30 - e)), |V| < 2^30, |V - v 2^(30-e)| <= 1/2.  V is split
-// into four balanced base-256 digits (int8): V = d0 2^24 + d1 2^16 + d2 2^8 + d3 with
-// d1..d3 in [-128, 127] and |d0| <= 64.  Then
-//     X . W = sum_{i,j} (a_i . b_j) 2^(8 (6 - i - j)),
-// and the 13 digit pairs with i + j <= 4 are multiplied by tcgen05 kind::i8 MMAs: int8 x int8
-// products accumulated in int32, which is exact (|class sum| < 5 * 2^14 * K < 2^31 for the
-// K <= 26,112 columns of one split).  One
-// tensor-memory accumulator per class c = i + j; the epilogue combines the five classes in
-// FP64 and scales by 2^(e_x + e_W - 60).  Error against the exact logit, before the FP32
-// rounding of the sum with the bias:
-//     2^(e_x - 31) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 62)      (rounding)
-//   + H (2^23 + 2^14) 2^(e_x + e_W - 60)                                        (pairs i+j > 4)
-//   + FP64 roundings of the combination and of the split-K sum (< H 2^(e_x + e_W - 48)),
-// in all at most 2^(e_x - 31) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 36).
+// Each token row x_t (BF16) is scaled by a power of two to 22-bit fixed point and each expert
+// row W_e (FP32) to 30-bit fixed point: with e the binary exponent of the row's largest
+// magnitude (max |v| < 2^e), X = RNE(x 2^(22 - e_x)), W = RNE(w 2^(30 - e_W)).  A BF16 value
+// has 8 significant bits, so X is exact for every element within 2^14 of the row's largest.
+// X is split into three balanced base-256 digits, X = a0 2^16 + a1 2^8 + a2, W into four,
+// W = b0 2^24 + b1 2^16 + b2 2^8 + b3 (digits in [-128, 127], |a0|, |b0| <= 64).  Then
+//     X . W = sum_{i,j} (a_i . b_j) 2^(8 (5 - i - j)),
+// and the 9 digit pairs with i + j <= 3 are multiplied by tcgen05 kind::i8 MMAs: int8 x int8
+// products accumulated in int32, which is exact (|class sum| < 3 * 2^14 * K < 2^31 for the
+// K <= 26,112 columns of one split).  One tensor-memory accumulator per class c = i + j (4 x 128
+// columns: 128 experts per CTA); the epilogue combines the classes in FP64 and scales by
+// 2^(e_x + e_W - 52).  Error against the exact logit, before the FP32 rounding of the sum with
+// the bias:
+//     sum_h |x_h - X_h 2^(e_x-22)| |W_eh| + sum_h |x_h| |W_eh - W_h 2^(e_W-30)|     (rounding)
+//       <= 2^(e_x - 23) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 54)
+//   + H (2^23 + 2^14) 2^(e_x + e_W - 52)                                 (pairs i + j > 3)
+//   + FP64 roundings of the combination and of the split-K sum (< H 2^(e_x + e_W - 50)),
+// in all at most 2^(e_x - 23) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 28).
 // A row with a non-finite element gets the exponent kExpNonFinite and NaN logits.
 #include "common.cuh"
 #include "kernels.h"
@@ -29,18 +31,19 @@ namespace {
 constexpr int kSliceThreads = 256;
 constexpr int kSliceMaxCtas = 1024;       // amax partials of the token rows
 constexpr int kTcM = 128;                 // tokens per tile
-constexpr int kTcN = 64;                  // experts per tile
+constexpr int kTcN = 128;                 // experts per tile
 constexpr int kTcStages = 2;
-constexpr int kDigits = 4;
-constexpr int kClasses = 5;               // digit-pair classes c = i + j <= 4
+constexpr int kXDigits = kRouterXDigits;  // 3: 22-bit token rows
+constexpr int kWDigits = kRouterWDigits;  // 4: 30-bit expert rows
+constexpr int kClasses = 4;               // digit-pair classes c = i + j <= 3
 constexpr int kTcThreads = 192;           // producer, MMA issuer, 4 epilogue warps
-constexpr uint32_t kTcTmemCols = 512;     // 5 x 64 columns used
+constexpr uint32_t kTcTmemCols = 512;     // 4 x 128 columns
 constexpr int kAPlaneBytes = kTcM * 128;  // one digit plane of the token tile, 128-byte K block
 constexpr int kBPlaneBytes = kTcN * 128;
 
 struct __align__(1024) TcSmem {
-  uint8_t a[kTcStages][kDigits][kAPlaneBytes];
-  uint8_t b[kTcStages][kDigits][kBPlaneBytes];
+  uint8_t a[kTcStages][kXDigits][kAPlaneBytes];
+  uint8_t b[kTcStages][kWDigits][kBPlaneBytes];
   uint64_t full[kTcStages];
   uint64_t empty[kTcStages];
   uint64_t acc_full;
@@ -77,6 +80,20 @@ __host__ __device__ constexpr uint32_t idesc_i8(uint32_t m, uint32_t n) {
 // and zero rows take the smallest normal exponent).
 __device__ __forceinline__ int row_exponent(uint32_t biased) { return (int)(biased > 1u ? biased : 1u) - 126; }
 
+// Three balanced base-256 digits of v * 2^shift, |v * 2^shift| < 2^22 (exact power-of-two
+// scaling in FP64, then round to nearest even), packed into one byte each of the three words'
+// byte lane `lane`.
+__device__ __forceinline__ void digits3(double v, double scale, uint32_t lane, uint32_t* d) {
+  int X = __double2int_rn(v * scale);
+  const int d2 = ((X + 128) & 255) - 128;
+  X = (X - d2) >> 8;
+  const int d1 = ((X + 128) & 255) - 128;
+  const int d0 = (X - d1) >> 8;
+  d[0] |= ((uint32_t)d0 & 255u) << (8 * lane);
+  d[1] |= ((uint32_t)d1 & 255u) << (8 * lane);
+  d[2] |= ((uint32_t)d2 & 255u) << (8 * lane);
+}
+
 // Four balanced base-256 digits of v * 2^shift (exact power-of-two scaling in FP64, then
 // round to nearest even), packed into one byte each of the four words' byte lane `lane`.
 __device__ __forceinline__ void digits4(double v, double scale, uint32_t lane, uint32_t* d) {
@@ -106,7 +123,7 @@ __device__ __forceinline__ uint32_t block_max(uint32_t m, uint32_t* s_red) {
 }
 }  // namespace
 
-// Token rows: BF16 x [T][H] -> digit planes [4][T][H], exponents [T]; CTA b also writes the
+// Token rows: BF16 x [T][H] -> digit planes [3][T][H], exponents [T]; CTA b also writes the
 // max |x| of its rows (BF16 magnitude bits) to amax_partials[b] for the quantiser's global scale.
 __global__ void __launch_bounds__(kSliceThreads) slice_x_kernel(RouterArgs a) {
   __shared__ uint32_t s_red[kSliceThreads / 32];
@@ -130,20 +147,20 @@ __global__ void __launch_bounds__(kSliceThreads) slice_x_kernel(RouterArgs a) {
     }
     const int e = row_exponent(be);
     if (threadIdx.x == 0) a.x_exp[t] = e;
-    const double scale = ldexp(1.0, 30 - e);
+    const double scale = ldexp(1.0, 22 - e);
     for (int v = threadIdx.x; v < n8; v += kSliceThreads) {
       const uint4 q = __ldg(src + v);
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-      uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+      uint32_t lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0};
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        digits4((double)__uint_as_float(w[j] << 16), scale, 2 * j, lo);
-        digits4((double)__uint_as_float(w[j] & 0xFFFF0000u), scale, 2 * j + 1, lo);
-        digits4((double)__uint_as_float(w[j + 2] << 16), scale, 2 * j, hi);
-        digits4((double)__uint_as_float(w[j + 2] & 0xFFFF0000u), scale, 2 * j + 1, hi);
+        digits3((double)__uint_as_float(w[j] << 16), scale, 2 * j, lo);
+        digits3((double)__uint_as_float(w[j] & 0xFFFF0000u), scale, 2 * j + 1, lo);
+        digits3((double)__uint_as_float(w[j + 2] << 16), scale, 2 * j, hi);
+        digits3((double)__uint_as_float(w[j + 2] & 0xFFFF0000u), scale, 2 * j + 1, hi);
       }
 #pragma unroll
-      for (int p = 0; p < kDigits; ++p)
+      for (int p = 0; p < kXDigits; ++p)
         reinterpret_cast<uint2*>(a.x_digits + ((int64_t)p * a.T + t) * a.H)[v] = make_uint2(lo[p], hi[p]);
     }
   }
@@ -182,15 +199,15 @@ __global__ void __launch_bounds__(kSliceThreads) slice_w_kernel(RouterArgs a) {
       digits4((double)f[4 + j], scale, j, hi);
     }
 #pragma unroll
-    for (int p2 = 0; p2 < kDigits; ++p2)
+    for (int p2 = 0; p2 < kWDigits; ++p2)
       reinterpret_cast<uint2*>(a.w_digits + ((int64_t)p2 * a.E + e_row) * a.H)[v] = make_uint2(lo[p2], hi[p2]);
   }
 }
 
-// One (token tile, expert tile, K split) per CTA.  Warp 0 loads the four digit planes of both
-// operands for each 128-byte K block (2 stages), warp 1 issues the 13 digit-pair MMAs per
-// K step into the five class accumulators, warps 2-5 combine the classes of their 32 token
-// rows in FP64 and write the split's partial logits.
+// One (token tile, expert tile, K split) per CTA.  Warp 0 loads the three token and four
+// expert digit planes of each 128-byte K block (2 stages of 112 KB), warp 1 issues the 9
+// digit-pair MMAs per K step into the four class accumulators, warps 2-5 combine the classes
+// of their 32 token rows in FP64 and write the split's partial logits.
 __global__ void __launch_bounds__(kTcThreads, 1)
 router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constant__ CUtensorMap tma_w,
                  const RouterArgs a) {
@@ -240,12 +257,13 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
           tc_set_abort(&s.abort_flag, a.status);
           break;
         }
-        mbar_arrive_expect_tx(&s.full[stage], kDigits * (kAPlaneBytes + kBPlaneBytes));
+        mbar_arrive_expect_tx(&s.full[stage], kXDigits * kAPlaneBytes + kWDigits * kBPlaneBytes);
 #pragma unroll
-        for (int p = 0; p < kDigits; ++p) {
+        for (int p = 0; p < kXDigits; ++p)
           tma_load_2d(s.a[stage][p], &tma_x, &s.full[stage], kb * 128, (int)(p * a.T) + t0, pol);
+#pragma unroll
+        for (int p = 0; p < kWDigits; ++p)
           tma_load_2d(s.b[stage][p], &tma_w, &s.full[stage], kb * 128, p * a.E + e0, pol);
-        }
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kTcStages) { stage = 0; phase ^= 1u; }
@@ -271,9 +289,9 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
 #pragma unroll
           for (int c = 0; c < kClasses; ++c) {
 #pragma unroll
-            for (int i = 0; i < kDigits; ++i) {
+            for (int i = 0; i < kXDigits; ++i) {
               const int j = c - i;
-              if (j < 0 || j >= kDigits) continue;
+              if (j < 0 || j >= kWDigits) continue;
               mma_i8(tmem + kTcN * c, desc_k_sw128(smem_u32(s.a[stage][i]) + 32 * k),
                      desc_k_sw128(smem_u32(s.b[stage][j]) + 32 * k), idesc, (started >> c) & 1u);
               started |= 1u << c;
@@ -313,12 +331,11 @@ router_i8_kernel(const __grid_constant__ CUtensorMap tma_x, const __grid_constan
           if (ex == kExpNonFinite || ew == kExpNonFinite) {
             v = __longlong_as_double(0x7FF8000000000000ll);
           } else {
-            v = (double)(int)C[4][j];
-            v = __dadd_rn(v, (double)(int)C[3][j] * 256.0);
-            v = __dadd_rn(v, (double)(int)C[2][j] * 65536.0);
-            v = __dadd_rn(v, (double)(int)C[1][j] * 16777216.0);
-            v = __dadd_rn(v, (double)(int)C[0][j] * 4294967296.0);
-            v = ldexp(v, ex + ew - 60 + 16);   // class c carries 2^(8 (6 - c)) = 2^(8 (4 - c)) 2^16
+            v = (double)(int)C[3][j];
+            v = __dadd_rn(v, (double)(int)C[2][j] * 256.0);
+            v = __dadd_rn(v, (double)(int)C[1][j] * 65536.0);
+            v = __dadd_rn(v, (double)(int)C[0][j] * 16777216.0);
+            v = ldexp(v, ex + ew - 52 + 16);   // class c carries 2^(8 (5 - c)) = 2^(8 (3 - c)) 2^16
           }
           out[e] = v;
         }
@@ -337,7 +354,7 @@ static int tc_tiles(int64_t T, int E) { return (int)(((T + kTcM - 1) / kTcM) * (
 
 // K split: doubled while the grid stays within one CTA per SM and every split keeps at least
 // two K blocks; also large enough that a split's class sums stay below 2^31 (at most 26,112
-// columns of K per split: 5 * 2^14 * 26,112 < 2^31).
+// columns of K per split: 3 * 2^14 * 26,112 < 2^31).
 int router_tc_ksplit(int64_t T, int E, int H) {
   const int tiles = tc_tiles(T, E);
   const int kb_total = H / 128;
@@ -353,8 +370,8 @@ cudaError_t launch_router_tc(RouterArgs a, cudaStream_t stream) {
   a.ksplit = router_tc_ksplit(a.T, a.E, a.H);
   a.k_slice = a.H / a.ksplit;
   CUtensorMap tma_x, tma_w;
-  if (make_tma_2d(&tma_x, a.x_digits, (uint64_t)a.H, (uint64_t)kDigits * a.T, kTcM) != 0 ||
-      make_tma_2d(&tma_w, a.w_digits, (uint64_t)a.H, (uint64_t)kDigits * a.E, kTcN) != 0)
+  if (make_tma_2d(&tma_x, a.x_digits, (uint64_t)a.H, (uint64_t)kXDigits * a.T, kTcM) != 0 ||
+      make_tma_2d(&tma_w, a.w_digits, (uint64_t)a.H, (uint64_t)kWDigits * a.E, kTcN) != 0)
     return cudaErrorInvalidValue;
   slice_x_kernel<<<(unsigned)router_tc_amax_partials(a.T), kSliceThreads, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();

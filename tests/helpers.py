@@ -42,18 +42,31 @@ def _row_exponents(v: np.ndarray) -> np.ndarray:
     return np.where(m == 0, -125, np.maximum(e, -125))
 
 
-def router_logit_bound_int(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
+def _fixed_point(v: np.ndarray, bits: int) -> np.ndarray:
+    """Each row scaled to `bits`-bit fixed point from its exponent and rounded to the nearest
+    integer (ties to even), in the row's own units: RNE(v 2^(bits - e)) 2^(e - bits)."""
+    e = _row_exponents(v)[:, None]
+    return np.ldexp(np.rint(np.ldexp(v, bits - e)), e - bits)
+
+
+def router_logit_bound_int(x: np.ndarray, wr: np.ndarray, bias, H: int, worst: bool = False) -> np.ndarray:
     """The documented bound of the integer tensor-core logits (T > 64):
-    2^-24 |logit| + 2^(e_x - 31) sum|W_e| + 2^(e_W - 31) sum|x_t| + H 2^(e_x + e_W - 36)."""
+    2^-24 |logit| + sum_h |x_h - x'_h| |W_eh| + sum_h |x_h| |W_eh - W'_eh| + H 2^(e_x + e_W - 28),
+    x' and W' the 22-bit and 30-bit fixed-point rows the kernel multiplies.  ``worst``: the two
+    rounding sums replaced by their worst case 2^(e_x - 23) sum|W_e| + 2^(e_W - 31) sum|x_t|
+    (row sums only: cheap at any T)."""
     ex = _row_exponents(x)[:, None].astype(np.float64)
     ew = _row_exponents(wr)[None, :].astype(np.float64)
     logit = x @ wr.T
     if bias is not None:
         logit = logit + np.asarray(bias, dtype=np.float64)[None, :]
-    sw = np.abs(wr).sum(axis=1)[None, :]
-    sx = np.abs(x).sum(axis=1)[:, None]
-    return (U * np.abs(logit) + np.exp2(ex - 31) * sw + np.exp2(ew - 31) * sx + H * np.exp2(ex + ew - 36)
-            + 2.0 ** -60)
+    if worst:
+        rx = np.exp2(ex - 23) * np.abs(wr).sum(axis=1)[None, :]
+        rw = np.exp2(ew - 31) * np.abs(x).sum(axis=1)[:, None]
+    else:
+        rx = np.abs(x - _fixed_point(x, 22)) @ np.abs(wr).T
+        rw = np.abs(x) @ np.abs(wr - _fixed_point(wr, 30)).T
+    return U * np.abs(logit) + rx + rw + H * np.exp2(ex + ew - 28) + 2.0 ** -60
 
 
 def router_logit_bound_fp32(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
@@ -67,8 +80,9 @@ def router_logit_bound_fp32(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.n
 
 
 def router_logit_bound(x: np.ndarray, wr: np.ndarray, bias, H: int) -> np.ndarray:
-    """A bound that holds for either logits path: the larger of the two documented ones."""
-    return np.maximum(router_logit_bound_fp32(x, wr, bias, H), router_logit_bound_int(x, wr, bias, H))
+    """A bound that holds for either logits path: the larger of the two documented ones (the
+    integer one in its worst-case form)."""
+    return np.maximum(router_logit_bound_fp32(x, wr, bias, H), router_logit_bound_int(x, wr, bias, H, worst=True))
 
 
 def check_routing(gpu_idx: np.ndarray, gpu_w: np.ndarray, r, x, wr, bias, shape, w_rtol=2e-6,

@@ -49,7 +49,7 @@ def test_decode_step_bytes_match_the_stated_figure():
 
 
 def test_stored_traffic_applies_only_to_its_sources_and_workload(monkeypatch):
-    with open(os.path.join(ROOT, "profiles", "gemm_gateup_traffic.txt")) as f:
+    with open(bench.TRAFFIC_FILE) as f:
         vals = dict(line.split()[:2] for line in f if line.strip() and not line.startswith("#"))
     if vals["source_sha256"] != bench.kernel_source_hash():
         # the kernels changed since the counters were taken: the line reports no traffic
@@ -118,10 +118,22 @@ def test_config_entry_reports_the_dominant_kernel():
     p = {"hbm_gbs": 6546.2, "bf16_tflops": 1615.2, "bf16_tflops_sustained": 1365.0, "source": "measured"}
     counts = np.full(BEAM.E, 1024, dtype=np.int64)
     alg = bench.algorithmic(BEAM, 32768, counts)
+    gemms = {"gateup": bench.kernel_roofline(alg["gateup_bytes"], alg["gateup_flops"], 3.3, p),
+             "down": bench.kernel_roofline(alg["down_bytes"], alg["down_flops"], 3.3, p)}
     m = {"workload": "w", "T_per_rank": 32768, "experts_hit": 256, "ms_per_step": 8.0, "value": 1.0,
-         "stage_ms": {}, "alg": alg, "layer_roofline": {},
-         "gemms": {"gateup": bench.kernel_roofline(alg["gateup_bytes"], alg["gateup_flops"], 3.3, p),
-                   "down": bench.kernel_roofline(alg["down_bytes"], alg["down_flops"], 3.3, p)}}
+         "stage_ms": {}, "alg": alg, "layer_roofline": {}, "gemms": gemms,
+         "dominant": {**gemms["gateup"], "kernel": bench.GATEUP_KERNEL}}
     e = bench.config_entry(m, None)
-    assert e["roofline"]["bound"] == "tensor" and e["roofline"]["frac"] == m["gemms"]["gateup"]["frac"]
+    assert e["roofline"]["bound"] == "tensor" and e["roofline"]["frac"] == gemms["gateup"]["frac"]
+    assert e["roofline"]["kernel"] == bench.GATEUP_KERNEL
     assert e["gemms"]["down"]["bound"] == "tensor"
+    # short segments: the one launch that runs both GEMMs, on both GEMMs' bytes
+    counts = np.zeros(BEAM.E, dtype=np.int64)
+    counts[:99] = 1
+    alg = bench.algorithmic(BEAM, 16, counts)
+    both = bench.kernel_roofline(alg["gateup_bytes"] + alg["down_bytes"], alg["gateup_flops"] + alg["down_flops"],
+                                 0.32, p)
+    m.update({"alg": alg, "dominant": {**both, "kernel": bench.EXPERTS_KERNEL}})
+    e = bench.config_entry(m, None)
+    assert e["roofline"]["bound"] == "hbm" and e["roofline"]["kernel"] == bench.EXPERTS_KERNEL
+    assert e["roofline"]["achieved"] == pytest.approx((alg["gateup_bytes"] + alg["down_bytes"]) / 0.32e-3 / 1e9)
