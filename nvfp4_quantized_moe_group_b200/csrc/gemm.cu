@@ -483,11 +483,6 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         const int K = gu ? pg.K : pd.K;
         const int kb_count = k_blocks(K);
         const uint32_t acc_par = (uint32_t)it & 1u;
-        if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u, wait_ns)) {
-          set_abort(&s.abort_flag, P0.status);
-          break;
-        }
-        tc_fence_after();
         const uint32_t acc = tmem;
         for (int kb = 0; kb < kb_count; ++kb) {
           if (aborted(&s.abort_flag) || !mbar_wait(&s.full[stage], phase, wait_ns)) {
@@ -499,6 +494,14 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           const uint32_t a0 = smem_u32(s.a[stage]);
           const uint32_t b0 = smem_u32(s.b[stage]);
           if constexpr (kFp8) {
+            if (kb == 0) {
+              if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u, wait_ns)) {
+                set_abort(&s.abort_flag, P0.status);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
             // four K = 32 instructions per 128-byte K block (32 bytes apart, like the FP4 steps)
             for (int k = 0; k < 4; ++k)
               mma_f8(acc, desc_k_sw128(a0 + 32 * k), desc_k_sw128(b0 + 32 * k), idesc, (kb | k) != 0 ? 1u : 0u);
@@ -519,6 +522,17 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
 #pragma unroll
             for (int j = 0; j < kNT; ++j)
               tc_cp_32x128b_x4(sfb_t + 4 * (kNT * k + j), desc_sf_block(sb + (j * 4 + k) * kAtomBytes));
+          }
+          // the first K block's scale copies go out before the wait for the accumulator (they
+          // write only this stage's scale columns), so they overlap the previous item's
+          // accumulator read-out
+          if (kb == 0) {
+            if (aborted(&s.abort_flag) || !mbar_wait(&s.acc_empty, acc_par ^ 1u, wait_ns)) {
+              set_abort(&s.abort_flag, P0.status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
           }
           for (int k = 0; k < ksteps; ++k) {
             mma_nvf4(acc, desc_k_sw128(a0 + 32 * k), desc_k_sw128(b0 + 32 * k), idesc, sfa_t + 4 * k,

@@ -80,11 +80,13 @@ __host__ __device__ constexpr uint32_t idesc_i8(uint32_t m, uint32_t n) {
 // and zero rows take the smallest normal exponent).
 __device__ __forceinline__ int row_exponent(uint32_t biased) { return (int)(biased > 1u ? biased : 1u) - 126; }
 
-// Three balanced base-256 digits of v * 2^shift, |v * 2^shift| < 2^22 (exact power-of-two
-// scaling in FP64, then round to nearest even), packed into one byte each of the three words'
-// byte lane `lane`.
-__device__ __forceinline__ void digits3(double v, double scale, uint32_t lane, uint32_t* d) {
-  int X = __double2int_rn(v * scale);
+// Three balanced base-256 digits of RNE(v 2^(s1 + s2)) for a BF16 value v with
+// |v 2^(s1 + s2)| < 2^22, the scaling applied as two FP32 multiplications by 2^s1 and 2^s2
+// (s1, s2 of the same sign, each within the normal range): exact, since an upward scaling
+// cannot overflow and a downward one only underflows values that round to 0 anyway.  Packed
+// into one byte each of the three words' byte lane `lane`.
+__device__ __forceinline__ void digits3(float v, float scale1, float scale2, uint32_t lane, uint32_t* d) {
+  int X = __float2int_rn(__fmul_rn(__fmul_rn(v, scale1), scale2));
   const int d2 = ((X + 128) & 255) - 128;
   X = (X - d2) >> 8;
   const int d1 = ((X + 128) & 255) - 128;
@@ -147,17 +149,20 @@ __global__ void __launch_bounds__(kSliceThreads) slice_x_kernel(RouterArgs a) {
     }
     const int e = row_exponent(be);
     if (threadIdx.x == 0) a.x_exp[t] = e;
-    const double scale = ldexp(1.0, 22 - e);
+    // 2^(22 - e) as 2^k1 * 2^k2, e in [-125, 128]: k1, k2 in [-53, 74]
+    const int k = 22 - e, k1 = k / 2, k2 = k - k1;
+    const float scale1 = __uint_as_float((uint32_t)(127 + k1) << 23);
+    const float scale2 = __uint_as_float((uint32_t)(127 + k2) << 23);
     for (int v = threadIdx.x; v < n8; v += kSliceThreads) {
       const uint4 q = __ldg(src + v);
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
       uint32_t lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0};
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        digits3((double)__uint_as_float(w[j] << 16), scale, 2 * j, lo);
-        digits3((double)__uint_as_float(w[j] & 0xFFFF0000u), scale, 2 * j + 1, lo);
-        digits3((double)__uint_as_float(w[j + 2] << 16), scale, 2 * j, hi);
-        digits3((double)__uint_as_float(w[j + 2] & 0xFFFF0000u), scale, 2 * j + 1, hi);
+        digits3(__uint_as_float(w[j] << 16), scale1, scale2, 2 * j, lo);
+        digits3(__uint_as_float(w[j] & 0xFFFF0000u), scale1, scale2, 2 * j + 1, lo);
+        digits3(__uint_as_float(w[j + 2] << 16), scale1, scale2, 2 * j, hi);
+        digits3(__uint_as_float(w[j + 2] & 0xFFFF0000u), scale1, scale2, 2 * j + 1, hi);
       }
 #pragma unroll
       for (int p = 0; p < kXDigits; ++p)
