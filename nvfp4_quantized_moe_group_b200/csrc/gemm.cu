@@ -20,8 +20,9 @@
 //             h = silu(g_x g_gate acc_gate) * (g_x g_up acc_up) in FP32, requantised to
 //             NVFP4 with the expert's static scale g_h (the down GEMM's A operand);
 //   down:     acc_out[token] += w * g_h * g_down * acc, FP32 additions into the token's row:
-//             with full segments each lane stages its row's 32-column piece in shared memory
-//             and adds it with one bulk reduction (cp.reduce.async.bulk .add.f32, 128 bytes);
+//             with full segments half the lanes at a time stage their row's 64-column piece in
+//             shared memory and add it with one bulk reduction (cp.reduce.async.bulk .add.f32,
+//             256 bytes);
 //             when segments hold few rows, vector reductions straight from the 16x256b register
 //             layout.
 // Every wait is bounded; a wait that runs out sets the timeout bit of the status word and
@@ -89,9 +90,9 @@ struct __align__(1024) Smem {
   uint8_t b[C::kStages][kNT * kTileBytes];
   uint8_t sfa[C::kStages][C::kSfaBytes];
   uint8_t sfb[C::kStages][C::kSfbBytes];
-  // down, full segments: per epilogue warp, 32 staged row pieces of 32 FP32 values, 144 bytes
-  // apart (16-byte aligned for the bulk reductions; the float4 stores of 8 consecutive lanes
-  // fall in 8 different bank groups)
+  // down, full segments: per epilogue warp, 16 staged row pieces of 64 FP32 values, 272 bytes
+  // apart (32 pieces of 32 values, 144 bytes apart, for FP8; 16-byte aligned for the bulk
+  // reductions, and the float4 stores of consecutive lanes fall in different bank groups)
   alignas(16) float stage_rows[C::kStaging ? kEpiWarps : 1][32 * 36];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
@@ -727,15 +728,16 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + half * (kN / 2) + c * 32, R[c]);
         tmem_ld_wait();
         release();
-        // each lane's row piece (32 columns, 128 bytes) staged in shared memory and added to the
-        // token's accumulator row by one bulk reduction (async proxy)
+        // row pieces staged in shared memory and added to the tokens' accumulator rows by bulk
+        // reductions (async proxy)
         const float scale = c0s;
-        float* mine = s.stage_rows[warp - 2] + lane * 36;
+        if constexpr (kFp8) {
+          // FP8: each lane's 32-column piece (128 bytes), one reduction per piece
+          float* mine = s.stage_rows[warp - 2] + lane * 36;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int c0 = half * (kN / 2) + c * 32;
-          if (c > 0) bulk_wait_read0();
-          if constexpr (kFp8) {
+          for (int c = 0; c < 4; ++c) {
+            const int c0 = half * (kN / 2) + c * 32;
+            if (c > 0) bulk_wait_read0();
             const float* wsc = P.w_scale + (int64_t)wk.e * P.n_total + wk.nt * kN + c0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -746,17 +748,39 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
                               __fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i + 2]), scale), w4.z),
                               __fmul_rn(__fmul_rn(__uint_as_float(R[c][4 * i + 3]), scale), w4.w));
             }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              *reinterpret_cast<float4*>(mine + 4 * i) =
-                  make_float4(__fmul_rn(__uint_as_float(R[c][4 * i]), scale), __fmul_rn(__uint_as_float(R[c][4 * i + 1]), scale),
-                              __fmul_rn(__uint_as_float(R[c][4 * i + 2]), scale), __fmul_rn(__uint_as_float(R[c][4 * i + 3]), scale));
+            if (token >= 0) {
+              fence_proxy_async_smem();
+              bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, mine, 128u);
+              bulk_commit();
+            }
           }
-          if (token >= 0) {
-            fence_proxy_async_smem();
-            bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, mine, 128u);
-            bulk_commit();
+        } else {
+          // 16 lanes at a time stage their row's 64 columns (256 bytes) and add each with one
+          // bulk reduction: the L2 takes bulk reductions at a rate per operation, so 256-byte
+          // operations move twice the bytes of 128-byte ones (T = 32768: 2.96 -> 2.73 ms)
+          float* slot = s.stage_rows[warp - 2] + (lane & 15) * 68;
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c0 = half * (kN / 2) + c2 * 64;
+#pragma unroll
+            for (int rd = 0; rd < 2; ++rd) {
+              if ((lane >> 4) == rd) {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                  for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4*>(slot + 32 * cc + 4 * i) =
+                        make_float4(__fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i]), scale), __fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i + 1]), scale),
+                                    __fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i + 2]), scale), __fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i + 3]), scale));
+                if (token >= 0) {
+                  fence_proxy_async_smem();
+                  bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, slot, 256u);
+                  bulk_commit();
+                  bulk_wait_read0();
+                }
+              }
+              __syncwarp();
+            }
           }
         }
         bulk_wait_read0();
