@@ -60,11 +60,11 @@ constexpr int kNT = kN / 128;                       // 128-row weight tiles per 
 // (per-tile counters), so no CTA idles at a boundary between two launches.
 enum : int { kModeDown = 0, kModeGateUp = 1, kModeFused = 2 };
 
-// kDecode: segments average fewer than 32 rows.  The epilogues then read the whole
-// accumulator before any arithmetic (gate/up) and reduce straight from the 16x256b register
-// layout (down), and the down GEMM keeps 4 stages.  With full segments the gate/up epilogue
-// frees the accumulator after its first 32-feature chunk, and the down GEMM stages 32-column
-// row pieces in shared memory for bulk reductions (3 stages): both measured faster there.
+// kDecode: segments average fewer than 32 rows.  The down epilogue then reduces straight from
+// the 16x256b register layout, and the down GEMM keeps 4 stages; with full segments it stages
+// row pieces in shared memory for bulk reductions (3 stages), measured faster there.  The
+// gate/up epilogue reads its whole share of the accumulator before any arithmetic in both
+// regimes (the accumulator is free for the next item's MMAs as early as possible).
 // The fused launch keeps 4 stages and reduces from registers in both regimes.
 //
 // kFp8: the FP8 W8A8 variant (E4M3 x E4M3 with FP32 accumulation, kind::f8f6f4): a 128-byte
@@ -657,36 +657,21 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
           // [128 half, +64) are their gate, [128 half + 64, +64) their up projections
           const int t = wk.nt * kNT + half;
           const int tcol = half * 128;
-          if constexpr (kDecode) {
-            // all four 32-column chunks into registers first, then the accumulator is released
-            uint32_t G0[32], U0[32], G1[32], U1[32];
-            tmem_ld_32x32b_x32(t_row + tcol, G0);
-            tmem_ld_32x32b_x32(t_row + tcol + 64, U0);
-            tmem_ld_32x32b_x32(t_row + tcol + 32, G1);
-            tmem_ld_32x32b_x32(t_row + tcol + 96, U1);
-            tmem_ld_wait();
-            release();
-            float h[32];
-            swiglu32(G0, U0, sg, su, h);
-            if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64, h);
-            quant_store32(h, gh, r_t, valid, row, t * 64, P, n_ct);
-            swiglu32(G1, U1, sg, su, h);
-            if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64 + 32, h);
-            quant_store32(h, gh, r_t, valid, row, t * 64 + 32, P, n_ct);
-          } else {
-#pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-              uint32_t G[32], U[32];
-              tmem_ld_32x32b_x32(t_row + tcol + 32 * pr, G);
-              tmem_ld_32x32b_x32(t_row + tcol + 64 + 32 * pr, U);
-              tmem_ld_wait();
-              if (pr == 1) release();
-              float h[32];
-              swiglu32(G, U, sg, su, h);
-              if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64 + 32 * pr, h);
-              quant_store32(h, gh, r_t, valid, row, t * 64 + 32 * pr, P, n_ct);
-            }
-          }
+          // all four 32-column chunks into registers first, then the accumulator is released
+          uint32_t G0[32], U0[32], G1[32], U1[32];
+          tmem_ld_32x32b_x32(t_row + tcol, G0);
+          tmem_ld_32x32b_x32(t_row + tcol + 64, U0);
+          tmem_ld_32x32b_x32(t_row + tcol + 32, G1);
+          tmem_ld_32x32b_x32(t_row + tcol + 96, U1);
+          tmem_ld_wait();
+          release();
+          float h[32];
+          swiglu32(G0, U0, sg, su, h);
+          if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64, h);
+          quant_store32(h, gh, r_t, valid, row, t * 64, P, n_ct);
+          swiglu32(G1, U1, sg, su, h);
+          if (P.h_dbg != nullptr && valid) store_h_dbg(P, wk, row_l, t * 64 + 32, h);
+          quant_store32(h, gh, r_t, valid, row, t * 64 + 32, P, n_ct);
         }
       } else if constexpr (!C::kStaging) {
         // two 16-lane blocks of this warp's rows, 128 columns each, in the 16x256b layout:
