@@ -147,11 +147,15 @@ __global__ void __launch_bounds__(1024) quantize_kernel(QuantizeArgs a) {
 #pragma unroll
     for (int i = 0; i < 2 * kBpl; ++i) codes[i] = 0;
     if (live) {
+      // every load of the lane in flight before the conversions (asm statements) start
       const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.cols + (int64_t)b * 16);
+      uint4 v[2 * kBpl];
+#pragma unroll
+      for (int i = 0; i < 2 * kBpl; ++i) v[i] = __ldg(src + i);
 #pragma unroll
       for (int k = 0; k < kBpl; ++k) {
-        const uint4 v0 = __ldg(src + 2 * k), v1 = __ldg(src + 2 * k + 1);
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t w[8] = {v[2 * k].x, v[2 * k].y, v[2 * k].z, v[2 * k].w,
+                               v[2 * k + 1].x, v[2 * k + 1].y, v[2 * k + 1].z, v[2 * k + 1].w};
         sl |= quantize_block(w, r_t, g, &codes[2 * k], &codes[2 * k + 1]) << (8 * k);
       }
     }
