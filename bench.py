@@ -824,9 +824,10 @@ def run_ep(args, world, rank, local):
             "data": "synthetic (seeded counter-hash inputs; random-init NVFP4 weights)",
             "config": {"workload": wl.describe() + f" per rank, expert parallel over {world} rank(s)",
                        "T_per_rank": T, "experts_per_rank": layer.e_count, "local_experts_hit": hit_local,
-                       "parallelism": f"ep{world} " + ("(all-gather tokens, reduce-scatter FP32 sums)"
-                                                      if args.exchange == "gather" else
-                                                      "(all-to-all of quantised pair rows and weighted output rows)"),
+                       "parallelism": f"ep{world} " + {
+                           "gather": "(all-gather tokens, reduce-scatter FP32 sums)",
+                           "peer": "(all-gather tokens, down GEMM adds the FP32 sums into the owning ranks' memory)",
+                           "all_to_all": "(all-to-all of quantised pair rows and weighted output rows)"}[args.exchange],
                        "l2": "no flush: every step streams the rank's routed experts' weights"},
             "roofline": {"bound": "hbm", "achieved": local_bytes / (ms / 1e3) / 1e9, "peak": p["hbm_gbs"],
                          "unit": "GB/s", "frac": local_bytes / (ms / 1e3) / (p["hbm_gbs"] * 1e9), "traffic": None,
@@ -994,8 +995,9 @@ def main():
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the ranks (each holds E/N experts) instead of one full replica "
                          "per GPU")
-    ap.add_argument("--exchange", choices=["gather", "all_to_all"], default="gather",
-                    help="with --ep: all-gather the tokens and reduce-scatter FP32 sums, or send each pair's "
+    ap.add_argument("--exchange", choices=["gather", "peer", "all_to_all"], default="gather",
+                    help="with --ep: all-gather the tokens and reduce-scatter FP32 sums; the same gather with the "
+                         "down GEMM adding the sums into the owning ranks' memory (peer); or send each pair's "
                          "quantised row to its expert's rank and its output row back (NCCL all-to-all)")
     args = ap.parse_args()
     if args.warmup < 3:

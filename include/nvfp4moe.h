@@ -354,6 +354,40 @@ NVFP4MOE_API int nvfp4moe_forward_partial(const nvfp4moe_experts* experts, const
                                           const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
 NVFP4MOE_API int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream);
 
+/* ------------------------------------ expert parallel, combine into peer memory ----
+ * nvfp4moe_forward_partial with the cross-rank sum folded into the down GEMM: instead of
+ * writing [T_all][H] FP32 sums for a reduce-scatter, the down GEMM's epilogue adds each pair's
+ * weighted row straight into the accumulator of the rank that owns the token, over NVLink (or
+ * into local memory for the caller's own rows), with the same FP32 reductions it uses for a
+ * local accumulator: the exchange overlaps the MMAs tile by tile and no reduce-scatter runs.
+ *
+ *   acc_peers      device array of n_peers pointers (8-byte aligned; pointers 16-byte
+ *                  aligned): rank d's FP32 accumulator [rows_per_peer][H], in this process's
+ *                  address space (its own allocation, or another GPU's memory mapped with
+ *                  nvfp4moe_ipc_open); token t of hidden_all is row t % rows_per_peer of rank
+ *                  t / rows_per_peer.  n_peers * rows_per_peer must equal T.
+ *   the other arguments as for nvfp4moe_forward_partial.
+ * Every owner's accumulator must hold zeros (or the values to add to) before any rank's call
+ * starts adding into it, and an owner reads its rows (nvfp4moe_finalize) only after every
+ * rank's call has completed: the caller orders both (a barrier between the ranks' streams).
+ * The ranks' additions into one row run in no fixed order, so the sums equal the single-GPU
+ * layer's up to the order of FP32 additions.  The call writes nothing else in the peers'
+ * memory, and reads none of it.  ERR_SHAPE when n_peers * rows_per_peer != T or n_peers < 1.
+ *
+ * nvfp4moe_ipc_get_handle / _open / _close: CUDA inter-process handles of device memory, for
+ * mapping the other ranks' accumulators.  get_handle: the handle (NVFP4MOE_IPC_HANDLE_BYTES
+ * opaque bytes) of the device allocation that contains dev_ptr, and dev_ptr's byte offset from
+ * that allocation's start.  open (in another process): maps that allocation and returns its
+ * start, to which the importer adds the offset.  close unmaps an address that open returned. */
+#define NVFP4MOE_IPC_HANDLE_BYTES 64
+NVFP4MOE_API int nvfp4moe_forward_partial_peer(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
+                                               const float* w_router, const float* logit_bias,
+                                               float* const* acc_peers, int32_t n_peers, int64_t rows_per_peer,
+                                               const nvfp4moe_debug* dbg, void* ws, size_t ws_bytes, void* stream);
+NVFP4MOE_API int nvfp4moe_ipc_get_handle(const void* dev_ptr, void* handle_out, int64_t* offset_out);
+NVFP4MOE_API int nvfp4moe_ipc_open(const void* handle, void** dev_ptr_out);
+NVFP4MOE_API int nvfp4moe_ipc_close(void* dev_ptr);
+
 /* ------------------------------- expert parallelism, all-to-all exchange of quantised rows ----
  * The exchange of the experts' placement across devices ("Reflection releases Beam ...",
  * section "Tool calling and multi-node setups": experts on the devices, a device count that

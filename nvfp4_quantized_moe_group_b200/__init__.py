@@ -18,14 +18,16 @@ Typical use (all tensors on one CUDA device; the current stream is used)::
 Also: ``quantize`` / ``route`` / ``route_noalloc`` (the layer's steps alone), ``forward_residual`` (RMSNorm in,
 weighted residual add out), ``quantize_weights_lh`` (local-Hessian weight scales),
 ``Fp8Experts`` / ``forward_fp8`` (the FP8 W8A8 variant), and ``ep.ExpertParallelLayer`` with
-``forward_partial`` / ``finalize`` or ``amax`` / ``ep_dispatch`` / ``ep_experts`` / ``ep_combine``
-(experts spread over the ranks of a process group; a gather exchange or an all-to-all one).
+``forward_partial`` / ``finalize``, ``forward_partial_peer`` / ``ipc_handle`` / ``ipc_open`` or ``amax`` /
+``ep_dispatch`` / ``ep_experts`` / ``ep_combine`` (experts spread over the ranks of a process group;
+a gather exchange, the same with the combine into the owners' memory inside the down GEMM, or an
+all-to-all one).
 """
 from ._lib import (  # noqa: F401
     Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, route_noalloc, forward,
     forward_residual, status_read, last_device_status, workspace_bytes, quantize_fp8, Fp8Experts, forward_fp8, forward_fp8_workspace_bytes,
     forward_partial, finalize, amax, ep_dispatch, ep_dispatch_workspace_bytes, ep_experts, ep_experts_workspace_bytes,
-    ep_combine,
+    ep_combine, forward_partial_peer, ipc_handle, ipc_open, ipc_close,
     status_string, last_launch_count, forward_workspace_bytes, route_workspace_bytes,
     quantize_workspace_bytes, swizzled_scale_bytes, declared_symbols, lib, LIB_PATH, StageTimer, STAGES,
     OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_WORKSPACE, ERR_NONFINITE, ERR_TIMEOUT, ERR_DEVICE,

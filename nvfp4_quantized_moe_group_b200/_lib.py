@@ -118,6 +118,11 @@ _SIGS = {
     "nvfp4moe_experts_range": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
     "nvfp4moe_forward_partial": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_finalize": (ctypes.c_int, [_P, _I64, _P, _P]),
+    "nvfp4moe_forward_partial_peer": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.c_int32, _I64,
+                                                     ctypes.POINTER(Debug), _P, _SZ, _P]),
+    "nvfp4moe_ipc_get_handle": (ctypes.c_int, [_P, _P, ctypes.POINTER(_I64)]),
+    "nvfp4moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(_P)]),
+    "nvfp4moe_ipc_close": (ctypes.c_int, [_P]),
     "nvfp4moe_forward_workspace_bytes": (_SZ, [ctypes.POINTER(Cfg), _I64]),
     "nvfp4moe_forward": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, ctypes.POINTER(Debug), _P, _SZ, _P]),
     "nvfp4moe_forward_residual": (ctypes.c_int, [_P, _P, _I64, _P, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
@@ -634,6 +639,51 @@ def forward_partial(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, b
     if debug:
         return acc_out, tensors
     return acc_out
+
+
+def forward_partial_peer(experts: Experts, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None,
+                         acc_peers: torch.Tensor, rows_per_peer: int, ws: torch.Tensor | None = None, stream=None):
+    """One rank's part of the layer with the cross-rank sum folded into the down GEMM
+    (nvfp4moe_forward_partial_peer): token t's weighted expert rows are added into row
+    t % rows_per_peer of the accumulator at acc_peers[t // rows_per_peer] (an int64 device
+    tensor of device addresses, one per rank)."""
+    cfg = experts.cfg
+    specs = _layer_specs(cfg, x, w_router, bias)
+    T, H = x.shape
+    dev = x.device
+    _require(*specs, (acc_peers, "acc_peers", torch.int64, (acc_peers.numel(),)), (ws, "ws", torch.uint8, None))
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(cfg, T), dev)
+    st = lib().nvfp4moe_forward_partial_peer(experts.handle, _ptr(x), T, _ptr(w_router), _ptr(bias), _ptr(acc_peers),
+                                             acc_peers.numel(), int(rows_per_peer), None, _ptr(ws), ws.numel(),
+                                             _stream(stream))
+    _check(st, "nvfp4moe_forward_partial_peer")
+
+
+IPC_HANDLE_BYTES = 64
+
+
+def ipc_handle(t: torch.Tensor) -> tuple[bytes, int]:
+    """The inter-process handle of the device allocation holding t and t's byte offset in it
+    (nvfp4moe_ipc_get_handle)."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_int64()
+    _check(lib().nvfp4moe_ipc_get_handle(ctypes.c_void_p(t.data_ptr()), buf, ctypes.byref(off)),
+           "nvfp4moe_ipc_get_handle")
+    return buf.raw, int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Maps another process's allocation (nvfp4moe_ipc_open); returns its device address here."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    ptr = ctypes.c_void_p()
+    _check(lib().nvfp4moe_ipc_open(handle, ctypes.byref(ptr)), "nvfp4moe_ipc_open")
+    return int(ptr.value)
+
+
+def ipc_close(address: int):
+    _check(lib().nvfp4moe_ipc_close(ctypes.c_void_p(address)), "nvfp4moe_ipc_close")
 
 
 def finalize(acc: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -666,14 +666,18 @@ size_t nvfp4moe_forward_workspace_bytes(const nvfp4moe_cfg* cfg, int64_t T_max) 
 // The layer; with res, finalize adds the output into the residual stream.
 // acc_out: NULL for the whole layer (BF16 out_bf16); otherwise the FP32 sums of the handle's
 // experts' contributions are left in acc_out [T][H] and there is no finalize.
+// acc_peers: the down GEMM adds each token's rows into the owning rank's accumulator instead
+// (the workspace's own accumulator is then unused), rows_per_peer tokens per rank.
 static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T, const float* w_router,
                         const float* logit_bias, void* out_bf16, const Residual* res, const nvfp4moe_debug* dbg,
-                        void* ws, size_t ws_bytes, void* stream, float* acc_out = nullptr) {
+                        void* ws, size_t ws_bytes, void* stream, float* acc_out = nullptr,
+                        float* const* acc_peers = nullptr, int64_t rows_per_peer = 0) {
   g_launches = 0;
   if (x == nullptr) return NVFP4MOE_ERR_ARG;
   const nvfp4moe_cfg& c = x->cfg;
   if (T < 1 || T > (1 << 20)) return NVFP4MOE_ERR_SHAPE;
-  if (hidden_bf16 == nullptr || w_router == nullptr || (out_bf16 == nullptr && acc_out == nullptr) || ws == nullptr)
+  if (hidden_bf16 == nullptr || w_router == nullptr ||
+      (out_bf16 == nullptr && acc_out == nullptr && acc_peers == nullptr) || ws == nullptr)
     return NVFP4MOE_ERR_ARG;
   if (!aligned(hidden_bf16, 16) || !aligned(w_router, 16) || !aligned(out_bf16, 16) || !aligned(acc_out, 16) ||
       !aligned(ws, kAlign))
@@ -873,6 +877,8 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
   gd.K = c.I;
   gd.n_total = c.H;
   gd.h_dbg = nullptr;
+  gd.acc_peers = acc_peers;
+  gd.rows_per_peer = rows_per_peer;
   // one launch for both GEMMs when segments are short (weight streaming dominates and the
   // boundary between two launches costs a few per cent); with full segments the down GEMM's
   // FP32 reductions, bound by the L2's reduction rate, slow the gate/up loads they would run
@@ -905,7 +911,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ++g_launches;
   }
 
-  if (acc_out == nullptr) {
+  if (acc_out == nullptr && acc_peers == nullptr) {
     FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,
                     res != nullptr ? res->a : 0.0f, res != nullptr ? res->b : 0.0f};
     ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
@@ -949,6 +955,67 @@ int nvfp4moe_forward_partial(const nvfp4moe_experts* x, const void* hidden_bf16,
   g_launches = 0;
   if (acc_out == nullptr) return NVFP4MOE_ERR_ARG;
   return forward_core(x, hidden_bf16, T, w_router, logit_bias, nullptr, nullptr, dbg, ws, ws_bytes, stream, acc_out);
+}
+
+int nvfp4moe_forward_partial_peer(const nvfp4moe_experts* x, const void* hidden_bf16, int64_t T,
+                                  const float* w_router, const float* logit_bias, float* const* acc_peers,
+                                  int32_t n_peers, int64_t rows_per_peer, const nvfp4moe_debug* dbg, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  if (acc_peers == nullptr || !aligned(acc_peers, 8)) return NVFP4MOE_ERR_ARG;
+  if (n_peers < 1 || rows_per_peer < 1 || (int64_t)n_peers * rows_per_peer != T) return NVFP4MOE_ERR_SHAPE;
+  if (dbg != nullptr && dbg->acc != nullptr) return NVFP4MOE_ERR_ARG;   // the sums are in the peers
+  return forward_core(x, hidden_bf16, T, w_router, logit_bias, nullptr, nullptr, dbg, ws, ws_bytes, stream, nullptr,
+                      acc_peers, rows_per_peer);
+}
+
+namespace {
+using AddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(ptr);
+  }
+  return fn;
+}
+}  // namespace
+
+int nvfp4moe_ipc_get_handle(const void* dev_ptr, void* handle_out, int64_t* offset_out) {
+  static_assert(sizeof(cudaIpcMemHandle_t) == NVFP4MOE_IPC_HANDLE_BYTES, "IPC handle size");
+  if (dev_ptr == nullptr || handle_out == nullptr || offset_out == nullptr) return NVFP4MOE_ERR_ARG;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  AddressRangeFn range = address_range_fn();
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range == nullptr || range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return NVFP4MOE_ERR_ARG;                                      // not device memory
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  std::memcpy(handle_out, &h, sizeof(h));
+  *offset_out = (int64_t)(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_ipc_open(const void* handle, void** dev_ptr_out) {
+  if (handle == nullptr || dev_ptr_out == nullptr) return NVFP4MOE_ERR_ARG;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  if (cudaIpcOpenMemHandle(dev_ptr_out, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  return NVFP4MOE_OK;
+}
+
+int nvfp4moe_ipc_close(void* dev_ptr) {
+  if (dev_ptr == nullptr) return NVFP4MOE_ERR_ARG;
+  int st = check_device();
+  if (st != NVFP4MOE_OK) return st;
+  return cudaIpcCloseMemHandle(dev_ptr) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
 }
 
 int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream) {

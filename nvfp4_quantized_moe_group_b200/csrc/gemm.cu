@@ -244,6 +244,14 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 // Orders this thread's generic-proxy global accesses with its async-proxy (TMA, bulk copy) ones.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
+// The FP32 accumulator row of a token: the launch's own accumulator, or the row in the owning
+// rank's accumulator (expert parallelism with the combine into peer memory).
+__device__ __forceinline__ float* acc_row(const GemmArgs& p, int token) {
+  if (p.acc_peers != nullptr)
+    return p.acc_peers[token / p.rows_per_peer] + (int64_t)(token % p.rows_per_peer) * p.H;
+  return p.acc + (int64_t)token * p.H;
+}
+
 __device__ __forceinline__ void set_abort(int* flag, uint32_t* status) {
   raise_status(status, kStatusTimeout);
   *reinterpret_cast<volatile int*>(flag) = 1;
@@ -691,7 +699,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             const int tok = __shfl_sync(0xffffffffu, token, r);
             const float sc = __shfl_sync(0xffffffffu, c0s, r);
             if (tok >= 0) {
-              float* dst = P.acc + (int64_t)tok * P.H + wk.nt * kN + half * (kN / 2) + cq;
+              float* dst = acc_row(P, tok) + wk.nt * kN + half * (kN / 2) + cq;
               const float* wsc = kFp8 ? P.w_scale + (int64_t)wk.e * P.n_total + wk.nt * kN + half * (kN / 2) + cq
                                       : nullptr;
 #pragma unroll
@@ -735,7 +743,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             }
             if (token >= 0) {
               fence_proxy_async_smem();
-              bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, mine, 128u);
+              bulk_reduce_add_f32(acc_row(P, token) + wk.nt * kN + c0, mine, 128u);
               bulk_commit();
             }
           }
@@ -759,7 +767,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
                                     __fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i + 2]), scale), __fmul_rn(__uint_as_float(R[2 * c2 + cc][4 * i + 3]), scale));
                 if (token >= 0) {
                   fence_proxy_async_smem();
-                  bulk_reduce_add_f32(P.acc + (int64_t)token * P.H + wk.nt * kN + c0, slot, 256u);
+                  bulk_reduce_add_f32(acc_row(P, token) + wk.nt * kN + c0, slot, 256u);
                   bulk_commit();
                   bulk_wait_read0();
                 }

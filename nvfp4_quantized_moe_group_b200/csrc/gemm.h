@@ -37,6 +37,8 @@ struct GemmArgs {
   int64_t zero_acc_elems;      // warps (a slice per work item; gate/up launch only)
   // down epilogue
   float* acc;                  // [T][H]
+  float* const* acc_peers;     // optional: token t's row is acc_peers[t / rows_per_peer] +
+  int64_t rows_per_peer;       //   (t % rows_per_peer) * H instead of acc + t * H
   const int32_t* row_pair;     // [rows_cap]
   const float* wts;            // [T*topk]
   const float* alpha_down;     // [E] = g_h * g_down

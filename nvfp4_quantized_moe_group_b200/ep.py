@@ -32,6 +32,17 @@ With ``exchange="all_to_all"`` (large batches) the pairs travel instead of the t
 Per step and rank that moves T topk (H/2 + H/16 + 8) bytes out and T topk H 4 bytes back,
 against G T H 2 gathered and G T H 4 reduce-scattered bytes for the gather exchange, and each
 rank routes and quantises T tokens instead of G T.
+
+With ``exchange="peer"`` the gather exchange's reduce-scatter disappears into the down GEMM:
+every rank maps the other ranks' FP32 accumulators into its address space once (CUDA
+inter-process handles exchanged through the process group), and each step
+
+  1. all-gathers the ranks' BF16 token rows, zeroes its own accumulator, and waits for every
+     rank to have done so (a collective on the stream);
+  2. nvfp4moe_forward_partial_peer: the rank's experts on all gathered tokens, the down
+     GEMM's epilogue adding each weighted row straight into the owning rank's accumulator
+     (over NVLink for other ranks' tokens), overlapped with the MMAs;
+  3. waits for every rank's additions (a second collective) and rounds its own rows to BF16.
 """
 from __future__ import annotations
 
@@ -61,13 +72,14 @@ class ExpertParallelLayer:
     def __init__(self, cfg: _lib.Cfg, group=None,
                  partial: Callable[[torch.Tensor, torch.Tensor, torch.Tensor | None], torch.Tensor] | None = None,
                  finalize: Callable[[torch.Tensor], torch.Tensor] | None = None,
-                 exchange: str = "gather", a2a_ops: dict | None = None):
-        """``exchange``: "gather" (all-gather the tokens, reduce-scatter FP32 sums) or
+                 exchange: str = "gather", a2a_ops: dict | None = None, peer_ops: dict | None = None):
+        """``exchange``: "gather" (all-gather the tokens, reduce-scatter FP32 sums), "peer" (the
+        same gather, the sums added into the owners' accumulators by the down GEMM) or
         "all_to_all" (send each pair's quantised row to its expert's rank and its weighted
-        output row back).  ``a2a_ops`` replaces the all-to-all path's library calls (keys
-        amax, dispatch, experts, combine; the signatures of the default methods below), to
-        exercise the exchange without a GPU."""
-        if exchange not in ("gather", "all_to_all"):
+        output row back).  ``a2a_ops`` / ``peer_ops`` replace those paths' library calls (keys
+        amax, dispatch, experts, combine / alloc, handle, open, close, partial_peer; the
+        signatures of the default methods below), to exercise the exchanges without a GPU."""
+        if exchange not in ("gather", "all_to_all", "peer"):
             raise ValueError(f"unknown exchange {exchange!r}")
         self.cfg = cfg
         self.group = group
@@ -75,6 +87,10 @@ class ExpertParallelLayer:
         self._a2a = {"amax": self._amax_cuda, "dispatch": self._dispatch_cuda, "experts": self._experts_cuda,
                      "combine": self._combine_cuda}
         self._a2a.update(a2a_ops or {})
+        self._p = {"alloc": self._peer_alloc_cuda, "handle": _lib.ipc_handle, "open": _lib.ipc_open,
+                   "close": _lib.ipc_close, "partial_peer": self._partial_peer_cuda}
+        self._p.update(peer_ops or {})
+        self._peer = None
         initialized = dist.is_available() and dist.is_initialized()
         self.world = dist.get_world_size(group) if initialized else 1
         self.rank = dist.get_rank(group) if initialized else 0
@@ -161,16 +177,80 @@ class ExpertParallelLayer:
         self._all_to_all(back, rows, sc, rc)
         return self._a2a["combine"](back, send["pos"], T)
 
+    # ----------------------------------------------- combine into the owners' memory ----
+    def _peer_alloc_cuda(self, T: int, H: int, device) -> torch.Tensor:
+        return torch.zeros((T, H), dtype=torch.float32, device=device)
+
+    def _partial_peer_cuda(self, x_all: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None,
+                           table: torch.Tensor, rows_per_peer: int):
+        ex = self.create_experts()
+        need = _lib.forward_workspace_bytes(self.cfg, x_all.shape[0])
+        if self._ws is None or self._ws.numel() < need or self._ws.device != x_all.device:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=x_all.device)
+        _lib.forward_partial_peer(ex, x_all, w_router, bias, table, rows_per_peer, ws=self._ws)
+
+    def _peer_setup(self, T: int, H: int, device) -> dict:
+        """This rank's accumulator [T, H] FP32 and the table of every rank's accumulator address
+        in this process (the other ranks' mapped through inter-process handles), made once per
+        token count."""
+        if self._peer is not None and self._peer["T"] == T:
+            return self._peer
+        self._peer_close()
+        acc = self._p["alloc"](T, H, device)
+        addrs, opened = [], []
+        if self.world == 1:
+            addrs = [acc.data_ptr()]
+        else:
+            mine = self._p["handle"](acc)
+            every = [None] * self.world
+            dist.all_gather_object(every, mine, group=self.group)
+            for r, (handle, offset) in enumerate(every):
+                if r == self.rank:
+                    addrs.append(acc.data_ptr())
+                else:
+                    base = self._p["open"](handle)
+                    opened.append(base)
+                    addrs.append(base + offset)
+        table = torch.tensor(addrs, dtype=torch.int64, device=device)
+        self._peer = {"T": T, "acc": acc, "table": table, "opened": opened}
+        return self._peer
+
+    def _peer_close(self):
+        if self._peer is not None:
+            for base in self._peer["opened"]:
+                self._p["close"](base)
+            self._peer = None
+
+    def _ranks_reached(self, device):
+        """Every rank's stream has reached this point (a collective ordered on the stream)."""
+        if self.world > 1:
+            dist.all_reduce(torch.zeros(1, device=device), group=self.group)
+
+    def forward_peer(self, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None) -> torch.Tensor:
+        """The gather exchange with the combine in the down GEMM: x [T, H] BF16 (T equal on every
+        rank) -> out [T, H] BF16."""
+        T, H = x.shape
+        p = self._peer_setup(T, H, x.device)
+        x_all = self.gather(x)
+        p["acc"].zero_()
+        self._ranks_reached(x.device)          # every owner's accumulator is zeroed
+        self._p["partial_peer"](x_all, w_router, bias, p["table"], T)
+        self._ranks_reached(x.device)          # every rank's additions are done
+        return self._finalize(p["acc"])
+
     def forward(self, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None = None) -> torch.Tensor:
         """x [T, H] BF16: this rank's tokens (T equal on every rank) -> out [T, H] BF16."""
         if self.exchange == "all_to_all":
             return self.forward_all_to_all(x, w_router, bias)
+        if self.exchange == "peer":
+            return self.forward_peer(x, w_router, bias)
         x_all = self.gather(x)
         partial = self._partial if self._partial is not None else self._partial_cuda
         acc = partial(x_all, w_router, bias)
         return self._finalize(self.scatter_sum(acc, x.shape[0]))
 
     def close(self):
+        self._peer_close()
         if self.experts is not None:
             self.experts.close()
             self.experts = None

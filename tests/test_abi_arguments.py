@@ -288,3 +288,34 @@ def test_expert_parallel_exchange_checks(lib):
     assert lib.nvfp4moe_ep_combine(MIS, A, 16, 8, 5120, A, None) == moe.ERR_ARG
     assert lib.nvfp4moe_ep_combine(A, A, 0, 8, 5120, A, None) == moe.OK
     assert lib.nvfp4moe_ep_combine(A, A, 16, 8, 5120, A, None) in NO_DEVICE
+
+
+def test_peer_combine_checks(lib):
+    """nvfp4moe_forward_partial_peer and the inter-process handle calls: host-side checks."""
+    f = lib.nvfp4moe_forward_partial_peer
+
+    def call(x=None, T=16, peers=A, n=2, rows=8, dbg=None):
+        return f(x, A, T, A, None, peers, n, rows, dbg, A, 1 << 30, None)
+
+    assert call(peers=None) == moe.ERR_ARG
+    assert call(peers=A + 4) == moe.ERR_ARG                     # the pointer table is 8-byte aligned
+    assert call(n=0) == moe.ERR_SHAPE
+    assert call(rows=0) == moe.ERR_SHAPE
+    assert call(n=3, rows=5) == moe.ERR_SHAPE                   # n_peers * rows_per_peer != T
+    d = moe._lib.Debug()
+    d.acc = A                                                   # the sums live in the peers
+    assert call(dbg=ctypes.byref(d)) == moe.ERR_ARG
+    assert call() == moe.ERR_ARG                                # no expert handle
+    assert lib.nvfp4moe_last_launch_count() == 0
+    buf = ctypes.create_string_buffer(64)
+    off = ctypes.c_int64()
+    assert lib.nvfp4moe_ipc_get_handle(None, buf, ctypes.byref(off)) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_get_handle(A, None, ctypes.byref(off)) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_get_handle(A, buf, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_get_handle(A, buf, ctypes.byref(off)) in NO_DEVICE
+    p = ctypes.c_void_p()
+    assert lib.nvfp4moe_ipc_open(None, ctypes.byref(p)) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_open(buf, None) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_open(buf, ctypes.byref(p)) in NO_DEVICE
+    assert lib.nvfp4moe_ipc_close(None) == moe.ERR_ARG
+    assert lib.nvfp4moe_ipc_close(A) in NO_DEVICE

@@ -175,6 +175,89 @@ def test_gloo_ranks_all_to_all_exchange(world):
         np.testing.assert_allclose(res[r][3], want, rtol=1e-12, atol=1e-12)
 
 
+def _rank_main_peer(rank, world, port, accs, out):
+    """One gloo rank of the gather exchange with the combine into the owners' memory: the
+    accumulators are shared CPU tensors (one per owner, made by the parent), the inter-process
+    handle calls are stand-ins that name the owner, and the library's call is replaced by the
+    oracle's sums of the rank's experts added into the owners' rows (in rank order, so that the
+    stand-in's plain additions do not race)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import nvfp4_quantized_moe_group_b200 as moe
+    from nvfp4_quantized_moe_group_b200.ep import ExpertParallelLayer
+    from workloads import TINY, activations, router_weight
+    from tests.helpers import oracle_layer, intermediate_scales
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        s = TINY
+        cfg = moe.Cfg(s.E, s.n_groups, s.topk_groups, s.topk, s.H, s.I, s.routed_scale)
+        g_h = intermediate_scales(s)
+        far = 1 << 40
+        log = {"opened": [], "closed": [], "zero_at_start": None}
+
+        def owner_of(addr):
+            return rank if addr == accs[rank].data_ptr() else (addr - far) >> 32
+
+        def partial_peer(x_all, w_router, bias, table, rows):
+            # every owner zeroed its accumulator before the first collective
+            log["zero_at_start"] = all(bool((accs[r] == 0).all()) for r in range(world))
+            ref = oracle_layer(s, x_all.float().numpy(), w_router.numpy(), None, g_h, workers=1,
+                               expert_range=(layer.e_begin, layer.e_count))["out"]
+            for turn in range(world):
+                if turn == rank:
+                    for t in range(x_all.shape[0]):
+                        accs[owner_of(int(table[t // rows]))][t % rows] += torch.from_numpy(ref[t])
+                dist.barrier()
+
+        ops = {"alloc": lambda T, H, device: accs[rank],
+               "handle": lambda acc: (b"owner %d" % rank, 0),
+               "open": lambda h: log["opened"].append(int(h.split()[1])) or far + (int(h.split()[1]) << 32),
+               "close": lambda addr: log["closed"].append(addr),
+               "partial_peer": partial_peer}
+        layer = ExpertParallelLayer(cfg, exchange="peer", peer_ops=ops, finalize=lambda acc: acc.to(torch.bfloat16))
+        wr = router_weight(s)
+        ys, xs = [], []
+        for step in range(2):                       # the second step reuses the mapped table
+            accs[rank].fill_(5.0)                   # stale values the step must clear
+            x = activations(T_RANK, s, seed=80 + 10 * step + rank)
+            ys.append(layer.forward(x, wr).float().numpy())
+            xs.append(x.float().numpy())
+        layer.close()
+        out[rank] = (log["opened"], log["closed"], log["zero_at_start"], ys, xs)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_peer_combine_exchange(world):
+    """The combine into the owners' memory on gloo ranks: each rank maps every other rank's
+    accumulator once, zeroes its own before a collective, the ranks add their experts' sums into
+    the owners' rows, and after a second collective every rank's rows are the oracle's whole
+    layer on its own tokens, on two consecutive steps; the mappings are released on close."""
+    accs = [torch.zeros((T_RANK, 256), dtype=torch.float64).share_memory_() for _ in range(world)]
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main_peer, args=(world, _free_port(), accs, out), nprocs=world, join=True)
+        res = dict(out)
+    sys.path.insert(0, ROOT)
+    from workloads import TINY, router_weight
+    from tests.helpers import oracle_layer, intermediate_scales, bf16_half_ulp
+    for r in range(world):
+        opened, closed, zero_at_start, ys, xs = res[r]
+        assert sorted(opened) == [q for q in range(world) if q != r]
+        assert len(closed) == world - 1
+        assert zero_at_start
+    for step in range(2):
+        x_all = np.concatenate([res[r][4][step] for r in range(world)])
+        ref = oracle_layer(TINY, x_all, router_weight(TINY).numpy(), None, intermediate_scales(TINY), workers=1)
+        for r in range(world):
+            want = ref["out"][r * T_RANK:(r + 1) * T_RANK]
+            got = res[r][3][step]
+            assert np.all(np.abs(got - want) <= 2 * bf16_half_ulp(want) + 1e-30)
+
+
 def test_expert_range_split():
     sys.path.insert(0, ROOT)
     from nvfp4_quantized_moe_group_b200.ep import expert_range

@@ -120,6 +120,77 @@ def test_beam_decode_eight_ranks():
     run_emulated(BEAM, 8, 16, sample=[0, 21, 47, 70, 101, 127])
 
 
+def run_peer_emulated(shape, G, T_rank, seed=90):
+    """The combine into the owners' memory (nvfp4moe_forward_partial_peer), G ranks emulated one
+    after another on one GPU: every rank's call adds its experts' weighted rows into the G
+    owners' accumulators (here all on this device, their addresses in one table).  The owners'
+    sums must equal the single-handle layer's FP32 sums up to the order of FP32 additions (the
+    gather emulation above checks each rank's share against the oracle), each owner must get
+    exactly its own tokens' rows, and the rounded rows must match nvfp4moe_forward within one
+    BF16 unit."""
+    full = gpu_experts(shape)
+    x_all = torch.cat([activations(T_rank, shape, seed=seed + r) for r in range(G)]).cuda()
+    wr = router_weight(shape).cuda()
+    acc_full = moe.forward_partial(full, x_all, wr)
+    out_full = moe.forward(full, x_all, wr)
+    # owners' accumulators with a canary row after each: nothing may land outside the owners' rows
+    store = torch.zeros((G, T_rank + 1, shape.H), dtype=torch.float32, device="cuda")
+    store[:, T_rank] = 7.0
+    table = torch.tensor([store[r].data_ptr() for r in range(G)], dtype=torch.int64, device="cuda")
+    for r in range(G):
+        e0, n = expert_range(shape.E, r, G)
+        ex = local_experts(shape, e0, n)
+        moe.forward_partial_peer(ex, x_all, wr, None, table, T_rank)
+        torch.cuda.synchronize()
+        ex.close()
+    assert bool((store[:, T_rank] == 7.0).all()), "a row outside the owners' token rows was written"
+    total = store[:, :T_rank].reshape(G * T_rank, shape.H).cpu().numpy()
+    af = acc_full.cpu().numpy()
+    row_scale = np.abs(af).max(axis=1, keepdims=True)
+    diff = np.abs(total - af)
+    assert np.all(diff <= 2.0 ** -16 * row_scale + 1e-30), f"max diff/row scale {np.max(diff / (row_scale + 1e-30)):.3g}"
+    out = torch.cat([moe.finalize(store[r, :T_rank].contiguous()) for r in range(G)]).float().cpu().numpy()
+    of = out_full.float().cpu().numpy()
+    bad = np.abs(out - of) > 2 * bf16_half_ulp(of) + 1e-30
+    assert bad.sum() <= max(4, 1e-4 * bad.size), f"{int(bad.sum())} outputs beyond one BF16 unit"
+
+
+@pytest.mark.parametrize("G,T_rank", [(2, 24), (4, 40)])
+def test_tiny_peer_combine_emulated(G, T_rank):
+    run_peer_emulated(TINY, G, T_rank)
+
+
+def test_beam_peer_combine_emulated():
+    """Beam on 4 emulated ranks with 300 tokens each: full segments (two GEMM launches, the
+    staged bulk reductions) into the owners' accumulators."""
+    run_peer_emulated(BEAM, 4, 300)
+
+
+def test_beam_peer_combine_decode_emulated():
+    """Beam decode on 8 emulated ranks with 16 tokens each: the one-launch GEMMs' register
+    reductions into the owners' accumulators."""
+    run_peer_emulated(BEAM, 8, 16)
+
+
+def test_single_rank_peer_exchange_matches_forward():
+    """ExpertParallelLayer(exchange="peer") without a process group: its own accumulator is the
+    only owner; the result is the whole layer."""
+    cfg = moe.make_cfg(TINY.E, TINY.n_groups, TINY.topk_groups, TINY.topk, TINY.H, TINY.I, TINY.routed_scale)
+    layer = ExpertParallelLayer(cfg, exchange="peer")
+    ex = layer.create_experts()
+    g_h = intermediate_scales(TINY)
+    for e in range(TINY.E):
+        ex.set_from_bf16(e, *(expert_weight(TINY, e, w, device="cuda") for w in ("gate", "up", "down")),
+                         float(g_h[e]))
+    x = activations(40, TINY, seed=9).cuda()
+    wr = router_weight(TINY).cuda()
+    want = moe.forward(gpu_experts(TINY), x, wr).float().cpu().numpy()
+    for _ in range(2):                          # the second step reuses the table and re-zeroes
+        got = layer.forward(x, wr).float().cpu().numpy()
+        assert np.all(np.abs(got - want) <= 2 * bf16_half_ulp(want) + 1e-30)
+    layer.close()
+
+
 def test_local_handle_rejects_foreign_experts_and_bad_ranges():
     cfg = moe.make_cfg(TINY.E, TINY.n_groups, TINY.topk_groups, TINY.topk, TINY.H, TINY.I, TINY.routed_scale)
     ex = moe.Experts(cfg, 8, 8)
