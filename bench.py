@@ -76,6 +76,25 @@ def stored_traffic(workload: str, experts_hit: int):
     return float(vals["dram_bytes_per_launch"]) / float(vals["experts_hit"]) * experts_hit
 
 
+def traffic_note(workload: str) -> str:
+    """Where the roofline's traffic figure comes from, or why there is none."""
+    name = os.path.relpath(TRAFFIC_FILE, ROOT)
+    if not os.path.exists(TRAFFIC_FILE):
+        return f"no ncu summary ({name} absent)"
+    vals = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if len(line) >= 2:
+                vals[line[0]] = line[1]
+    if vals.get("workload") != workload:
+        return f"none: {name} covers the {vals.get('workload')} workload, not {workload}"
+    if vals.get("source_sha256") != kernel_source_hash():
+        return (f"none: {name} was captured on GEMM sources hashing to {vals.get('source_sha256', '?')[:12]}, "
+                f"these hash to {kernel_source_hash()[:12]} (counters not retaken since the change)")
+    return f"{name}: one ncu capture, scaled by the experts hit"
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -651,6 +670,7 @@ def run_ours(args, world, rank, local):
         roof["spec_peak"] = HBM_SPEC_GBS
     roof["traffic"] = stored_traffic(args.workload if not args.experts else f"{args.workload}-e{shape.E}",
                                      alg["experts_hit"])
+    roof["traffic_source"] = traffic_note(args.workload if not args.experts else f"{args.workload}-e{shape.E}")
     roof["kernel"] = gu["kernel"]
     roof["duration_source"] = (f"CUDA events around the GEMM launch of each of {args.steps} steps of a second "
                                "timed region right after the headline one (same inputs), on the launching stream")

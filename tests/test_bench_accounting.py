@@ -54,7 +54,10 @@ def test_stored_traffic_applies_only_to_its_sources_and_workload(monkeypatch):
     if vals["source_sha256"] != bench.kernel_source_hash():
         # the kernels changed since the counters were taken: the line reports no traffic
         assert bench.stored_traffic("decode", 99) is None
+        assert bench.traffic_note("decode").startswith("none: ") and "hash" in bench.traffic_note("decode")
         monkeypatch.setattr(bench, "kernel_source_hash", lambda: vals["source_sha256"])
+    assert "one ncu capture" in bench.traffic_note("decode")
+    assert bench.traffic_note("prefill").startswith("none: ")
     t = bench.stored_traffic("decode", 99)
     assert t == float(vals["dram_bytes_per_launch"]) / float(vals["experts_hit"]) * 99
     assert bench.stored_traffic("prefill", 99) is None
