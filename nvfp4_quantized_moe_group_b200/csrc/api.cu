@@ -51,10 +51,10 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int check_device() {
   int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_failed();
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   return (major == 10 && minor == 0) ? NVFP4MOE_OK : NVFP4MOE_ERR_DEVICE;
 }
 
@@ -455,12 +455,12 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return cuda_failed();
   int blocks = 0;
   if (g_in == nullptr) {
     blocks = amax_partial_blocks(rows * cols);
     if (launch_amax_partial(x_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess)
-      return NVFP4MOE_ERR_CUDA;
+      return cuda_failed();
     ++g_launches;
   }
   QuantizeArgs a{};
@@ -479,7 +479,7 @@ int nvfp4moe_quantize(const void* x_bf16, int64_t rows, int64_t cols, const floa
   a.g_scratch = q.g;
   a.zero_out = nullptr;
   a.status = &q.hdr->status;
-  if (launch_quantize(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_quantize(a, s) != cudaSuccess) return cuda_failed();
   g_launches += quantize_launch_count(a);
   return NVFP4MOE_OK;
 }
@@ -502,12 +502,12 @@ int nvfp4moe_quantize_weights_lh(const void* w_bf16, int64_t rows, int64_t cols,
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return cuda_failed();
   const int blocks = amax_partial_blocks(rows * cols);
-  if (launch_amax_partial(w_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_amax_partial(w_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return cuda_failed();
   LhArgs la{static_cast<const uint16_t*>(w_bf16), rows, cols, hess_blocks, m, q.partials, blocks, codes, scales,
             g_out, &q.hdr->status};
-  if (launch_lh_quantize(la, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_lh_quantize(la, s) != cudaSuccess) return cuda_failed();
   g_launches = 2;
   return NVFP4MOE_OK;
 }
@@ -533,7 +533,7 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(r.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(r.hdr, 1, s) != cudaSuccess) return cuda_failed();
   if (T == 0) return NVFP4MOE_OK;
   RouterArgs a{};
   a.x = static_cast<const uint16_t*>(hidden_bf16);
@@ -551,7 +551,7 @@ int nvfp4moe_route(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int64_t T, 
   a.routed_scale = cfg->routed_scale;
   a.status = &r.hdr->status;
   set_router_tc(a, r.tc, r.x_digits);
-  if (launch_router(a, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_router(a, s) != cudaSuccess) return cuda_failed();
   g_launches += router_launch_count(a);
   return NVFP4MOE_OK;
 }
@@ -584,7 +584,7 @@ int nvfp4moe_experts_create_local(const nvfp4moe_cfg* cfg, int32_t e_begin, int3
   ok = ok && cudaMemset(x->w13_codes, 0, w13) == cudaSuccess && cudaMemset(x->wd_codes, 0, wd) == cudaSuccess;
   if (!ok) {
     nvfp4moe_experts_destroy(x);
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   }
   *out = x;
   return NVFP4MOE_OK;
@@ -625,16 +625,16 @@ int nvfp4moe_experts_set(nvfp4moe_experts* x, int32_t e_global, const nvfp4moe_e
       launch_tile_weights(t->up_codes, (int)I, (int)(H / 2), w13, kG, 2, 1, s) != cudaSuccess ||
       launch_tile_weights(t->down_codes, (int)H, (int)(I / 2), x->wd_codes + (size_t)e * wd_expert, (int)H, 1, 0,
                           s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   uint8_t* w13sf = x->w13_sf + (size_t)e * 2 * I * H / 16;
   if (launch_repack_sf(t->gate_scales, (int)I, (int)(H / 16), w13sf, H / 64, kG, 2, 0, s) != cudaSuccess ||
       launch_repack_sf(t->up_scales, (int)I, (int)(H / 16), w13sf, H / 64, kG, 2, 1, s) != cudaSuccess ||
       launch_repack_sf(t->down_scales, (int)H, (int)(I / 16), x->wd_sf + (size_t)e * H * I / 16, I / 64, (int)H,
                        1, 0, s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   set_expert_scalars_kernel<<<1, 1, 0, s>>>(x->g_gate, x->g_up, x->g_h, x->alpha_down, e, t->g_gate, t->g_up,
                                             t->g_h, t->g_down);
-  if (cudaGetLastError() != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return cuda_failed();
   g_launches += 7;
   return NVFP4MOE_OK;
 }
@@ -699,13 +699,13 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
       make_tma_2d(&tma_a32, f.a_codes, c.H / 2, f.rows_cap, 32) != 0 ||
       make_tma_2d(&tma_h, f.hq_codes, c.I / 2, f.rows_cap, kBlockM) != 0 ||
       make_tma_2d(&tma_h32, f.hq_codes, c.I / 2, f.rows_cap, 32) != 0)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
 
   const StageEvents ev{dbg != nullptr ? dbg->events : nullptr, s};
   // status word, front-end barrier, the GEMM work counters and the row-tile counters that follow
   // the header
   if (reset_status(f.hdr, (int)(sizeof(WsHeader) / 4 + f.rows_cap / kBlockM), s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   const bool keep_xq = dbg != nullptr && (dbg->xq_codes != nullptr || dbg->xq_scales != nullptr);
   const bool decode_cfg = T * c.topk < 32 * c.E;   // segments average fewer than 32 rows
   // two GEMM launches (else one for both, see below); the gate/up launch then zeroes the FP32
@@ -751,7 +751,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ev.mark(NVFP4MOE_STAGE_AMAX, 0);
     ev.mark(NVFP4MOE_STAGE_AMAX, 1);
     ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
-    if (launch_front(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_front(fa, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
     for (int stage : {NVFP4MOE_STAGE_PERMUTE, NVFP4MOE_STAGE_QUANTIZE, NVFP4MOE_STAGE_GATHER}) {
       ev.mark(stage, 0);
@@ -784,7 +784,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ev.mark(NVFP4MOE_STAGE_AMAX, 0);
     ev.mark(NVFP4MOE_STAGE_AMAX, 1);
     ev.mark(NVFP4MOE_STAGE_ROUTE, 0);
-    if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_router(r, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_ROUTE, 1);
     g_launches += router_launch_count(r);
 
@@ -804,7 +804,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     pa.inv = f.inv;
     pa.row_pair = f.row_pair;
     ev.mark(NVFP4MOE_STAGE_PERMUTE, 0);
-    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_PERMUTE, 1);
 
     // quantise x and write each token's row into its expert-segment rows (zeroes the
@@ -833,7 +833,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     q.seg_codes = f.a_codes;
     q.seg_sf = f.a_sf;
     ev.mark(NVFP4MOE_STAGE_QUANTIZE, 0);
-    if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_quantize(q, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_QUANTIZE, 1);
     ev.mark(NVFP4MOE_STAGE_GATHER, 0);
     ev.mark(NVFP4MOE_STAGE_GATHER, 1);
@@ -890,12 +890,12 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
       gz.zero_acc = f.acc;
       gz.zero_acc_elems = T * c.H;
     }
-    if (launch_gemm_gateup(tma_a, tma_a32, gz, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_gemm_gateup(tma_a, tma_a32, gz, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
     ++g_launches;
     ev.mark(NVFP4MOE_STAGE_DOWN, 0);
     gd.work_counter = &f.hdr->work[1];
-    if (launch_gemm_down(tma_h, tma_h32, gd, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_gemm_down(tma_h, tma_h32, gd, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_DOWN, 1);
     ++g_launches;
   } else {
@@ -904,7 +904,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     ev.mark(NVFP4MOE_STAGE_GATEUP, 0);
     if (launch_gemm_fused(tma_a, tma_a32, tma_h, tma_h32, g, gd, f.dep, kFusedLagPerSm * grid, grid, s) !=
         cudaSuccess)
-      return NVFP4MOE_ERR_CUDA;
+      return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_GATEUP, 1);
     ev.mark(NVFP4MOE_STAGE_DOWN, 0);
     ev.mark(NVFP4MOE_STAGE_DOWN, 1);
@@ -915,7 +915,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
     FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, res != nullptr ? res->h : nullptr,
                     res != nullptr ? res->a : 0.0f, res != nullptr ? res->b : 0.0f};
     ev.mark(NVFP4MOE_STAGE_FINALIZE, 0);
-    if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_finalize(fa, s) != cudaSuccess) return cuda_failed();
     ev.mark(NVFP4MOE_STAGE_FINALIZE, 1);
     ++g_launches;
   }
@@ -938,7 +938,7 @@ static int forward_core(const nvfp4moe_experts* x, const void* hidden_bf16, int6
                              dbg->hq_codes, dbg->hq_scales, s) == cudaSuccess;
     if (dbg->acc && dbg->acc != f.acc)
       ok &= cudaMemcpyAsync(dbg->acc, f.acc, T * c.H * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
-    if (!ok) return NVFP4MOE_ERR_CUDA;
+    if (!ok) return cuda_failed();
   }
   return NVFP4MOE_OK;
 }
@@ -995,7 +995,7 @@ int nvfp4moe_ipc_get_handle(const void* dev_ptr, void* handle_out, int64_t* offs
   if (range == nullptr || range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
     return NVFP4MOE_ERR_ARG;                                      // not device memory
   cudaIpcMemHandle_t h;
-  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return cuda_failed();
   std::memcpy(handle_out, &h, sizeof(h));
   *offset_out = (int64_t)(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
   return NVFP4MOE_OK;
@@ -1007,7 +1007,7 @@ int nvfp4moe_ipc_open(const void* handle, void** dev_ptr_out) {
   if (st != NVFP4MOE_OK) return st;
   cudaIpcMemHandle_t h;
   std::memcpy(&h, handle, sizeof(h));
-  if (cudaIpcOpenMemHandle(dev_ptr_out, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaIpcOpenMemHandle(dev_ptr_out, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return cuda_failed();
   return NVFP4MOE_OK;
 }
 
@@ -1015,7 +1015,7 @@ int nvfp4moe_ipc_close(void* dev_ptr) {
   if (dev_ptr == nullptr) return NVFP4MOE_ERR_ARG;
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
-  return cudaIpcCloseMemHandle(dev_ptr) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
+  return cudaIpcCloseMemHandle(dev_ptr) == cudaSuccess ? NVFP4MOE_OK : cuda_failed();
 }
 
 int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream) {
@@ -1026,7 +1026,7 @@ int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, void* stream)
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   FinalizeArgs fa{acc, static_cast<uint16_t*>(out_bf16), n, nullptr, 0.0f, 0.0f};
-  if (launch_finalize(fa, static_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_finalize(fa, static_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_failed();
   g_launches = 1;
   return NVFP4MOE_OK;
 }
@@ -1051,14 +1051,14 @@ int nvfp4moe_forward_residual(const nvfp4moe_experts* x, const void* h_bf16, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the status word is reset by the forward that follows; the norm raises nothing
   RmsNormArgs na{static_cast<const uint16_t*>(h_bf16), gamma, eps, T, c.H, f.x_norm};
-  if (launch_rmsnorm(na, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_rmsnorm(na, s) != cudaSuccess) return cuda_failed();
   const Residual r{static_cast<const uint16_t*>(h_bf16), (float)std::sqrt((double)(step_k - 1) / (double)step_k),
                    (float)(1.0 / std::sqrt((double)step_k))};
   st = forward_core(x, f.x_norm, T, w_router, logit_bias, h_out_bf16, &r, dbg, ws, ws_bytes, stream);
   g_launches += 1;
   if (st == NVFP4MOE_OK && dbg != nullptr && dbg->x_norm != nullptr &&
       cudaMemcpyAsync(dbg->x_norm, f.x_norm, (size_t)T * c.H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   return st;
 }
 
@@ -1075,9 +1075,9 @@ int nvfp4moe_quantize_fp8(const void* x_bf16, int64_t rows, int64_t cols, uint8_
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(q.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(q.hdr, 1, s) != cudaSuccess) return cuda_failed();
   Fp8RowsArgs fa{static_cast<const uint16_t*>(x_bf16), rows, cols, codes, scales, &q.hdr->status};
-  if (launch_fp8_quantize_rows(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_fp8_quantize_rows(fa, s) != cudaSuccess) return cuda_failed();
   g_launches = 1;
   return NVFP4MOE_OK;
 }
@@ -1103,7 +1103,7 @@ int nvfp4moe_fp8_experts_create(const nvfp4moe_cfg* cfg, nvfp4moe_fp8_experts** 
                   cudaMemset(x->wd_scale, 0, (size_t)E * H * sizeof(float)) == cudaSuccess;
   if (!ok) {
     nvfp4moe_fp8_experts_destroy(x);
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   }
   *out = x;
   return NVFP4MOE_OK;
@@ -1128,14 +1128,14 @@ int nvfp4moe_fp8_experts_set(nvfp4moe_fp8_experts* x, int32_t e, const nvfp4moe_
       launch_tile_weights(t->up_codes, (int)I, (int)H, w13, kG, 2, 1, s) != cudaSuccess ||
       launch_tile_weights(t->down_codes, (int)H, (int)I, x->wd_codes + (size_t)e * H * I, (int)H, 1, 0, s) !=
           cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   float* sc = x->w13_scale + (size_t)e * 2 * I;
   const size_t gb = kG * sizeof(float);
   if (cudaMemcpy2DAsync(sc, 2 * gb, t->gate_scales, gb, gb, I / kG, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
       cudaMemcpy2DAsync(sc + kG, 2 * gb, t->up_scales, gb, gb, I / kG, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(x->wd_scale + (size_t)e * H, t->down_scales, H * sizeof(float), cudaMemcpyDeviceToDevice,
                       s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   g_launches = 3;
   return NVFP4MOE_OK;
 }
@@ -1176,9 +1176,9 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
       make_tma_2d(&tma_a32, f.a_codes, c.H, f.rows_cap, 32) != 0 ||
       make_tma_2d(&tma_h, f.hq, c.I, f.rows_cap, kBlockM) != 0 ||
       make_tma_2d(&tma_h32, f.hq, c.I, f.rows_cap, 32) != 0)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   // status word, front-end barrier and the two GEMM work counters
-  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(f.hdr, 4, s) != cudaSuccess) return cuda_failed();
 
   if (front_supported(T, c.E, c.H)) {
     // small T: routing and grouping in the fused front-end launch (its NVFP4 quantisation
@@ -1209,7 +1209,7 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
     fa.acc = f.acc;
     fa.status = &f.hdr->status;
     fa.barrier = &f.hdr->barrier;
-    if (launch_front(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_front(fa, s) != cudaSuccess) return cuda_failed();
     ++g_launches;
   } else {
     RouterArgs r{};
@@ -1230,7 +1230,7 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
     r.amax_partials = f.partials;
     r.status = &f.hdr->status;
     set_router_tc(r, f.tc, f.a_codes);
-    if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_router(r, s) != cudaSuccess) return cuda_failed();
     g_launches += router_launch_count(r);
 
     PermArgs pa{};
@@ -1247,14 +1247,14 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
     pa.perm = f.perm;
     pa.inv = f.inv;
     pa.row_pair = f.row_pair;
-    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+    if (launch_permute(pa, s, &g_launches) != cudaSuccess) return cuda_failed();
   }
 
   Fp8ScatterArgs qa{static_cast<const uint16_t*>(hidden_bf16), T, c.H, c.topk, f.idx, f.inv, f.offsets,
                     f.mtile_prefix, f.a_codes, f.a_scale, f.acc,
                     dbg != nullptr ? dbg->xq8_codes : nullptr, dbg != nullptr ? dbg->xq8_scales : nullptr,
                     &f.hdr->status};
-  if (launch_fp8_quantize_scatter(qa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_fp8_quantize_scatter(qa, s) != cudaSuccess) return cuda_failed();
   ++g_launches;
 
   const int grid = num_sms();
@@ -1277,18 +1277,18 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
   g.w_scale = x->w13_scale;
   g.h32 = f.h32;
   g.work_counter = &f.hdr->work[0];
-  if (launch_gemm_gateup_fp8(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup_fp8(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
   Fp8RequantArgs ra{f.h32, f.rows_cap, c.I, f.row_pair, f.mtile_prefix, c.E, f.hq, f.h_scale, &f.hdr->status};
-  if (launch_fp8_requant_rows(ra, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_fp8_requant_rows(ra, s) != cudaSuccess) return cuda_failed();
   g.b_tiles = x->wd_codes;
   g.K = c.I;
   g.n_total = c.H;
   g.w_scale = x->wd_scale;
   g.h_scale = f.h_scale;
   g.work_counter = &f.hdr->work[1];
-  if (launch_gemm_down_fp8(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_down_fp8(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
   FinalizeArgs fa{f.acc, static_cast<uint16_t*>(out_bf16), T * c.H, nullptr, 0.0f, 0.0f};
-  if (launch_finalize(fa, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_finalize(fa, s) != cudaSuccess) return cuda_failed();
   g_launches += 4;
 
   if (dbg != nullptr) {
@@ -1299,16 +1299,16 @@ int nvfp4moe_forward_fp8(const nvfp4moe_fp8_experts* x, const void* hidden_bf16,
     if (dbg->offsets)
       ok &= cudaMemcpyAsync(dbg->offsets, f.offsets, (c.E + 1) * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
     if (dbg->perm) ok &= cudaMemcpyAsync(dbg->perm, f.perm, pairs * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
-    if (!ok) return NVFP4MOE_ERR_CUDA;
+    if (!ok) return cuda_failed();
   }
   return NVFP4MOE_OK;
 }
 
 int nvfp4moe_status_read(const void* ws, void* stream) {
   if (ws == nullptr) return NVFP4MOE_ERR_ARG;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_failed();
   uint32_t v = 0;
-  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_failed();
   if (v & kStatusTimeout) return NVFP4MOE_ERR_TIMEOUT;
   if (v & kStatusBadInput) return NVFP4MOE_ERR_ARG;
   if (v & kStatusNonFinite) return NVFP4MOE_ERR_NONFINITE;
@@ -1351,10 +1351,10 @@ int nvfp4moe_amax(const void* x_bf16, int64_t rows, int64_t cols, uint32_t* amax
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (rows == 0) return cudaMemsetAsync(amax_bits, 0, 4, s) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
+  if (rows == 0) return cudaMemsetAsync(amax_bits, 0, 4, s) == cudaSuccess ? NVFP4MOE_OK : cuda_failed();
   const int blocks = amax_partial_blocks(rows * cols);
-  if (launch_amax_partial(x_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  if (launch_amax_reduce(q.partials, blocks, amax_bits, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_amax_partial(x_bf16, rows * cols, q.partials, blocks, s) != cudaSuccess) return cuda_failed();
+  if (launch_amax_reduce(q.partials, blocks, amax_bits, s) != cudaSuccess) return cuda_failed();
   g_launches = 2;
   return NVFP4MOE_OK;
 }
@@ -1386,7 +1386,7 @@ int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* h
   st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(d.hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(d.hdr, 1, s) != cudaSuccess) return cuda_failed();
   // route this rank's tokens
   RouterArgs r{};
   r.x = static_cast<const uint16_t*>(hidden_bf16);
@@ -1404,7 +1404,7 @@ int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* h
   r.routed_scale = c.routed_scale;
   r.status = &d.hdr->status;
   set_router_tc(r, d.tc, nullptr);
-  if (launch_router(r, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_router(r, s) != cudaSuccess) return cuda_failed();
   g_launches += router_launch_count(r);
   // group its pairs by expert: the stable expert-major order is also destination-rank order
   PermArgs pa{};
@@ -1421,7 +1421,7 @@ int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* h
   pa.perm = d.perm;
   pa.inv = d.inv;
   pa.row_pair = d.row_pair;
-  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return cuda_failed();
   // quantise the tokens with the global scale of all ranks' tokens (from their amax)
   QuantizeArgs q{};
   q.x = static_cast<const uint16_t*>(hidden_bf16);
@@ -1437,7 +1437,7 @@ int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* h
   q.n_col_tiles = c.H / 64;
   q.g_out = d.g;
   q.status = &d.hdr->status;
-  if (launch_quantize(q, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_quantize(q, s) != cudaSuccess) return cuda_failed();
   g_launches += quantize_launch_count(q);
   // pack the pairs' rows in send order, with their metadata and the per-rank counts
   EpPackArgs pk{};
@@ -1458,7 +1458,7 @@ int nvfp4moe_ep_dispatch(const nvfp4moe_cfg* cfg, int32_t n_ranks, const void* h
   pk.send_w = send_w;
   pk.send_pos = send_pos;
   pk.rank_counts = rank_counts;
-  if (launch_ep_pack(pk, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_ep_pack(pk, s) != cudaSuccess) return cuda_failed();
   g_launches += 2;
   return NVFP4MOE_OK;
 }
@@ -1489,18 +1489,18 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   int st = check_device();
   if (st != NVFP4MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (reset_status(f.hdr, 4, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(f.hdr, 4, s) != cudaSuccess) return cuda_failed();
   if (n_rows == 0) return NVFP4MOE_OK;
   CUtensorMap tma_a, tma_a32, tma_h, tma_h32;
   if (make_tma_2d(&tma_a, f.a_codes, cl.H / 2, f.rows_cap, kBlockM) != 0 ||
       make_tma_2d(&tma_a32, f.a_codes, cl.H / 2, f.rows_cap, 32) != 0 ||
       make_tma_2d(&tma_h, f.hq_codes, cl.I / 2, f.rows_cap, kBlockM) != 0 ||
       make_tma_2d(&tma_h32, f.hq_codes, cl.I / 2, f.rows_cap, 32) != 0)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   // the expert indices come from other ranks: checked on the device (an index outside the
   // handle's experts is replaced by 0 and raises NVFP4MOE_ERR_ARG in the status word)
   if (launch_check_indices(expert, n_rows, cl.E, f.expert, &f.hdr->status, s) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   ++g_launches;
   // group the received rows by local expert (stable: source rank, then its order)
   PermArgs pa{};
@@ -1517,12 +1517,12 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   pa.perm = f.perm;
   pa.inv = f.inv;
   pa.row_pair = f.row_pair;
-  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
-  if (launch_global_scale(amax_bits, 1, f.g_x, &f.hdr->status, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_permute(pa, s, &g_launches) != cudaSuccess) return cuda_failed();
+  if (launch_global_scale(amax_bits, 1, f.g_x, &f.hdr->status, s) != cudaSuccess) return cuda_failed();
   ++g_launches;
   RowsToSegmentsArgs ra{codes, scales, f.expert, f.inv, f.offsets, f.mtile_prefix, n_rows, cl.H, cl.H / 64,
                         f.a_codes, f.a_sf, out_rows};
-  if (launch_rows_to_segments(ra, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_rows_to_segments(ra, s) != cudaSuccess) return cuda_failed();
   ++g_launches;
   const int grid = num_sms();
   const bool decode_cfg = n_rows < 32 * (int64_t)cl.E;
@@ -1550,7 +1550,7 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   g.topk = 1;
   g.H = cl.H;
   g.work_counter = &f.hdr->work[0];
-  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_gateup(tma_a, tma_a32, g, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
   ++g_launches;
   g.b_tiles = x->wd_codes;
   g.sfa = f.hq_sf;
@@ -1558,7 +1558,7 @@ int nvfp4moe_ep_experts(const nvfp4moe_experts* x, const uint8_t* codes, const u
   g.K = cl.I;
   g.n_total = cl.H;
   g.work_counter = &f.hdr->work[1];
-  if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (launch_gemm_down(tma_h, tma_h32, g, grid, decode_cfg, s) != cudaSuccess) return cuda_failed();
   ++g_launches;
   return NVFP4MOE_OK;
 }
@@ -1574,7 +1574,7 @@ int nvfp4moe_ep_combine(const float* rows, const int32_t* send_pos, int64_t T, i
   if (st != NVFP4MOE_OK) return st;
   if (launch_ep_combine(rows, send_pos, T, topk, H, static_cast<uint16_t*>(out_bf16), static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   g_launches = 1;
   return NVFP4MOE_OK;
 }

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "gemm.h"
+#include "nvfp4moe.h"
 
 namespace nvfp4moe {
 
@@ -296,5 +297,13 @@ int num_sms();
 // Zeroes the first `words` 32-bit words of a call's status header on the stream and records
 // the status word as this host thread's latest (read by nvfp4moe_last_device_status).
 cudaError_t reset_status(void* header, int words, cudaStream_t stream);
+
+// A failed runtime call (an allocation, an IPC mapping, a copy) stays the host thread's last
+// CUDA error, and the launch checks of the next call read that word: every entry point that
+// returns NVFP4MOE_ERR_CUDA goes through here, so the next call does not report it again.
+inline int cuda_failed() {
+  (void)cudaGetLastError();
+  return NVFP4MOE_ERR_CUDA;
+}
 
 }  // namespace nvfp4moe

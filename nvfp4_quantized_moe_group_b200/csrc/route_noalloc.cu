@@ -33,12 +33,12 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // host code the symbol itself is only a host-side stand-in for that address).
 int scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_failed();
   if (dev < 0 || dev >= kMaxDevices) return NVFP4MOE_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return NVFP4MOE_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return cuda_failed();
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -68,7 +68,7 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return NVFP4MOE_ERR_CUDA;
+    return cuda_failed();
   if (major != 10 || minor != 0) return NVFP4MOE_ERR_DEVICE;
   void* scratch = nullptr;
   st = scratch_address(&scratch);
@@ -77,7 +77,7 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
   WsHeader* hdr = static_cast<WsHeader*>(scratch);
   // the array keeps the previous call's contents: the status word starts at zero; the
   // partial sums are overwritten before they are read
-  if (reset_status(hdr, 1, s) != cudaSuccess) return NVFP4MOE_ERR_CUDA;
+  if (reset_status(hdr, 1, s) != cudaSuccess) return cuda_failed();
   if (T == 0) return NVFP4MOE_OK;
   RouterArgs a{};
   a.x = static_cast<const uint16_t*>(hidden_bf16);
@@ -94,7 +94,7 @@ int nvfp4moe_route_noalloc(const nvfp4moe_cfg* cfg, const void* hidden_bf16, int
   a.topk = cfg->topk;
   a.routed_scale = cfg->routed_scale;
   a.status = &hdr->status;
-  return launch_router(a, s) == cudaSuccess ? NVFP4MOE_OK : NVFP4MOE_ERR_CUDA;
+  return launch_router(a, s) == cudaSuccess ? NVFP4MOE_OK : cuda_failed();
 }
 
 }  // extern "C"

@@ -112,3 +112,24 @@ def test_poisoned_workspace_gives_the_clean_result(shape, T):
         assert torch.equal(d0[key], d1[key]), key
     assert bool(torch.isfinite(out1.float()).all())
     assert _within_one_bf16_unit(out1, out0)
+
+
+def test_failed_allocation_leaves_no_error_for_the_next_call():
+    """A runtime call that fails inside the library (here the expert weights' allocation for a
+    shape far beyond the device's memory: 256 experts of H = I = 32768, 275 GB of codes) returns
+    NVFP4MOE_ERR_CUDA and leaves the thread's last CUDA error clear, so neither the library's
+    next call nor torch's next launch reports it as its own."""
+    ex = gpu_experts(TINY)
+    x = activations(16, TINY, seed=35).cuda()
+    wr = router_weight(TINY).cuda()
+    ws = torch.zeros(moe.forward_workspace_bytes(ex.cfg, 16), dtype=torch.uint8, device="cuda")
+    ref = moe.forward(ex, x, wr, ws=ws)
+    torch.cuda.synchronize()
+    with pytest.raises(moe.NvFp4MoeError) as err:
+        moe.Experts(moe.Cfg(256, 8, 4, 8, 32768, 32768, 2.5))
+    assert err.value.status == moe.ERR_CUDA
+    y = x.clone()                                  # a torch launch right after the failure
+    got = moe.forward(ex, y, wr, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.status_read(ws) == moe.OK
+    assert _within_one_bf16_unit(got, ref)
