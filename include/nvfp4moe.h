@@ -378,7 +378,10 @@ NVFP4MOE_API int nvfp4moe_finalize(const float* acc, int64_t n, void* out_bf16, 
  * mapping the other ranks' accumulators.  get_handle: the handle (NVFP4MOE_IPC_HANDLE_BYTES
  * opaque bytes) of the device allocation that contains dev_ptr, and dev_ptr's byte offset from
  * that allocation's start.  open (in another process): maps that allocation and returns its
- * start, to which the importer adds the offset.  close unmaps an address that open returned. */
+ * start, to which the importer adds the offset.  close unmaps an address that open returned.
+ * Errors: ERR_ARG for a null argument or an address that is not device memory; ERR_CUDA when
+ * CUDA refuses the handle or the mapping (inter-process handles cover memory from cudaMalloc,
+ * not from the virtual-memory calls); ERR_DEVICE off a B200. */
 #define NVFP4MOE_IPC_HANDLE_BYTES 64
 NVFP4MOE_API int nvfp4moe_forward_partial_peer(const nvfp4moe_experts* experts, const void* hidden_bf16, int64_t T,
                                                const float* w_router, const float* logit_bias,

@@ -78,7 +78,10 @@ class ExpertParallelLayer:
         "all_to_all" (send each pair's quantised row to its expert's rank and its weighted
         output row back).  ``a2a_ops`` / ``peer_ops`` replace those paths' library calls (keys
         amax, dispatch, experts, combine / alloc, handle, open, close, partial_peer; the
-        signatures of the default methods below), to exercise the exchanges without a GPU."""
+        signatures of the default methods below), to exercise the exchanges without a GPU.
+        The peer exchange maps the accumulators through CUDA inter-process handles, which cover
+        memory from cudaMalloc only: torch's caching allocator without expandable segments
+        (with them the handle call fails and raises)."""
         if exchange not in ("gather", "all_to_all", "peer"):
             raise ValueError(f"unknown exchange {exchange!r}")
         self.cfg = cfg
