@@ -141,6 +141,11 @@ CASES = [
     ("weights-over-all-experts", "router", "route",
      "cfg.routed_scale * ss / ss.sum()", "cfg.routed_scale * ss / s[t].sum()"),
     ("routed-scale-dropped", "router", "route", "cfg.routed_scale * ss / ss.sum()", "ss / ss.sum()"),
+    ("weights-not-normalised", "router", "route", "cfg.routed_scale * ss / ss.sum()", "cfg.routed_scale * ss"),
+    ("selection-in-index-order", "router", "route", "idx[t] = sel", "idx[t] = np.sort(sel)"),
+    ("bias-after-sigmoid", "router", "route",
+     "logits = logits + np.asarray(bias, dtype=np.float64)[None, :]",
+     "logits = _sigmoid(logits) + np.asarray(bias, dtype=np.float64)[None, :]"),
     ("group-margin-wrong-neighbour", "router", "route",
      "gscore[t, gorder[KG - 1]] - gscore[t, gorder[KG]]", "gscore[t, gorder[0]] - gscore[t, gorder[KG]]"),
     ("expert-margin-off-by-one", "router", "route",

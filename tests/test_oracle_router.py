@@ -101,6 +101,31 @@ def test_bias_shifts_selection():
     assert np.all(r.idx[:, 0] == 17)
 
 
+def test_bias_is_a_logit_offset():
+    """The skewed workload's per-expert bias is added to the logits before the sigmoid: it
+    routes exactly like one more input column of ones whose router weights are the bias.
+    Inputs are integers scaled by powers of two, so both forms give the same FP64 logits."""
+    rng = np.random.default_rng(5)
+    x = rng.integers(-8, 9, size=(40, 32)) / 8.0
+    wr = rng.integers(-8, 9, size=(32, 32)) / 64.0
+    bias = rng.integers(-16, 17, size=32) / 8.0
+    cfg = _cfg(32, 8, 4, 8)
+    r = oracle.route(x, wr, cfg, bias=bias)
+    r1 = oracle.route(np.hstack([x, np.ones((40, 1))]), np.hstack([wr, bias[:, None]]), cfg)
+    np.testing.assert_array_equal(r.idx, r1.idx)
+    np.testing.assert_array_equal(r.w, r1.w)
+
+
+def test_bias_alone_gives_sigmoid_of_bias():
+    """With x = 0 the scores are the sigmoid of the bias, and the weights its normalised
+    selection scaled by 2.5 (closed form)."""
+    bias = np.linspace(-2.0, 2.0, 16)
+    r = oracle.route(np.zeros((1, 8)), np.zeros((16, 8)), _cfg(16, 1, 1, 4), bias=bias)
+    sig = 1.0 / (1.0 + np.exp(-bias))
+    assert list(r.idx[0]) == [15, 14, 13, 12]
+    np.testing.assert_allclose(r.w[0], 2.5 * sig[[15, 14, 13, 12]] / sig[12:].sum(), rtol=1e-15)
+
+
 def test_ties_go_to_lower_index():
     x = np.ones((1, 4))
     wr = np.zeros((8, 4))                 # every score equal
