@@ -78,7 +78,9 @@ def _tiny_layer(T=24):
     x = activations(T, shape).float().numpy()
     wr = router_weight(shape).numpy()
     ex = {e: tuple(_qt(expert_weight(shape, e, w)) for w in ("gate", "up", "down")) for e in range(shape.E)}
-    g_h = np.full(shape.E, np.float32(0.002), dtype=np.float32)
+    # a different static scale per expert, so that an expert's h quantised with another
+    # expert's scale shows
+    g_h = (np.float32(0.002) * (1 + np.arange(shape.E, dtype=np.float32) / shape.E)).astype(np.float32)
     return shape, x, wr, ex, g_h
 
 

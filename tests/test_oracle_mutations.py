@@ -125,6 +125,17 @@ CASES = [
     ("unpack-nibbles-swapped", "formats", "unpack_codes",
      "out[:, 0::2] = codes & 0xF\n    out[:, 1::2] = codes >> 4",
      "out[:, 0::2] = codes >> 4\n    out[:, 1::2] = codes & 0xF"),
+    ("swizzle-column-tile-stride", "formats", "swizzle_scales",
+     "(c // 4) * 512 + (r % 32)", "(c // 4) * 128 + (r % 32)"),
+    ("scale-per-row", "formats", "quantize",
+     "amax_b = np.max(np.abs(xb), axis=2) if x.size",
+     "amax_b = np.repeat(np.max(np.abs(xb), axis=(1, 2))[:, None], cols // 16, axis=1) if x.size"),
+    ("zero-tensor-scale-zero", "formats", "global_scale", "if a == 0:\n        return F32(1.0)",
+     "if a == 0:\n        return F32(0.0)"),
+    ("e2m1-rounds-down", "formats", "e2m1_encode",
+     "mid = (_E2M1_MAG[i] + _E2M1_MAG[i + 1]) / 2", "mid = _E2M1_MAG[i + 1]"),
+    ("scale-from-first-value", "formats", "quantize",
+     "amax_b = np.max(np.abs(xb), axis=2) if x.size", "amax_b = np.abs(xb[:, :, 0]) if x.size"),
     ("scale-bytes-per-32", "formats", "nvfp4_tensor_bytes",
      "rows * cols // 16", "rows * cols // 32"),
     # router
@@ -169,6 +180,14 @@ CASES = [
     ("h-dynamic-scale", "moe", "expert_mlp",
      "hq_codes, hq_scales, _ = quantize(h.astype(np.float32), g=g_h)",
      "hq_codes, hq_scales, g_h = quantize(h.astype(np.float32))"),
+    ("g_h-of-expert-0", "moe", "moe_forward",
+     "res = expert_mlp(xhat, gate, up, down, np.float32(g_h[e]))",
+     "res = expert_mlp(xhat, gate, up, down, np.float32(g_h[0]))"),
+    ("gate-and-up-both-gate", "moe", "expert_mlp", "uv = xhat @ Wu.T", "uv = xhat @ Wg.T"),
+    ("counts-shifted", "moe", "permutation",
+     "counts = np.bincount(flat, minlength=E).astype(np.int64)",
+     "counts = np.roll(np.bincount(flat, minlength=E).astype(np.int64), 1)"),
+    ("combine-unweighted", "moe", "moe_forward", "out[i] += r.w[t, j] * res[\"y\"][n]", "out[i] += res[\"y\"][n]"),
     ("weights-of-expert-0", "moe", "moe_forward", "gate, up, down = experts(e)", "gate, up, down = experts(0)"),
     # FP8 variant
     ("fp8-fnuz-max", "fp8", "row_scales", "(amax / F32(E4M3_MAX))", "(amax / F32(240.0))"),
