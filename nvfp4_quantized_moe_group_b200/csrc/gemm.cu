@@ -19,7 +19,8 @@
 //   gate/up:  each 128-column half holds 64 gate and 64 up columns of the same features:
 //             h = silu(g_x g_gate acc_gate) * (g_x g_up acc_up) in FP32, requantised to
 //             NVFP4 with the expert's static scale g_h (the down GEMM's A operand);
-//   down:     acc_out[token] += w * g_h * g_down * acc, FP32 additions into the token's row:
+//   down:     acc_out[token] += w * g_h * g_down * acc, FP32 additions into the token's row
+//             (given a table of the ranks' accumulators, the row in the owning rank's one):
 //             with full segments half the lanes at a time stage their row's 64-column piece in
 //             shared memory and add it with one bulk reduction (cp.reduce.async.bulk .add.f32,
 //             256 bytes);
