@@ -20,9 +20,11 @@ def _cuda():
     moe.lib()
 
 
-def _run(shape, T, rms_rows=False, bias=None, max_flag_frac=0.1):
+def _run(shape, T, rms_rows=False, bias=None, max_flag_frac=0.1, bf16_router=False):
     x = activations(T, shape, rms_rows=rms_rows)
     wr = router_weight(shape)
+    if bf16_router:
+        wr = wr.bfloat16().float()
     cfg = moe.make_cfg(shape.E, shape.n_groups, shape.topk_groups, shape.topk, shape.H, shape.I,
                        shape.routed_scale)
     idx, w = moe.route(cfg, x.cuda(), wr.cuda(), None if bias is None else bias.cuda())
@@ -57,6 +59,14 @@ def test_beam_skewed_zipf_bias():
     idx, _ = _run(BEAM, 16384, bias=zipf_bias(256))
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=256)
     assert counts.max() > 8 * counts.mean()           # the bias concentrates the load
+
+
+@pytest.mark.parametrize("T", [16, 4096])
+def test_bf16_valued_router_weights(T):
+    """A router kept in BF16 (the quantisation page leaves routers in BF16) is the special case
+    of FP32 router rows whose values are BF16: both logit paths (T <= 64 and the integer one)
+    route it under the same protocol."""
+    _run(BEAM, T, rms_rows=T == 16, bf16_router=True)
 
 
 def test_ragged_token_counts():
