@@ -21,7 +21,8 @@ weighted residual add out), ``quantize_weights_lh`` (local-Hessian weight scales
 ``forward_partial`` / ``finalize``, ``forward_partial_peer`` / ``ipc_handle`` / ``ipc_open`` or ``amax`` /
 ``ep_dispatch`` / ``ep_experts`` / ``ep_combine`` (experts spread over the ranks of a process group;
 a gather exchange, the same with the combine into the owners' memory inside the down GEMM, or an
-all-to-all one).
+all-to-all one), and ``tp.TensorParallelLayer`` (every expert's intermediate features split over
+the ranks, an all-reduce of the FP32 sums).
 """
 from ._lib import (  # noqa: F401
     Cfg, Experts, NvFp4MoeError, cfg_default, make_cfg, quantize, quantize_weights_lh, route, route_noalloc, forward,
