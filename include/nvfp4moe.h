@@ -30,6 +30,9 @@
  * Conventions for every call:
  *   * Tensor pointers are DEVICE pointers owned by the caller unless stated otherwise;
  *     row-major, densely packed.  BF16 is the IEEE bfloat16 bit pattern (uint16).
+ *   * Calls run on the calling thread's current CUDA device: device pointers are memory
+ *     of that device (or, for nvfp4moe_forward_partial_peer's table, memory mapped into
+ *     it) and `stream` is a stream of that device.
  *   * `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are asynchronous
  *     on it and allocate nothing; they return after enqueueing work.
  *   * Argument and shape errors are reported synchronously by the return code and

@@ -187,7 +187,8 @@ def _ptr(t):
 def _require(*specs):
     """Raise TypeError unless every (tensor, name, dtype, shape) of ``specs`` whose tensor is
     not None is a contiguous tensor of that dtype and shape (shape None: any), and all of them
-    are CUDA tensors on the first one's device.  Types and shapes are checked before devices.
+    are CUDA tensors on the first one's device, the current device.  Types and shapes are
+    checked before devices.
     The library receives raw pointers, so a tensor of the wrong type or size would be read out
     of bounds rather than rejected."""
     present = [s for s in specs if s[0] is not None]
@@ -203,6 +204,11 @@ def _require(*specs):
     for t, name, _, _ in present:
         if not t.is_cuda or t.device != present[0][0].device:
             raise TypeError(f"{name} must be a CUDA tensor on {present[0][0].device}, got {t.device}")
+    # the library launches on the current device: tensors of another one would be read
+    # through addresses that device does not map
+    if present and present[0][0].device.index != torch.cuda.current_device():
+        raise TypeError(f"the tensors are on {present[0][0].device} but the current device is "
+                        f"cuda:{torch.cuda.current_device()}: call under torch.cuda.device({present[0][0].device})")
 
 
 def _rows(x, name: str, min_rows: int = 1) -> int:
