@@ -141,3 +141,28 @@ def test_missing_library_fails_loudly(monkeypatch):
         _lib.lib()
     with pytest.raises(ImportError):
         _lib.cfg_default()
+
+
+class _OnCuda1(torch.Tensor):
+    """A CPU tensor that reports itself as memory of cuda:1 (the device check reads only
+    these two attributes)."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+    @property
+    def device(self):
+        return torch.device("cuda", 1)
+
+
+def test_tensors_of_another_device_than_the_current_one(monkeypatch):
+    """The library launches on the current device, so tensors of another device are refused
+    before any pointer reaches it."""
+    from nvfp4_quantized_moe_group_b200 import _lib
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    x = torch.zeros((4, 256), dtype=torch.bfloat16).as_subclass(_OnCuda1)
+    with pytest.raises(TypeError, match=r"on cuda:1 but the current device is cuda:0"):
+        _lib._require((x, "x", torch.bfloat16, (4, 256)))
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    _lib._require((x, "x", torch.bfloat16, (4, 256)))
